@@ -1,0 +1,203 @@
+/*
+ * moe.h -- C ABI of libmoe: the forward hot path of one sparse MoE layer
+ * (256 routed experts, top-6, plus 2 shared experts normalised jointly) and
+ * its auxiliary-loss-free bias update, as hand-written CUDA kernels for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one of "Inkling, Dissected" (engineermaxxing.com),
+ * §02 "Anatomy of one MoE layer" and §02b "Sigmoid, not softmax":
+ *     s_i = sigmoid(x . w_i)                       for all routed + shared experts
+ *     kept = top-k over routed i of (s_i + b_i)    (the bias steers selection only)
+ *     g_i  = s_i / sum_{j in kept U shared} s_j    (one joint normalisation)
+ *     out  = sum_{i in kept U shared} g_i * E_i(x),  E_i(x) = W2_i gelu(W1_i x)
+ * followed by §02e "The aux-loss-free bias":
+ *     b_i <- b_i + gamma * sign(Lbar - L_i),  L_i = tokens that picked i,
+ *     Lbar = (total selections) / n_routed.
+ * "Under the hood" (huggingface.co blog), "The routing strategy", adds that the
+ * shared experts join the normalisation but are never top-k candidates.
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - All tensor pointers are DEVICE pointers to caller-owned memory, row-major,
+ *    16-byte aligned.  The library allocates nothing and keeps no pointer after
+ *    a call returns.
+ *  - bf16 tensors are passed as moe_bf16 (the 16-bit pattern).
+ *  - Every call is asynchronous on the given cudaStream_t (passed as void*;
+ *    NULL = legacy default stream).  No call synchronises the host.
+ *  - Return value: MOE_OK or a negative MOE_ERR_* code.  Argument errors are
+ *    detected on the host before anything is launched; nothing is launched
+ *    when a call fails validation.  Calls never abort, exit or trap.
+ *  - Errors found on the device (a bounded wait that ran out, an expert index
+ *    out of range, inconsistent counts) set bits in a per-device status word
+ *    that moe_get_status() reads and clears.
+ *  - T = 0 (no tokens) is valid: the call does nothing except what it states
+ *    (moe_router_topk still zeroes counts).
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size or k   */
+#define MOE_ERR_UNSUPPORTED (-2) /* shape outside what the kernels handle      */
+#define MOE_ERR_CUDA (-3)        /* a CUDA runtime/driver call failed          */
+#define MOE_ERR_TIMEOUT (-4)     /* reported by moe_get_status: a device wait ran out */
+#define MOE_ERR_DEVICE (-5)      /* reported by moe_get_status: other device-side error */
+#define MOE_ERR_SCRATCH (-6)     /* scratch buffer smaller than required       */
+
+/* device status bits (moe_get_status) */
+#define MOE_STATUS_TIMEOUT 0x1u        /* a bounded mbarrier wait gave up          */
+#define MOE_STATUS_BAD_EXPERT 0x2u     /* permute saw an expert id outside [0,n)   */
+#define MOE_STATUS_COUNT_MISMATCH 0x4u /* permute's counts differ from topk_idx    */
+
+/* expert nonlinearity */
+#define MOE_ACT_GELU_TANH 0 /* gelu(u) = u/2 (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3))) */
+
+/* limits */
+#define MOE_MAX_TOP_K 8
+#define MOE_MAX_ROUTED 256
+#define MOE_MAX_SHARED 8
+#define MOE_MAX_GROUPS 1024
+
+/*
+ * moe_router_topk -- router scores, biased top-k, joint gates, load counts.
+ * "Inkling, Dissected" §02b (router formula and per-token sketch); "Under the
+ * hood", "The routing strategy", steps 1-4; loads L_i of §02e.
+ *
+ *   x          [T, d] bf16          hidden states
+ *   w_router   [n_routed + n_shared, d] bf16; rows 0..n_routed-1 routed,
+ *              the next n_shared rows the shared experts
+ *   bias       [n_routed] fp32      balancing bias b (selection only)
+ *   logit_offset [n_routed] fp32 or NULL: added to the routed logits before the
+ *              sigmoid (a workload input for skewed routing, not part of the method)
+ *   route_scale must be 1.0 (gates sum to 1)
+ *   topk_idx   [T, top_k] int32 out: kept routed experts, descending s_i + b_i,
+ *              ties to the lower index
+ *   gates      [T, top_k + n_shared] fp32 out: g of the kept experts in topk
+ *              order, then the shared experts in index order; per token they sum to 1
+ *   counts     [n_routed] int32 out: L_i; zeroed by this call, then accumulated
+ *   scores_out [T, n_routed + n_shared] fp32 or NULL: s_i for debugging
+ * Logits are accumulated in fp32 from bf16 products (tcgen05 tensor cores);
+ * s, s + b and the gates are fp32.
+ * Limits: d % 64 == 0, 1 <= top_k <= min(MOE_MAX_TOP_K, n_routed),
+ * n_routed <= 256, n_shared <= 8, n_routed + n_shared <= 272.
+ */
+int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const float* logit_offset,
+                    int T, int d, int n_routed, int n_shared, int top_k, float route_scale, int32_t* topk_idx,
+                    float* gates, int32_t* counts, float* scores_out, void* stream);
+
+/*
+ * moe_permute -- dispatch: group the T*top_k (token, slot) pairs by expert.
+ * "Inkling, Dissected" §02 (every token goes to exactly its top-k routed
+ * experts; dispatch precedes the experts) and §02d (tokens are queued per expert).
+ *
+ *   x          [T, d] bf16
+ *   topk_idx   [T, top_k] int32 (from moe_router_topk)
+ *   counts     [n_routed] int32 or NULL: if given, checked against topk_idx
+ *              (MOE_STATUS_COUNT_MISMATCH on the device if they differ); the
+ *              layout is always derived from topk_idx itself
+ *   offsets    [n_routed + 1] int32 out: rows of expert e are offsets[e] .. offsets[e+1]-1
+ *   x_perm     [T*top_k, d] bf16 out: row r = x[row_token[r]]
+ *   row_token  [T*top_k] int32 out
+ *   token_row  [T, top_k] int32 out: the row each (token, slot) went to
+ *   scratch    device buffer of at least moe_permute_scratch_bytes(T, n_routed)
+ *              bytes, caller-owned, contents need not be initialised
+ * Within an expert, rows are in increasing token order (deterministic).
+ * Limits: d % 8 == 0, n_routed <= 256, 1 <= top_k <= 8.
+ */
+size_t moe_permute_scratch_bytes(int T, int n_routed);
+int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d, int n_routed,
+                int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token, int32_t* token_row, void* scratch,
+                size_t scratch_bytes, void* stream);
+
+/*
+ * moe_grouped_ffn -- the expert MLPs, y = W2_e gelu(W1_e x), for groups of rows.
+ * "Inkling, Dissected" §02: an expert is two matrix multiplies with a
+ * nonlinearity between them (GELU, tanh form, here).
+ *
+ *   rows       [n_rows, d] bf16 input rows
+ *   offsets    [n_groups + 1] int32 or NULL.
+ *              Non-NULL: group g is rows offsets[g] .. offsets[g+1]-1 (device
+ *              values, e.g. from moe_permute), expert expert_base + g; h_scratch
+ *              is [n_rows, d_ff] and y is [n_rows, d].
+ *              NULL: every group sees all n_rows rows (the shared experts);
+ *              h_scratch is [n_groups, n_rows, d_ff] and y is [n_groups, n_rows, d].
+ *   w1         [*, d_ff, d] bf16 all experts' first matrices (K-major)
+ *   w2         [*, d, d_ff] bf16 all experts' second matrices (K-major)
+ *   expert_base index of the first expert used (group g uses expert_base + g)
+ *   activation MOE_ACT_GELU_TANH
+ *   h_scratch  bf16 hidden activations (caller-owned), written then read
+ * Tensor cores (tcgen05, bf16 in, fp32 accumulate); h is rounded to bf16
+ * between the two matmuls; y is bf16.
+ * Limits: d % 64 == 0, d_ff % 64 == 0, n_groups <= MOE_MAX_GROUPS.
+ */
+int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, int n_rows, int expert_base,
+                    const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff, int activation, moe_bf16* h_scratch,
+                    moe_bf16* y, void* stream);
+
+/*
+ * moe_combine -- gate-weighted sum of the contributors, back in token order.
+ * "Inkling, Dissected" §02 (the layer output is the weighted sum of the 8
+ * contributing experts) and §02b sketch (out += g_k * e_k(x)).
+ *
+ *   y_perm     [T*top_k, d] bf16 routed expert outputs in dispatch order
+ *   token_row  [T, top_k] int32 (from moe_permute)
+ *   gates      [T, top_k + n_shared] fp32 (from moe_router_topk)
+ *   y_shared   [n_shared, T, d] bf16 or NULL (then n_shared must be 0)
+ *   out        [T, d] bf16: out[t] = sum_j g[t,j] y_perm[token_row[t,j]]
+ *              + sum_s g[t,top_k+s] y_shared[s,t], accumulated in fp32
+ * Limits: d % 8 == 0, 1 <= top_k <= 8, n_shared <= 8.
+ */
+int moe_combine(const moe_bf16* y_perm, const int32_t* token_row, const float* gates, const moe_bf16* y_shared,
+                int T, int d, int top_k, int n_shared, moe_bf16* out, void* stream);
+
+/*
+ * moe_bias_update -- the aux-loss-free balancing controller, in place.
+ * "Inkling, Dissected" §02e: b_i <- b_i + gamma * sign(Lbar - L_i).
+ * Lbar = top_k * T / n_routed; the sign is taken in integers as
+ * sign(top_k*T - n_routed*counts[i]) (sign(0) = 0), and b_i is updated in fp32:
+ * b_i = fl32(b_i + fl32(gamma) * sign).  Runs after the forward, for the next batch.
+ *   counts [n_routed] int32, bias [n_routed] fp32 (in/out).
+ */
+int moe_bias_update(const int32_t* counts, int n_routed, int T, int top_k, float gamma, float* bias, void* stream);
+
+/* Human-readable text for a MOE_* return code. */
+const char* moe_status_string(int code);
+
+/*
+ * moe_get_status -- synchronise `stream`, then read and clear this device's
+ * status word (MOE_STATUS_* bits) into *device_status.  Returns MOE_OK,
+ * MOE_ERR_TIMEOUT if the timeout bit was set, MOE_ERR_DEVICE if another bit
+ * was set, or MOE_ERR_CUDA.
+ */
+int moe_get_status(void* stream, int* device_status);
+
+/*
+ * moe_set_wait_timeout_ns -- limit, in nanoseconds, on every device-side wait
+ * of the kernels launched afterwards (default 2e9).  A wait that runs out sets
+ * MOE_STATUS_TIMEOUT and its kernel winds down and returns.
+ */
+int moe_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * moe_debug_bounded_wait -- launch one CTA that waits on a shared-memory
+ * barrier which nothing ever completes, through the same bounded wait the
+ * GEMM kernels use; it must give up after timeout_ns and set
+ * MOE_STATUS_TIMEOUT.  For testing the failure path without faulting a GPU.
+ */
+int moe_debug_bounded_wait(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

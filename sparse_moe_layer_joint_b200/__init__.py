@@ -1,0 +1,236 @@
+"""Python binding of libmoe (the C ABI declared in include/moe.h).
+
+Argument marshalling only: every step of the MoE layer runs in the library's
+CUDA kernels.  Tensors are torch CUDA tensors (PyTorch supplies device memory
+and streams, nothing else); each function takes the same arguments, in the same
+order, as its C counterpart, with pointers replaced by tensors and the stream
+defaulting to torch's current stream.  A non-zero return code raises MoEError.
+
+Importing this module fails loudly if libmoe.so has not been built; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                      "(there is no non-CUDA implementation of this layer)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_TIMEOUT = -4
+MOE_ERR_DEVICE = -5
+MOE_ERR_SCRATCH = -6
+MOE_STATUS_TIMEOUT = 0x1
+MOE_STATUS_BAD_EXPERT = 0x2
+MOE_STATUS_COUNT_MISMATCH = 0x4
+MOE_ACT_GELU_TANH = 0
+
+_vp, _i32, _u64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_float, ctypes.c_size_t
+
+_lib.moe_router_topk.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _vp]
+_lib.moe_permute_scratch_bytes.argtypes = [_i32, _i32]
+_lib.moe_permute_scratch_bytes.restype = _sz
+_lib.moe_permute.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_grouped_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
+_lib.moe_bias_update.argtypes = [_vp, _i32, _i32, _i32, _f32, _vp, _vp]
+_lib.moe_status_string.argtypes = [_i32]
+_lib.moe_status_string.restype = ctypes.c_char_p
+_lib.moe_get_status.argtypes = [_vp, ctypes.POINTER(_i32)]
+_lib.moe_set_wait_timeout_ns.argtypes = [_u64]
+_lib.moe_debug_bounded_wait.argtypes = [_u64, _vp]
+for _f in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_bias_update", "moe_get_status",
+           "moe_set_wait_timeout_ns", "moe_debug_bounded_wait"):
+    getattr(_lib, _f).restype = _i32
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {code}: {status_string(code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/moe.h declares."""
+    with open(HEADER_PATH) as fh:
+        text = fh.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(moe_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def status_string(code: int) -> str:
+    return _lib.moe_status_string(int(code)).decode()
+
+
+def _p(t) -> Optional[int]:
+    """Device address of a tensor (or an int address); None for None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, rc: int):
+    if rc != MOE_OK:
+        raise MoEError(fn, rc)
+
+
+# ---------------------------------------------------------------------------
+# the five calls of the layer, same names and argument order as the C ABI
+# ---------------------------------------------------------------------------
+def moe_router_topk(x, w_router, bias, logit_offset, T: int, d: int, n_routed: int, n_shared: int, top_k: int,
+                    route_scale: float, topk_idx, gates, counts, scores_out=None, stream=None):
+    _check("moe_router_topk", _lib.moe_router_topk(
+        _p(x), _p(w_router), _p(bias), _p(logit_offset), T, d, n_routed, n_shared, top_k, route_scale,
+        _p(topk_idx), _p(gates), _p(counts), _p(scores_out), _stream(stream)))
+
+
+def moe_permute_scratch_bytes(T: int, n_routed: int) -> int:
+    return int(_lib.moe_permute_scratch_bytes(T, n_routed))
+
+
+def moe_permute(x, topk_idx, counts, T: int, d: int, n_routed: int, top_k: int, offsets, x_perm, row_token,
+                token_row, scratch, scratch_bytes: int, stream=None):
+    _check("moe_permute", _lib.moe_permute(
+        _p(x), _p(topk_idx), _p(counts), T, d, n_routed, top_k, _p(offsets), _p(x_perm), _p(row_token),
+        _p(token_row), _p(scratch), scratch_bytes, _stream(stream)))
+
+
+def moe_grouped_ffn(rows, offsets, n_groups: int, n_rows: int, expert_base: int, w1, w2, d: int, d_ff: int,
+                    activation: int, h_scratch, y, stream=None):
+    _check("moe_grouped_ffn", _lib.moe_grouped_ffn(
+        _p(rows), _p(offsets), n_groups, n_rows, expert_base, _p(w1), _p(w2), d, d_ff, activation, _p(h_scratch),
+        _p(y), _stream(stream)))
+
+
+def moe_combine(y_perm, token_row, gates, y_shared, T: int, d: int, top_k: int, n_shared: int, out, stream=None):
+    _check("moe_combine", _lib.moe_combine(
+        _p(y_perm), _p(token_row), _p(gates), _p(y_shared), T, d, top_k, n_shared, _p(out), _stream(stream)))
+
+
+def moe_bias_update(counts, n_routed: int, T: int, top_k: int, gamma: float, bias, stream=None):
+    _check("moe_bias_update", _lib.moe_bias_update(_p(counts), n_routed, T, top_k, gamma, _p(bias), _stream(stream)))
+
+
+def moe_get_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status bits."""
+    v = _i32(0)
+    rc = _lib.moe_get_status(_stream(stream), ctypes.byref(v))
+    if rc not in (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE):
+        raise MoEError("moe_get_status", rc)
+    return v.value
+
+
+def moe_set_wait_timeout_ns(ns: int):
+    _check("moe_set_wait_timeout_ns", _lib.moe_set_wait_timeout_ns(int(ns)))
+
+
+def moe_debug_bounded_wait(timeout_ns: int, stream=None):
+    _check("moe_debug_bounded_wait", _lib.moe_debug_bounded_wait(int(timeout_ns), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# host orchestration of one layer forward: the calls above, in the pages'
+# order, on two streams (shared experts beside the routed path)
+# ---------------------------------------------------------------------------
+@dataclass
+class LayerShape:
+    T: int
+    d: int
+    d_ff: int
+    n_routed: int = 256
+    n_shared: int = 2
+    top_k: int = 6
+
+
+class MoELayer:
+    """Device buffers for one layer shape and the call sequence of a forward.
+
+    Weights are caller-owned torch tensors: w_router [n_routed + n_shared, d],
+    w1 [n_routed + n_shared, d_ff, d], w2 [n_routed + n_shared, d, d_ff] (bf16),
+    bias [n_routed] fp32 (updated in place by ``bias_update``).
+    """
+
+    def __init__(self, shape: LayerShape, device="cuda"):
+        import torch
+
+        self.shape = s = shape
+        dev = torch.device(device)
+        R = s.T * s.top_k
+        bf = torch.bfloat16
+        self.topk_idx = torch.empty((s.T, s.top_k), dtype=torch.int32, device=dev)
+        self.gates = torch.empty((s.T, s.top_k + s.n_shared), dtype=torch.float32, device=dev)
+        self.counts = torch.empty((s.n_routed,), dtype=torch.int32, device=dev)
+        self.offsets = torch.empty((s.n_routed + 1,), dtype=torch.int32, device=dev)
+        self.x_perm = torch.empty((max(R, 1), s.d), dtype=bf, device=dev)
+        self.row_token = torch.empty((max(R, 1),), dtype=torch.int32, device=dev)
+        self.token_row = torch.empty((s.T, s.top_k), dtype=torch.int32, device=dev)
+        self.scratch_bytes = moe_permute_scratch_bytes(s.T, s.n_routed)
+        self.scratch = torch.empty((self.scratch_bytes,), dtype=torch.uint8, device=dev)
+        self.h = torch.empty((max(R, 1), s.d_ff), dtype=bf, device=dev)
+        self.y_perm = torch.empty((max(R, 1), s.d), dtype=bf, device=dev)
+        self.h_shared = torch.empty((max(s.n_shared, 1), s.T, s.d_ff), dtype=bf, device=dev)
+        self.y_shared = torch.empty((max(s.n_shared, 1), s.T, s.d), dtype=bf, device=dev)
+        self.out = torch.empty((s.T, s.d), dtype=bf, device=dev)
+        self.side = torch.cuda.Stream(device=dev)
+        self.ev_start = torch.cuda.Event()
+        self.ev_shared = torch.cuda.Event()
+
+    def forward(self, x, w_router, w1, w2, bias, logit_offset=None, stream=None, scores_out=None):
+        """Router -> permute -> routed experts (stream A) | shared experts (stream B) -> combine."""
+        import torch
+
+        s = self.shape
+        main = stream if stream is not None else torch.cuda.current_stream()
+        T, d, f, k = s.T, s.d, s.d_ff, s.top_k
+        self.ev_start.record(main)
+        # shared experts see every token: start them beside the routed path
+        if s.n_shared > 0:
+            self.side.wait_event(self.ev_start)
+            moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h_shared,
+                            self.y_shared, stream=self.side)
+            self.ev_shared.record(self.side)
+        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, 1.0, self.topk_idx,
+                        self.gates, self.counts, scores_out, stream=main)
+        moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, self.x_perm, self.row_token,
+                    self.token_row, self.scratch, self.scratch_bytes, stream=main)
+        moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h,
+                        self.y_perm, stream=main)
+        if s.n_shared > 0:
+            main.wait_event(self.ev_shared)
+        moe_combine(self.y_perm, self.token_row, self.gates, self.y_shared if s.n_shared > 0 else None, T, d, k,
+                    s.n_shared, self.out, stream=main)
+        return self.out
+
+    def bias_update(self, bias, gamma: float, stream=None):
+        s = self.shape
+        moe_bias_update(self.counts, s.n_routed, s.T, s.top_k, gamma, bias, stream=stream)

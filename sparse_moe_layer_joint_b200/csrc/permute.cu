@@ -1,0 +1,211 @@
+// permute.cu -- dispatch: group the T*k (token, slot) pairs by expert, rows of
+// one expert in increasing token order ("Inkling, Dissected" §02: each token
+// goes to exactly its k routed experts; §02d: tokens queue per expert).
+//
+// Three launches, all deterministic (no atomics decide a position):
+//   1. chunk_hist   one CTA per 256-token chunk: hist[c][e] = picks of e in chunk c
+//   2. chunk_scan   one CTA: offsets[e] = exclusive scan over experts of the
+//                   per-expert totals; base[c][e] = offsets[e] + picks of e in
+//                   chunks before c; optional check of the caller's counts
+//   3. scatter      one CTA per chunk: each warp takes 32 tokens; a per-warp
+//                   bitmask per expert (bit = lane) gives each pick its rank
+//                   among earlier lanes, a prefix over the 8 warps gives the
+//                   rank among earlier warps; then the warp copies x rows to
+//                   their destinations with 16-byte loads/stores, reading each
+//                   x row once and writing it k times.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace perm {
+
+constexpr int CHUNK = 256;  // tokens per chunk (8 warps x 32)
+constexpr int THREADS = 256;
+constexpr int WARPS = THREADS / 32;
+constexpr int ROW_VEC = 8;  // uint4 per lane per pass of the row copy
+
+__global__ void __launch_bounds__(THREADS) chunk_hist_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
+                                                             int n_routed, int32_t* __restrict__ hist,
+                                                             unsigned int* status) {
+  __shared__ int h[MOE_MAX_ROUTED];
+  for (int e = threadIdx.x; e < MOE_MAX_ROUTED; e += THREADS) h[e] = 0;
+  __syncthreads();
+  const int c = blockIdx.x;
+  const int t0 = c * CHUNK;
+  const int n = min(CHUNK, T - t0) * k;
+  const int32_t* src = topk_idx + (size_t)t0 * k;
+  bool bad = false;
+  for (int i = threadIdx.x; i < n; i += THREADS) {
+    int e = src[i];
+    if (e >= 0 && e < n_routed)
+      atomicAdd(&h[e], 1);
+    else
+      bad = true;
+  }
+  if (bad) set_status(status, MOE_STATUS_BAD_EXPERT);
+  __syncthreads();
+  for (int e = threadIdx.x; e < n_routed; e += THREADS) hist[(size_t)c * n_routed + e] = h[e];
+}
+
+// One CTA of 256 threads; thread e owns expert e.
+__global__ void __launch_bounds__(THREADS) chunk_scan_kernel(const int32_t* __restrict__ hist, int n_chunks,
+                                                             int n_routed, const int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ base, unsigned int* status) {
+  __shared__ int tot[MOE_MAX_ROUTED];
+  __shared__ int warp_sum[WARPS];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < n_routed) {
+    for (int c = 0; c < n_chunks; ++c) total += hist[(size_t)c * n_routed + e];
+    if (counts != nullptr && counts[e] != total) set_status(status, MOE_STATUS_COUNT_MISMATCH);
+  }
+  // exclusive scan of totals over experts
+  const int lane = e & 31, w = e >> 5;
+  int v = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_sum[w] = v;
+  __syncthreads();
+  int before = 0;
+  for (int i = 0; i < w; ++i) before += warp_sum[i];
+  const int excl = before + v - total;
+  tot[e] = excl;
+  if (e < n_routed) offsets[e] = excl;
+  if (e == n_routed - 1) offsets[n_routed] = excl + total;
+  __syncthreads();
+  if (e < n_routed) {
+    int run = tot[e];
+    for (int c = 0; c < n_chunks; ++c) {
+      base[(size_t)c * n_routed + e] = run;
+      run += hist[(size_t)c * n_routed + e];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS) scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
+                                                          const int32_t* __restrict__ base, int T, int d_vec, int k,
+                                                          int n_routed, uint4* __restrict__ x_perm,
+                                                          int32_t* __restrict__ row_token,
+                                                          int32_t* __restrict__ token_row) {
+  __shared__ uint32_t mask[WARPS][MOE_MAX_ROUTED];
+  __shared__ int pre[WARPS][MOE_MAX_ROUTED];
+  const int c = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < WARPS * MOE_MAX_ROUTED; i += THREADS) (&mask[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = c * CHUNK + warp * 32 + lane;
+  const bool valid = t < T;
+  int ex[MOE_MAX_TOP_K];
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+    ex[j] = -1;
+    if (j < k && valid) {
+      int e = topk_idx[(size_t)t * k + j];
+      if (e >= 0 && e < n_routed) {
+        ex[j] = e;
+        atomicOr(&mask[warp][e], 1u << lane);
+      }
+    }
+  }
+  __syncthreads();
+  // prefix over warps, per expert
+  for (int e = threadIdx.x; e < n_routed; e += THREADS) {
+    int run = base[(size_t)c * n_routed + e];
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      pre[w][e] = run;
+      run += __popc(mask[w][e]);
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  int pos[MOE_MAX_TOP_K];
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+    pos[j] = -1;
+    if (ex[j] >= 0) {
+      pos[j] = pre[warp][ex[j]] + __popc(mask[warp][ex[j]] & lt);
+      token_row[(size_t)t * k + j] = pos[j];
+      row_token[pos[j]] = t;
+    } else if (j < k && valid) {
+      token_row[(size_t)t * k + j] = -1;
+    }
+  }
+  // row copies: the warp walks its 32 tokens; each lane moves 16-byte pieces
+  for (int src = 0; src < 32; ++src) {
+    const int ts = c * CHUNK + warp * 32 + src;
+    if (ts >= T) break;
+    int dst[MOE_MAX_TOP_K];
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOP_K; ++j) dst[j] = __shfl_sync(0xffffffffu, pos[j], src);
+    const uint4* xs = x + (size_t)ts * d_vec;
+    for (int v0 = 0; v0 < d_vec; v0 += 32 * ROW_VEC) {
+      uint4 buf[ROW_VEC];
+#pragma unroll
+      for (int q = 0; q < ROW_VEC; ++q) {
+        int vi = v0 + q * 32 + lane;
+        if (vi < d_vec) buf[q] = __ldg(xs + vi);
+      }
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+        if (j < k && dst[j] >= 0) {
+          uint4* xd = x_perm + (size_t)dst[j] * d_vec;
+#pragma unroll
+          for (int q = 0; q < ROW_VEC; ++q) {
+            int vi = v0 + q * 32 + lane;
+            if (vi < d_vec) xd[vi] = buf[q];
+          }
+        }
+      }
+    }
+  }
+}
+
+}  // namespace perm
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_permute_scratch_bytes(int T, int n_routed) {
+  if (T <= 0 || n_routed <= 0) return 256;
+  size_t n_chunks = ((size_t)T + perm::CHUNK - 1) / perm::CHUNK;
+  return 2 * n_chunks * (size_t)n_routed * sizeof(int32_t) + 256;
+}
+
+extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                           int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
+                           int32_t* token_row, void* scratch, size_t scratch_bytes, void* stream) {
+  using namespace moe::perm;
+  if (T < 0 || d <= 0 || n_routed < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
+  if (top_k > MOE_MAX_TOP_K || top_k > n_routed || n_routed > MOE_MAX_ROUTED) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!x || !topk_idx || !offsets || !x_perm || !row_token || !token_row || !scratch) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned4(topk_idx) || !aligned4(counts) || !aligned4(offsets) ||
+      !aligned4(row_token) || !aligned4(token_row) || !aligned16(scratch))
+    return MOE_ERR_INVALID_ARG;
+  if ((long long)T * top_k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (scratch_bytes < moe_permute_scratch_bytes(T, n_routed)) return MOE_ERR_SCRATCH;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (T == 0) {
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (n_routed + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  unsigned int* status = status_ptr();
+  if (!status) return MOE_ERR_CUDA;
+  const int n_chunks = (T + CHUNK - 1) / CHUNK;
+  int32_t* hist = reinterpret_cast<int32_t*>(scratch);
+  int32_t* base = hist + (size_t)n_chunks * n_routed;
+  chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
+  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, counts, offsets, base, status);
+  scatter_kernel<<<n_chunks, THREADS, 0, s>>>(reinterpret_cast<const uint4*>(x), topk_idx, base, T, d / 8, top_k,
+                                               n_routed, reinterpret_cast<uint4*>(x_perm), row_token, token_row);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

@@ -1,0 +1,346 @@
+// router.cu -- router GEMM with the routing fused into its epilogue
+// ("Inkling, Dissected" §02b: s_i = sigmoid(x . w_i); keep the top 6 by
+// s_i + b_i; g_i = s_i / sum over kept U shared; "Under the hood", "The
+// routing strategy": 256 routed + 2 shared scores, top-k over routed only).
+//
+// One CTA per 128 tokens.  The logits of all n_routed + n_shared experts for
+// the CTA's tokens are one 128 x 272 fp32 accumulator in TMEM: a tcgen05 MMA
+// with N = 256 (experts 0..255) and one with N = 16 (experts 256..271, zero
+// rows past the last expert) per 16-deep K step, fed by TMA through a 4-stage
+// ring.  In the epilogue each of the 128 epilogue threads owns one token (its
+// TMEM lane): it reads its 258 logits 32 at a time, applies the sigmoid, adds
+// the bias for selection, keeps a register top-k list (strict '>' while
+// scanning experts in index order, so ties keep the lower index), then forms
+// the joint gates and counts its picks in a shared-memory histogram that is
+// added to the global counts once per CTA.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "moe.h"
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace router {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B0_ROWS = 256;
+constexpr int B1_ROWS = 16;
+constexpr int B0_BYTES = B0_ROWS * BK * 2;
+constexpr int B1_BYTES = B1_ROWS * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B0_BYTES + B1_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct Params {
+  const float* bias;
+  const float* offset;  // nullable
+  int T, d, n_routed, n_shared;
+  int32_t* topk_idx;
+  float* gates;
+  int32_t* counts;
+  float* scores;  // nullable
+  uint64_t timeout_ns;
+  unsigned int* status;
+};
+
+struct SmemTail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float bias[MOE_MAX_ROUTED];
+  float off[MOE_MAX_ROUTED];
+  int hist[MOE_MAX_ROUTED];
+  float shared_s[BM][MOE_MAX_SHARED];
+};
+
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+
+__device__ __forceinline__ float sigmoid_f32(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+template <int K>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    router_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                  const __grid_constant__ CUtensorMap tmB1, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemTail* st = reinterpret_cast<SmemTail*>(smem + STAGES * STAGE_BYTES);
+  auto stageA = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto stageB0 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+  auto stageB1 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B0_BYTES; };
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int E = p.n_routed + p.n_shared;
+  const bool two = E > B0_ROWS;
+  const int m0 = blockIdx.x * BM;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&st->full[s], 1);
+      mbar_init(&st->empty[s], 1);
+    }
+    mbar_init(&st->tfull, 1);
+    mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    fence_barrier_init();
+  }
+  for (int i = tid; i < MOE_MAX_ROUTED; i += NUM_THREADS) {
+    st->bias[i] = i < p.n_routed ? p.bias[i] : 0.0f;
+    st->off[i] = (p.offset != nullptr && i < p.n_routed) ? p.offset[i] : 0.0f;
+    st->hist[i] = 0;
+  }
+  if (warp == 1) tmem_alloc(&st->tmem_base, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = st->tmem_base;
+  const int num_kb = p.d / BK;
+  volatile int* abort_flag = &st->abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB0);
+      if (two) tma_prefetch_desc(&tmB1);
+      const uint32_t bytes = (uint32_t)(A_BYTES + B0_BYTES + (two ? B1_BYTES : 0));
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&st->full[stage], bytes);
+        tma_load_2d(stageA(stage), &tmA, &st->full[stage], kb * BK, m0);
+        tma_load_2d(stageB0(stage), &tmB0, &st->full[stage], kb * BK, 0);
+        if (two) tma_load_2d(stageB1(stage), &tmB1, &st->full[stage], kb * BK, B0_ROWS);
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        int zero = 0;
+        for (long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+          mbar_wait(&st->full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.timeout_ns, &zero, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc0 = make_idesc_bf16(BM, B0_ROWS);
+      constexpr uint32_t idesc1 = make_idesc_bf16(BM, B1_ROWS);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&st->full[stage], phase, p.timeout_ns, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = smem_u32(stageA(stage));
+        const uint32_t b0 = smem_u32(stageB0(stage));
+        const uint32_t b1 = smem_u32(stageB1(stage));
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
+          mma_bf16_ss(tmem_base, make_desc_sw128(a + k * 32), make_desc_sw128(b0 + k * 32), idesc0, acc);
+          if (two)
+            mma_bf16_ss(tmem_base + B0_ROWS, make_desc_sw128(a + k * 32), make_desc_sw128(b1 + k * 32), idesc1,
+                        acc);
+        }
+        mma_commit(&st->empty[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) mma_commit(&st->tfull);
+      int zero = 0;
+      mma_commit(&st->drain);
+      mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
+    }
+  } else {
+    // ================= epilogue: one token per thread =================
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int t = m0 + row;
+    const bool valid = t < p.T;
+    const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    if (mbar_wait(&st->tfull, 0, p.timeout_ns, abort_flag, p.status)) {
+      tc_fence_after();
+      float val[K], sc[K];
+      int id[K];
+#pragma unroll
+      for (int q = 0; q < K; ++q) {
+        val[q] = -INFINITY;
+        sc[q] = 0.0f;
+        id[q] = 0x7fffffff;
+      }
+      float* srow = (p.scores != nullptr && valid) ? p.scores + (size_t)t * E : nullptr;
+      auto consume = [&](int i, float z) {
+        if (i < p.n_routed) {
+          float s = sigmoid_f32(z + st->off[i]);
+          float sel = s + st->bias[i];
+          if (srow) srow[i] = s;
+          if (sel > val[K - 1]) {
+            val[K - 1] = sel;
+            sc[K - 1] = s;
+            id[K - 1] = i;
+#pragma unroll
+            for (int q = K - 1; q > 0; --q) {
+              if (val[q] > val[q - 1]) {
+                float tv = val[q]; val[q] = val[q - 1]; val[q - 1] = tv;
+                float ts = sc[q]; sc[q] = sc[q - 1]; sc[q - 1] = ts;
+                int ti = id[q]; id[q] = id[q - 1]; id[q - 1] = ti;
+              }
+            }
+          }
+        } else if (i < E) {
+          float s = sigmoid_f32(z);
+          if (srow) srow[i] = s;
+          st->shared_s[row][i - p.n_routed] = s;
+        }
+      };
+      const int lim = E < B0_ROWS ? E : B0_ROWS;
+#pragma unroll 1
+      for (int c0 = 0; c0 < lim; c0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < lim) consume(c0 + j, v[j]);
+      }
+      if (two) {
+        float v[16];
+        tmem_ld16(taddr + B0_ROWS, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (B0_ROWS + j < E) consume(B0_ROWS + j, v[j]);
+      }
+      if (valid) {
+        // joint denominator: a sum over the contributor set, in ascending index
+        float den = 0.0f;
+        int prev = -1;
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+          int best = 0x7fffffff;
+          float bs = 0.0f;
+#pragma unroll
+          for (int r = 0; r < K; ++r)
+            if (id[r] > prev && id[r] < best) {
+              best = id[r];
+              bs = sc[r];
+            }
+          den += bs;
+          prev = best;
+        }
+        for (int q = 0; q < p.n_shared; ++q) den += st->shared_s[row][q];
+        const int G = K + p.n_shared;
+        int32_t* ti = p.topk_idx + (size_t)t * K;
+        float* gt = p.gates + (size_t)t * G;
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+          ti[q] = id[q];
+          gt[q] = __fdiv_rn(sc[q], den);
+          if (id[q] < p.n_routed) atomicAdd(&st->hist[id[q]], 1);  // unset only for non-finite scores
+        }
+        for (int q = 0; q < p.n_shared; ++q) gt[K + q] = __fdiv_rn(st->shared_s[row][q], den);
+      }
+    }
+    named_bar_sync(1, 128);
+    for (int e = row; e < p.n_routed; e += 128) {
+      int c = st->hist[e];
+      if (c) atomicAdd(&p.counts[e], c);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int K>
+int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const Params& p, int grid,
+           cudaStream_t s) {
+  auto kfn = router_kernel<K>;
+  int rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES);
+  if (rc != MOE_OK) return rc;
+  kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace router
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                               const float* logit_offset, int T, int d, int n_routed, int n_shared, int top_k,
+                               float route_scale, int32_t* topk_idx, float* gates, int32_t* counts,
+                               float* scores_out, void* stream) {
+  using namespace moe::router;
+  if (!x || !w_router || !bias || !topk_idx || !gates || !counts) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(gates) ||
+      !aligned4(counts) || !aligned4(logit_offset) || !aligned4(scores_out))
+    return MOE_ERR_INVALID_ARG;
+  if (T < 0 || d <= 0 || n_routed < 1 || n_shared < 0 || top_k < 1) return MOE_ERR_INVALID_ARG;
+  if (top_k > MOE_MAX_TOP_K || top_k > n_routed) return MOE_ERR_INVALID_ARG;
+  if (route_scale != 1.0f) return MOE_ERR_UNSUPPORTED;
+  if (n_routed > MOE_MAX_ROUTED || n_shared > MOE_MAX_SHARED || n_routed + n_shared > B0_ROWS + B1_ROWS)
+    return MOE_ERR_UNSUPPORTED;
+  if (d % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * n_routed, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (T == 0) return MOE_OK;
+
+  const int E = n_routed + n_shared;
+  CUtensorMap tA, tB0, tB1;
+  int rc;
+  if ((rc = encode_tmap_bf16(&tA, x, 2, (uint64_t)d, (uint64_t)T, 1, BK, BM)) != MOE_OK) return rc;
+  if ((rc = encode_tmap_bf16(&tB0, w_router, 2, (uint64_t)d, (uint64_t)E, 1, BK, B0_ROWS)) != MOE_OK) return rc;
+  if ((rc = encode_tmap_bf16(&tB1, w_router, 2, (uint64_t)d, (uint64_t)E, 1, BK, B1_ROWS)) != MOE_OK) return rc;
+
+  Params p{};
+  p.bias = bias;
+  p.offset = logit_offset;
+  p.T = T;
+  p.d = d;
+  p.n_routed = n_routed;
+  p.n_shared = n_shared;
+  p.topk_idx = topk_idx;
+  p.gates = gates;
+  p.counts = counts;
+  p.scores = scores_out;
+  p.timeout_ns = wait_timeout_ns();
+  p.status = status_ptr();
+  if (!p.status) return MOE_ERR_CUDA;
+  const int grid = (T + BM - 1) / BM;
+  switch (top_k) {
+    case 1: return launch<1>(tA, tB0, tB1, p, grid, s);
+    case 2: return launch<2>(tA, tB0, tB1, p, grid, s);
+    case 3: return launch<3>(tA, tB0, tB1, p, grid, s);
+    case 4: return launch<4>(tA, tB0, tB1, p, grid, s);
+    case 5: return launch<5>(tA, tB0, tB1, p, grid, s);
+    case 6: return launch<6>(tA, tB0, tB1, p, grid, s);
+    case 7: return launch<7>(tA, tB0, tB1, p, grid, s);
+    default: return launch<8>(tA, tB0, tB1, p, grid, s);
+  }
+}

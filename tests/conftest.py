@@ -11,17 +11,15 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: takes more than a few seconds")
-
-
-@pytest.fixture(scope="session", autouse=True)
-def _built_libs():
-    """Build the CPU-side libraries (generator, oracle) in-tree if stale."""
+    # build the in-tree libraries if stale (no-op when up to date), before the
+    # test modules import them
     import moe_inputs.build
     import oracle.build
+    import sparse_moe_layer_joint_b200.build as moe_build
 
     moe_inputs.build.build()
     oracle.build.build()
-    yield
+    moe_build.build()
 
 
 def cuda_ok():

@@ -1,0 +1,113 @@
+"""The C ABI without a GPU: the library loads, exports every function
+include/moe.h declares, and rejects bad arguments on the host (nothing is
+launched for a call that fails validation, so these run on a CPU-only box)."""
+import ctypes
+
+import pytest
+
+import sparse_moe_layer_joint_b200 as moe
+
+NULL = None
+A16 = 0x10000      # a 16-byte aligned, never dereferenced fake device address
+MIS = 0x10004      # misaligned by 4
+
+
+def test_every_declared_function_is_exported():
+    names = moe.header_functions()
+    assert {"moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_bias_update"} <= set(names)
+    for n in names:
+        assert hasattr(moe.lib(), n), n
+
+
+def test_status_strings():
+    for code in (moe.MOE_OK, moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_UNSUPPORTED, moe.MOE_ERR_CUDA,
+                 moe.MOE_ERR_TIMEOUT, moe.MOE_ERR_DEVICE, moe.MOE_ERR_SCRATCH):
+        assert moe.status_string(code) and moe.status_string(code) != "unknown status"
+    assert moe.status_string(12345) == "unknown status"
+
+
+def test_permute_scratch_size():
+    assert moe.moe_permute_scratch_bytes(0, 256) >= 0
+    a = moe.moe_permute_scratch_bytes(65536, 256)
+    assert a >= 2 * 256 * 256 * 4
+    assert moe.moe_permute_scratch_bytes(257, 256) > moe.moe_permute_scratch_bytes(256, 256)
+
+
+L = moe.lib()
+
+
+def router(**kw):
+    a = dict(x=A16, w=A16, b=A16, off=NULL, T=4, d=64, nr=256, ns=2, k=6, rs=1.0, idx=A16, g=A16, c=A16, sc=NULL,
+             s=NULL)
+    a.update(kw)
+    return L.moe_router_topk(a["x"], a["w"], a["b"], a["off"], a["T"], a["d"], a["nr"], a["ns"], a["k"], a["rs"],
+                             a["idx"], a["g"], a["c"], a["sc"], a["s"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(x=MIS), moe.MOE_ERR_INVALID_ARG),
+    (dict(w=MIS), moe.MOE_ERR_INVALID_ARG),
+    (dict(c=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(off=0x10002), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=9), moe.MOE_ERR_INVALID_ARG),
+    (dict(nr=4, k=5), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(d=100), moe.MOE_ERR_UNSUPPORTED),
+    (dict(nr=300), moe.MOE_ERR_UNSUPPORTED),
+    (dict(ns=9), moe.MOE_ERR_UNSUPPORTED),
+    (dict(rs=8.0), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_router_rejects(kw, code):
+    assert router(**kw) == code
+
+
+def test_permute_rejects():
+    ok = dict(x=A16, idx=A16, cnt=NULL, T=8, d=64, nr=256, k=6, off=A16, xp=A16, rt=A16, tr=A16, scr=A16,
+              sb=1 << 20, s=NULL)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.moe_permute(a["x"], a["idx"], a["cnt"], a["T"], a["d"], a["nr"], a["k"], a["off"], a["xp"],
+                             a["rt"], a["tr"], a["scr"], a["sb"], a["s"])
+
+    assert call(x=NULL) == moe.MOE_ERR_INVALID_ARG
+    assert call(xp=MIS) == moe.MOE_ERR_INVALID_ARG
+    assert call(k=9) == moe.MOE_ERR_INVALID_ARG
+    assert call(d=12) == moe.MOE_ERR_UNSUPPORTED
+    assert call(sb=16) == moe.MOE_ERR_SCRATCH
+    assert call(scr=NULL) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_grouped_ffn_rejects_and_empty_is_noop():
+    def call(rows=A16, off=A16, G=256, n=100, base=0, w1=A16, w2=A16, d=64, f=64, act=0, h=A16, y=A16):
+        return L.moe_grouped_ffn(rows, off, G, n, base, w1, w2, d, f, act, h, y, NULL)
+
+    assert call(rows=NULL) == moe.MOE_ERR_INVALID_ARG
+    assert call(w1=MIS) == moe.MOE_ERR_INVALID_ARG
+    assert call(act=3) == moe.MOE_ERR_INVALID_ARG
+    assert call(d=96) == moe.MOE_ERR_UNSUPPORTED
+    assert call(f=100) == moe.MOE_ERR_UNSUPPORTED
+    assert call(G=5000) == moe.MOE_ERR_UNSUPPORTED
+    assert call(n=-1) == moe.MOE_ERR_INVALID_ARG
+    # no rows or no groups: nothing to do, nothing launched
+    assert call(n=0) == moe.MOE_OK
+    assert call(G=0) == moe.MOE_OK
+
+
+def test_combine_and_bias_update_reject():
+    assert L.moe_combine(A16, A16, A16, NULL, 4, 64, 6, 2, A16, NULL) == moe.MOE_ERR_INVALID_ARG  # y_shared missing
+    assert L.moe_combine(A16, A16, A16, A16, 4, 60, 6, 2, A16, NULL) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_combine(MIS, A16, A16, A16, 4, 64, 6, 2, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(A16, A16, A16, A16, 0, 64, 6, 2, A16, NULL) == moe.MOE_OK   # T = 0
+    assert L.moe_bias_update(NULL, 256, 4, 6, 1e-3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_bias_update(A16, 0, 4, 6, 1e-3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_bias_update(A16, 256, 4, 6, float("nan"), A16, NULL) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_wait_timeout_setting():
+    assert L.moe_set_wait_timeout_ns(0) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_set_wait_timeout_ns(2_000_000_000) == moe.MOE_OK
+    assert L.moe_debug_bounded_wait(0, NULL) == moe.MOE_ERR_INVALID_ARG
