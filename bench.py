@@ -1,0 +1,330 @@
+"""Benchmark: MoE-layer forward tokens/s on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|mid|skew|tiny]
+                    [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of T tokens: router
+(scores, biased top-6, joint gates, counts) -> dispatch -> routed experts
+(tcgen05 grouped GEMMs) beside the shared experts (second stream) -> combine
+-> bias update.  Inputs are seeded synthetic tensors of the workload's shape,
+generated in HBM before timing; every input (x 0.94 GB, weights 15 GB at the
+prefill size) is far larger than the 126 MB L2, so no L2 flush is needed.
+
+With N > 1 (torchrun, one process per GPU) each rank runs the layer on its own
+T tokens (data-parallel replicas of the same weights: weak scaling); the load
+counts are summed over ranks with one NCCL all-reduce (256 int32) before the
+bias update, so every replica keeps the same bias.
+
+--impl reference times the CPU oracle (fp64, the layer's plain definition) on
+the host cores on a bounded sample of the same workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200; % BF16 tensor peak (prefill), % HBM BW (decode)"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "src": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED, "src": "fallback"}
+
+
+def config_of(w, world):
+    return {"workload": w.name, "description": w.description, "T_per_gpu": w.T, "global_tokens": w.T * world,
+            "d": w.d, "d_ff": w.f, "n_routed": w.n_routed, "n_shared": w.n_shared, "top_k": w.k,
+            "activation": "gelu_tanh", "parallelism": f"dp{world} (replicas, counts all-reduced)" if world > 1
+            else "single GPU", "l2": "inputs larger than L2 (no flush)", "seed": w.seed}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm: the CUDA path through libmoe
+# ---------------------------------------------------------------------------
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_moe_layer_joint_b200 as moe
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    t = mi.torch_workload(w, device=dev)
+    if rank > 0:  # each replica gets its own tokens: rows rank*T .. of one global x stream
+        mi.gpu_normal_bf16(t["x"].data_ptr(), t["x"].numel(), w.seed, mi.STREAM_X, rank * w.T * w.d, w.std_x,
+                           stream.cuda_stream)
+    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev)
+    bias0 = t["bias"].clone()
+    ffn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def step(i=None, x=None):
+        layer.forward(t["x"] if x is None else x, t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"],
+                      ffn_events=None if i is None else ffn_ev[i])
+        if world > 1:
+            dist.all_reduce(layer.counts)
+        layer.bias_update(t["bias"], w.gamma)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = moe.moe_get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} after warm-up")
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ffn_ev)
+
+    # end to end through the public API: pinned host x in, host out back, every step
+    x_host = t["x"].cpu().pin_memory()
+    out_host = torch.empty_like(layer.out, device="cpu").pin_memory()
+    x_dev = torch.empty_like(t["x"])
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x=x_dev)
+        out_host.copy_(layer.out, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x=x_dev)
+        out_host.copy_(layer.out, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e2.elapsed_time(e3) / args.steps
+    st = moe.moe_get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} after timing")
+
+    vals = torch.tensor([ms, e2e_ms, ffn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, ffn_ms = vals.tolist()
+
+    # the dominant kernel: the routed experts' grouped GEMMs (both launches of
+    # one moe_grouped_ffn call), algorithmic FLOPs = 2 GEMMs x 2 * rows * d * d_ff
+    pk = peaks()
+    rows = w.T * w.k
+    ffn_flops = 2 * 2.0 * rows * w.d * w.f
+    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
+    roofline = {"kernel": "grouped_gemm_kernel x2 (routed experts: GEMM1+GELU, GEMM2)", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
+                "peak_source": f"{pk['src']} bf16 sustained (MEASURED_PEAKS.json)" if pk["src"] == "measured"
+                else "fallback bf16 sustained", "traffic": None,
+                "ms_per_launch_pair": round(ffn_ms, 4),
+                "layer_tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1)}
+    if w.name in ("decode", "mid"):
+        roofline["note"] = "HBM-bound workload; see DESIGN.md for its byte roofline"
+    line = {
+        "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox, random-init weights)",
+        "config": config_of(w, world), "clocks": clk,
+        "e2e": {"value": round(world * w.T / (e2e_ms * 1e-3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": w.T * w.d * 2, "d2h_bytes_per_step": w.T * w.d * 2,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": moe.MoELayer.LAUNCHES_PER_STEP * args.steps,
+        "roofline": roofline,
+    }
+    del bias0
+    return line
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def oracle_sample(w, n_tokens, seed_offset=0):
+    """Prepare a bounded sample: n_tokens tokens of the workload and the host
+    weights of every expert they use (generated before any timing)."""
+    import oracle
+
+    tokens = (np.arange(n_tokens) * 7919 + seed_offset) % w.T
+    b = mi.host_bias(w)
+    off = mi.host_logit_offset(w)
+    r = oracle.route_workload(w, b, tokens, off)
+    experts = sorted(set(int(e) for e in np.unique(r["contrib"])))
+    weights = {"w1": {e: mi.host_w1(w, e) for e in experts}, "w2": {e: mi.host_w2(w, e) for e in experts}}
+    return tokens, b, off, weights
+
+
+def oracle_forward_timed(w, tokens, b, off, weights):
+    import oracle
+
+    t0 = time.perf_counter()
+    oracle.forward_tokens(w, tokens, b, off, weights=weights)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, n_tokens=4):
+    tokens, b, off, weights = oracle_sample(w, n_tokens)
+    dt = oracle_forward_timed(w, tokens, b, off, weights)
+    return {"value": round(len(tokens) / dt, 4), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{len(tokens)} tokens of the {w.name} workload (full layer: fp64 router over 258 experts, "
+                      f"top-{w.k}, joint gates, 8 expert MLPs each), wall {dt:.2f} s; expert weights generated "
+                      "before timing"}
+
+
+def run_reference(args, w):
+    tokens, b, off, weights = oracle_sample(w, 2)
+    per_step = 1
+    for i in range(args.warmup):
+        oracle_forward_timed(w, tokens[i % len(tokens):i % len(tokens) + per_step], b, off, weights)
+    total = 0.0
+    for i in range(args.steps):
+        j = i % len(tokens)
+        total += oracle_forward_timed(w, tokens[j:j + per_step], b, off, weights)
+    ms = total / args.steps * 1e3
+    v = round(per_step / (ms * 1e-3), 4)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, random-init weights)",
+        "config": config_of(w, 1),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"each step: {per_step} token of the {w.name} workload through the fp64 oracle "
+                                   "(router + 8 expert MLPs + combine), weights generated before timing"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = mi.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, w, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(w)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -205,31 +205,41 @@ class MoELayer:
         self.ev_start = torch.cuda.Event()
         self.ev_shared = torch.cuda.Event()
 
-    def forward(self, x, w_router, w1, w2, bias, logit_offset=None, stream=None, scores_out=None):
-        """Router -> permute -> routed experts (stream A) | shared experts (stream B) -> combine."""
+    def forward(self, x, w_router, w1, w2, bias, logit_offset=None, stream=None, scores_out=None,
+                ffn_events=None):
+        """Router -> [fork] permute -> routed experts (main stream) | shared experts
+        (side stream) -> [join] combine.  ``ffn_events`` = (start, end) torch events
+        recorded around the routed experts' call on the main stream."""
         import torch
 
         s = self.shape
         main = stream if stream is not None else torch.cuda.current_stream()
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
-        self.ev_start.record(main)
-        # shared experts see every token: start them beside the routed path
+        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, 1.0, self.topk_idx,
+                        self.gates, self.counts, scores_out, stream=main)
+        # shared experts see every token: run them beside dispatch and the routed experts
         if s.n_shared > 0:
+            self.ev_start.record(main)
             self.side.wait_event(self.ev_start)
             moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h_shared,
                             self.y_shared, stream=self.side)
             self.ev_shared.record(self.side)
-        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, 1.0, self.topk_idx,
-                        self.gates, self.counts, scores_out, stream=main)
         moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, self.x_perm, self.row_token,
                     self.token_row, self.scratch, self.scratch_bytes, stream=main)
+        if ffn_events is not None:
+            ffn_events[0].record(main)
         moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h,
                         self.y_perm, stream=main)
+        if ffn_events is not None:
+            ffn_events[1].record(main)
         if s.n_shared > 0:
             main.wait_event(self.ev_shared)
         moe_combine(self.y_perm, self.token_row, self.gates, self.y_shared if s.n_shared > 0 else None, T, d, k,
                     s.n_shared, self.out, stream=main)
         return self.out
+
+    # kernels of libmoe launched by one forward + bias update
+    LAUNCHES_PER_STEP = 1 + 3 + 2 + 2 + 1 + 1
 
     def bias_update(self, bias, gamma: float, stream=None):
         s = self.shape
