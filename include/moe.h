@@ -120,6 +120,37 @@ int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* count
                 size_t scratch_bytes, void* stream);
 
 /*
+ * moe_permute_noalloc -- moe_permute for callers that cannot allocate device
+ * memory.  No counterpart in the paper: it exists for the library's users, not
+ * the method.
+ *
+ * Some callers have no way to obtain a scratch buffer: a plugin running inside
+ * a host application that owns every device allocation and lends it none, a
+ * process that reserved all of HBM for its own pool at start-up, or a latency
+ * loop that must not call cudaMalloc/cudaFree (they can synchronise the
+ * device).  This entry point takes the same arguments as moe_permute minus the
+ * scratch buffer and gives identical results; its scratch lives in a fixed
+ * device array inside libmoe of MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES (1 MiB),
+ * which every GPU that loads the library holds until the process exits.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - Limit: moe_permute_scratch_bytes(T, n_routed) must not exceed 1 MiB
+ *    (with 256 routed experts: T <= 130816 tokens); larger calls return
+ *    MOE_ERR_SCRATCH and launch nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; nothing in it needs clearing, because each call writes every
+ *    part it reads.  Calls whose kernels overlap on the GPU (for instance on
+ *    two streams without ordering between them) race on the array: order them.
+ * Inputs and outputs are caller-owned device buffers exactly as for moe_permute.
+ */
+#define MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES (1 << 20)
+int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                        int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
+                        int32_t* token_row, void* stream);
+
+/*
  * moe_grouped_ffn -- the expert MLPs, y = W2_e gelu(W1_e x), for groups of rows.
  * "Inkling, Dissected" §02: an expert is two matrix multiplies with a
  * nonlinearity between them (GELU, tanh form, here).

@@ -45,6 +45,7 @@ _lib.moe_router_topk.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i3
 _lib.moe_permute_scratch_bytes.argtypes = [_i32, _i32]
 _lib.moe_permute_scratch_bytes.restype = _sz
 _lib.moe_permute.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_permute_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_grouped_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
 _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_bias_update.argtypes = [_vp, _i32, _i32, _i32, _f32, _vp, _vp]
@@ -53,7 +54,7 @@ _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_get_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.moe_set_wait_timeout_ns.argtypes = [_u64]
 _lib.moe_debug_bounded_wait.argtypes = [_u64, _vp]
-for _f in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_bias_update", "moe_get_status",
+for _f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine", "moe_bias_update", "moe_get_status",
            "moe_set_wait_timeout_ns", "moe_debug_bounded_wait"):
     getattr(_lib, _f).restype = _i32
 
@@ -123,6 +124,18 @@ def moe_permute(x, topk_idx, counts, T: int, d: int, n_routed: int, top_k: int, 
     _check("moe_permute", _lib.moe_permute(
         _p(x), _p(topk_idx), _p(counts), T, d, n_routed, top_k, _p(offsets), _p(x_perm), _p(row_token),
         _p(token_row), _p(scratch), scratch_bytes, _stream(stream)))
+
+
+def moe_permute_noalloc(x, topk_idx, counts, T: int, d: int, n_routed: int, top_k: int, offsets, x_perm, row_token,
+                        token_row, stream=None):
+    """moe_permute without a scratch argument, for callers that cannot allocate
+    device memory: the scratch is a fixed 1 MiB device array inside libmoe
+    (limit: moe_permute_scratch_bytes(T, n_routed) <= 1 MiB).  Calls on one
+    device share that array, so calls that could overlap on the GPU must be
+    ordered; the first call on a device should come before any stream capture."""
+    _check("moe_permute_noalloc", _lib.moe_permute_noalloc(
+        _p(x), _p(topk_idx), _p(counts), T, d, n_routed, top_k, _p(offsets), _p(x_perm), _p(row_token),
+        _p(token_row), _stream(stream)))
 
 
 def moe_grouped_ffn(rows, offsets, n_groups: int, n_rows: int, expert_base: int, w1, w2, d: int, d_ff: int,

@@ -209,3 +209,73 @@ extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int
                                                n_routed, reinterpret_cast<uint4*>(x_perm), row_token, token_row);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the same three launches, with the scratch held in this
+// file's device array instead of a caller buffer (for callers that cannot
+// allocate device memory).  The array's host-side name is not a device
+// address: its address is fetched once per device with cudaGetSymbolAddress,
+// with that device current, and passed to the kernels.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace moe {
+namespace perm {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of this device's copy of the array (set up on first use).
+static int noalloc_scratch(void** out) {
+  int dev;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace perm
+}  // namespace moe
+
+extern "C" int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                                   int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
+                                   int32_t* token_row, void* stream) {
+  using namespace moe::perm;
+  if (T < 0 || d <= 0 || n_routed < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
+  if (top_k > MOE_MAX_TOP_K || top_k > n_routed || n_routed > MOE_MAX_ROUTED) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!x || !topk_idx || !offsets || !x_perm || !row_token || !token_row) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned4(topk_idx) || !aligned4(counts) || !aligned4(offsets) ||
+      !aligned4(row_token) || !aligned4(token_row))
+    return MOE_ERR_INVALID_ARG;
+  if ((long long)T * top_k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (moe_permute_scratch_bytes(T, n_routed) > (size_t)MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES) return MOE_ERR_SCRATCH;
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (T == 0) {
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (n_routed + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  unsigned int* status = status_ptr();
+  if (!status) return MOE_ERR_CUDA;
+  // Every part of the scratch that is read is written first in the same call
+  // (hist by chunk_hist, base by chunk_scan), so nothing needs clearing.
+  const int n_chunks = (T + CHUNK - 1) / CHUNK;
+  int32_t* hist = reinterpret_cast<int32_t*>(scratch);
+  int32_t* base = hist + (size_t)n_chunks * n_routed;
+  chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
+  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, counts, offsets, base, status);
+  scatter_kernel<<<n_chunks, THREADS, 0, s>>>(reinterpret_cast<const uint4*>(x), topk_idx, base, T, d / 8, top_k,
+                                               n_routed, reinterpret_cast<uint4*>(x_perm), row_token, token_row);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
