@@ -283,6 +283,47 @@ def run_reference(args, w):
     }
 
 
+def run_kernel_case(args):
+    """The grouped expert GEMMs alone, on a prefill-shaped slice small enough to
+    profile (32 experts x 1536 rows, d 7168, d_ff 2048: 3.5 GB on the device,
+    inputs larger than L2).  Prints one diagnostic JSON line (not a bench line)."""
+    import torch
+
+    import sparse_moe_layer_joint_b200 as moe
+
+    G, per, d, f = 32, 1536, 7168, 2048
+    n = G * per
+    dev = torch.device("cuda", 0)
+    s = torch.cuda.current_stream(dev).cuda_stream
+    rows = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+    w1 = torch.empty((G, f, d), dtype=torch.bfloat16, device=dev)
+    w2 = torch.empty((G, d, f), dtype=torch.bfloat16, device=dev)
+    mi.gpu_normal_bf16(rows.data_ptr(), rows.numel(), 0, mi.STREAM_TEST_ROWS, 0, 1.0, s)
+    mi.gpu_normal_bf16(w1.data_ptr(), w1.numel(), 0, mi.STREAM_W1, 0, d ** -0.5, s)
+    mi.gpu_normal_bf16(w2.data_ptr(), w2.numel(), 0, mi.STREAM_W2, 0, f ** -0.5, s)
+    offsets = torch.arange(0, n + 1, per, dtype=torch.int32, device=dev)
+    h = torch.empty((n, f), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+
+    def call():
+        moe.moe_grouped_ffn(rows, offsets, G, n, 0, w1, w2, d, f, moe.MOE_ACT_GELU_TANH, h, y)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2 * 2.0 * n * d * f
+    print(json.dumps({"kernel_case": "grouped_ffn", "experts": G, "rows_per_expert": per, "d": d, "d_ff": f,
+                      "ms_per_call": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                      "status": moe.moe_get_status()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -291,6 +332,8 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=["grouped_ffn"], default=None,
+                    help="time one kernel alone on a small profiling case instead of the layer")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -298,6 +341,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = mi.WORKLOADS[args.workload]
+
+    if args.kernel_case is not None:
+        run_kernel_case(args)
+        return
 
     if args.impl == "reference":
         if rank == 0:
