@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "moe.h"
 #include "moe_internal.h"
@@ -292,6 +293,242 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant: a cluster of 2 CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256).  CTA rank r holds A rows
+// r*128 .. r*128+127 of the tile and B rows (output columns) r*128 ..
+// r*128+127 in its own shared memory, and receives accumulator rows r*128 ..
+// in its own TMEM.  Each CTA's producer loads its halves; every load signals
+// the leader's (rank 0) full barrier, whose producer expects both halves'
+// bytes.  The leader's single MMA thread issues for the pair and commits to
+// both CTAs' empty / accumulator-full barriers; both CTAs' epilogue warps
+// release the accumulator on the leader's barrier.  Per CTA and K step this
+// halves the B operand's shared-memory traffic of the 1-CTA kernel.
+// ---------------------------------------------------------------------------
+constexpr int P_BM = 256;                      // tile rows per pair
+constexpr int P_HALF = 128;                    // rows (of A and of B) per CTA
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = P_HALF * BK * 2;     // 16 KB
+constexpr int P_B_BYTES = P_HALF * BK * 2;     // 16 KB
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+
+struct SmemTailPair {
+  uint64_t full[P_STAGES];
+  uint64_t empty[P_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int off[MOE_MAX_GROUPS + 1];
+  int prefix[MOE_MAX_GROUPS + 1];
+};
+
+constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * P_STAGE_BYTES + sizeof(SmemTailPair);
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smemA = smem;
+  uint8_t* smemB = smem + P_STAGES * P_A_BYTES;
+  SmemTailPair* st = reinterpret_cast<SmemTailPair*>(smem + P_STAGES * P_STAGE_BYTES);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const bool identity = (p.offsets == nullptr);
+
+  if (tid == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&st->full[s], 1);
+      mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&st->tfull[a], 1);
+      mbar_init(&st->tempty[a], 8);  // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (!identity) {
+    for (int i = tid; i <= p.n_groups; i += NUM_THREADS) {
+      int v = p.offsets[i];
+      st->off[i] = v < 0 ? 0 : (v > p.n_rows ? p.n_rows : v);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.n_groups; base += 32) {
+      int g = base + lane;
+      int cnt = 0;
+      if (g < p.n_groups) {
+        int rows = identity ? p.n_rows : st->off[g + 1] - st->off[g];
+        cnt = rows > 0 ? (rows + P_BM - 1) / P_BM : 0;
+      }
+      int v = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (g < p.n_groups) st->prefix[g + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) st->prefix[0] = 0;
+  }
+  __syncthreads();
+  const int total_tiles = st->prefix[p.n_groups] * p.n_tiles_n;
+  if (pair >= total_tiles) return;  // both CTAs of the pair leave together, before any cluster traffic
+
+  if (warp == 1) tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM taken in both
+  tc_fence_after();
+  const uint32_t tmem_base = st->tmem_base;
+  const int num_kb = (p.K + BK - 1) / BK;
+  volatile int* abort_flag = &st->abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        TileInfo ti = tile_info(tile, st->prefix, p.n_groups, p.n_tiles_n);
+        int a_row = (identity ? ti.g * p.a_group_stride : st->off[ti.g]) + ti.m * P_BM + (int)rank * P_HALF;
+        int b_row = ti.nt * BN + (int)rank * P_HALF;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&st->full[stage], 2 * P_STAGE_BYTES);
+          tma_load_2d_pair(smemA + stage * P_A_BYTES, &tmA, &st->full[stage], kb * BK, a_row);
+          tma_load_3d_pair(smemB + stage * P_B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc_bf16(P_BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&st->full[stage], phase, p.timeout_ns, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smemA + stage * P_A_BYTES);
+          const uint32_t b_addr = smem_u32(smemB + stage * P_B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            mma_bf16_ss_pair(d_tmem, make_desc_sw128(a_addr + k * 32), make_desc_sw128(b_addr + k * 32), idesc,
+                             (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair(&st->empty[stage], 0x3);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&st->tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      int zero = 0;
+      mma_commit_pair(&st->drain, 0x1);
+      mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row_in_tile = (int)rank * P_HALF + quarter * 32 + lane;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&st->tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&st->tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      TileInfo ti = tile_info(tile, st->prefix, p.n_groups, p.n_tiles_n);
+      int rows_g = identity ? p.n_rows : st->off[ti.g + 1] - st->off[ti.g];
+      int c_base = identity ? ti.g * p.c_group_stride : st->off[ti.g];
+      int r = ti.m * P_BM + row_in_tile;
+      int c_row = c_base + r;
+      bool valid = (r < rows_g) && (c_row < p.c_row_limit);
+      if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      __nv_bfloat16* crow = p.C + (size_t)c_row * p.ldc;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int col0 = ti.nt * BN + ch * 32;
+        if (col0 >= p.N) break;
+        float v[32];
+        tmem_ld32(taddr + ch * 32, v);
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float a = v[2 * i], b = v[2 * i + 1];
+            if (EPI == EPI_GELU) {
+              a = gelu_tanh_f32(a);
+              b = gelu_tanh_f32(b);
+            }
+            pk[i] = pack_bf16x2(a, b);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // every MMA of the pair has landed and both CTAs are done with each other's memory
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int EPI>
+int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const Params& p, int grid, cudaStream_t stream) {
+  auto kfn = grouped_gemm_pair_kernel<EPI>;
+  int rc = ensure_smem_attr((const void*)kfn, P_SMEM_BYTES);
+  if (rc != MOE_OK) return rc;
+  kfn<<<grid, NUM_THREADS, P_SMEM_BYTES, stream>>>(tmA, tmB, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 template <int EPI>
 int launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const Params& p, int grid, cudaStream_t stream) {
   auto kfn = grouped_gemm_kernel<EPI>;
@@ -331,19 +568,39 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   const __nv_bfloat16* w1e = reinterpret_cast<const __nv_bfloat16*>(w1) + (size_t)expert_base * d_ff * d;
   const __nv_bfloat16* w2e = reinterpret_cast<const __nv_bfloat16*>(w2) + (size_t)expert_base * d * d_ff;
 
+  // Kernel variant.  CTA pairs (cta_group::2, 256 x 256 tiles) halve each CTA's shared-memory
+  // operand traffic and win when groups are large (compute-bound); with few rows per group the
+  // work is weight streaming and single CTAs (128 x 256 tiles, more weight bytes in flight per
+  // SM) win.  MOE_GEMM_CTA=1 or =2 forces one of them.
+  const char* env = getenv("MOE_GEMM_CTA");
+  const long long rows_per_group = identity ? n_rows : n_rows / n_groups;
+  bool pair = rows_per_group >= 256;
+  if (env && env[0] == '1' && env[1] == '\0') pair = false;
+  if (env && env[0] == '2' && env[1] == '\0') pair = true;
+  const uint32_t b_box = pair ? (uint32_t)P_HALF : (uint32_t)BN;
+  const int tile_m = pair ? P_BM : BM;
+
   CUtensorMap tA1, tB1, tA2, tB2;
   // GEMM1: A = rows [n_rows, d], B = W1 [n_groups, d_ff, d]
   if ((rc = encode_tmap_bf16(&tA1, rows, 2, (uint64_t)d, (uint64_t)n_rows, 1, BK, BM)) != MOE_OK) return rc;
-  if ((rc = encode_tmap_bf16(&tB1, w1e, 3, (uint64_t)d, (uint64_t)d_ff, (uint64_t)n_groups, BK, BN)) != MOE_OK)
+  if ((rc = encode_tmap_bf16(&tB1, w1e, 3, (uint64_t)d, (uint64_t)d_ff, (uint64_t)n_groups, BK, b_box)) != MOE_OK)
     return rc;
   // GEMM2: A = H [h_rows, d_ff], B = W2 [n_groups, d, d_ff]
   if ((rc = encode_tmap_bf16(&tA2, h_scratch, 2, (uint64_t)d_ff, (uint64_t)h_rows, 1, BK, BM)) != MOE_OK)
     return rc;
-  if ((rc = encode_tmap_bf16(&tB2, w2e, 3, (uint64_t)d_ff, (uint64_t)d, (uint64_t)n_groups, BK, BN)) != MOE_OK)
+  if ((rc = encode_tmap_bf16(&tB2, w2e, 3, (uint64_t)d_ff, (uint64_t)d, (uint64_t)n_groups, BK, b_box)) != MOE_OK)
     return rc;
 
   // upper bound on m-tiles: every group may add one partial tile
-  long long mtiles = identity ? (long long)n_groups * ((n_rows + BM - 1) / BM) : (n_rows + BM - 1) / BM + n_groups;
+  long long mtiles = identity ? (long long)n_groups * ((n_rows + tile_m - 1) / tile_m)
+                              : (n_rows + tile_m - 1) / tile_m + n_groups;
+  auto grid_for = [&](long long tiles) -> int {
+    if (pair) {
+      long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+      return (int)(2 * pairs);
+    }
+    return (int)(tiles < sms ? tiles : sms);
+  };
 
   Params p1{};
   p1.offsets = offsets;
@@ -360,9 +617,9 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   p1.timeout_ns = wait_timeout_ns();
   p1.status = status_ptr();
   if (!p1.status) return MOE_ERR_CUDA;
-  long long t1 = mtiles * p1.n_tiles_n;
-  int grid1 = (int)(t1 < sms ? t1 : sms);
-  if ((rc = launch<EPI_GELU>(tA1, tB1, p1, grid1, s)) != MOE_OK) return rc;
+  const int grid1 = grid_for(mtiles * p1.n_tiles_n);
+  rc = pair ? launch_pair<EPI_GELU>(tA1, tB1, p1, grid1, s) : launch<EPI_GELU>(tA1, tB1, p1, grid1, s);
+  if (rc != MOE_OK) return rc;
 
   Params p2 = p1;
   p2.a_group_stride = n_rows;
@@ -373,7 +630,6 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   p2.n_tiles_n = (d + BN - 1) / BN;
   p2.C = reinterpret_cast<__nv_bfloat16*>(y);
   p2.ldc = d;
-  long long t2 = mtiles * p2.n_tiles_n;
-  int grid2 = (int)(t2 < sms ? t2 : sms);
-  return launch<EPI_NONE>(tA2, tB2, p2, grid2, s);
+  const int grid2 = grid_for(mtiles * p2.n_tiles_n);
+  return pair ? launch_pair<EPI_NONE>(tA2, tB2, p2, grid2, s) : launch<EPI_NONE>(tA2, tB2, p2, grid2, s);
 }

@@ -187,14 +187,22 @@ def _ffn_weights(E, d, f, seed):
     return w1, w2
 
 
+@pytest.fixture(params=["pair", "single"])
+def gemm_variant(request, monkeypatch):
+    """Both grouped-GEMM kernels: CTA pairs (default) and single CTAs."""
+    monkeypatch.setenv("MOE_GEMM_CTA", "1" if request.param == "single" else "2")
+    return request.param
+
+
 @pytest.mark.parametrize("sizes,d,f", [
     ([0, 1, 127, 128, 129, 300, 0, 5], 256, 128),
     ([200, 37, 0, 513], 512, 768),
     ([64] * 16, 128, 256),
     ([1000], 1024, 512),
     ([3, 0, 0, 0, 250, 7], 2048, 1024),
+    ([129, 255, 256, 257, 0, 511, 1], 256, 256),
 ])
-def test_grouped_ffn_parity(sizes, d, f):
+def test_grouped_ffn_parity(sizes, d, f, gemm_variant):
     G = len(sizes)
     n = int(sum(sizes))
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
@@ -216,7 +224,7 @@ def test_grouped_ffn_parity(sizes, d, f):
 
 
 @pytest.mark.parametrize("n,G,d,f", [(1, 2, 64, 64), (300, 2, 256, 128), (1030, 3, 512, 256)])
-def test_grouped_ffn_identity_groups(n, G, d, f):
+def test_grouped_ffn_identity_groups(n, G, d, f, gemm_variant):
     """offsets = NULL: every group (expert) sees all rows, as the shared experts do."""
     rows = mi.normal_bf16(n * d, 6, mi.STREAM_TEST_ROWS).reshape(n, d)
     w1, w2 = _ffn_weights(G + 5, d, f, 6)
@@ -228,7 +236,7 @@ def test_grouped_ffn_identity_groups(n, G, d, f):
         check_output(yg[g], oracle.expert(rows, w1[5 + g], w2[5 + g]), f"group {g}")
 
 
-def test_grouped_ffn_special_weights():
+def test_grouped_ffn_special_weights(gemm_variant):
     """W2 = 0 gives exactly 0; W1 = W2 = I (d = d_ff) gives bf16(gelu(x))."""
     n, d = 260, 128
     rows = mi.normal_bf16(n * d, 7, mi.STREAM_TEST_ROWS).reshape(n, d)
