@@ -196,13 +196,14 @@ def run_ours(args, w, rank, world, local_rank):
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
     ms, e2e_ms, ffn_ms = vals.tolist()
 
-    # the dominant kernel: the routed experts' grouped GEMMs (both launches of
-    # one moe_grouped_ffn call), algorithmic FLOPs = 2 GEMMs x 2 * rows * d * d_ff
+    # the dominant kernel: the experts' grouped GEMMs (both launches of one
+    # moe_experts_ffn call), algorithmic FLOPs = 2 GEMMs x 2 * rows * d * d_ff
+    # over the T*k routed and T*n_shared shared (token, expert) rows
     pk = peaks()
-    rows = w.T * w.k
+    rows = w.T * (w.k + w.n_shared)
     ffn_flops = 2 * 2.0 * rows * w.d * w.f
     achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
-    roofline = {"kernel": "grouped_gemm_kernel x2 (routed experts: GEMM1+GELU, GEMM2)", "bound": "tensor",
+    roofline = {"kernel": "grouped_gemm_kernel x2 (all 258 experts: GEMM1+GELU, GEMM2)", "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
                 "peak_source": f"{pk['src']} bf16 sustained (MEASURED_PEAKS.json)" if pk["src"] == "measured"
@@ -219,7 +220,7 @@ def run_ours(args, w, rank, world, local_rank):
         "e2e": {"value": round(world * w.T / (e2e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": w.T * w.d * 2, "d2h_bytes_per_step": w.T * w.d * 2,
                 "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": moe.MoELayer.LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": layer.launches_per_step() * args.steps,
         "roofline": roofline,
     }
     del bias0
@@ -305,23 +306,35 @@ def run_kernel_case(args):
     h = torch.empty((n, f), dtype=torch.bfloat16, device=dev)
     y = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
 
-    def call():
-        moe.moe_grouped_ffn(rows, offsets, G, n, 0, w1, w2, d, f, moe.MOE_ACT_GELU_TANH, h, y)
+    if args.kernel_case == "grouped_ffn":
+        def call():
+            moe.moe_grouped_ffn(rows, offsets, G, n, 0, w1, w2, d, f, moe.MOE_ACT_GELU_TANH, h, y)
+    else:
+        # comparison only (not the product path): the same two GEMMs per expert through cuBLAS
+        xr, hr, yr = rows.view(G, per, d), h.view(G, per, f), y.view(G, per, d)
+
+        def call():
+            torch.bmm(xr, w1.transpose(1, 2), out=hr)
+            torch.bmm(hr, w2.transpose(1, 2), out=yr)
 
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         call()
     e1.record()
     torch.cuda.synchronize()
+    clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     flops = 2 * 2.0 * n * d * f
-    print(json.dumps({"kernel_case": "grouped_ffn", "experts": G, "rows_per_expert": per, "d": d, "d_ff": f,
+    print(json.dumps({"kernel_case": args.kernel_case, "experts": G, "rows_per_expert": per, "d": d, "d_ff": f,
                       "ms_per_call": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
-                      "status": moe.moe_get_status()}), flush=True)
+                      "clocks": clk, "status": moe.moe_get_status()}), flush=True)
 
 
 def main():
@@ -332,7 +345,7 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["grouped_ffn"], default=None,
+    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas"], default=None,
                     help="time one kernel alone on a small profiling case instead of the layer")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -176,6 +176,27 @@ int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, 
                     moe_bf16* y, void* stream);
 
 /*
+ * moe_experts_ffn -- every expert of the layer in one pair of launches: the
+ * n_routed routed experts on their dispatched rows and the n_shared shared
+ * experts on all T tokens ("Inkling, Dissected" §02: each token goes to its 6
+ * routed experts and to both shared experts; an expert is two matmuls with a
+ * nonlinearity).  The same grouped GEMM as moe_grouped_ffn, with the shared
+ * experts' tiles scheduled in the same persistent launches as the routed ones.
+ *
+ *   x          [T, d] bf16 (shared experts' input)
+ *   x_perm     [T*top_k, d] bf16, offsets [n_routed + 1] int32 (from moe_permute)
+ *   w1, w2     [n_routed + n_shared, d_ff, d] and [n_routed + n_shared, d, d_ff]
+ *              bf16: routed experts first, then the shared experts
+ *   h_scratch  [T*top_k + n_shared*T, d_ff] bf16 (caller-owned)
+ *   y_perm     [T*top_k, d] bf16 out (routed, dispatch order)
+ *   y_shared   [n_shared, T, d] bf16 out
+ * Limits: d % 64 == 0, d_ff % 64 == 0, n_routed + n_shared <= MOE_MAX_GROUPS.
+ */
+int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* offsets, int T, int n_routed,
+                    int n_shared, int top_k, const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff, int activation,
+                    moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared, void* stream);
+
+/*
  * moe_combine -- gate-weighted sum of the contributors, back in token order.
  * "Inkling, Dissected" §02 (the layer output is the weighted sum of the 8
  * contributing experts) and §02b sketch (out += g_k * e_k(x)).

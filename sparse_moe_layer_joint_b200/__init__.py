@@ -47,6 +47,8 @@ _lib.moe_permute_scratch_bytes.restype = _sz
 _lib.moe_permute.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_permute_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_grouped_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.moe_experts_ffn.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp,
+                                 _vp]
 _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_bias_update.argtypes = [_vp, _i32, _i32, _i32, _f32, _vp, _vp]
 _lib.moe_status_string.argtypes = [_i32]
@@ -54,7 +56,7 @@ _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_get_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.moe_set_wait_timeout_ns.argtypes = [_u64]
 _lib.moe_debug_bounded_wait.argtypes = [_u64, _vp]
-for _f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine", "moe_bias_update", "moe_get_status",
+for _f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_experts_ffn", "moe_combine", "moe_bias_update", "moe_get_status",
            "moe_set_wait_timeout_ns", "moe_debug_bounded_wait"):
     getattr(_lib, _f).restype = _i32
 
@@ -145,6 +147,13 @@ def moe_grouped_ffn(rows, offsets, n_groups: int, n_rows: int, expert_base: int,
         _p(y), _stream(stream)))
 
 
+def moe_experts_ffn(x, x_perm, offsets, T: int, n_routed: int, n_shared: int, top_k: int, w1, w2, d: int, d_ff: int,
+                    activation: int, h_scratch, y_perm, y_shared, stream=None):
+    _check("moe_experts_ffn", _lib.moe_experts_ffn(
+        _p(x), _p(x_perm), _p(offsets), T, n_routed, n_shared, top_k, _p(w1), _p(w2), d, d_ff, activation,
+        _p(h_scratch), _p(y_perm), _p(y_shared), _stream(stream)))
+
+
 def moe_combine(y_perm, token_row, gates, y_shared, T: int, d: int, top_k: int, n_shared: int, out, stream=None):
     _check("moe_combine", _lib.moe_combine(
         _p(y_perm), _p(token_row), _p(gates), _p(y_shared), T, d, top_k, n_shared, _p(out), _stream(stream)))
@@ -193,10 +202,11 @@ class MoELayer:
     bias [n_routed] fp32 (updated in place by ``bias_update``).
     """
 
-    def __init__(self, shape: LayerShape, device="cuda"):
+    def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True):
         import torch
 
         self.shape = s = shape
+        self.fused_experts = fused_experts
         dev = torch.device(device)
         R = s.T * s.top_k
         bf = torch.bfloat16
@@ -209,7 +219,8 @@ class MoELayer:
         self.token_row = torch.empty((s.T, s.top_k), dtype=torch.int32, device=dev)
         self.scratch_bytes = moe_permute_scratch_bytes(s.T, s.n_routed)
         self.scratch = torch.empty((self.scratch_bytes,), dtype=torch.uint8, device=dev)
-        self.h = torch.empty((max(R, 1), s.d_ff), dtype=bf, device=dev)
+        # hidden rows: routed rows, then (fused path) the shared experts' rows
+        self.h = torch.empty((max(R + s.n_shared * s.T, 1), s.d_ff), dtype=bf, device=dev)
         self.y_perm = torch.empty((max(R, 1), s.d), dtype=bf, device=dev)
         self.h_shared = torch.empty((max(s.n_shared, 1), s.T, s.d_ff), dtype=bf, device=dev)
         self.y_shared = torch.empty((max(s.n_shared, 1), s.T, s.d), dtype=bf, device=dev)
@@ -220,9 +231,13 @@ class MoELayer:
 
     def forward(self, x, w_router, w1, w2, bias, logit_offset=None, stream=None, scores_out=None,
                 ffn_events=None):
-        """Router -> [fork] permute -> routed experts (main stream) | shared experts
-        (side stream) -> [join] combine.  ``ffn_events`` = (start, end) torch events
-        recorded around the routed experts' call on the main stream."""
+        """Router -> dispatch -> experts -> combine, on the given (default: current) stream.
+
+        With ``fused_experts`` (default) the routed and shared experts run in one
+        pair of grouped-GEMM launches (moe_experts_ffn).  Otherwise the shared
+        experts run beside dispatch and the routed experts on a second stream
+        (moe_grouped_ffn twice).  ``ffn_events`` = (start, end) torch events
+        recorded around the expert launches on the main stream."""
         import torch
 
         s = self.shape
@@ -230,8 +245,8 @@ class MoELayer:
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
         moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, 1.0, self.topk_idx,
                         self.gates, self.counts, scores_out, stream=main)
-        # shared experts see every token: run them beside dispatch and the routed experts
-        if s.n_shared > 0:
+        side = s.n_shared > 0 and not self.fused_experts
+        if side:
             self.ev_start.record(main)
             self.side.wait_event(self.ev_start)
             moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h_shared,
@@ -241,18 +256,25 @@ class MoELayer:
                     self.token_row, self.scratch, self.scratch_bytes, stream=main)
         if ffn_events is not None:
             ffn_events[0].record(main)
-        moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h,
-                        self.y_perm, stream=main)
+        if self.fused_experts:
+            moe_experts_ffn(x, self.x_perm, self.offsets, T, s.n_routed, s.n_shared, k, w1, w2, d, f,
+                            MOE_ACT_GELU_TANH, self.h, self.y_perm, self.y_shared, stream=main)
+        else:
+            moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, MOE_ACT_GELU_TANH,
+                            self.h, self.y_perm, stream=main)
         if ffn_events is not None:
             ffn_events[1].record(main)
-        if s.n_shared > 0:
+        if side:
             main.wait_event(self.ev_shared)
         moe_combine(self.y_perm, self.token_row, self.gates, self.y_shared if s.n_shared > 0 else None, T, d, k,
                     s.n_shared, self.out, stream=main)
         return self.out
 
     # kernels of libmoe launched by one forward + bias update
-    LAUNCHES_PER_STEP = 1 + 3 + 2 + 2 + 1 + 1
+    def launches_per_step(self) -> int:
+        """libmoe kernels one forward + bias update launches."""
+        experts = 2 if self.fused_experts else 4
+        return 1 + 3 + experts + 1 + 1
 
     def bias_update(self, bias, gamma: float, stream=None):
         s = self.shape

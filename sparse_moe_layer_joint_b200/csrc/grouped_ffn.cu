@@ -1,23 +1,41 @@
 // grouped_ffn.cu -- the expert MLPs y = W2_e gelu(W1_e x) over groups of rows
-// ("Inkling, Dissected" §02: an expert is two matmuls with a nonlinearity),
-// as two launches of one persistent, warp-specialised tcgen05 grouped GEMM:
+// ("Inkling, Dissected" §02: an expert is two matmuls with a nonlinearity), as
+// two launches of one persistent, warp-specialised tcgen05 grouped GEMM:
 //
 //   GEMM1:  H[rows of e] = gelu(X[rows of e] . W1_e^T)   (bf16 out, GELU fused)
 //   GEMM2:  Y[rows of e] =      H[rows of e] . W2_e^T    (bf16 out)
 //
-// Per CTA (one per SM, persistent over a static round-robin of 128x256 tiles):
-//   warp 0      TMA producer: A (128 x 64) and B (256 x 64) bf16 tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (full/empty mbarriers)
-//   warp 1      TMEM owner + MMA issuer: tcgen05.mma.cta_group::1.kind::f16,
-//               M=128 N=256 K=16, fp32 accumulators in TMEM, two accumulator
-//               buffers (512 columns) so the epilogue of tile i overlaps the
-//               main loop of tile i+1
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, activation, bf16
-//               rounding, 16-byte stores of each row's 64-byte chunk
-// Ragged groups: a tile's A rows run past its group into the next group's rows
-// (or past the tensor, where TMA fills zeros); the epilogue writes only the
-// group's own rows.  The tile list is built on the device from the group
+// Groups.  A launch covers G_r "routed" groups, whose rows are given by device
+// offsets (the dispatch layout), followed by G_s "shared" groups that each see
+// the same `shared_rows` rows (every token).  Group g uses expert g of the
+// weight tensors it is given, so one launch can run the 256 routed and the 2
+// shared experts of the layer together.  The tile list, (group, row tile,
+// column tile) with the column index fastest, is built on the device from the
 // offsets, so the host never reads the per-expert counts.
+//
+// Per CTA (persistent, static round-robin over tiles):
+//   warp 0      TMA producer into a shared-memory ring of A and B tiles
+//               (128-byte swizzle, full/empty mbarriers)
+//   warp 1      TMEM owner + MMA issuer (one thread): tcgen05.mma kind::f16,
+//               bf16 in, fp32 accumulators in TMEM, two 256-column
+//               accumulator buffers so the epilogue of tile i overlaps the
+//               main loop of tile i+1
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, activation, bf16,
+//               16-byte stores of each row's 64-byte chunk
+// Two variants:
+//   PAIR = false  one CTA per 128 x 256 tile (4-stage ring of 48 KB)
+//   PAIR = true   a cluster of two CTAs per 256 x 256 tile with
+//                 tcgen05.mma.cta_group::2 (M = 256): CTA rank r holds A rows
+//                 r*128.. and B rows (output columns) r*128.. in its own
+//                 shared memory and accumulator rows r*128.. in its own TMEM;
+//                 both CTAs' loads signal the leader's full barrier, the
+//                 leader's MMA thread issues for the pair and commits to both
+//                 CTAs' barriers, both epilogues release the accumulator on
+//                 the leader.  Per CTA this halves the B operand's shared-
+//                 memory traffic (6-stage ring of 32 KB).
+// Ragged groups: a tile's A rows may run past its group (into the next
+// group's rows, or past the tensor where TMA fills zeros); the epilogue writes
+// only the group's own rows.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,47 +49,93 @@
 namespace moe {
 namespace gffn {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BN = 256;  // output columns per tile
+constexpr int BK = 64;   // reduction depth per stage (one 128-byte swizzle atom)
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_NONE = 1;
 
+template <bool PAIR>
+struct Cfg {
+  static constexpr int TILE_M = PAIR ? 256 : 128;  // rows per tile (per pair, or per CTA)
+  static constexpr int A_ROWS = 128;               // A rows held by one CTA
+  static constexpr int B_ROWS = PAIR ? 128 : 256;  // B rows (output columns) held by one CTA
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int A_BYTES = A_ROWS * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // bytes landing on the (leader's) full barrier
+};
+
 struct Params {
-  const int* offsets;  // [n_groups + 1] or null (every group sees rows 0..n_rows-1)
-  int n_groups;
-  int n_rows;          // rows of A for offsets mode; rows per group in identity mode
-  int a_group_stride;  // identity mode: A row base of group g = g * a_group_stride
-  int c_group_stride;  // identity mode: C row base of group g = g * c_group_stride
-  int c_row_limit;     // rows of C (writes at or past it are skipped)
-  int N;               // output columns
-  int K;               // reduction length
+  const int* offsets;  // [G_r + 1] routed group row offsets (device); unused when G_r == 0
+  int G_r;             // routed groups
+  int G_s;             // shared groups
+  int routed_rows;     // offsets are clamped to [0, routed_rows]
+  int shared_rows;     // rows of every shared group
+  int a_sh_map;        // A tensor map of shared groups: 0 = tmA0 (as routed), 1 = tmA1
+  int a_sh_base, a_sh_stride;  // A row of shared group s, row r: a_sh_base + s*a_sh_stride + r
+  __nv_bfloat16* C0;           // routed output: row off[g] + r
+  int c0_limit;
+  __nv_bfloat16* C1;           // shared output: row c1_base + s*c1_stride + r
+  int c1_base, c1_stride, c1_limit;
+  int N;  // output columns
+  int K;  // reduction length
   int n_tiles_n;
-  __nv_bfloat16* C;
   int ldc;
   uint64_t timeout_ns;
   unsigned int* status;
 };
 
+struct GroupTables {
+  int off[MOE_MAX_GROUPS + 1];
+  int prefix[MOE_MAX_GROUPS + 1];  // prefix[g] = row tiles of groups < g
+};
+
+template <bool PAIR>
 struct SmemTail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[Cfg<PAIR>::STAGES];
+  uint64_t empty[Cfg<PAIR>::STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  int off[MOE_MAX_GROUPS + 1];
-  int prefix[MOE_MAX_GROUPS + 1];
+  GroupTables gt;
 };
 
-constexpr size_t SMEM_BYTES = 1024 /* alignment slack */ + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+template <bool PAIR>
+constexpr size_t smem_bytes() {
+  return 1024 /* alignment slack */ + (size_t)Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + sizeof(SmemTail<PAIR>);
+}
+
+struct Group {
+  int rows;
+  int a_map;
+  int a_base;
+  int c_sel;
+  int c_base;
+};
+
+__device__ __forceinline__ Group group_info(const Params& p, const GroupTables& gt, int g) {
+  Group G;
+  if (g < p.G_r) {
+    G.rows = gt.off[g + 1] - gt.off[g];
+    G.a_map = 0;
+    G.a_base = gt.off[g];
+    G.c_sel = 0;
+    G.c_base = gt.off[g];
+  } else {
+    const int s = g - p.G_r;
+    G.rows = p.shared_rows;
+    G.a_map = p.a_sh_map;
+    G.a_base = p.a_sh_base + s * p.a_sh_stride;
+    G.c_sel = 1;
+    G.c_base = p.c1_base + s * p.c1_stride;
+  }
+  return G;
+}
 
 struct TileInfo {
   int g, m, nt;
@@ -81,7 +145,7 @@ __device__ __forceinline__ TileInfo tile_info(int tile, const int* prefix, int n
   TileInfo ti;
   int mt = tile / n_tiles_n;
   ti.nt = tile - mt * n_tiles_n;
-  int lo = 0, hi = n_groups;  // largest g with prefix[g] <= mt
+  int lo = 0, hi = n_groups;  // largest g with prefix[g] <= mt (never an empty group)
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
     if (prefix[mid] <= mt)
@@ -94,50 +158,23 @@ __device__ __forceinline__ TileInfo tile_info(int tile, const int* prefix, int n
   return ti;
 }
 
-template <int EPI>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* smemA = smem;
-  uint8_t* smemB = smem + STAGES * A_BYTES;
-  SmemTail* st = reinterpret_cast<SmemTail*>(smem + STAGES * STAGE_BYTES);
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const bool identity = (p.offsets == nullptr);
-
-  // ---- setup: barriers, group table, m-tile prefix ----
-  if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&st->full[s], 1);
-      mbar_init(&st->empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&st->tfull[a], 1);
-      mbar_init(&st->tempty[a], 128);
-    }
-    mbar_init(&st->drain, 1);
-    st->abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (!identity) {
-    for (int i = tid; i <= p.n_groups; i += NUM_THREADS) {
-      int v = p.offsets[i];
-      st->off[i] = v < 0 ? 0 : (v > p.n_rows ? p.n_rows : v);
-    }
+// Load the routed offsets and build the row-tile prefix over all groups.
+template <int TILE_M>
+__device__ __forceinline__ void build_tables(const Params& p, GroupTables& gt, int tid, int warp, int lane) {
+  for (int i = tid; i <= p.G_r && p.G_r > 0; i += NUM_THREADS) {
+    int v = p.offsets[i];
+    gt.off[i] = v < 0 ? 0 : (v > p.routed_rows ? p.routed_rows : v);
   }
   __syncthreads();
+  const int G = p.G_r + p.G_s;
   if (warp == 0) {
     int carry = 0;
-    for (int base = 0; base < p.n_groups; base += 32) {
+    for (int base = 0; base < G; base += 32) {
       int g = base + lane;
       int cnt = 0;
-      if (g < p.n_groups) {
-        int rows = identity ? p.n_rows : st->off[g + 1] - st->off[g];
-        cnt = rows > 0 ? (rows + BM - 1) / BM : 0;
+      if (g < G) {
+        int rows = g < p.G_r ? gt.off[g + 1] - gt.off[g] : p.shared_rows;
+        cnt = rows > 0 ? (rows + TILE_M - 1) / TILE_M : 0;
       }
       int v = cnt;
 #pragma unroll
@@ -145,18 +182,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int u = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += u;
       }
-      if (g < p.n_groups) st->prefix[g + 1] = carry + v;
+      if (g < G) gt.prefix[g + 1] = carry + v;
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
-    if (lane == 0) st->prefix[0] = 0;
+    if (lane == 0) gt.prefix[0] = 0;
   }
   __syncthreads();
-  const int total_tiles = st->prefix[p.n_groups] * p.n_tiles_n;
-  if ((int)blockIdx.x >= total_tiles) return;  // uniform across the CTA, before TMEM is taken
+}
 
-  if (warp == 1) tmem_alloc(&st->tmem_base, TMEM_COLS);
+template <int EPI, bool PAIR>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmB, const Params p) {
+  using C = Cfg<PAIR>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smemA = smem;
+  uint8_t* smemB = smem + C::STAGES * C::A_BYTES;
+  SmemTail<PAIR>* st = reinterpret_cast<SmemTail<PAIR>*>(smem + C::STAGES * C::STAGE_BYTES);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // pair or CTA index
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&st->full[s], 1);
+      mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&st->tfull[a], 1);
+      mbar_init(&st->tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
+    }
+    mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    fence_barrier_init();
+  }
+  build_tables<C::TILE_M>(p, st->gt, tid, warp, lane);
+  const int G = p.G_r + p.G_s;
+  const int total_tiles = st->gt.prefix[G] * p.n_tiles_n;
+  if (unit >= total_tiles) return;  // uniform across the CTA (and the pair), before TMEM is taken
+
+  if (warp == 1) {
+    if (PAIR)
+      tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
+    else
+      tmem_alloc(&st->tmem_base, TMEM_COLS);
+  }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync_all();  // both CTAs' barriers initialised and TMEM taken before any cross-CTA traffic
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = st->tmem_base;
   const int num_kb = (p.K + BK - 1) / BK;
@@ -165,48 +246,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
-      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmA0);
+      if (p.G_s > 0 && p.a_sh_map == 1) tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB);
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        TileInfo ti = tile_info(tile, st->prefix, p.n_groups, p.n_tiles_n);
-        int a_row = (identity ? ti.g * p.a_group_stride : st->off[ti.g]) + ti.m * BM;
-        int n0 = ti.nt * BN;
+      for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
+        const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
+        const Group gr = group_info(p, st->gt, ti.g);
+        const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
+        const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
+        const int b_row = ti.nt * BN + (int)rank * C::B_ROWS;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&st->full[stage], STAGE_BYTES);
-          tma_load_2d(smemA + stage * A_BYTES, &tmA, &st->full[stage], kb * BK, a_row);
-          tma_load_3d(smemB + stage * B_BYTES, &tmB, &st->full[stage], kb * BK, n0, ti.g);
+          if (leader) mbar_arrive_expect_tx(&st->full[stage], C::TX_BYTES);
+          if (PAIR) {
+            tma_load_2d_pair(smemA + stage * C::A_BYTES, am, &st->full[stage], kb * BK, a_row);
+            tma_load_3d_pair(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+          } else {
+            tma_load_2d(smemA + stage * C::A_BYTES, am, &st->full[stage], kb * BK, a_row);
+            tma_load_3d(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+          }
           ++issued;
-          if (++stage == STAGES) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (!ok) {
+      if (!ok && !PAIR) {
         // wind down: let the copies already issued land before the CTA exits
         int zero = 0;
-        for (long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
-          mbar_wait(&st->full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.timeout_ns, &zero, p.status);
+        for (long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
+          mbar_wait(&st->full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), p.timeout_ns, &zero, p.status);
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_bf16(BM, BN);
+    // ================= MMA issuer (the pair's leader) =================
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc_bf16(C::TILE_M, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
         if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -216,46 +305,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smemA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(smemB + stage * B_BYTES);
+          const uint32_t a_addr = smem_u32(smemA + stage * C::A_BYTES);
+          const uint32_t b_addr = smem_u32(smemB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            mma_bf16_ss(d_tmem, make_desc_sw128(a_addr + k * 32), make_desc_sw128(b_addr + k * 32), idesc,
-                        (kb | k) != 0 ? 1u : 0u);
+            const uint64_t ad = make_desc_sw128(a_addr + k * 32);
+            const uint64_t bd = make_desc_sw128(b_addr + k * 32);
+            if (PAIR)
+              mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          mma_commit(&st->empty[stage]);
-          if (++stage == STAGES) {
+          if (PAIR)
+            mma_commit_pair(&st->empty[stage], 0x3);
+          else
+            mma_commit(&st->empty[stage]);
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&st->tfull[acc]);
+        if (PAIR)
+          mma_commit_pair(&st->tfull[acc], 0x3);
+        else
+          mma_commit(&st->tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // no MMA may still be running when TMEM is released
       int zero = 0;
-      mma_commit(&st->drain);
+      if (PAIR)
+        mma_commit_pair(&st->drain, 0x1);
+      else
+        mma_commit(&st->drain);
       mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
     }
   } else {
     // ================= epilogue (warps 2..5) =================
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int row_in_tile = quarter * 32 + lane;
+    const int row_in_tile = (int)rank * C::A_ROWS + quarter * 32 + lane;
+    const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(&st->tempty[0]), 0) : 0u;
+    const uint32_t tempty1 = PAIR ? mapa_shared(smem_u32(&st->tempty[1]), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      TileInfo ti = tile_info(tile, st->prefix, p.n_groups, p.n_tiles_n);
-      int rows_g = identity ? p.n_rows : st->off[ti.g + 1] - st->off[ti.g];
-      int c_base = identity ? ti.g * p.c_group_stride : st->off[ti.g];
-      int r = ti.m * BM + row_in_tile;
-      int c_row = c_base + r;
-      bool valid = (r < rows_g) && (c_row < p.c_row_limit);
+    for (int tile = unit; tile < total_tiles; tile += n_units) {
+      const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
+      const Group gr = group_info(p, st->gt, ti.g);
+      const int r = ti.m * C::TILE_M + row_in_tile;
+      const int c_row = gr.c_base + r;
+      __nv_bfloat16* cbase = gr.c_sel ? p.C1 : p.C0;
+      const int climit = gr.c_sel ? p.c1_limit : p.c0_limit;
+      const bool valid = (r < gr.rows) && (c_row < climit);
       if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      __nv_bfloat16* crow = p.C + (size_t)c_row * p.ldc;
+      __nv_bfloat16* crow = cbase + (size_t)c_row * p.ldc;
 #pragma unroll 1
       for (int ch = 0; ch < BN / 32; ++ch) {
         const int col0 = ti.nt * BN + ch * 32;
@@ -279,274 +384,112 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&st->tempty[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(acc == 0 ? tempty0 : tempty1);
+        else
+          mbar_arrive(&st->tempty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
-  __syncthreads();
+  tc_fence_before();
+  if (PAIR)
+    cluster_sync_all();  // every MMA of the pair has landed; both CTAs are done with each other's memory
+  else
+    __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-// ---------------------------------------------------------------------------
-// CTA-pair variant: a cluster of 2 CTAs computes a 256 x 256 tile with
-// tcgen05.mma.cta_group::2 (M = 256, N = 256).  CTA rank r holds A rows
-// r*128 .. r*128+127 of the tile and B rows (output columns) r*128 ..
-// r*128+127 in its own shared memory, and receives accumulator rows r*128 ..
-// in its own TMEM.  Each CTA's producer loads its halves; every load signals
-// the leader's (rank 0) full barrier, whose producer expects both halves'
-// bytes.  The leader's single MMA thread issues for the pair and commits to
-// both CTAs' empty / accumulator-full barriers; both CTAs' epilogue warps
-// release the accumulator on the leader's barrier.  Per CTA and K step this
-// halves the B operand's shared-memory traffic of the 1-CTA kernel.
-// ---------------------------------------------------------------------------
-constexpr int P_BM = 256;                      // tile rows per pair
-constexpr int P_HALF = 128;                    // rows (of A and of B) per CTA
-constexpr int P_STAGES = 6;
-constexpr int P_A_BYTES = P_HALF * BK * 2;     // 16 KB
-constexpr int P_B_BYTES = P_HALF * BK * 2;     // 16 KB
-constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+template <int EPI, bool PAIR>
+int launch_one(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const Params& p, int grid,
+               cudaStream_t stream) {
+  auto kfn = grouped_gemm_kernel<EPI, PAIR>;
+  constexpr size_t bytes = smem_bytes<PAIR>();
+  int rc = ensure_smem_attr((const void*)kfn, bytes);
+  if (rc != MOE_OK) return rc;
+  if (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kfn, a0, a1, b, p) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    kfn<<<grid, NUM_THREADS, bytes, stream>>>(a0, a1, b, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
-struct SmemTailPair {
-  uint64_t full[P_STAGES];
-  uint64_t empty[P_STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort_flag;
-  int off[MOE_MAX_GROUPS + 1];
-  int prefix[MOE_MAX_GROUPS + 1];
+// Everything one GEMM launch needs from the host.
+struct GemmSpec {
+  const void* a0;
+  uint64_t a0_rows;
+  const void* a1;  // may be null (then a0's map is passed twice)
+  uint64_t a1_rows;
+  const void* b;   // weights of the launch's group 0: [G, N, K]
+  Params p;
 };
 
-constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * P_STAGE_BYTES + sizeof(SmemTailPair);
+// Kernel variant.  CTA pairs (cta_group::2, 256 x 256 tiles) halve each CTA's shared-memory operand
+// traffic and win when groups are large (compute-bound); with few rows per group the work is weight
+// streaming and single CTAs (128 x 256 tiles, more weight bytes in flight per SM) win.
+// MOE_GEMM_CTA=1 or =2 forces one of them.
+bool choose_pair(long long rows, int groups) {
+  bool pair = groups > 0 && rows / groups >= 256;
+  const char* env = getenv("MOE_GEMM_CTA");
+  if (env && env[0] == '1' && env[1] == '\0') pair = false;
+  if (env && env[0] == '2' && env[1] == '\0') pair = true;
+  return pair;
+}
 
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* smemA = smem;
-  uint8_t* smemB = smem + P_STAGES * P_A_BYTES;
-  SmemTailPair* st = reinterpret_cast<SmemTailPair*>(smem + P_STAGES * P_STAGE_BYTES);
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = (rank == 0);
-  const int pair = blockIdx.x >> 1;
-  const int n_pairs = gridDim.x >> 1;
-  const bool identity = (p.offsets == nullptr);
-
-  if (tid == 0) {
-    for (int s = 0; s < P_STAGES; ++s) {
-      mbar_init(&st->full[s], 1);
-      mbar_init(&st->empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&st->tfull[a], 1);
-      mbar_init(&st->tempty[a], 8);  // 4 epilogue warps x 2 CTAs
-    }
-    mbar_init(&st->drain, 1);
-    st->abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (!identity) {
-    for (int i = tid; i <= p.n_groups; i += NUM_THREADS) {
-      int v = p.offsets[i];
-      st->off[i] = v < 0 ? 0 : (v > p.n_rows ? p.n_rows : v);
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int carry = 0;
-    for (int base = 0; base < p.n_groups; base += 32) {
-      int g = base + lane;
-      int cnt = 0;
-      if (g < p.n_groups) {
-        int rows = identity ? p.n_rows : st->off[g + 1] - st->off[g];
-        cnt = rows > 0 ? (rows + P_BM - 1) / P_BM : 0;
-      }
-      int v = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-      }
-      if (g < p.n_groups) st->prefix[g + 1] = carry + v;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-    if (lane == 0) st->prefix[0] = 0;
-  }
-  __syncthreads();
-  const int total_tiles = st->prefix[p.n_groups] * p.n_tiles_n;
-  if (pair >= total_tiles) return;  // both CTAs of the pair leave together, before any cluster traffic
-
-  if (warp == 1) tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
-  tc_fence_before();
-  cluster_sync_all();  // barriers of both CTAs initialised, TMEM taken in both
-  tc_fence_after();
-  const uint32_t tmem_base = st->tmem_base;
-  const int num_kb = (p.K + BK - 1) / BK;
-  volatile int* abort_flag = &st->abort_flag;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
-        TileInfo ti = tile_info(tile, st->prefix, p.n_groups, p.n_tiles_n);
-        int a_row = (identity ? ti.g * p.a_group_stride : st->off[ti.g]) + ti.m * P_BM + (int)rank * P_HALF;
-        int b_row = ti.nt * BN + (int)rank * P_HALF;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(&st->full[stage], 2 * P_STAGE_BYTES);
-          tma_load_2d_pair(smemA + stage * P_A_BYTES, &tmA, &st->full[stage], kb * BK, a_row);
-          tma_load_3d_pair(smemB + stage * P_B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
-          if (++stage == P_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc_bf16(P_BM, BN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
-        if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&st->full[stage], phase, p.timeout_ns, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smemA + stage * P_A_BYTES);
-          const uint32_t b_addr = smem_u32(smemB + stage * P_B_BYTES);
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            mma_bf16_ss_pair(d_tmem, make_desc_sw128(a_addr + k * 32), make_desc_sw128(b_addr + k * 32), idesc,
-                             (kb | k) != 0 ? 1u : 0u);
-          }
-          mma_commit_pair(&st->empty[stage], 0x3);
-          if (++stage == P_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        mma_commit_pair(&st->tfull[acc], 0x3);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      }
-      int zero = 0;
-      mma_commit_pair(&st->drain, 0x1);
-      mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
-    }
+int run_gemm(const GemmSpec& g, bool pair, int sms, long long tiles_upper, cudaStream_t s) {
+  const uint32_t b_box = pair ? (uint32_t)Cfg<true>::B_ROWS : (uint32_t)Cfg<false>::B_ROWS;
+  CUtensorMap a0, a1, b;
+  int rc;
+  const uint64_t K = (uint64_t)g.p.K, N = (uint64_t)g.p.N;
+  if ((rc = encode_tmap_bf16(&a0, g.a0, 2, K, g.a0_rows, 1, BK, 128)) != MOE_OK) return rc;
+  if (g.a1) {
+    if ((rc = encode_tmap_bf16(&a1, g.a1, 2, K, g.a1_rows, 1, BK, 128)) != MOE_OK) return rc;
   } else {
-    const int quarter = warp & 3;
-    const int row_in_tile = (int)rank * P_HALF + quarter * 32 + lane;
-    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&st->tempty[0]), 0);
-    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&st->tempty[1]), 0);
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
-      TileInfo ti = tile_info(tile, st->prefix, p.n_groups, p.n_tiles_n);
-      int rows_g = identity ? p.n_rows : st->off[ti.g + 1] - st->off[ti.g];
-      int c_base = identity ? ti.g * p.c_group_stride : st->off[ti.g];
-      int r = ti.m * P_BM + row_in_tile;
-      int c_row = c_base + r;
-      bool valid = (r < rows_g) && (c_row < p.c_row_limit);
-      if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      __nv_bfloat16* crow = p.C + (size_t)c_row * p.ldc;
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int col0 = ti.nt * BN + ch * 32;
-        if (col0 >= p.N) break;
-        float v[32];
-        tmem_ld32(taddr + ch * 32, v);
-        if (valid) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a = v[2 * i], b = v[2 * i + 1];
-            if (EPI == EPI_GELU) {
-              a = gelu_tanh_f32(a);
-              b = gelu_tanh_f32(b);
-            }
-            pk[i] = pack_bf16x2(a, b);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
-    }
+    a1 = a0;
   }
-
-  tc_fence_before();
-  cluster_sync_all();  // every MMA of the pair has landed and both CTAs are done with each other's memory
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  if ((rc = encode_tmap_bf16(&b, g.b, 3, K, N, (uint64_t)(g.p.G_r + g.p.G_s), BK, b_box)) != MOE_OK) return rc;
+  long long units = tiles_upper * g.p.n_tiles_n;
+  if (pair) {
+    long long pairs = units < sms / 2 ? units : sms / 2;
+    return launch_one<EPI, true>(a0, a1, b, g.p, (int)(2 * pairs), s);
   }
-}
-
-template <int EPI>
-int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const Params& p, int grid, cudaStream_t stream) {
-  auto kfn = grouped_gemm_pair_kernel<EPI>;
-  int rc = ensure_smem_attr((const void*)kfn, P_SMEM_BYTES);
-  if (rc != MOE_OK) return rc;
-  kfn<<<grid, NUM_THREADS, P_SMEM_BYTES, stream>>>(tmA, tmB, p);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
-template <int EPI>
-int launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const Params& p, int grid, cudaStream_t stream) {
-  auto kfn = grouped_gemm_kernel<EPI>;
-  int rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES);
-  if (rc != MOE_OK) return rc;
-  kfn<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_one<EPI, false>(a0, a1, b, g.p, (int)(units < sms ? units : sms), s);
 }
 
 }  // namespace gffn
 }  // namespace moe
 
 using namespace moe;
+using namespace moe::gffn;
 
 extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, int n_rows,
                                int expert_base, const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff,
                                int activation, moe_bf16* h_scratch, moe_bf16* y, void* stream) {
-  using namespace moe::gffn;
   if (n_groups < 0 || n_rows < 0 || expert_base < 0 || d <= 0 || d_ff <= 0) return MOE_ERR_INVALID_ARG;
   if (activation != MOE_ACT_GELU_TANH) return MOE_ERR_INVALID_ARG;
   if (!aligned16(rows) || !aligned16(w1) || !aligned16(w2) || !aligned16(h_scratch) || !aligned16(y))
@@ -564,72 +507,140 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   int dev, sms;
   int rc = device_info(&dev, &sms);
   if (rc != MOE_OK) return rc;
+  unsigned int* status = status_ptr();
+  if (!status) return MOE_ERR_CUDA;
 
-  const __nv_bfloat16* w1e = reinterpret_cast<const __nv_bfloat16*>(w1) + (size_t)expert_base * d_ff * d;
-  const __nv_bfloat16* w2e = reinterpret_cast<const __nv_bfloat16*>(w2) + (size_t)expert_base * d * d_ff;
+  const bool pair = choose_pair(h_rows, n_groups);
+  const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
+  const long long tiles_upper = identity ? (long long)n_groups * ((n_rows + tile_m - 1) / tile_m)
+                                         : (n_rows + tile_m - 1) / tile_m + n_groups;
 
-  // Kernel variant.  CTA pairs (cta_group::2, 256 x 256 tiles) halve each CTA's shared-memory
-  // operand traffic and win when groups are large (compute-bound); with few rows per group the
-  // work is weight streaming and single CTAs (128 x 256 tiles, more weight bytes in flight per
-  // SM) win.  MOE_GEMM_CTA=1 or =2 forces one of them.
-  const char* env = getenv("MOE_GEMM_CTA");
-  const long long rows_per_group = identity ? n_rows : n_rows / n_groups;
-  bool pair = rows_per_group >= 256;
-  if (env && env[0] == '1' && env[1] == '\0') pair = false;
-  if (env && env[0] == '2' && env[1] == '\0') pair = true;
-  const uint32_t b_box = pair ? (uint32_t)P_HALF : (uint32_t)BN;
-  const int tile_m = pair ? P_BM : BM;
+  Params p{};
+  p.offsets = offsets;
+  p.G_r = identity ? 0 : n_groups;
+  p.G_s = identity ? n_groups : 0;
+  p.routed_rows = n_rows;
+  p.shared_rows = n_rows;
+  p.a_sh_map = 0;
+  p.timeout_ns = wait_timeout_ns();
+  p.status = status;
 
-  CUtensorMap tA1, tB1, tA2, tB2;
-  // GEMM1: A = rows [n_rows, d], B = W1 [n_groups, d_ff, d]
-  if ((rc = encode_tmap_bf16(&tA1, rows, 2, (uint64_t)d, (uint64_t)n_rows, 1, BK, BM)) != MOE_OK) return rc;
-  if ((rc = encode_tmap_bf16(&tB1, w1e, 3, (uint64_t)d, (uint64_t)d_ff, (uint64_t)n_groups, BK, b_box)) != MOE_OK)
-    return rc;
-  // GEMM2: A = H [h_rows, d_ff], B = W2 [n_groups, d, d_ff]
-  if ((rc = encode_tmap_bf16(&tA2, h_scratch, 2, (uint64_t)d_ff, (uint64_t)h_rows, 1, BK, BM)) != MOE_OK)
-    return rc;
-  if ((rc = encode_tmap_bf16(&tB2, w2e, 3, (uint64_t)d_ff, (uint64_t)d, (uint64_t)n_groups, BK, b_box)) != MOE_OK)
-    return rc;
+  GemmSpec g1{};
+  g1.a0 = rows;
+  g1.a0_rows = (uint64_t)n_rows;
+  g1.b = reinterpret_cast<const __nv_bfloat16*>(w1) + (size_t)expert_base * d_ff * d;
+  g1.p = p;
+  g1.p.a_sh_base = 0;
+  g1.p.a_sh_stride = 0;  // every shared group reads rows 0..n_rows-1
+  g1.p.C0 = g1.p.C1 = reinterpret_cast<__nv_bfloat16*>(h_scratch);
+  g1.p.c0_limit = g1.p.c1_limit = (int)h_rows;
+  g1.p.c1_base = 0;
+  g1.p.c1_stride = n_rows;
+  g1.p.N = d_ff;
+  g1.p.K = d;
+  g1.p.n_tiles_n = (d_ff + BN - 1) / BN;
+  g1.p.ldc = d_ff;
+  if ((rc = run_gemm<EPI_GELU>(g1, pair, sms, tiles_upper, s)) != MOE_OK) return rc;
 
-  // upper bound on m-tiles: every group may add one partial tile
-  long long mtiles = identity ? (long long)n_groups * ((n_rows + tile_m - 1) / tile_m)
-                              : (n_rows + tile_m - 1) / tile_m + n_groups;
-  auto grid_for = [&](long long tiles) -> int {
-    if (pair) {
-      long long pairs = tiles < sms / 2 ? tiles : sms / 2;
-      return (int)(2 * pairs);
-    }
-    return (int)(tiles < sms ? tiles : sms);
-  };
+  GemmSpec g2{};
+  g2.a0 = h_scratch;
+  g2.a0_rows = (uint64_t)h_rows;
+  g2.b = reinterpret_cast<const __nv_bfloat16*>(w2) + (size_t)expert_base * d * d_ff;
+  g2.p = p;
+  g2.p.a_sh_base = 0;
+  g2.p.a_sh_stride = n_rows;
+  g2.p.C0 = g2.p.C1 = reinterpret_cast<__nv_bfloat16*>(y);
+  g2.p.c0_limit = g2.p.c1_limit = (int)h_rows;
+  g2.p.c1_base = 0;
+  g2.p.c1_stride = n_rows;
+  g2.p.N = d;
+  g2.p.K = d_ff;
+  g2.p.n_tiles_n = (d + BN - 1) / BN;
+  g2.p.ldc = d;
+  return run_gemm<EPI_NONE>(g2, pair, sms, tiles_upper, s);
+}
 
-  Params p1{};
-  p1.offsets = offsets;
-  p1.n_groups = n_groups;
-  p1.n_rows = n_rows;
-  p1.a_group_stride = 0;
-  p1.c_group_stride = n_rows;
-  p1.c_row_limit = (int)h_rows;
-  p1.N = d_ff;
-  p1.K = d;
-  p1.n_tiles_n = (d_ff + BN - 1) / BN;
-  p1.C = reinterpret_cast<__nv_bfloat16*>(h_scratch);
-  p1.ldc = d_ff;
-  p1.timeout_ns = wait_timeout_ns();
-  p1.status = status_ptr();
-  if (!p1.status) return MOE_ERR_CUDA;
-  const int grid1 = grid_for(mtiles * p1.n_tiles_n);
-  rc = pair ? launch_pair<EPI_GELU>(tA1, tB1, p1, grid1, s) : launch<EPI_GELU>(tA1, tB1, p1, grid1, s);
+extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* offsets, int T,
+                               int n_routed, int n_shared, int top_k, const moe_bf16* w1, const moe_bf16* w2, int d,
+                               int d_ff, int activation, moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared,
+                               void* stream) {
+  if (T < 0 || n_routed < 0 || n_shared < 0 || top_k < 1 || d <= 0 || d_ff <= 0) return MOE_ERR_INVALID_ARG;
+  if (activation != MOE_ACT_GELU_TANH) return MOE_ERR_INVALID_ARG;
+  if (n_routed + n_shared > MOE_MAX_GROUPS) return MOE_ERR_UNSUPPORTED;
+  if (d % 64 != 0 || d_ff % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!w1 || !w2 || !h_scratch || !aligned16(w1) || !aligned16(w2) || !aligned16(h_scratch))
+    return MOE_ERR_INVALID_ARG;
+  if (n_routed > 0 && (!x_perm || !offsets || !y_perm || !aligned16(x_perm) || !aligned4(offsets) ||
+                       !aligned16(y_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (n_shared > 0 && (!x || !y_shared || !aligned16(x) || !aligned16(y_shared))) return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * top_k;
+  const long long h_rows = R + (long long)n_shared * T;
+  if (h_rows > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (T == 0 || n_routed + n_shared == 0) return MOE_OK;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  int dev, sms;
+  int rc = device_info(&dev, &sms);
   if (rc != MOE_OK) return rc;
+  unsigned int* status = status_ptr();
+  if (!status) return MOE_ERR_CUDA;
 
-  Params p2 = p1;
-  p2.a_group_stride = n_rows;
-  p2.c_group_stride = n_rows;
-  p2.c_row_limit = (int)h_rows;
-  p2.N = d;
-  p2.K = d_ff;
-  p2.n_tiles_n = (d + BN - 1) / BN;
-  p2.C = reinterpret_cast<__nv_bfloat16*>(y);
-  p2.ldc = d;
-  const int grid2 = grid_for(mtiles * p2.n_tiles_n);
-  return pair ? launch_pair<EPI_NONE>(tA2, tB2, p2, grid2, s) : launch<EPI_NONE>(tA2, tB2, p2, grid2, s);
+  const int G = n_routed + n_shared;
+  const bool pair = choose_pair(h_rows, G);
+  const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
+  const long long tiles_upper =
+      (R + tile_m - 1) / tile_m + n_routed + (long long)n_shared * ((T + tile_m - 1) / tile_m);
+
+  Params p{};
+  p.offsets = offsets;
+  p.G_r = n_routed;
+  p.G_s = n_shared;
+  p.routed_rows = (int)R;
+  p.shared_rows = T;
+  p.timeout_ns = wait_timeout_ns();
+  p.status = status;
+
+  // GEMM1: routed rows from x_perm (map 0), shared rows from x (map 1); H = [routed rows | shared s rows]
+  GemmSpec g1{};
+  g1.a0 = n_routed > 0 ? (const void*)x_perm : (const void*)x;
+  g1.a0_rows = n_routed > 0 ? (uint64_t)R : (uint64_t)T;
+  g1.a1 = n_shared > 0 ? (const void*)x : nullptr;
+  g1.a1_rows = (uint64_t)T;
+  g1.b = w1;
+  g1.p = p;
+  g1.p.a_sh_map = n_routed > 0 ? 1 : 0;
+  g1.p.a_sh_base = 0;
+  g1.p.a_sh_stride = 0;
+  g1.p.C0 = g1.p.C1 = reinterpret_cast<__nv_bfloat16*>(h_scratch);
+  g1.p.c0_limit = (int)R;
+  g1.p.c1_base = (int)R;
+  g1.p.c1_stride = T;
+  g1.p.c1_limit = (int)h_rows;
+  g1.p.N = d_ff;
+  g1.p.K = d;
+  g1.p.n_tiles_n = (d_ff + BN - 1) / BN;
+  g1.p.ldc = d_ff;
+  if ((rc = run_gemm<EPI_GELU>(g1, pair, sms, tiles_upper, s)) != MOE_OK) return rc;
+
+  // GEMM2: all A rows from H (map 0); routed outputs to y_perm, shared outputs to y_shared
+  GemmSpec g2{};
+  g2.a0 = h_scratch;
+  g2.a0_rows = (uint64_t)h_rows;
+  g2.b = w2;
+  g2.p = p;
+  g2.p.a_sh_map = 0;
+  g2.p.a_sh_base = (int)R;
+  g2.p.a_sh_stride = T;
+  g2.p.C0 = reinterpret_cast<__nv_bfloat16*>(y_perm);
+  g2.p.c0_limit = (int)R;
+  g2.p.C1 = reinterpret_cast<__nv_bfloat16*>(y_shared);
+  g2.p.c1_base = 0;
+  g2.p.c1_stride = T;
+  g2.p.c1_limit = n_shared * T;
+  g2.p.N = d;
+  g2.p.K = d_ff;
+  g2.p.n_tiles_n = (d + BN - 1) / BN;
+  g2.p.ldc = d;
+  return run_gemm<EPI_NONE>(g2, pair, sms, tiles_upper, s);
 }

@@ -97,6 +97,21 @@ def test_grouped_ffn_rejects_and_empty_is_noop():
     assert call(G=0) == moe.MOE_OK
 
 
+def test_experts_ffn_rejects():
+    def call(x=A16, xp=A16, off=A16, T=64, nr=256, ns=2, k=6, w1=A16, w2=A16, d=64, f=64, act=0, h=A16, yp=A16,
+             ys=A16):
+        return L.moe_experts_ffn(x, xp, off, T, nr, ns, k, w1, w2, d, f, act, h, yp, ys, NULL)
+
+    assert call(xp=NULL) == moe.MOE_ERR_INVALID_ARG
+    assert call(ys=NULL) == moe.MOE_ERR_INVALID_ARG
+    assert call(off=0x10002) == moe.MOE_ERR_INVALID_ARG
+    assert call(d=96) == moe.MOE_ERR_UNSUPPORTED
+    assert call(nr=1024, ns=8) == moe.MOE_ERR_UNSUPPORTED
+    assert call(k=0) == moe.MOE_ERR_INVALID_ARG
+    assert call(T=0) == moe.MOE_OK
+    assert call(nr=0, ns=0) == moe.MOE_OK
+
+
 def test_combine_and_bias_update_reject():
     assert L.moe_combine(A16, A16, A16, NULL, 4, 64, 6, 2, A16, NULL) == moe.MOE_ERR_INVALID_ARG  # y_shared missing
     assert L.moe_combine(A16, A16, A16, A16, 4, 60, 6, 2, A16, NULL) == moe.MOE_ERR_UNSUPPORTED

@@ -17,9 +17,9 @@ if torch.cuda.is_available():
     import sparse_moe_layer_joint_b200 as moe
 
 
-def _layer(w, with_weights=True):
+def _layer(w, with_weights=True, fused=True):
     t = mi.torch_workload(w, with_weights=with_weights)
-    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k))
+    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), fused_experts=fused)
     return t, layer
 
 
@@ -43,9 +43,9 @@ def _check_dispatch_properties(layer, x_bits, T, k, n_routed):
     np.testing.assert_array_equal(xp, x_bits[rt[sample]])
 
 
-def _run_and_check(name, tokens=None, check_all_routing=True):
+def _run_and_check(name, tokens=None, check_all_routing=True, fused=True):
     w = mi.WORKLOADS[name]
-    t, layer = _layer(w)
+    t, layer = _layer(w, fused=fused)
     bias0 = t["bias"].clone()
     out = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
     layer.bias_update(t["bias"], w.gamma)
@@ -78,6 +78,11 @@ def _run_and_check(name, tokens=None, check_all_routing=True):
 
 def test_layer_tiny_all_tokens():
     _run_and_check("tiny")
+
+
+def test_layer_tiny_two_streams():
+    """The shared experts on a second stream (two moe_grouped_ffn calls) instead of the fused launch."""
+    _run_and_check("tiny", fused=False)
 
 
 @pytest.mark.slow

@@ -253,6 +253,40 @@ def test_grouped_ffn_special_weights(gemm_variant):
     np.testing.assert_allclose(yg[100:], ref, rtol=2 ** -7, atol=2e-3)
 
 
+@pytest.mark.parametrize("T,n_routed,n_shared,k,d,f", [
+    (300, 16, 2, 3, 256, 128), (1000, 8, 2, 2, 512, 256), (64, 64, 2, 6, 256, 256), (700, 4, 0, 2, 128, 128),
+    (129, 0, 2, 1, 128, 192),
+])
+def test_experts_ffn_parity(T, n_routed, n_shared, k, d, f, gemm_variant):
+    """Routed experts on dispatched rows and shared experts on all tokens, one pair of launches."""
+    E = n_routed + n_shared
+    x = mi.normal_bf16(T * d, 11, mi.STREAM_X).reshape(T, d)
+    w1, w2 = _ffn_weights(E, d, f, 11)
+    R = T * k
+    h = torch.empty((R + n_shared * T, f), dtype=torch.bfloat16, device="cuda")
+    y_perm = torch.full((max(R, 1), d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y_sh = torch.full((max(n_shared, 1), T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    if n_routed:
+        topk = _random_topk(T, k, n_routed, 12)
+        dp = oracle.dispatch(topk, n_routed)
+        xp = x[dp["row_token"]]
+        moe.moe_experts_ffn(dev_bf16(x), dev_bf16(xp), _i32(dp["offsets"]), T, n_routed, n_shared, k, dev_bf16(w1),
+                            dev_bf16(w2), d, f, moe.MOE_ACT_GELU_TANH, h, y_perm, y_sh)
+    else:
+        moe.moe_experts_ffn(dev_bf16(x), None, None, T, 0, n_shared, k, dev_bf16(w1), dev_bf16(w2), d, f,
+                            moe.MOE_ACT_GELU_TANH, h, y_perm, y_sh)
+    assert moe.moe_get_status() == 0
+    if n_routed:
+        yp = host_bf16_f64(y_perm)
+        off = dp["offsets"]
+        for e in range(n_routed):
+            if off[e] < off[e + 1]:
+                check_output(yp[off[e]:off[e + 1]], oracle.expert(xp[off[e]:off[e + 1]], w1[e], w2[e]), f"routed {e}")
+    ys = host_bf16_f64(y_sh)
+    for sidx in range(n_shared):
+        check_output(ys[sidx], oracle.expert(x, w1[n_routed + sidx], w2[n_routed + sidx]), f"shared {sidx}")
+
+
 # ---------------------------------------------------------------------------
 # combine
 # ---------------------------------------------------------------------------
