@@ -151,6 +151,7 @@ def run_ours(args, w, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after warm-up")
 
+    bias_at_start = t["bias"].clone()   # to replay the timed steps afterwards
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
@@ -166,6 +167,18 @@ def run_ours(args, w, rank, world, local_rank):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ffn_ev)
+
+    # replay the timed steps (routing is deterministic) to learn which experts each
+    # step touched: the expert GEMMs read only those experts' weights
+    t["bias"].copy_(bias_at_start)
+    local_counts = torch.empty((args.steps, w.n_routed), dtype=torch.int32, device=dev)
+    for i in range(args.steps):
+        layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
+        local_counts[i].copy_(layer.counts)
+        if world > 1:
+            dist.all_reduce(layer.counts)
+        layer.bias_update(t["bias"], w.gamma)
+    touched = (local_counts > 0).sum(dim=1).double().mean().item()
 
     # end to end through the public API: pinned host x in, host out back, every step
     x_host = t["x"].cpu().pin_memory()
@@ -196,22 +209,33 @@ def run_ours(args, w, rank, world, local_rank):
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
     ms, e2e_ms, ffn_ms = vals.tolist()
 
-    # the dominant kernel: the experts' grouped GEMMs (both launches of one
-    # moe_experts_ffn call), algorithmic FLOPs = 2 GEMMs x 2 * rows * d * d_ff
-    # over the T*k routed and T*n_shared shared (token, expert) rows
+    # the dominant kernels: the experts' grouped GEMMs (both launches of one
+    # moe_experts_ffn call).  Algorithmic work per step: FLOPs = 2 GEMMs x 2 * rows * d * d_ff
+    # over the T*k routed and T*n_shared shared (token, expert) rows; bytes = weights of the
+    # touched routed experts and the shared experts + A rows read + hidden written and read
+    # + outputs written (bf16)
     pk = peaks()
     rows = w.T * (w.k + w.n_shared)
     ffn_flops = 2 * 2.0 * rows * w.d * w.f
-    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
-    roofline = {"kernel": "grouped_gemm_kernel x2 (all 258 experts: GEMM1+GELU, GEMM2)", "bound": "tensor",
-                "achieved": round(achieved, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
-                "peak_source": f"{pk['src']} bf16 sustained (MEASURED_PEAKS.json)" if pk["src"] == "measured"
-                else "fallback bf16 sustained", "traffic": None,
-                "ms_per_launch_pair": round(ffn_ms, 4),
-                "layer_tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1)}
-    if w.name in ("decode", "mid"):
-        roofline["note"] = "HBM-bound workload; see DESIGN.md for its byte roofline"
+    ffn_bytes = ((touched + w.n_shared) * 2 * w.d * w.f * 2
+                 + rows * w.d * 2 + rows * w.f * 2 * 2 + rows * w.d * 2)
+    tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
+    gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
+    kernel = "grouped_gemm_kernel x2 (all experts: GEMM1+GELU, GEMM2)"
+    tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1),
+                   "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                   "frac": round(tflops / pk["bf16_tflops_sustained"], 4),
+                   "peak_source": f"{pk['src']} bf16 sustained (MEASURED_PEAKS.json)" if pk["src"] == "measured"
+                   else "fallback bf16 sustained", "traffic": None,
+                   "flop_per_launch_pair": ffn_flops, "ms_per_launch_pair": round(ffn_ms, 4)}
+    hbm_roof = {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / pk["hbm_gbs"], 4),
+                "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)", "traffic": None,
+                "bytes_per_launch_pair": round(ffn_bytes), "touched_routed_experts_mean": round(touched, 2),
+                "ms_per_launch_pair": round(ffn_ms, 4)}
+    weight_bound = w.name in ("decode", "mid")
+    roofline = hbm_roof if weight_bound else tensor_roof
+    roofline["layer_tflops"] = round(w.flops() / (ms * 1e-3) / 1e12, 1)
     line = {
         "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
@@ -222,6 +246,7 @@ def run_ours(args, w, rank, world, local_rank):
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": layer.launches_per_step() * args.steps,
         "roofline": roofline,
+        "roofline_other": tensor_roof if weight_bound else hbm_roof,
     }
     del bias0
     return line
@@ -296,17 +321,27 @@ def run_kernel_case(args):
     n = G * per
     dev = torch.device("cuda", 0)
     s = torch.cuda.current_stream(dev).cuda_stream
-    rows = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
-    w1 = torch.empty((G, f, d), dtype=torch.bfloat16, device=dev)
-    w2 = torch.empty((G, d, f), dtype=torch.bfloat16, device=dev)
-    mi.gpu_normal_bf16(rows.data_ptr(), rows.numel(), 0, mi.STREAM_TEST_ROWS, 0, 1.0, s)
-    mi.gpu_normal_bf16(w1.data_ptr(), w1.numel(), 0, mi.STREAM_W1, 0, d ** -0.5, s)
-    mi.gpu_normal_bf16(w2.data_ptr(), w2.numel(), 0, mi.STREAM_W2, 0, f ** -0.5, s)
-    offsets = torch.arange(0, n + 1, per, dtype=torch.int32, device=dev)
-    h = torch.empty((n, f), dtype=torch.bfloat16, device=dev)
-    y = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+    if args.kernel_case != "router":
+        rows = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+        w1 = torch.empty((G, f, d), dtype=torch.bfloat16, device=dev)
+        w2 = torch.empty((G, d, f), dtype=torch.bfloat16, device=dev)
+        mi.gpu_normal_bf16(rows.data_ptr(), rows.numel(), 0, mi.STREAM_TEST_ROWS, 0, 1.0, s)
+        mi.gpu_normal_bf16(w1.data_ptr(), w1.numel(), 0, mi.STREAM_W1, 0, d ** -0.5, s)
+        mi.gpu_normal_bf16(w2.data_ptr(), w2.numel(), 0, mi.STREAM_W2, 0, f ** -0.5, s)
+        offsets = torch.arange(0, n + 1, per, dtype=torch.int32, device=dev)
+        h = torch.empty((n, f), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
 
-    if args.kernel_case == "grouped_ffn":
+    if args.kernel_case == "router":
+        # the router alone on the chosen workload's tokens (diagnostic / profiling case)
+        w = mi.WORKLOADS[args.workload]
+        t = mi.torch_workload(w, with_weights=False)
+        layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k))
+
+        def call():
+            moe.moe_router_topk(t["x"], t["w_r"], t["bias"], t["logit_offset"], w.T, w.d, w.n_routed, w.n_shared,
+                                w.k, 1.0, layer.topk_idx, layer.gates, layer.counts)
+    elif args.kernel_case == "grouped_ffn":
         def call():
             moe.moe_grouped_ffn(rows, offsets, G, n, 0, w1, w2, d, f, moe.MOE_ACT_GELU_TANH, h, y)
     else:
@@ -325,12 +360,19 @@ def run_kernel_case(args):
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
+    h0 = time.perf_counter()
     for _ in range(args.steps):
         call()
+    host_us = (time.perf_counter() - h0) / args.steps * 1e6
     e1.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
+    if args.kernel_case == "router":
+        print(json.dumps({"kernel_case": "router", "workload": args.workload, "us_per_call": round(ms * 1e3, 2),
+                          "host_us_per_call": round(host_us, 2),
+                          "clocks": clk, "status": moe.moe_get_status()}), flush=True)
+        return
     flops = 2 * 2.0 * n * d * f
     print(json.dumps({"kernel_case": args.kernel_case, "experts": G, "rows_per_expert": per, "d": d, "d_ff": f,
                       "ms_per_call": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
@@ -345,7 +387,7 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas"], default=None,
+    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "router"], default=None,
                     help="time one kernel alone on a small profiling case instead of the layer")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -106,7 +106,9 @@ int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, const float* bi
  *              (MOE_STATUS_COUNT_MISMATCH on the device if they differ); the
  *              layout is always derived from topk_idx itself
  *   offsets    [n_routed + 1] int32 out: rows of expert e are offsets[e] .. offsets[e+1]-1
- *   x_perm     [T*top_k, d] bf16 out: row r = x[row_token[r]]
+ *   x_perm     [T*top_k, d] bf16 out: row r = x[row_token[r]]; may be NULL (then x
+ *              may be NULL too): only the index outputs are produced, for
+ *              moe_experts_ffn to gather the rows itself
  *   row_token  [T*top_k] int32 out
  *   token_row  [T, top_k] int32 out: the row each (token, slot) went to
  *   scratch    device buffer of at least moe_permute_scratch_bytes(T, n_routed)
@@ -183,8 +185,13 @@ int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, 
  * nonlinearity).  The same grouped GEMM as moe_grouped_ffn, with the shared
  * experts' tiles scheduled in the same persistent launches as the routed ones.
  *
- *   x          [T, d] bf16 (shared experts' input)
- *   x_perm     [T*top_k, d] bf16, offsets [n_routed + 1] int32 (from moe_permute)
+ *   x          [T, d] bf16 (the shared experts' input, and the routed experts' when
+ *              x_perm is NULL)
+ *   x_perm     [T*top_k, d] bf16 (from moe_permute) or NULL: then the routed rows
+ *              are gathered from x through row_token by the GEMM's own loads
+ *              (TMA tile::gather4), and moe_permute need not copy rows
+ *   row_token  [T*top_k] int32 (from moe_permute); used when x_perm is NULL
+ *   offsets    [n_routed + 1] int32 (from moe_permute)
  *   w1, w2     [n_routed + n_shared, d_ff, d] and [n_routed + n_shared, d, d_ff]
  *              bf16: routed experts first, then the shared experts
  *   h_scratch  [T*top_k + n_shared*T, d_ff] bf16 (caller-owned)
@@ -192,9 +199,10 @@ int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, 
  *   y_shared   [n_shared, T, d] bf16 out
  * Limits: d % 64 == 0, d_ff % 64 == 0, n_routed + n_shared <= MOE_MAX_GROUPS.
  */
-int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* offsets, int T, int n_routed,
-                    int n_shared, int top_k, const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff, int activation,
-                    moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared, void* stream);
+int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* row_token, const int32_t* offsets,
+                    int T, int n_routed, int n_shared, int top_k, const moe_bf16* w1, const moe_bf16* w2, int d,
+                    int d_ff, int activation, moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared,
+                    void* stream);
 
 /*
  * moe_combine -- gate-weighted sum of the contributors, back in token order.

@@ -47,8 +47,8 @@ _lib.moe_permute_scratch_bytes.restype = _sz
 _lib.moe_permute.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_permute_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_grouped_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
-_lib.moe_experts_ffn.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp,
-                                 _vp]
+_lib.moe_experts_ffn.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp,
+                                 _vp, _vp]
 _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_bias_update.argtypes = [_vp, _i32, _i32, _i32, _f32, _vp, _vp]
 _lib.moe_status_string.argtypes = [_i32]
@@ -147,11 +147,11 @@ def moe_grouped_ffn(rows, offsets, n_groups: int, n_rows: int, expert_base: int,
         _p(y), _stream(stream)))
 
 
-def moe_experts_ffn(x, x_perm, offsets, T: int, n_routed: int, n_shared: int, top_k: int, w1, w2, d: int, d_ff: int,
-                    activation: int, h_scratch, y_perm, y_shared, stream=None):
+def moe_experts_ffn(x, x_perm, row_token, offsets, T: int, n_routed: int, n_shared: int, top_k: int, w1, w2, d: int,
+                    d_ff: int, activation: int, h_scratch, y_perm, y_shared, stream=None):
     _check("moe_experts_ffn", _lib.moe_experts_ffn(
-        _p(x), _p(x_perm), _p(offsets), T, n_routed, n_shared, top_k, _p(w1), _p(w2), d, d_ff, activation,
-        _p(h_scratch), _p(y_perm), _p(y_shared), _stream(stream)))
+        _p(x), _p(x_perm), _p(row_token), _p(offsets), T, n_routed, n_shared, top_k, _p(w1), _p(w2), d, d_ff,
+        activation, _p(h_scratch), _p(y_perm), _p(y_shared), _stream(stream)))
 
 
 def moe_combine(y_perm, token_row, gates, y_shared, T: int, d: int, top_k: int, n_shared: int, out, stream=None):
@@ -202,11 +202,15 @@ class MoELayer:
     bias [n_routed] fp32 (updated in place by ``bias_update``).
     """
 
-    def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True):
+    def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True, gather_rows: bool = False):
         import torch
 
         self.shape = s = shape
         self.fused_experts = fused_experts
+        # with the fused experts, GEMM1 can gather the routed rows from x itself (no x_perm copy);
+        # measured slower on B200 at every workload here (32 row gathers per stage bound the TMA
+        # unit), so the default copies the rows in moe_permute and loads tiles
+        self.gather_rows = gather_rows and fused_experts
         dev = torch.device(device)
         R = s.T * s.top_k
         bf = torch.bfloat16
@@ -252,12 +256,13 @@ class MoELayer:
             moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h_shared,
                             self.y_shared, stream=self.side)
             self.ev_shared.record(self.side)
-        moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, self.x_perm, self.row_token,
+        x_perm = None if self.gather_rows else self.x_perm
+        moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, x_perm, self.row_token,
                     self.token_row, self.scratch, self.scratch_bytes, stream=main)
         if ffn_events is not None:
             ffn_events[0].record(main)
         if self.fused_experts:
-            moe_experts_ffn(x, self.x_perm, self.offsets, T, s.n_routed, s.n_shared, k, w1, w2, d, f,
+            moe_experts_ffn(x, x_perm, self.row_token, self.offsets, T, s.n_routed, s.n_shared, k, w1, w2, d, f,
                             MOE_ACT_GELU_TANH, self.h, self.y_perm, self.y_shared, stream=main)
         else:
             moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, MOE_ACT_GELU_TANH,
@@ -274,7 +279,8 @@ class MoELayer:
     def launches_per_step(self) -> int:
         """libmoe kernels one forward + bias update launches."""
         experts = 2 if self.fused_experts else 4
-        return 1 + 3 + experts + 1 + 1
+        permute = 3 if self.gather_rows else 4
+        return 1 + permute + experts + 1 + 1
 
     def bias_update(self, bias, gamma: float, stream=None):
         s = self.shape

@@ -88,8 +88,45 @@ int ensure_smem_attr(const void* kernel, size_t bytes) {
   return MOE_OK;
 }
 
+namespace {
+
+// Encoded descriptors are pure functions of (base, shape, box); repeated calls
+// on the same buffers (every layer step) reuse them instead of re-encoding.
+struct TmapKey {
+  const void* base;
+  int rank;
+  uint64_t dim0, dim1, dim2;
+  uint32_t box0, box1;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rank == o.rank && dim0 == o.dim0 && dim1 == o.dim1 && dim2 == o.dim2 &&
+           box0 == o.box0 && box1 == o.box1;
+  }
+};
+
+constexpr int kTmapCacheSize = 64;
+struct TmapEntry {
+  bool used = false;
+  TmapKey key;
+  CUtensorMap map;
+};
+TmapEntry g_tmap_cache[kTmapCacheSize];
+int g_tmap_next = 0;
+std::mutex g_tmap_mu;
+
+}  // namespace
+
 int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                      uint32_t box0, uint32_t box1) {
+  const TmapKey key{base, rank, dim0, dim1, rank == 3 ? dim2 : 1, box0, box1};
+  {
+    std::lock_guard<std::mutex> lk(g_tmap_mu);
+    for (int i = 0; i < kTmapCacheSize; ++i) {
+      if (g_tmap_cache[i].used && g_tmap_cache[i].key == key) {
+        *map = g_tmap_cache[i].map;
+        return MOE_OK;
+      }
+    }
+  }
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return MOE_ERR_CUDA;
   cuuint64_t dims[3] = {dim0, dim1, dim2};
@@ -100,7 +137,14 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_tmap_mu);
+  TmapEntry& e = g_tmap_cache[g_tmap_next];
+  g_tmap_next = (g_tmap_next + 1) % kTmapCacheSize;
+  e.used = true;
+  e.key = key;
+  e.map = *map;
+  return MOE_OK;
 }
 
 namespace {

@@ -70,6 +70,8 @@ struct Cfg {
 
 struct Params {
   const int* offsets;  // [G_r + 1] routed group row offsets (device); unused when G_r == 0
+  const int* gather_rows;  // non-null: routed A rows are gathered, row r of group g = gather_rows[off[g] + r]
+  int gather_limit;        // gathered row indices are clamped to [0, gather_limit)
   int G_r;             // routed groups
   int G_s;             // shared groups
   int routed_rows;     // offsets are clamped to [0, routed_rows]
@@ -244,47 +246,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = &st->abort_flag;
 
   if (warp == 0) {
-    // ================= TMA producer =================
+    // ================= TMA producer (whole warp; lane 0 issues tiles, every lane a row gather) ===========
     if (lane == 0) {
       tma_prefetch_desc(&tmA0);
       if (p.G_s > 0 && p.a_sh_map == 1) tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB);
-      int stage = 0;
-      uint32_t phase = 0;
-      long issued = 0;
-      bool ok = true;
-      for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
-        const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
-        const Group gr = group_info(p, st->gt, ti.g);
-        const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
-        const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
-        const int b_row = ti.nt * BN + (int)rank * C::B_ROWS;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(&st->full[stage], C::TX_BYTES);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool ok = true;
+    for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
+      const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
+      const Group gr = group_info(p, st->gt, ti.g);
+      const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
+      const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
+      const int b_row = ti.nt * BN + (int)rank * C::B_ROWS;
+      const bool gather = p.gather_rows != nullptr && ti.g < p.G_r;
+      int gr0 = 0, gr1 = 0, gr2 = 0, gr3 = 0;  // this lane's four source rows (rows 4*lane.. of the CTA's A tile)
+      if (gather) {
+        const int r0 = ti.m * C::TILE_M + (int)rank * C::A_ROWS + 4 * lane;  // row within the group
+        auto src = [&](int j) -> int {
+          if (r0 + j >= gr.rows) return 0;  // past the group: any valid row, masked in the epilogue
+          int v = __ldg(p.gather_rows + gr.a_base + r0 + j);
+          return v < 0 ? 0 : (v >= p.gather_limit ? p.gather_limit - 1 : v);
+        };
+        gr0 = src(0);
+        gr1 = src(1);
+        gr2 = src(2);
+        gr3 = src(3);
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (lane == 0) ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (lane == 0 && leader) mbar_arrive_expect_tx(&st->full[stage], C::TX_BYTES);
+        __syncwarp();
+        uint8_t* a_dst = smemA + stage * C::A_BYTES;
+        if (gather) {
+          if (PAIR)
+            tma_gather4_pair(a_dst + lane * 512, am, &st->full[stage], kb * BK, gr0, gr1, gr2, gr3);
+          else
+            tma_gather4(a_dst + lane * 512, am, &st->full[stage], kb * BK, gr0, gr1, gr2, gr3);
+        }
+        if (lane == 0) {
           if (PAIR) {
-            tma_load_2d_pair(smemA + stage * C::A_BYTES, am, &st->full[stage], kb * BK, a_row);
+            if (!gather) tma_load_2d_pair(a_dst, am, &st->full[stage], kb * BK, a_row);
             tma_load_3d_pair(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
           } else {
-            tma_load_2d(smemA + stage * C::A_BYTES, am, &st->full[stage], kb * BK, a_row);
+            if (!gather) tma_load_2d(a_dst, am, &st->full[stage], kb * BK, a_row);
             tma_load_3d(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
           }
-          ++issued;
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      if (!ok && !PAIR) {
-        // wind down: let the copies already issued land before the CTA exits
-        int zero = 0;
-        for (long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
-          mbar_wait(&st->full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), p.timeout_ns, &zero, p.status);
-      }
+    }
+    if (!ok && !PAIR && lane == 0) {
+      // wind down: let the copies already issued land before the CTA exits
+      int zero = 0;
+      for (long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
+        mbar_wait(&st->full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), p.timeout_ns, &zero, p.status);
     }
   } else if (warp == 1) {
     // ================= MMA issuer (the pair's leader) =================
@@ -442,6 +467,7 @@ int launch_one(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& 
 struct GemmSpec {
   const void* a0;
   uint64_t a0_rows;
+  uint32_t a0_box_rows;  // 128 for tiled A loads, 1 for row gathers
   const void* a1;  // may be null (then a0's map is passed twice)
   uint64_t a1_rows;
   const void* b;   // weights of the launch's group 0: [G, N, K]
@@ -466,7 +492,8 @@ int run_gemm(const GemmSpec& g, bool pair, int sms, long long tiles_upper, cudaS
   CUtensorMap a0, a1, b;
   int rc;
   const uint64_t K = (uint64_t)g.p.K, N = (uint64_t)g.p.N;
-  if ((rc = encode_tmap_bf16(&a0, g.a0, 2, K, g.a0_rows, 1, BK, 128)) != MOE_OK) return rc;
+  if ((rc = encode_tmap_bf16(&a0, g.a0, 2, K, g.a0_rows, 1, BK, g.a0_box_rows ? g.a0_box_rows : 128)) != MOE_OK)
+    return rc;
   if (g.a1) {
     if ((rc = encode_tmap_bf16(&a1, g.a1, 2, K, g.a1_rows, 1, BK, 128)) != MOE_OK) return rc;
   } else {
@@ -560,18 +587,20 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   return run_gemm<EPI_NONE>(g2, pair, sms, tiles_upper, s);
 }
 
-extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* offsets, int T,
-                               int n_routed, int n_shared, int top_k, const moe_bf16* w1, const moe_bf16* w2, int d,
-                               int d_ff, int activation, moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared,
-                               void* stream) {
+extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* row_token,
+                               const int32_t* offsets, int T, int n_routed, int n_shared, int top_k,
+                               const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff, int activation,
+                               moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared, void* stream) {
   if (T < 0 || n_routed < 0 || n_shared < 0 || top_k < 1 || d <= 0 || d_ff <= 0) return MOE_ERR_INVALID_ARG;
   if (activation != MOE_ACT_GELU_TANH) return MOE_ERR_INVALID_ARG;
   if (n_routed + n_shared > MOE_MAX_GROUPS) return MOE_ERR_UNSUPPORTED;
   if (d % 64 != 0 || d_ff % 64 != 0) return MOE_ERR_UNSUPPORTED;
   if (!w1 || !w2 || !h_scratch || !aligned16(w1) || !aligned16(w2) || !aligned16(h_scratch))
     return MOE_ERR_INVALID_ARG;
-  if (n_routed > 0 && (!x_perm || !offsets || !y_perm || !aligned16(x_perm) || !aligned4(offsets) ||
-                       !aligned16(y_perm)))
+  const bool gather = (x_perm == nullptr);  // routed rows gathered from x through row_token
+  if (n_routed > 0 && (!offsets || !y_perm || !aligned16(x_perm) || !aligned4(offsets) || !aligned16(y_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (n_routed > 0 && gather && (!x || !row_token || !aligned16(x) || !aligned4(row_token)))
     return MOE_ERR_INVALID_ARG;
   if (n_shared > 0 && (!x || !y_shared || !aligned16(x) || !aligned16(y_shared))) return MOE_ERR_INVALID_ARG;
   const long long R = (long long)T * top_k;
@@ -601,15 +630,20 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
 
-  // GEMM1: routed rows from x_perm (map 0), shared rows from x (map 1); H = [routed rows | shared s rows]
+  // GEMM1: routed rows from x_perm, or gathered from x through row_token (map 0), shared rows from x
+  // (map 1); H = [routed rows | shared s rows]
   GemmSpec g1{};
-  g1.a0 = n_routed > 0 ? (const void*)x_perm : (const void*)x;
-  g1.a0_rows = n_routed > 0 ? (uint64_t)R : (uint64_t)T;
+  const bool routed_gather = n_routed > 0 && gather;
+  g1.a0 = (n_routed > 0 && !gather) ? (const void*)x_perm : (const void*)x;
+  g1.a0_rows = (n_routed > 0 && !gather) ? (uint64_t)R : (uint64_t)T;
+  g1.a0_box_rows = routed_gather ? 1u : 128u;
   g1.a1 = n_shared > 0 ? (const void*)x : nullptr;
   g1.a1_rows = (uint64_t)T;
   g1.b = w1;
   g1.p = p;
-  g1.p.a_sh_map = n_routed > 0 ? 1 : 0;
+  g1.p.gather_rows = routed_gather ? row_token : nullptr;
+  g1.p.gather_limit = T;
+  g1.p.a_sh_map = (n_routed > 0 || n_shared == 0) ? 1 : 0;
   g1.p.a_sh_base = 0;
   g1.p.a_sh_stride = 0;
   g1.p.C0 = g1.p.C1 = reinterpret_cast<__nv_bfloat16*>(h_scratch);

@@ -2,17 +2,18 @@
 // one expert in increasing token order ("Inkling, Dissected" §02: each token
 // goes to exactly its k routed experts; §02d: tokens queue per expert).
 //
-// Three launches, all deterministic (no atomics decide a position):
+// Four launches, all deterministic (no atomics decide a position):
 //   1. chunk_hist   one CTA per 256-token chunk: hist[c][e] = picks of e in chunk c
 //   2. chunk_scan   one CTA: offsets[e] = exclusive scan over experts of the
 //                   per-expert totals; base[c][e] = offsets[e] + picks of e in
 //                   chunks before c; optional check of the caller's counts
-//   3. scatter      one CTA per chunk: each warp takes 32 tokens; a per-warp
+//   3. rank         one CTA per chunk: each warp takes 32 tokens; a per-warp
 //                   bitmask per expert (bit = lane) gives each pick its rank
-//                   among earlier lanes, a prefix over the 8 warps gives the
-//                   rank among earlier warps; then the warp copies x rows to
-//                   their destinations with 16-byte loads/stores, reading each
-//                   x row once and writing it k times.
+//                   among earlier lanes, a prefix over the 8 warps its rank
+//                   among earlier warps -> token_row, row_token
+//   4. copy_rows    grid-wide over (token, 256-vector slice) units: each x
+//                   slice is read once with 16-byte loads and written to the
+//                   token's k rows.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,7 +27,6 @@ namespace perm {
 constexpr int CHUNK = 256;  // tokens per chunk (8 warps x 32)
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
-constexpr int ROW_VEC = 8;  // uint4 per lane per pass of the row copy
 
 __global__ void __launch_bounds__(THREADS) chunk_hist_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
                                                              int n_routed, int32_t* __restrict__ hist,
@@ -90,11 +90,10 @@ __global__ void __launch_bounds__(THREADS) chunk_scan_kernel(const int32_t* __re
   }
 }
 
-__global__ void __launch_bounds__(THREADS) scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
-                                                          const int32_t* __restrict__ base, int T, int d_vec, int k,
-                                                          int n_routed, uint4* __restrict__ x_perm,
-                                                          int32_t* __restrict__ row_token,
-                                                          int32_t* __restrict__ token_row) {
+__global__ void __launch_bounds__(THREADS) rank_kernel(const int32_t* __restrict__ topk_idx,
+                                                       const int32_t* __restrict__ base, int T, int k, int n_routed,
+                                                       int32_t* __restrict__ row_token,
+                                                       int32_t* __restrict__ token_row) {
   __shared__ uint32_t mask[WARPS][MOE_MAX_ROUTED];
   __shared__ int pre[WARPS][MOE_MAX_ROUTED];
   const int c = blockIdx.x;
@@ -127,46 +126,62 @@ __global__ void __launch_bounds__(THREADS) scatter_kernel(const uint4* __restric
   }
   __syncthreads();
   const uint32_t lt = (1u << lane) - 1u;
-  int pos[MOE_MAX_TOP_K];
 #pragma unroll
   for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
-    pos[j] = -1;
     if (ex[j] >= 0) {
-      pos[j] = pre[warp][ex[j]] + __popc(mask[warp][ex[j]] & lt);
-      token_row[(size_t)t * k + j] = pos[j];
-      row_token[pos[j]] = t;
+      const int pos = pre[warp][ex[j]] + __popc(mask[warp][ex[j]] & lt);
+      token_row[(size_t)t * k + j] = pos;
+      row_token[pos] = t;
     } else if (j < k && valid) {
       token_row[(size_t)t * k + j] = -1;
     }
   }
-  // row copies: the warp walks its 32 tokens; each lane moves 16-byte pieces
-  for (int src = 0; src < 32; ++src) {
-    const int ts = c * CHUNK + warp * 32 + src;
-    if (ts >= T) break;
-    int dst[MOE_MAX_TOP_K];
+}
+
+// x_perm[token_row[t][j]] = x[t] for every slot j: unit u = (token, slice of
+// 256 16-byte vectors); each thread reads one vector and writes it k times.
+__global__ void __launch_bounds__(THREADS) copy_rows_kernel(const uint4* __restrict__ x,
+                                                            const int32_t* __restrict__ token_row, int T, int d_vec,
+                                                            int k, int n_rows, uint4* __restrict__ x_perm) {
+  const int n_slices = (d_vec + THREADS - 1) / THREADS;
+  const long long units = (long long)T * n_slices;
+  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+    const int t = (int)(u / n_slices);
+    const int v = (int)(u - (long long)t * n_slices) * THREADS + threadIdx.x;
+    if (v >= d_vec) continue;
+    const uint4 val = __ldg(x + (size_t)t * d_vec + v);
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_TOP_K; ++j) dst[j] = __shfl_sync(0xffffffffu, pos[j], src);
-    const uint4* xs = x + (size_t)ts * d_vec;
-    for (int v0 = 0; v0 < d_vec; v0 += 32 * ROW_VEC) {
-      uint4 buf[ROW_VEC];
-#pragma unroll
-      for (int q = 0; q < ROW_VEC; ++q) {
-        int vi = v0 + q * 32 + lane;
-        if (vi < d_vec) buf[q] = __ldg(xs + vi);
-      }
-#pragma unroll
-      for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
-        if (j < k && dst[j] >= 0) {
-          uint4* xd = x_perm + (size_t)dst[j] * d_vec;
-#pragma unroll
-          for (int q = 0; q < ROW_VEC; ++q) {
-            int vi = v0 + q * 32 + lane;
-            if (vi < d_vec) xd[vi] = buf[q];
-          }
-        }
+    for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+      if (j < k) {
+        const int r = __ldg(token_row + (size_t)t * k + j);
+        if (r >= 0 && r < n_rows) x_perm[(size_t)r * d_vec + v] = val;
       }
     }
   }
+}
+
+// The launches shared by moe_permute and moe_permute_noalloc.
+static int launch_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                          int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
+                          int32_t* token_row, void* scratch, cudaStream_t s) {
+  unsigned int* status = status_ptr();
+  if (!status) return MOE_ERR_CUDA;
+  int dev, sms;
+  int rc = device_info(&dev, &sms);
+  if (rc != MOE_OK) return rc;
+  const int n_chunks = (T + CHUNK - 1) / CHUNK;
+  int32_t* hist = reinterpret_cast<int32_t*>(scratch);
+  int32_t* base = hist + (size_t)n_chunks * n_routed;
+  chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
+  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, counts, offsets, base, status);
+  rank_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, base, T, top_k, n_routed, row_token, token_row);
+  if (x_perm == nullptr) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;  // indices only
+  const int d_vec = d / 8;
+  const long long units = (long long)T * ((d_vec + THREADS - 1) / THREADS);
+  const int grid = (int)(units < (long long)sms * 8 ? units : (long long)sms * 8);
+  copy_rows_kernel<<<grid, THREADS, 0, s>>>(reinterpret_cast<const uint4*>(x), token_row, T, d_vec, top_k,
+                                            T * top_k, reinterpret_cast<uint4*>(x_perm));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace perm
@@ -187,7 +202,7 @@ extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int
   if (T < 0 || d <= 0 || n_routed < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
   if (top_k > MOE_MAX_TOP_K || top_k > n_routed || n_routed > MOE_MAX_ROUTED) return MOE_ERR_INVALID_ARG;
   if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
-  if (!x || !topk_idx || !offsets || !x_perm || !row_token || !token_row || !scratch) return MOE_ERR_INVALID_ARG;
+  if (!topk_idx || !offsets || !row_token || !token_row || !scratch || (x_perm && !x)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm) || !aligned4(topk_idx) || !aligned4(counts) || !aligned4(offsets) ||
       !aligned4(row_token) || !aligned4(token_row) || !aligned16(scratch))
     return MOE_ERR_INVALID_ARG;
@@ -198,16 +213,8 @@ extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int
     if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (n_routed + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  unsigned int* status = status_ptr();
-  if (!status) return MOE_ERR_CUDA;
-  const int n_chunks = (T + CHUNK - 1) / CHUNK;
-  int32_t* hist = reinterpret_cast<int32_t*>(scratch);
-  int32_t* base = hist + (size_t)n_chunks * n_routed;
-  chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
-  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, counts, offsets, base, status);
-  scatter_kernel<<<n_chunks, THREADS, 0, s>>>(reinterpret_cast<const uint4*>(x), topk_idx, base, T, d / 8, top_k,
-                                               n_routed, reinterpret_cast<uint4*>(x_perm), row_token, token_row);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_permute(x, topk_idx, counts, T, d, n_routed, top_k, offsets, x_perm, row_token, token_row, scratch,
+                        s);
 }
 
 // ---------------------------------------------------------------------------
@@ -252,7 +259,7 @@ extern "C" int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, c
   if (T < 0 || d <= 0 || n_routed < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
   if (top_k > MOE_MAX_TOP_K || top_k > n_routed || n_routed > MOE_MAX_ROUTED) return MOE_ERR_INVALID_ARG;
   if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
-  if (!x || !topk_idx || !offsets || !x_perm || !row_token || !token_row) return MOE_ERR_INVALID_ARG;
+  if (!topk_idx || !offsets || !row_token || !token_row || (x_perm && !x)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm) || !aligned4(topk_idx) || !aligned4(counts) || !aligned4(offsets) ||
       !aligned4(row_token) || !aligned4(token_row))
     return MOE_ERR_INVALID_ARG;
@@ -266,16 +273,8 @@ extern "C" int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, c
     if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (n_routed + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  unsigned int* status = status_ptr();
-  if (!status) return MOE_ERR_CUDA;
   // Every part of the scratch that is read is written first in the same call
   // (hist by chunk_hist, base by chunk_scan), so nothing needs clearing.
-  const int n_chunks = (T + CHUNK - 1) / CHUNK;
-  int32_t* hist = reinterpret_cast<int32_t*>(scratch);
-  int32_t* base = hist + (size_t)n_chunks * n_routed;
-  chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
-  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, counts, offsets, base, status);
-  scatter_kernel<<<n_chunks, THREADS, 0, s>>>(reinterpret_cast<const uint4*>(x), topk_idx, base, T, d / 8, top_k,
-                                               n_routed, reinterpret_cast<uint4*>(x_perm), row_token, token_row);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_permute(x, topk_idx, counts, T, d, n_routed, top_k, offsets, x_perm, row_token, token_row, scratch,
+                        s);
 }

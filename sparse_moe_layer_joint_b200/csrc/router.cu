@@ -3,16 +3,23 @@
 // s_i + b_i; g_i = s_i / sum over kept U shared; "Under the hood", "The
 // routing strategy": 256 routed + 2 shared scores, top-k over routed only).
 //
-// One CTA per 128 tokens.  The logits of all n_routed + n_shared experts for
-// the CTA's tokens are one 128 x 272 fp32 accumulator in TMEM: a tcgen05 MMA
-// with N = 256 (experts 0..255) and one with N = 16 (experts 256..271, zero
-// rows past the last expert) per 16-deep K step, fed by TMA through a 4-stage
-// ring.  In the epilogue each of the 128 epilogue threads owns one token (its
-// TMEM lane): it reads its 258 logits 32 at a time, applies the sigmoid, adds
-// the bias for selection, keeps a register top-k list (strict '>' while
-// scanning experts in index order, so ties keep the lower index), then forms
-// the joint gates and counts its picks in a shared-memory histogram that is
-// added to the global counts once per CTA.
+// The logits of all n_routed + n_shared experts for 128 tokens are one
+// 128 x 272 fp32 accumulator in TMEM: a tcgen05 MMA with N = 256 (experts
+// 0..255) and one with N = 16 (experts 256..271, zero rows past the last
+// expert) per 16-deep K step, fed by TMA through a 4-stage ring.
+//
+// Split-K across a cluster.  When there are few 128-token tiles (decode, mid
+// sizes) a cluster of S CTAs (S = 2, 4 or 8) shares one tile: CTA c runs the
+// MMAs of the c-th slice of K, then writes its partial 128 x 272 tile into its
+// shared memory; after a cluster barrier, CTA c owns rows c*128/S .. of the
+// tile and sums their S partials in cluster-rank order through distributed
+// shared memory (a fixed order, so the result does not depend on timing).
+//
+// Routing epilogue, one token per thread: sigmoid, + b for selection, a
+// register top-k list (strict '>' while scanning experts in index order, so
+// ties keep the lower index), the joint gates (denominator summed over the
+// contributors in ascending expert index) and a shared-memory histogram of
+// the picks, added to the global counts once per CTA.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -37,11 +44,14 @@ constexpr int B1_BYTES = B1_ROWS * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B0_BYTES + B1_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int RED_COLS = B0_ROWS + B1_ROWS;  // 272 columns of a partial tile row
+constexpr int MAX_SPLIT = 8;
 
 struct Params {
   const float* bias;
   const float* offset;  // nullable
   int T, d, n_routed, n_shared;
+  int ksplit;           // CTAs (cluster size) sharing one 128-token tile: 1, 2, 4 or 8
   int32_t* topk_idx;
   float* gates;
   int32_t* counts;
@@ -63,9 +73,102 @@ struct SmemTail {
   float shared_s[BM][MOE_MAX_SHARED];
 };
 
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+// The stage ring, idle once the MMAs are done, also holds the split-K partial
+// tile [128][272] fp32 and the reduced rows [128/S][272] fp32 (S >= 2).
+constexpr size_t SPLIT_BYTES = (size_t)BM * RED_COLS * 4 + (size_t)(BM / 2) * RED_COLS * 4;
+constexpr size_t RING_BYTES =
+    (size_t)STAGES * STAGE_BYTES > SPLIT_BYTES ? (size_t)STAGES * STAGE_BYTES : SPLIT_BYTES;
+
+constexpr size_t SMEM_BYTES = 1024 + RING_BYTES + sizeof(SmemTail);
+static_assert(SMEM_BYTES <= 227 * 1024, "router shared memory");
 
 __device__ __forceinline__ float sigmoid_f32(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// One token's routing state: the running top-k of (s + b) over routed experts.
+template <int K>
+struct TopK {
+  float val[K], sc[K];
+  int id[K];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      val[q] = -INFINITY;
+      sc[q] = 0.0f;
+      id[q] = 0x7fffffff;
+    }
+  }
+  __device__ __forceinline__ void push(int i, float s, float sel) {
+    if (sel > val[K - 1]) {
+      val[K - 1] = sel;
+      sc[K - 1] = s;
+      id[K - 1] = i;
+#pragma unroll
+      for (int q = K - 1; q > 0; --q) {
+        if (val[q] > val[q - 1]) {
+          float tv = val[q]; val[q] = val[q - 1]; val[q - 1] = tv;
+          float ts = sc[q]; sc[q] = sc[q - 1]; sc[q - 1] = ts;
+          int ti = id[q]; id[q] = id[q - 1]; id[q - 1] = ti;
+        }
+      }
+    }
+  }
+};
+
+// Score expert i of a token from its logit z: routed experts enter the top-k,
+// shared experts only keep their affinity for the joint normalisation.
+template <int K>
+__device__ __forceinline__ void consume(const Params& p, SmemTail* st, TopK<K>& tk, int row, float* srow, int i,
+                                        float z) {
+  if (i < p.n_routed) {
+    float s = sigmoid_f32(z + st->off[i]);
+    if (srow) srow[i] = s;
+    tk.push(i, s, s + st->bias[i]);
+  } else if (i < p.n_routed + p.n_shared) {
+    float s = sigmoid_f32(z);
+    if (srow) srow[i] = s;
+    st->shared_s[row][i - p.n_routed] = s;
+  }
+}
+
+// Joint gates and outputs for one token.
+template <int K>
+__device__ __forceinline__ void finish(const Params& p, SmemTail* st, TopK<K>& tk, int row, int t) {
+  // the denominator is a sum over the contributor set, in ascending expert index
+  float den = 0.0f;
+  int prev = -1;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    int best = 0x7fffffff;
+    float bs = 0.0f;
+#pragma unroll
+    for (int r = 0; r < K; ++r)
+      if (tk.id[r] > prev && tk.id[r] < best) {
+        best = tk.id[r];
+        bs = tk.sc[r];
+      }
+    den += bs;
+    prev = best;
+  }
+  for (int q = 0; q < p.n_shared; ++q) den += st->shared_s[row][q];
+  const int G = K + p.n_shared;
+  int32_t* ti = p.topk_idx + (size_t)t * K;
+  float* gt = p.gates + (size_t)t * G;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    ti[q] = tk.id[q];
+    gt[q] = __fdiv_rn(tk.sc[q], den);
+    if (tk.id[q] < p.n_routed) atomicAdd(&st->hist[tk.id[q]], 1);  // unset only for non-finite scores
+  }
+  for (int q = 0; q < p.n_shared; ++q) gt[K + q] = __fdiv_rn(st->shared_s[row][q], den);
+}
 
 template <int K>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -73,17 +176,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmB1, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SmemTail* st = reinterpret_cast<SmemTail*>(smem + STAGES * STAGE_BYTES);
+  SmemTail* st = reinterpret_cast<SmemTail*>(smem + RING_BYTES);
   auto stageA = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stageB0 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
   auto stageB1 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B0_BYTES; };
+  float* red = reinterpret_cast<float*>(smem);   // [BM][RED_COLS] split-K partial
+  float* zsum = red + (size_t)BM * RED_COLS;      // [BM/S][RED_COLS] reduced rows
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int E = p.n_routed + p.n_shared;
   const bool two = E > B0_ROWS;
-  const int m0 = blockIdx.x * BM;
+  const int S = p.ksplit;
+  const uint32_t crank = S > 1 ? cluster_ctarank() : 0u;
+  const int m0 = (blockIdx.x / S) * BM;
+  const int kb_per = (p.d / BK) / S;
+  const int kb0 = (int)crank * kb_per;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -105,7 +214,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = st->tmem_base;
-  const int num_kb = p.d / BK;
   volatile int* abort_flag = &st->abort_flag;
 
   if (warp == 0) {
@@ -118,7 +226,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = kb0; kb < kb0 + kb_per; ++kb) {
         if (!mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status)) {
           ok = false;
           break;
@@ -146,7 +254,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = 0; kb < kb_per; ++kb) {
         if (!mbar_wait(&st->full[stage], phase, p.timeout_ns, abort_flag, p.status)) {
           ok = false;
           break;
@@ -175,95 +283,111 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
     }
   } else {
-    // ================= epilogue: one token per thread =================
+    // ================= epilogue warps =================
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const int t = m0 + row;
-    const bool valid = t < p.T;
+    const int row = quarter * 32 + lane;  // this thread's TMEM lane
     const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const int lim = E < B0_ROWS ? E : B0_ROWS;
     if (mbar_wait(&st->tfull, 0, p.timeout_ns, abort_flag, p.status)) {
       tc_fence_after();
-      float val[K], sc[K];
-      int id[K];
-#pragma unroll
-      for (int q = 0; q < K; ++q) {
-        val[q] = -INFINITY;
-        sc[q] = 0.0f;
-        id[q] = 0x7fffffff;
-      }
-      float* srow = (p.scores != nullptr && valid) ? p.scores + (size_t)t * E : nullptr;
-      auto consume = [&](int i, float z) {
-        if (i < p.n_routed) {
-          float s = sigmoid_f32(z + st->off[i]);
-          float sel = s + st->bias[i];
-          if (srow) srow[i] = s;
-          if (sel > val[K - 1]) {
-            val[K - 1] = sel;
-            sc[K - 1] = s;
-            id[K - 1] = i;
-#pragma unroll
-            for (int q = K - 1; q > 0; --q) {
-              if (val[q] > val[q - 1]) {
-                float tv = val[q]; val[q] = val[q - 1]; val[q - 1] = tv;
-                float ts = sc[q]; sc[q] = sc[q - 1]; sc[q - 1] = ts;
-                int ti = id[q]; id[q] = id[q - 1]; id[q - 1] = ti;
-              }
-            }
-          }
-        } else if (i < E) {
-          float s = sigmoid_f32(z);
-          if (srow) srow[i] = s;
-          st->shared_s[row][i - p.n_routed] = s;
-        }
-      };
-      const int lim = E < B0_ROWS ? E : B0_ROWS;
+      if (S == 1) {
+        // one token per thread, straight from TMEM
+        const int t = m0 + row;
+        const bool valid = t < p.T;
+        TopK<K> tk;
+        tk.init();
+        float* srow = (p.scores != nullptr && valid) ? p.scores + (size_t)t * E : nullptr;
 #pragma unroll 1
-      for (int c0 = 0; c0 < lim; c0 += 32) {
-        float v[32];
-        tmem_ld32(taddr + c0, v);
+        for (int c0 = 0; c0 < lim; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c0 + j < lim) consume(c0 + j, v[j]);
-      }
-      if (two) {
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < lim) consume<K>(p, st, tk, row, srow, c0 + j, v[j]);
+        }
+        if (two) {
+          float v[16];
+          tmem_ld16(taddr + B0_ROWS, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (B0_ROWS + j < E) consume<K>(p, st, tk, row, srow, B0_ROWS + j, v[j]);
+        }
+        if (valid) finish<K>(p, st, tk, row, t);
+      } else {
+        // split-K: park this CTA's partial tile row in shared memory (the stage ring is idle now)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        float* dst = red + (size_t)row * RED_COLS;
+#pragma unroll 1
+        for (int c0 = 0; c0 < B0_ROWS; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
         float v[16];
-        tmem_ld16(taddr + B0_ROWS, v);
+        if (two) {
+          tmem_ld16(taddr + B0_ROWS, v);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (B0_ROWS + j < E) consume(B0_ROWS + j, v[j]);
-      }
-      if (valid) {
-        // joint denominator: a sum over the contributor set, in ascending index
-        float den = 0.0f;
-        int prev = -1;
-#pragma unroll
-        for (int q = 0; q < K; ++q) {
-          int best = 0x7fffffff;
-          float bs = 0.0f;
-#pragma unroll
-          for (int r = 0; r < K; ++r)
-            if (id[r] > prev && id[r] < best) {
-              best = id[r];
-              bs = sc[r];
-            }
-          den += bs;
-          prev = best;
+          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
         }
-        for (int q = 0; q < p.n_shared; ++q) den += st->shared_s[row][q];
-        const int G = K + p.n_shared;
-        int32_t* ti = p.topk_idx + (size_t)t * K;
-        float* gt = p.gates + (size_t)t * G;
 #pragma unroll
-        for (int q = 0; q < K; ++q) {
-          ti[q] = id[q];
-          gt[q] = __fdiv_rn(sc[q], den);
-          if (id[q] < p.n_routed) atomicAdd(&st->hist[id[q]], 1);  // unset only for non-finite scores
-        }
-        for (int q = 0; q < p.n_shared; ++q) gt[K + q] = __fdiv_rn(st->shared_s[row][q], den);
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(dst + B0_ROWS + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
     }
+  }
+
+  if (S > 1) {
+    tc_fence_before();
+    cluster_sync_all();  // every CTA's partial tile is in its shared memory
+    if (warp >= 2) {
+      const int e = tid - 64;          // 0..127
+      const int rows_per = BM / S;     // rows this CTA finishes
+      const int r_local = e / S;       // S threads per row
+      const int part = e - r_local * S;
+      const int row = (int)crank * rows_per + r_local;
+      // 1. sum the S partials of this CTA's rows (float4 columns part, part + S, ...), in rank order
+      const uint32_t red_local = smem_u32(red + (size_t)row * RED_COLS);
+      for (int f = part; f < RED_COLS / 4; f += S) {
+        float4 q[MAX_SPLIT];
+#pragma unroll
+        for (int c = 0; c < MAX_SPLIT; ++c)  // all remote loads in flight at once
+          if (c < S) q[c] = ld_dsmem_f4(mapa_shared(red_local + f * 16, (uint32_t)c));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < MAX_SPLIT; ++c) {
+          if (c < S) {
+            acc.x += q[c].x;
+            acc.y += q[c].y;
+            acc.z += q[c].z;
+            acc.w += q[c].w;
+          }
+        }
+        *reinterpret_cast<float4*>(zsum + (size_t)r_local * RED_COLS + 4 * f) = acc;
+      }
+      named_bar_sync(1, 128);
+      // 2. route the rows: one thread per token
+      if (e < rows_per) {
+        const int rr = (int)crank * rows_per + e;
+        const int t = m0 + rr;
+        if (t < p.T) {
+          TopK<K> tk;
+          tk.init();
+          float* srow = p.scores != nullptr ? p.scores + (size_t)t * E : nullptr;
+          const float* z = zsum + (size_t)e * RED_COLS;
+          for (int i = 0; i < E; ++i) consume<K>(p, st, tk, rr, srow, i, z[i]);
+          finish<K>(p, st, tk, rr, t);
+        }
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while another may still read its partial
+  }
+
+  if (warp >= 2) {
     named_bar_sync(1, 128);
-    for (int e = row; e < p.n_routed; e += 128) {
+    for (int e = tid - 64; e < p.n_routed; e += 128) {
       int c = st->hist[e];
       if (c) atomicAdd(&p.counts[e], c);
     }
@@ -283,8 +407,30 @@ int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, c
   auto kfn = router_kernel<K>;
   int rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES);
   if (rc != MOE_OK) return rc;
-  kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kfn, a, b0, b1, p) != cudaSuccess) return MOE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Cluster size sharing one tile: the largest S in {1, 2, 4, 8} that keeps all
+// CTAs resident at once (one per SM), divides the K blocks, and leaves each CTA
+// at least two of them.
+int choose_ksplit(int n_mtiles, int num_kb, int sms) {
+  int S = 1;
+  while (S < MAX_SPLIT && (long long)n_mtiles * S * 2 <= sms && num_kb % (S * 2) == 0 && num_kb / (S * 2) >= 2)
+    S *= 2;
+  return S;
 }
 
 }  // namespace router
@@ -310,14 +456,17 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * n_routed, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (T == 0) return MOE_OK;
+  int dev, sms;
+  int rc = device_info(&dev, &sms);
+  if (rc != MOE_OK) return rc;
 
   const int E = n_routed + n_shared;
   CUtensorMap tA, tB0, tB1;
-  int rc;
   if ((rc = encode_tmap_bf16(&tA, x, 2, (uint64_t)d, (uint64_t)T, 1, BK, BM)) != MOE_OK) return rc;
   if ((rc = encode_tmap_bf16(&tB0, w_router, 2, (uint64_t)d, (uint64_t)E, 1, BK, B0_ROWS)) != MOE_OK) return rc;
   if ((rc = encode_tmap_bf16(&tB1, w_router, 2, (uint64_t)d, (uint64_t)E, 1, BK, B1_ROWS)) != MOE_OK) return rc;
 
+  const int n_mtiles = (T + BM - 1) / BM;
   Params p{};
   p.bias = bias;
   p.offset = logit_offset;
@@ -325,6 +474,7 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   p.d = d;
   p.n_routed = n_routed;
   p.n_shared = n_shared;
+  p.ksplit = choose_ksplit(n_mtiles, d / BK, sms);
   p.topk_idx = topk_idx;
   p.gates = gates;
   p.counts = counts;
@@ -332,7 +482,7 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   p.timeout_ns = wait_timeout_ns();
   p.status = status_ptr();
   if (!p.status) return MOE_ERR_CUDA;
-  const int grid = (T + BM - 1) / BM;
+  const int grid = n_mtiles * p.ksplit;
   switch (top_k) {
     case 1: return launch<1>(tA, tB0, tB1, p, grid, s);
     case 2: return launch<2>(tA, tB0, tB1, p, grid, s);

@@ -75,6 +75,7 @@ def test_permute_rejects():
 
     assert call(x=NULL) == moe.MOE_ERR_INVALID_ARG
     assert call(xp=MIS) == moe.MOE_ERR_INVALID_ARG
+    assert call(tr=NULL) == moe.MOE_ERR_INVALID_ARG
     assert call(k=9) == moe.MOE_ERR_INVALID_ARG
     assert call(d=12) == moe.MOE_ERR_UNSUPPORTED
     assert call(sb=16) == moe.MOE_ERR_SCRATCH
@@ -98,11 +99,12 @@ def test_grouped_ffn_rejects_and_empty_is_noop():
 
 
 def test_experts_ffn_rejects():
-    def call(x=A16, xp=A16, off=A16, T=64, nr=256, ns=2, k=6, w1=A16, w2=A16, d=64, f=64, act=0, h=A16, yp=A16,
-             ys=A16):
-        return L.moe_experts_ffn(x, xp, off, T, nr, ns, k, w1, w2, d, f, act, h, yp, ys, NULL)
+    def call(x=A16, xp=A16, rt=A16, off=A16, T=64, nr=256, ns=2, k=6, w1=A16, w2=A16, d=64, f=64, act=0, h=A16,
+             yp=A16, ys=A16):
+        return L.moe_experts_ffn(x, xp, rt, off, T, nr, ns, k, w1, w2, d, f, act, h, yp, ys, NULL)
 
-    assert call(xp=NULL) == moe.MOE_ERR_INVALID_ARG
+    assert call(xp=NULL, rt=NULL) == moe.MOE_ERR_INVALID_ARG   # gathering needs row_token
+    assert call(xp=0x10008) == moe.MOE_ERR_INVALID_ARG
     assert call(ys=NULL) == moe.MOE_ERR_INVALID_ARG
     assert call(off=0x10002) == moe.MOE_ERR_INVALID_ARG
     assert call(d=96) == moe.MOE_ERR_UNSUPPORTED

@@ -17,9 +17,10 @@ if torch.cuda.is_available():
     import sparse_moe_layer_joint_b200 as moe
 
 
-def _layer(w, with_weights=True, fused=True):
+def _layer(w, with_weights=True, fused=True, gather=False):
     t = mi.torch_workload(w, with_weights=with_weights)
-    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), fused_experts=fused)
+    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), fused_experts=fused,
+                         gather_rows=gather)
     return t, layer
 
 
@@ -38,14 +39,15 @@ def _check_dispatch_properties(layer, x_bits, T, k, n_routed):
     for e in range(n_routed):
         r = rt[off[e]:off[e + 1]]
         assert (np.diff(r) > 0).all()
-    sample = np.linspace(0, T * k - 1, min(T * k, 512)).astype(np.int64)
-    xp = host_bf16_bits(layer.x_perm[torch.from_numpy(sample).cuda()])
-    np.testing.assert_array_equal(xp, x_bits[rt[sample]])
+    if not layer.gather_rows:  # the rows were copied (otherwise the GEMM gathers them itself)
+        sample = np.linspace(0, T * k - 1, min(T * k, 512)).astype(np.int64)
+        xp = host_bf16_bits(layer.x_perm[torch.from_numpy(sample).cuda()])
+        np.testing.assert_array_equal(xp, x_bits[rt[sample]])
 
 
-def _run_and_check(name, tokens=None, check_all_routing=True, fused=True):
+def _run_and_check(name, tokens=None, check_all_routing=True, fused=True, gather=False):
     w = mi.WORKLOADS[name]
-    t, layer = _layer(w, fused=fused)
+    t, layer = _layer(w, fused=fused, gather=gather)
     bias0 = t["bias"].clone()
     out = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
     layer.bias_update(t["bias"], w.gamma)
@@ -83,6 +85,16 @@ def test_layer_tiny_all_tokens():
 def test_layer_tiny_two_streams():
     """The shared experts on a second stream (two moe_grouped_ffn calls) instead of the fused launch."""
     _run_and_check("tiny", fused=False)
+
+
+def test_layer_tiny_gathered_rows():
+    """Fused experts gathering the routed rows from x (TMA row gathers) instead of reading copied rows."""
+    _run_and_check("tiny", gather=True)
+
+
+@pytest.mark.slow
+def test_layer_mid_gathered_rows():
+    _run_and_check("mid", tokens=np.arange(0, 4096, 97), gather=True)
 
 
 @pytest.mark.slow
@@ -137,7 +149,7 @@ def test_layer_skew_sampled_and_bias_trajectory():
 
 def test_layer_is_deterministic_and_writes_every_row():
     w = mi.WORKLOADS["tiny"]
-    t, layer = _layer(w)
+    t, layer = _layer(w, gather=False)
     layer.out.fill_(float("nan"))
     layer.x_perm.fill_(float("nan"))
     o1 = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"]).clone()

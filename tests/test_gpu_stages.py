@@ -152,6 +152,23 @@ def test_permute_parity(T, k, n_routed, d):
     np.testing.assert_array_equal(host_bf16_bits(xp), x[ref["row_token"]])
 
 
+def test_permute_indices_only():
+    """x_perm = NULL: the same offsets / row_token / token_row, no row copy."""
+    T, k, n = 1000, 6, 256
+    topk = _random_topk(T, k, n, 21)
+    ref = oracle.dispatch(topk, n)
+    off = torch.full((n + 1,), -5, dtype=torch.int32, device="cuda")
+    rt = torch.full((T * k,), -5, dtype=torch.int32, device="cuda")
+    tr = torch.full((T, k), -5, dtype=torch.int32, device="cuda")
+    nb = moe.moe_permute_scratch_bytes(T, n)
+    scratch = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    moe.moe_permute(None, _i32(topk), None, T, 64, n, k, off, None, rt, tr, scratch, nb)
+    assert moe.moe_get_status() == 0
+    np.testing.assert_array_equal(off.cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(rt.cpu().numpy(), ref["row_token"])
+    np.testing.assert_array_equal(tr.cpu().numpy(), ref["token_row"])
+
+
 def test_permute_reports_bad_inputs():
     T, k, n = 300, 2, 16
     topk = _random_topk(T, k, n, 5)
@@ -257,8 +274,10 @@ def test_grouped_ffn_special_weights(gemm_variant):
     (300, 16, 2, 3, 256, 128), (1000, 8, 2, 2, 512, 256), (64, 64, 2, 6, 256, 256), (700, 4, 0, 2, 128, 128),
     (129, 0, 2, 1, 128, 192),
 ])
-def test_experts_ffn_parity(T, n_routed, n_shared, k, d, f, gemm_variant):
-    """Routed experts on dispatched rows and shared experts on all tokens, one pair of launches."""
+@pytest.mark.parametrize("gather", [False, True])
+def test_experts_ffn_parity(T, n_routed, n_shared, k, d, f, gemm_variant, gather):
+    """Routed experts on dispatched rows (copied by moe_permute, or gathered by the GEMM
+    itself through row_token) and shared experts on all tokens, one pair of launches."""
     E = n_routed + n_shared
     x = mi.normal_bf16(T * d, 11, mi.STREAM_X).reshape(T, d)
     w1, w2 = _ffn_weights(E, d, f, 11)
@@ -270,10 +289,11 @@ def test_experts_ffn_parity(T, n_routed, n_shared, k, d, f, gemm_variant):
         topk = _random_topk(T, k, n_routed, 12)
         dp = oracle.dispatch(topk, n_routed)
         xp = x[dp["row_token"]]
-        moe.moe_experts_ffn(dev_bf16(x), dev_bf16(xp), _i32(dp["offsets"]), T, n_routed, n_shared, k, dev_bf16(w1),
-                            dev_bf16(w2), d, f, moe.MOE_ACT_GELU_TANH, h, y_perm, y_sh)
+        moe.moe_experts_ffn(dev_bf16(x), None if gather else dev_bf16(xp), _i32(dp["row_token"]),
+                            _i32(dp["offsets"]), T, n_routed, n_shared, k, dev_bf16(w1), dev_bf16(w2), d, f,
+                            moe.MOE_ACT_GELU_TANH, h, y_perm, y_sh)
     else:
-        moe.moe_experts_ffn(dev_bf16(x), None, None, T, 0, n_shared, k, dev_bf16(w1), dev_bf16(w2), d, f,
+        moe.moe_experts_ffn(dev_bf16(x), None, None, None, T, 0, n_shared, k, dev_bf16(w1), dev_bf16(w2), d, f,
                             moe.MOE_ACT_GELU_TANH, h, y_perm, y_sh)
     assert moe.moe_get_status() == 0
     if n_routed:
