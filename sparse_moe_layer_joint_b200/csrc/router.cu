@@ -15,11 +15,12 @@
 // tile and sums their S partials in cluster-rank order through distributed
 // shared memory (a fixed order, so the result does not depend on timing).
 //
-// Routing epilogue, one token per thread: sigmoid, + b for selection, a
-// register top-k list (strict '>' while scanning experts in index order, so
-// ties keep the lower index), the joint gates (denominator summed over the
-// contributors in ascending expert index) and a shared-memory histogram of
-// the picks, added to the global counts once per CTA.
+// Routing epilogue: the logit tile is parked in shared memory (the stage ring
+// is idle by then) and each epilogue warp routes one token at a time: sigmoid,
+// + b for selection, k rounds of a warp-wide argmax (ties keep the lower
+// index), the joint gates (denominator summed over the contributors in
+// ascending expert index) and a shared-memory histogram of the picks, added to
+// the global counts once per CTA.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -92,82 +93,106 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
-// One token's routing state: the running top-k of (s + b) over routed experts.
+// Route one token with one warp.  z: the token's logits in shared memory
+// (RED_COLS floats).  Lane l scores routed experts 8l .. 8l+7; then k rounds of
+// a warp-wide argmax of s + b (a strict '>' scan within a lane, and the lower
+// index on equal values across lanes, so ties keep the lower index) pick the
+// experts in descending order.  Lane 0 forms the joint gates (denominator summed
+// over the contributors in ascending expert index) and writes the outputs.
 template <int K>
-struct TopK {
-  float val[K], sc[K];
+__device__ __forceinline__ void route_token_warp(const Params& p, SmemTail* st, const float* z, int t, int lane) {
+  const int E = p.n_routed + p.n_shared;
+  float s[8], sel[8];
+  const float4* z4 = reinterpret_cast<const float4*>(z + 8 * lane);
+  const float4 za = z4[0], zb = z4[1];
+  const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+  float* srow = p.scores != nullptr ? p.scores + (size_t)t * E : nullptr;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int i = 8 * lane + j;
+    if (i < p.n_routed) {
+      s[j] = sigmoid_f32(zz[j] + st->off[i]);
+      sel[j] = s[j] + st->bias[i];
+      if (srow) srow[i] = s[j];
+    } else {
+      s[j] = 0.0f;
+      sel[j] = -INFINITY;
+    }
+  }
+  // shared experts' affinities (lanes 0 .. n_shared-1)
+  float sh = 0.0f;
+  if (lane < p.n_shared) {
+    sh = sigmoid_f32(z[p.n_routed + lane]);
+    if (srow) srow[p.n_routed + lane] = sh;
+  }
   int id[K];
-  __device__ __forceinline__ void init() {
+  float sc[K];
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (sel[j] > bv) {
+        bv = sel[j];
+        bi = 8 * lane + j;
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    float sw = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (8 * lane + j == bi) {
+        sw = s[j];
+        sel[j] = -INFINITY;
+      }
+    const int owner = (bi >= 0 && bi < 256) ? (bi >> 3) : 0;
+    sc[q] = __shfl_sync(0xffffffffu, sw, owner);
+    id[q] = bi;
+  }
+  float shv[MOE_MAX_SHARED];
+#pragma unroll
+  for (int q = 0; q < MOE_MAX_SHARED; ++q) shv[q] = __shfl_sync(0xffffffffu, sh, q);
+  if (lane == 0) {
+    // the denominator is a sum over the contributor set, in ascending expert index
+    float den = 0.0f;
+    int prev = -1;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      val[q] = -INFINITY;
-      sc[q] = 0.0f;
-      id[q] = 0x7fffffff;
-    }
-  }
-  __device__ __forceinline__ void push(int i, float s, float sel) {
-    if (sel > val[K - 1]) {
-      val[K - 1] = sel;
-      sc[K - 1] = s;
-      id[K - 1] = i;
+      int best = 0x7fffffff;
+      float bs = 0.0f;
 #pragma unroll
-      for (int q = K - 1; q > 0; --q) {
-        if (val[q] > val[q - 1]) {
-          float tv = val[q]; val[q] = val[q - 1]; val[q - 1] = tv;
-          float ts = sc[q]; sc[q] = sc[q - 1]; sc[q - 1] = ts;
-          int ti = id[q]; id[q] = id[q - 1]; id[q - 1] = ti;
+      for (int r = 0; r < K; ++r)
+        if (id[r] > prev && id[r] < best) {
+          best = id[r];
+          bs = sc[r];
         }
-      }
+      den += bs;
+      prev = best;
     }
-  }
-};
-
-// Score expert i of a token from its logit z: routed experts enter the top-k,
-// shared experts only keep their affinity for the joint normalisation.
-template <int K>
-__device__ __forceinline__ void consume(const Params& p, SmemTail* st, TopK<K>& tk, int row, float* srow, int i,
-                                        float z) {
-  if (i < p.n_routed) {
-    float s = sigmoid_f32(z + st->off[i]);
-    if (srow) srow[i] = s;
-    tk.push(i, s, s + st->bias[i]);
-  } else if (i < p.n_routed + p.n_shared) {
-    float s = sigmoid_f32(z);
-    if (srow) srow[i] = s;
-    st->shared_s[row][i - p.n_routed] = s;
-  }
-}
-
-// Joint gates and outputs for one token.
-template <int K>
-__device__ __forceinline__ void finish(const Params& p, SmemTail* st, TopK<K>& tk, int row, int t) {
-  // the denominator is a sum over the contributor set, in ascending expert index
-  float den = 0.0f;
-  int prev = -1;
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
-    int best = 0x7fffffff;
-    float bs = 0.0f;
+    for (int q = 0; q < MOE_MAX_SHARED; ++q)
+      if (q < p.n_shared) den += shv[q];
+    const int G = K + p.n_shared;
+    int32_t* ti = p.topk_idx + (size_t)t * K;
+    float* gt = p.gates + (size_t)t * G;
 #pragma unroll
-    for (int r = 0; r < K; ++r)
-      if (tk.id[r] > prev && tk.id[r] < best) {
-        best = tk.id[r];
-        bs = tk.sc[r];
-      }
-    den += bs;
-    prev = best;
-  }
-  for (int q = 0; q < p.n_shared; ++q) den += st->shared_s[row][q];
-  const int G = K + p.n_shared;
-  int32_t* ti = p.topk_idx + (size_t)t * K;
-  float* gt = p.gates + (size_t)t * G;
+    for (int q = 0; q < K; ++q) {
+      ti[q] = id[q];
+      gt[q] = __fdiv_rn(sc[q], den);
+      if (id[q] >= 0 && id[q] < p.n_routed) atomicAdd(&st->hist[id[q]], 1);  // unset only for non-finite scores
+    }
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
-    ti[q] = tk.id[q];
-    gt[q] = __fdiv_rn(tk.sc[q], den);
-    if (tk.id[q] < p.n_routed) atomicAdd(&st->hist[tk.id[q]], 1);  // unset only for non-finite scores
+    for (int q = 0; q < MOE_MAX_SHARED; ++q)
+      if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[q], den);
   }
-  for (int q = 0; q < p.n_shared; ++q) gt[K + q] = __fdiv_rn(st->shared_s[row][q], den);
 }
 
 template <int K>
@@ -180,7 +205,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto stageA = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stageB0 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
   auto stageB1 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B0_BYTES; };
-  float* red = reinterpret_cast<float*>(smem);   // [BM][RED_COLS] split-K partial
+  float* red = reinterpret_cast<float*>(smem);   // [BM][RED_COLS] logits (split-K: this CTA's partial)
   float* zsum = red + (size_t)BM * RED_COLS;      // [BM/S][RED_COLS] reduced rows
 
   const int tid = threadIdx.x;
@@ -283,63 +308,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
     }
   } else {
-    // ================= epilogue warps =================
+    // ================= epilogue warps: park this CTA's logit tile in shared memory =================
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // this thread's TMEM lane
     const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const int lim = E < B0_ROWS ? E : B0_ROWS;
     if (mbar_wait(&st->tfull, 0, p.timeout_ns, abort_flag, p.status)) {
       tc_fence_after();
-      if (S == 1) {
-        // one token per thread, straight from TMEM
-        const int t = m0 + row;
-        const bool valid = t < p.T;
-        TopK<K> tk;
-        tk.init();
-        float* srow = (p.scores != nullptr && valid) ? p.scores + (size_t)t * E : nullptr;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the stage ring is idle now
+      float* dst = red + (size_t)row * RED_COLS;
 #pragma unroll 1
-        for (int c0 = 0; c0 < lim; c0 += 32) {
-          float v[32];
-          tmem_ld32(taddr + c0, v);
+      for (int c0 = 0; c0 < B0_ROWS; c0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + c0, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < lim) consume<K>(p, st, tk, row, srow, c0 + j, v[j]);
-        }
-        if (two) {
-          float v[16];
-          tmem_ld16(taddr + B0_ROWS, v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (B0_ROWS + j < E) consume<K>(p, st, tk, row, srow, B0_ROWS + j, v[j]);
-        }
-        if (valid) finish<K>(p, st, tk, row, t);
-      } else {
-        // split-K: park this CTA's partial tile row in shared memory (the stage ring is idle now)
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        float* dst = red + (size_t)row * RED_COLS;
-#pragma unroll 1
-        for (int c0 = 0; c0 < B0_ROWS; c0 += 32) {
-          float v[32];
-          tmem_ld32(taddr + c0, v);
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        }
-        float v[16];
-        if (two) {
-          tmem_ld16(taddr + B0_ROWS, v);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(dst + B0_ROWS + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
+      float v[16];
+      if (two) {
+        tmem_ld16(taddr + B0_ROWS, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(dst + B0_ROWS + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
 
-  if (S > 1) {
+  if (S == 1) {
+    if (warp >= 2) {
+      named_bar_sync(1, 128);
+      for (int r = warp - 2; r < BM; r += 4) {  // one token per warp
+        const int t = m0 + r;
+        if (t < p.T) route_token_warp<K>(p, st, red + (size_t)r * RED_COLS, t, lane);
+      }
+    }
+  } else {
     tc_fence_before();
     cluster_sync_all();  // every CTA's partial tile is in its shared memory
     if (warp >= 2) {
@@ -368,18 +374,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *reinterpret_cast<float4*>(zsum + (size_t)r_local * RED_COLS + 4 * f) = acc;
       }
       named_bar_sync(1, 128);
-      // 2. route the rows: one thread per token
-      if (e < rows_per) {
-        const int rr = (int)crank * rows_per + e;
-        const int t = m0 + rr;
-        if (t < p.T) {
-          TopK<K> tk;
-          tk.init();
-          float* srow = p.scores != nullptr ? p.scores + (size_t)t * E : nullptr;
-          const float* z = zsum + (size_t)e * RED_COLS;
-          for (int i = 0; i < E; ++i) consume<K>(p, st, tk, rr, srow, i, z[i]);
-          finish<K>(p, st, tk, rr, t);
-        }
+      // 2. route the rows: one token per warp
+      for (int r = warp - 2; r < rows_per; r += 4) {
+        const int t = m0 + (int)crank * rows_per + r;
+        if (t < p.T) route_token_warp<K>(p, st, zsum + (size_t)r * RED_COLS, t, lane);
       }
     }
     cluster_sync_all();  // no CTA leaves while another may still read its partial
