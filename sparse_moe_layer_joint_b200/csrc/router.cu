@@ -16,15 +16,18 @@
 // shared memory (a fixed order, so the result does not depend on timing).
 //
 // Routing epilogue: the logit tile is parked in shared memory (the stage ring
-// is idle by then) and each epilogue warp routes one token at a time: sigmoid,
-// + b for selection, k rounds of a warp-wide argmax (ties keep the lower
-// index), the joint gates (denominator summed over the contributors in
-// ascending expert index) and a shared-memory histogram of the picks, added to
-// the global counts once per CTA.
+// is idle by then).  With a whole tile per CTA each epilogue thread routes one
+// token (register top-k list); after a split-K reduction, with 128/S rows per
+// CTA, each epilogue warp routes one token at a time (k rounds of a warp-wide
+// argmax).  Both keep the lower index on ties, form the joint gates with the
+// denominator summed over the contributors in ascending expert index, and
+// count the picks in a shared-memory histogram added to the global counts once
+// per CTA.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "moe.h"
@@ -45,7 +48,9 @@ constexpr int B1_BYTES = B1_ROWS * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B0_BYTES + B1_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int RED_COLS = B0_ROWS + B1_ROWS;  // 272 columns of a partial tile row
+constexpr int RED_COLS = B0_ROWS + B1_ROWS;  // 272 logit columns per tile row
+constexpr int RED_LD = RED_COLS + 4;         // row stride in shared memory: 16-byte reads of 8 consecutive rows
+                                             // (one per thread) fall in distinct bank groups
 constexpr int MAX_SPLIT = 8;
 
 struct Params {
@@ -68,22 +73,25 @@ struct SmemTail {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float bias[MOE_MAX_ROUTED];
-  float off[MOE_MAX_ROUTED];
+  alignas(16) float bias[MOE_MAX_ROUTED];  // read as float4
+  alignas(16) float off[MOE_MAX_ROUTED];
   int hist[MOE_MAX_ROUTED];
   float shared_s[BM][MOE_MAX_SHARED];
 };
 
 // The stage ring, idle once the MMAs are done, also holds the split-K partial
 // tile [128][272] fp32 and the reduced rows [128/S][272] fp32 (S >= 2).
-constexpr size_t SPLIT_BYTES = (size_t)BM * RED_COLS * 4 + (size_t)(BM / 2) * RED_COLS * 4;
+constexpr size_t SPLIT_BYTES = (size_t)BM * RED_LD * 4 + (size_t)(BM / 2) * RED_LD * 4;
 constexpr size_t RING_BYTES =
     (size_t)STAGES * STAGE_BYTES > SPLIT_BYTES ? (size_t)STAGES * STAGE_BYTES : SPLIT_BYTES;
 
 constexpr size_t SMEM_BYTES = 1024 + RING_BYTES + sizeof(SmemTail);
 static_assert(SMEM_BYTES <= 227 * 1024, "router shared memory");
+static_assert(RING_BYTES % 16 == 0 && offsetof(SmemTail, bias) % 16 == 0 && offsetof(SmemTail, off) % 16 == 0,
+              "float4 reads of bias / offset need 16-byte alignment");
+static_assert((RED_LD * 4) % 16 == 0, "logit rows are read as float4");
 
-__device__ __forceinline__ float sigmoid_f32(float z) { return 1.0f / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float sigmoid_f32(float z) { return __frcp_rn(1.0f + __expf(-z)); }
 
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   float4 v;
@@ -91,6 +99,104 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
   return v;
+}
+
+// Route one token with one thread.  z: the token's logits in shared memory.
+// Scores are computed 32 experts at a time (independent, so their latencies
+// overlap); each is then offered to a sorted register top-k list, with a
+// single compare against the current k-th value rejecting most of them.
+// Scanning experts in index order with a strict '>' keeps the lower index on
+// ties.  Then the joint gates (denominator summed over the contributors in
+// ascending expert index), the outputs and the pick histogram.
+template <int K>
+__device__ __forceinline__ void route_token(const Params& p, SmemTail* st, const float* z, int t) {
+  const int E = p.n_routed + p.n_shared;
+  float* srow = p.scores != nullptr ? p.scores + (size_t)t * E : nullptr;
+  float val[K], sc[K];
+  int id[K];
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    val[q] = -INFINITY;
+    sc[q] = 0.0f;
+    id[q] = 0x7fffffff;
+  }
+  for (int c0 = 0; c0 < p.n_routed; c0 += 32) {
+    float sv[32], sl[32];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 z4 = *reinterpret_cast<const float4*>(z + c0 + j);
+      const float4 o4 = *reinterpret_cast<const float4*>(st->off + c0 + j);
+      const float4 b4 = *reinterpret_cast<const float4*>(st->bias + c0 + j);
+      sv[j + 0] = sigmoid_f32(z4.x + o4.x);
+      sv[j + 1] = sigmoid_f32(z4.y + o4.y);
+      sv[j + 2] = sigmoid_f32(z4.z + o4.z);
+      sv[j + 3] = sigmoid_f32(z4.w + o4.w);
+      sl[j + 0] = sv[j + 0] + b4.x;
+      sl[j + 1] = sv[j + 1] + b4.y;
+      sl[j + 2] = sv[j + 2] + b4.z;
+      sl[j + 3] = sv[j + 3] + b4.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int i = c0 + j;
+      if (i < p.n_routed) {
+        if (srow) srow[i] = sv[j];
+        if (sl[j] > val[K - 1]) {
+          val[K - 1] = sl[j];
+          sc[K - 1] = sv[j];
+          id[K - 1] = i;
+#pragma unroll
+          for (int q = K - 1; q > 0; --q) {
+            if (val[q] > val[q - 1]) {
+              float tv = val[q]; val[q] = val[q - 1]; val[q - 1] = tv;
+              float ts = sc[q]; sc[q] = sc[q - 1]; sc[q - 1] = ts;
+              int ti = id[q]; id[q] = id[q - 1]; id[q - 1] = ti;
+            }
+          }
+        }
+      }
+    }
+  }
+  float shv[MOE_MAX_SHARED];
+#pragma unroll
+  for (int q = 0; q < MOE_MAX_SHARED; ++q) {
+    shv[q] = 0.0f;
+    if (q < p.n_shared) {
+      shv[q] = sigmoid_f32(z[p.n_routed + q]);
+      if (srow) srow[p.n_routed + q] = shv[q];
+    }
+  }
+  // the denominator is a sum over the contributor set, in ascending expert index
+  float den = 0.0f;
+  int prev = -1;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    int best = 0x7fffffff;
+    float bs = 0.0f;
+#pragma unroll
+    for (int r = 0; r < K; ++r)
+      if (id[r] > prev && id[r] < best) {
+        best = id[r];
+        bs = sc[r];
+      }
+    den += bs;
+    prev = best;
+  }
+#pragma unroll
+  for (int q = 0; q < MOE_MAX_SHARED; ++q)
+    if (q < p.n_shared) den += shv[q];
+  const int G = K + p.n_shared;
+  int32_t* ti = p.topk_idx + (size_t)t * K;
+  float* gt = p.gates + (size_t)t * G;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    ti[q] = id[q];
+    gt[q] = __fdiv_rn(sc[q], den);
+    if (id[q] >= 0 && id[q] < p.n_routed) atomicAdd(&st->hist[id[q]], 1);  // unset only for non-finite scores
+  }
+#pragma unroll
+  for (int q = 0; q < MOE_MAX_SHARED; ++q)
+    if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[q], den);
 }
 
 // Route one token with one warp.  z: the token's logits in shared memory
@@ -205,8 +311,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto stageA = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stageB0 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
   auto stageB1 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B0_BYTES; };
-  float* red = reinterpret_cast<float*>(smem);   // [BM][RED_COLS] logits (split-K: this CTA's partial)
-  float* zsum = red + (size_t)BM * RED_COLS;      // [BM/S][RED_COLS] reduced rows
+  float* red = reinterpret_cast<float*>(smem);   // [BM][RED_LD] logits (split-K: this CTA's partial)
+  float* zsum = red + (size_t)BM * RED_LD;        // [BM/S][RED_LD] reduced rows
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -315,7 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (mbar_wait(&st->tfull, 0, p.timeout_ns, abort_flag, p.status)) {
       tc_fence_after();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the stage ring is idle now
-      float* dst = red + (size_t)row * RED_COLS;
+      float* dst = red + (size_t)row * RED_LD;
 #pragma unroll 1
       for (int c0 = 0; c0 < B0_ROWS; c0 += 32) {
         float v[32];
@@ -339,11 +445,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (S == 1) {
     if (warp >= 2) {
-      named_bar_sync(1, 128);
-      for (int r = warp - 2; r < BM; r += 4) {  // one token per warp
-        const int t = m0 + r;
-        if (t < p.T) route_token_warp<K>(p, st, red + (size_t)r * RED_COLS, t, lane);
-      }
+      // each thread routes the row it parked (its TMEM lane)
+      const int r = (warp & 3) * 32 + lane;
+      const int t = m0 + r;
+      if (t < p.T) route_token<K>(p, st, red + (size_t)r * RED_LD, t);
     }
   } else {
     tc_fence_before();
@@ -355,7 +460,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int part = e - r_local * S;
       const int row = (int)crank * rows_per + r_local;
       // 1. sum the S partials of this CTA's rows (float4 columns part, part + S, ...), in rank order
-      const uint32_t red_local = smem_u32(red + (size_t)row * RED_COLS);
+      const uint32_t red_local = smem_u32(red + (size_t)row * RED_LD);
       for (int f = part; f < RED_COLS / 4; f += S) {
         float4 q[MAX_SPLIT];
 #pragma unroll
@@ -371,13 +476,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             acc.w += q[c].w;
           }
         }
-        *reinterpret_cast<float4*>(zsum + (size_t)r_local * RED_COLS + 4 * f) = acc;
+        *reinterpret_cast<float4*>(zsum + (size_t)r_local * RED_LD + 4 * f) = acc;
       }
       named_bar_sync(1, 128);
-      // 2. route the rows: one token per warp
+      // 2. route the rows: with only 128/S of them, one token per warp (all lanes busy)
       for (int r = warp - 2; r < rows_per; r += 4) {
         const int t = m0 + (int)crank * rows_per + r;
-        if (t < p.T) route_token_warp<K>(p, st, zsum + (size_t)r * RED_COLS, t, lane);
+        if (t < p.T) route_token_warp<K>(p, st, zsum + (size_t)r * RED_LD, t, lane);
       }
     }
     cluster_sync_all();  // no CTA leaves while another may still read its partial
