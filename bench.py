@@ -121,6 +121,7 @@ def run_ours(args, w, rank, world, local_rank):
     import torch.distributed as dist
 
     import sparse_moe_layer_joint_b200 as moe
+    from sparse_moe_layer_joint_b200 import dp
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -129,16 +130,15 @@ def run_ours(args, w, rank, world, local_rank):
     if rank > 0:  # each replica gets its own tokens: rows rank*T .. of one global x stream
         mi.gpu_normal_bf16(t["x"].data_ptr(), t["x"].numel(), w.seed, mi.STREAM_X, rank * w.T * w.d, w.std_x,
                            stream.cuda_stream)
-    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev)
+    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev,
+                         gather_rows=args.gather_rows)
     bias0 = t["bias"].clone()
     ffn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
     def step(i=None, x=None):
         layer.forward(t["x"] if x is None else x, t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"],
                       ffn_events=None if i is None else ffn_ev[i])
-        if world > 1:
-            dist.all_reduce(layer.counts)
-        layer.bias_update(t["bias"], w.gamma)
+        dp.bias_step(layer, t["bias"], w.gamma)
 
     def barrier():
         if world > 1:
@@ -175,27 +175,51 @@ def run_ours(args, w, rank, world, local_rank):
     for i in range(args.steps):
         layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
         local_counts[i].copy_(layer.counts)
-        if world > 1:
-            dist.all_reduce(layer.counts)
-        layer.bias_update(t["bias"], w.gamma)
+        dp.bias_step(layer, t["bias"], w.gamma)
     touched = (local_counts > 0).sum(dim=1).double().mean().item()
 
-    # end to end through the public API: pinned host x in, host out back, every step
+    # end to end through the public API: every step copies its x in from pinned host memory and
+    # its output back to pinned host memory.  Like a serving loop, the copies of neighbouring steps
+    # overlap the current step: x and out are double-buffered on the device, the H2D copies run on
+    # one stream and the D2H copies on another, with events so that no buffer is overwritten
+    # before it has been consumed.
     x_host = t["x"].cpu().pin_memory()
-    out_host = torch.empty_like(layer.out, device="cpu").pin_memory()
-    x_dev = torch.empty_like(t["x"])
-    for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x=x_dev)
-        out_host.copy_(layer.out, non_blocking=True)
+    out_host = [torch.empty((w.T, w.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(t["x"]) for _ in range(2)]
+    out_dev = [torch.empty_like(layer.out) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("x_ready", "x_free", "out_ready", "out_free")}
+    for b in range(2):
+        ev["x_free"][b].record(stream)
+        ev["out_free"][b].record(stream)
+
+    def e2e_step(i):
+        b = i % 2
+        s_in.wait_event(ev["x_free"][b])
+        with torch.cuda.stream(s_in):
+            x_dev[b].copy_(x_host, non_blocking=True)
+        ev["x_ready"][b].record(s_in)
+        stream.wait_event(ev["x_ready"][b])
+        stream.wait_event(ev["out_free"][b])
+        layer.forward(x_dev[b], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"], out=out_dev[b])
+        dp.bias_step(layer, t["bias"], w.gamma)
+        ev["x_free"][b].record(stream)
+        ev["out_ready"][b].record(stream)
+        s_out.wait_event(ev["out_ready"][b])
+        with torch.cuda.stream(s_out):
+            out_host[b].copy_(out_dev[b], non_blocking=True)
+        ev["out_free"][b].record(s_out)
+
+    for i in range(2):
+        e2e_step(i)
     barrier()
     torch.cuda.synchronize()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x=x_dev)
-        out_host.copy_(layer.out, non_blocking=True)
+    s_in.wait_stream(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_stream(s_out)   # the last output is on the host before the clock stops
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -240,10 +264,12 @@ def run_ours(args, w, rank, world, local_rank):
         "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox, random-init weights)",
-        "config": config_of(w, world), "clocks": clk,
+        "config": dict(config_of(w, world), dispatch="rows gathered by GEMM1 (cp.async)" if args.gather_rows
+                       else "rows copied by moe_permute"), "clocks": clk,
         "e2e": {"value": round(world * w.T / (e2e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": w.T * w.d * 2, "d2h_bytes_per_step": w.T * w.d * 2,
-                "ms_per_step": round(e2e_ms, 4)},
+                "ms_per_step": round(e2e_ms, 4),
+                "note": "pinned host x in and out every step; copies of neighbouring steps overlap compute"},
         "gpu_launches": layer.launches_per_step() * args.steps,
         "roofline": roofline,
         "roofline_other": tensor_roof if weight_bound else hbm_roof,
@@ -387,6 +413,8 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gather-rows", action="store_true",
+                    help="GEMM1 gathers the routed rows from x (cp.async) instead of reading rows copied by dispatch")
     ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "router"], default=None,
                     help="time one kernel alone on a small profiling case instead of the layer")
     args = ap.parse_args()

@@ -234,14 +234,15 @@ class MoELayer:
         self.ev_shared = torch.cuda.Event()
 
     def forward(self, x, w_router, w1, w2, bias, logit_offset=None, stream=None, scores_out=None,
-                ffn_events=None):
+                ffn_events=None, out=None):
         """Router -> dispatch -> experts -> combine, on the given (default: current) stream.
 
         With ``fused_experts`` (default) the routed and shared experts run in one
         pair of grouped-GEMM launches (moe_experts_ffn).  Otherwise the shared
         experts run beside dispatch and the routed experts on a second stream
         (moe_grouped_ffn twice).  ``ffn_events`` = (start, end) torch events
-        recorded around the expert launches on the main stream."""
+        recorded around the expert launches on the main stream.  ``out``: a [T, d]
+        bf16 tensor to write the result into (default: this layer's own buffer)."""
         import torch
 
         s = self.shape
@@ -271,9 +272,10 @@ class MoELayer:
             ffn_events[1].record(main)
         if side:
             main.wait_event(self.ev_shared)
+        dst = self.out if out is None else out
         moe_combine(self.y_perm, self.token_row, self.gates, self.y_shared if s.n_shared > 0 else None, T, d, k,
-                    s.n_shared, self.out, stream=main)
-        return self.out
+                    s.n_shared, dst, stream=main)
+        return dst
 
     # kernels of libmoe launched by one forward + bias update
     def launches_per_step(self) -> int:
@@ -282,6 +284,9 @@ class MoELayer:
         permute = 3 if self.gather_rows else 4
         return 1 + permute + experts + 1 + 1
 
-    def bias_update(self, bias, gamma: float, stream=None):
+    def bias_update(self, bias, gamma: float, stream=None, T_total: Optional[int] = None):
+        """b += gamma * sign(Lbar - L) from this layer's counts; T_total: the batch's token
+        count when the counts were summed over data-parallel ranks (default: this layer's T)."""
         s = self.shape
-        moe_bias_update(self.counts, s.n_routed, s.T, s.top_k, gamma, bias, stream=stream)
+        moe_bias_update(self.counts, s.n_routed, s.T if T_total is None else T_total, s.top_k, gamma, bias,
+                        stream=stream)

@@ -66,12 +66,16 @@ struct Cfg {
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // bytes landing on the (leader's) full barrier
+  static constexpr uint32_t TX_B_BYTES = (PAIR ? 2 : 1) * B_BYTES;     // when A rows arrive by cp.async instead
+  static constexpr int GATHER_LAG = STAGES - 2;  // stages of row copies a producer lane keeps in flight
+  static constexpr int GATHER_ARRIVALS = 32 * (PAIR ? 2 : 1);  // producer lanes arriving per stage
 };
 
 struct Params {
   const int* offsets;  // [G_r + 1] routed group row offsets (device); unused when G_r == 0
   const int* gather_rows;  // non-null: routed A rows are gathered, row r of group g = gather_rows[off[g] + r]
   int gather_limit;        // gathered row indices are clamped to [0, gather_limit)
+  const __nv_bfloat16* gather_src;  // rows gathered from here (row stride K)
   int G_r;             // routed groups
   int G_s;             // shared groups
   int routed_rows;     // offsets are clamped to [0, routed_rows]
@@ -212,8 +216,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (tid == 0) {
+    // gathering launches: the producer lanes of both CTAs also arrive once per stage
+    const uint32_t full_count = 1u + (p.gather_rows != nullptr ? (uint32_t)C::GATHER_ARRIVALS : 0u);
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&st->full[s], 1);
+      mbar_init(&st->full[s], full_count);
       mbar_init(&st->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -246,7 +252,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = &st->abort_flag;
 
   if (warp == 0) {
-    // ================= TMA producer (whole warp; lane 0 issues tiles, every lane a row gather) ===========
+    // ================= producer (whole warp) =================
+    // Tiles arrive by TMA (lane 0).  In gathering launches the routed groups' A rows are instead
+    // copied by the lanes with cp.async, in 16-byte chunks placed in the 128-byte swizzled layout;
+    // every lane commits one copy group per stage and, GATHER_LAG stages later, once that group has
+    // landed, arrives on the stage's full barrier (the pair leader's).
+    const bool gathering = p.gather_rows != nullptr;
     if (lane == 0) {
       tma_prefetch_desc(&tmA0);
       if (p.G_s > 0 && p.a_sh_map == 1) tma_prefetch_desc(&tmA1);
@@ -256,38 +267,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0;
     long issued = 0;
     bool ok = true;
-    for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
+    const bool active = gathering || lane == 0;  // without gathers, lane 0 alone produces
+    auto lane_arrive = [&](long it) {  // this lane's arrival for stage iteration `it`
+      fence_proxy_async_smem();
+      uint64_t* bar = &st->full[it % C::STAGES];
+      if (PAIR)
+        mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
+      else
+        mbar_arrive(bar);
+    };
+    for (int tile = unit; active && tile < total_tiles && ok; tile += n_units) {
       const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
       const Group gr = group_info(p, st->gt, ti.g);
       const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
       const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
       const int b_row = ti.nt * BN + (int)rank * C::B_ROWS;
-      const bool gather = p.gather_rows != nullptr && ti.g < p.G_r;
-      int gr0 = 0, gr1 = 0, gr2 = 0, gr3 = 0;  // this lane's four source rows (rows 4*lane.. of the CTA's A tile)
+      const bool gather = gathering && ti.g < p.G_r;
+      // gathered rows: copy instruction q moves rows 4q .. 4q+3 of the CTA's A tile, eight lanes per
+      // row (lane l: row 4q + l/8, 16-byte chunk l%8), so each instruction reads four whole 128-byte
+      // row pieces; this lane's 32 source rows are kept as indices
+      int srow_idx[32];
       if (gather) {
-        const int r0 = ti.m * C::TILE_M + (int)rank * C::A_ROWS + 4 * lane;  // row within the group
-        auto src = [&](int j) -> int {
-          if (r0 + j >= gr.rows) return 0;  // past the group: any valid row, masked in the epilogue
-          int v = __ldg(p.gather_rows + gr.a_base + r0 + j);
-          return v < 0 ? 0 : (v >= p.gather_limit ? p.gather_limit - 1 : v);
-        };
-        gr0 = src(0);
-        gr1 = src(1);
-        gr2 = src(2);
-        gr3 = src(3);
+        const int r_base = ti.m * C::TILE_M + (int)rank * C::A_ROWS;  // tile row 0 within the group
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int r = r_base + 4 * q + (lane >> 3);
+          int v = 0;  // rows past the group: any valid row, masked in the epilogue
+          if (r < gr.rows) {
+            v = __ldg(p.gather_rows + gr.a_base + r);
+            v = v < 0 ? 0 : (v >= p.gather_limit ? p.gather_limit - 1 : v);
+          }
+          srow_idx[q] = v;
+        }
       }
       for (int kb = 0; kb < num_kb; ++kb) {
         if (lane == 0) ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (gathering) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        if (lane == 0 && leader) mbar_arrive_expect_tx(&st->full[stage], C::TX_BYTES);
-        __syncwarp();
+        if (lane == 0 && leader) mbar_arrive_expect_tx(&st->full[stage], gather ? C::TX_B_BYTES : C::TX_BYTES);
+        if (gathering) __syncwarp();
         uint8_t* a_dst = smemA + stage * C::A_BYTES;
         if (gather) {
-          if (PAIR)
-            tma_gather4_pair(a_dst + lane * 512, am, &st->full[stage], kb * BK, gr0, gr1, gr2, gr3);
-          else
-            tma_gather4(a_dst + lane * 512, am, &st->full[stage], kb * BK, gr0, gr1, gr2, gr3);
+          const uint32_t a_base = smem_u32(a_dst);
+          const int c = lane & 7;
+          const __nv_bfloat16* src = p.gather_src + kb * BK + c * 8;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int row = 4 * q + (lane >> 3);
+            cp_async_16(a_base + row * 128 + ((c ^ (row & 7)) << 4), src + (size_t)srow_idx[q] * p.K);
+          }
         }
         if (lane == 0) {
           if (PAIR) {
@@ -298,6 +326,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_3d(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
           }
         }
+        if (gathering) {
+          cp_async_commit();  // one group per stage (empty for TMA-loaded tiles)
+          if (issued >= C::GATHER_LAG) {
+            cp_async_wait<C::GATHER_LAG>();
+            lane_arrive(issued - C::GATHER_LAG);
+          }
+        }
         ++issued;
         if (++stage == C::STAGES) {
           stage = 0;
@@ -305,7 +340,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-    if (!ok && !PAIR && lane == 0) {
+    if (gathering) {
+      // the last stages' copies: wait for all of them, then arrive for each
+      cp_async_wait<0>();
+      if (ok)
+        for (long it = issued > C::GATHER_LAG ? issued - C::GATHER_LAG : 0; it < issued; ++it) lane_arrive(it);
+    }
+    if (!ok && !PAIR && lane == 0 && !gathering) {
       // wind down: let the copies already issued land before the CTA exits
       int zero = 0;
       for (long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
@@ -330,6 +371,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
+          fence_proxy_async_smem();  // rows copied by cp.async are read by the tensor core (async proxy)
           const uint32_t a_addr = smem_u32(smemA + stage * C::A_BYTES);
           const uint32_t b_addr = smem_u32(smemB + stage * C::B_BYTES);
 #pragma unroll
@@ -636,13 +678,14 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   const bool routed_gather = n_routed > 0 && gather;
   g1.a0 = (n_routed > 0 && !gather) ? (const void*)x_perm : (const void*)x;
   g1.a0_rows = (n_routed > 0 && !gather) ? (uint64_t)R : (uint64_t)T;
-  g1.a0_box_rows = routed_gather ? 1u : 128u;
+  g1.a0_box_rows = 128u;
   g1.a1 = n_shared > 0 ? (const void*)x : nullptr;
   g1.a1_rows = (uint64_t)T;
   g1.b = w1;
   g1.p = p;
   g1.p.gather_rows = routed_gather ? row_token : nullptr;
   g1.p.gather_limit = T;
+  g1.p.gather_src = reinterpret_cast<const __nv_bfloat16*>(x);
   g1.p.a_sh_map = (n_routed > 0 || n_shared == 0) ? 1 : 0;
   g1.p.a_sh_base = 0;
   g1.p.a_sh_stride = 0;

@@ -1,0 +1,72 @@
+"""The data-parallel exchange on CPU (gloo, world size 2): each rank routes its
+half of the batch with the oracle, the per-expert loads are summed with
+sparse_moe_layer_joint_b200.dp, and the bias update on every rank equals the
+single-process update on the whole batch (the rule of §02e counts the batch's
+loads)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out_dir):
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+
+    import moe_inputs as mi
+    import oracle
+    from sparse_moe_layer_joint_b200 import dp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = mi.WORKLOADS["tiny"]
+        T_local = w.T // world
+        tokens = np.arange(rank * T_local, (rank + 1) * T_local)
+        b = mi.host_bias(w)
+        r = oracle.route_workload(w, b, tokens=tokens)
+        counts = torch.from_numpy(oracle.load_counts(r["topk_idx"], w.n_routed).astype(np.int32))
+        dp.global_counts(counts)
+        T_total = dp.total_tokens(T_local)
+        nb = oracle.bias_update(counts.numpy(), b, T_total, w.k, w.gamma)
+        np.save(os.path.join(out_dir, f"bias_{rank}.npy"), nb)
+        np.save(os.path.join(out_dir, f"counts_{rank}.npy"), counts.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_agree_with_the_whole_batch(tmp_path):
+    import moe_inputs as mi
+    import oracle
+
+    world = 2
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    w = mi.WORKLOADS["tiny"]
+    b = mi.host_bias(w)
+    full = oracle.route_workload(w, b)
+    counts = oracle.load_counts(full["topk_idx"], w.n_routed)
+    expect = oracle.bias_update(counts, b, w.T, w.k, w.gamma)
+    for rank in range(world):
+        np.testing.assert_array_equal(np.load(tmp_path / f"counts_{rank}.npy"), counts)
+        np.testing.assert_array_equal(np.load(tmp_path / f"bias_{rank}.npy").view(np.uint32), expect.view(np.uint32))
+
+
+def test_single_process_is_a_no_op():
+    from sparse_moe_layer_joint_b200 import dp
+
+    c = torch.arange(4, dtype=torch.int32)
+    assert dp.world_size() == 1
+    assert dp.global_counts(c) is c and c.tolist() == [0, 1, 2, 3]
+    assert dp.total_tokens(100) == 100
