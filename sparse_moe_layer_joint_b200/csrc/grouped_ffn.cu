@@ -371,7 +371,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          fence_proxy_async_smem();  // rows copied by cp.async are read by the tensor core (async proxy)
+          // rows copied by cp.async (generic proxy) are read by the tensor core (async proxy)
+          if (p.gather_rows != nullptr) fence_proxy_async_smem();
           const uint32_t a_addr = smem_u32(smemA + stage * C::A_BYTES);
           const uint32_t b_addr = smem_u32(smemB + stage * C::B_BYTES);
 #pragma unroll
