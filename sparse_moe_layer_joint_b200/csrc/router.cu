@@ -199,74 +199,108 @@ __device__ __forceinline__ void route_token(const Params& p, SmemTail* st, const
     if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[q], den);
 }
 
-// Route one token with one warp.  z: the token's logits in shared memory
-// (RED_COLS floats).  Lane l scores routed experts 8l .. 8l+7; then k rounds of
-// a warp-wide argmax of s + b (a strict '>' scan within a lane, and the lower
-// index on equal values across lanes, so ties keep the lower index) pick the
-// experts in descending order.  Lane 0 forms the joint gates (denominator summed
-// over the contributors in ascending expert index) and writes the outputs.
-template <int K>
-__device__ __forceinline__ void route_token_warp(const Params& p, SmemTail* st, const float* z, int t, int lane) {
+// Route NT tokens with one warp, their work interleaved so the latencies of the
+// NT independent shuffle chains overlap.  z: the first token's logits in shared
+// memory (rows ld floats apart); t0: its token index; n_valid <= NT tokens are
+// real.  Lane l scores routed experts 8l .. 8l+7 of every token; then k rounds
+// of a warp-wide argmax of s + b (a strict '>' scan within a lane, and the
+// lower index on equal values across lanes, so ties keep the lower index)
+// pick each token's experts in descending order.  Lane n then forms token n's
+// joint gates (denominator summed over the contributors in ascending expert
+// index) and writes its outputs.
+template <int K, int NT>
+__device__ __forceinline__ void route_tokens_warp(const Params& p, SmemTail* st, const float* z, int ld, int t0,
+                                                  int n_valid, int lane) {
   const int E = p.n_routed + p.n_shared;
-  float s[8], sel[8];
-  const float4* z4 = reinterpret_cast<const float4*>(z + 8 * lane);
-  const float4 za = z4[0], zb = z4[1];
-  const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-  float* srow = p.scores != nullptr ? p.scores + (size_t)t * E : nullptr;
+  float s[NT][8], sel[NT][8];
+  float4 o4[2], b4[2];
+  o4[0] = *reinterpret_cast<const float4*>(st->off + 8 * lane);
+  o4[1] = *reinterpret_cast<const float4*>(st->off + 8 * lane + 4);
+  b4[0] = *reinterpret_cast<const float4*>(st->bias + 8 * lane);
+  b4[1] = *reinterpret_cast<const float4*>(st->bias + 8 * lane + 4);
+  const float off[8] = {o4[0].x, o4[0].y, o4[0].z, o4[0].w, o4[1].x, o4[1].y, o4[1].z, o4[1].w};
+  const float bia[8] = {b4[0].x, b4[0].y, b4[0].z, b4[0].w, b4[1].x, b4[1].y, b4[1].z, b4[1].w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int i = 8 * lane + j;
-    if (i < p.n_routed) {
-      s[j] = sigmoid_f32(zz[j] + st->off[i]);
-      sel[j] = s[j] + st->bias[i];
-      if (srow) srow[i] = s[j];
-    } else {
-      s[j] = 0.0f;
-      sel[j] = -INFINITY;
+  for (int n = 0; n < NT; ++n) {
+    const float4* z4 = reinterpret_cast<const float4*>(z + (size_t)n * ld + 8 * lane);
+    const float4 za = z4[0], zb = z4[1];
+    const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+    float* srow = (p.scores != nullptr && n < n_valid) ? p.scores + (size_t)(t0 + n) * E : nullptr;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = 8 * lane + j;
+      if (i < p.n_routed) {
+        s[n][j] = sigmoid_f32(zz[j] + off[j]);
+        sel[n][j] = s[n][j] + bia[j];
+        if (srow) srow[i] = s[n][j];
+      } else {
+        s[n][j] = 0.0f;
+        sel[n][j] = -INFINITY;
+      }
     }
   }
-  // shared experts' affinities (lanes 0 .. n_shared-1)
-  float sh = 0.0f;
-  if (lane < p.n_shared) {
-    sh = sigmoid_f32(z[p.n_routed + lane]);
-    if (srow) srow[p.n_routed + lane] = sh;
+  // shared experts' affinities: lane q < n_shared holds shared expert q of every token
+  float sh[NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    sh[n] = 0.0f;
+    if (lane < p.n_shared) {
+      sh[n] = sigmoid_f32(z[(size_t)n * ld + p.n_routed + lane]);
+      if (p.scores != nullptr && n < n_valid) p.scores[(size_t)(t0 + n) * E + p.n_routed + lane] = sh[n];
+    }
   }
-  int id[K];
-  float sc[K];
+  int id[NT][K];
+  float sc[NT][K];
 #pragma unroll
   for (int q = 0; q < K; ++q) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    float bv[NT];
+    int bi[NT];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (sel[j] > bv) {
-        bv = sel[j];
-        bi = 8 * lane + j;
-      }
+    for (int n = 0; n < NT; ++n) {
+      bv[n] = -INFINITY;
+      bi[n] = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (sel[n][j] > bv[n]) {
+          bv[n] = sel[n][j];
+          bi[n] = 8 * lane + j;
+        }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv[n], o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi[n], o);
+        if (ov > bv[n] || (ov == bv[n] && oi < bi[n])) {
+          bv[n] = ov;
+          bi[n] = oi;
+        }
       }
     }
-    float sw = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (8 * lane + j == bi) {
-        sw = s[j];
-        sel[j] = -INFINITY;
-      }
-    const int owner = (bi >= 0 && bi < 256) ? (bi >> 3) : 0;
-    sc[q] = __shfl_sync(0xffffffffu, sw, owner);
-    id[q] = bi;
+    for (int n = 0; n < NT; ++n) {
+      float sw = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (8 * lane + j == bi[n]) {
+          sw = s[n][j];
+          sel[n][j] = -INFINITY;
+        }
+      const int owner = (bi[n] >= 0 && bi[n] < 256) ? (bi[n] >> 3) : 0;
+      sc[n][q] = __shfl_sync(0xffffffffu, sw, owner);
+      id[n][q] = bi[n];
+    }
   }
-  float shv[MOE_MAX_SHARED];
+  float shv[NT][MOE_MAX_SHARED];
 #pragma unroll
-  for (int q = 0; q < MOE_MAX_SHARED; ++q) shv[q] = __shfl_sync(0xffffffffu, sh, q);
-  if (lane == 0) {
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int q = 0; q < MOE_MAX_SHARED; ++q) shv[n][q] = __shfl_sync(0xffffffffu, sh[n], q);
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    if (lane != n || n >= n_valid) continue;  // lane n finishes token n
+    const int t = t0 + n;
     // the denominator is a sum over the contributor set, in ascending expert index
     float den = 0.0f;
     int prev = -1;
@@ -276,28 +310,28 @@ __device__ __forceinline__ void route_token_warp(const Params& p, SmemTail* st, 
       float bs = 0.0f;
 #pragma unroll
       for (int r = 0; r < K; ++r)
-        if (id[r] > prev && id[r] < best) {
-          best = id[r];
-          bs = sc[r];
+        if (id[n][r] > prev && id[n][r] < best) {
+          best = id[n][r];
+          bs = sc[n][r];
         }
       den += bs;
       prev = best;
     }
 #pragma unroll
     for (int q = 0; q < MOE_MAX_SHARED; ++q)
-      if (q < p.n_shared) den += shv[q];
+      if (q < p.n_shared) den += shv[n][q];
     const int G = K + p.n_shared;
     int32_t* ti = p.topk_idx + (size_t)t * K;
     float* gt = p.gates + (size_t)t * G;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      ti[q] = id[q];
-      gt[q] = __fdiv_rn(sc[q], den);
-      if (id[q] >= 0 && id[q] < p.n_routed) atomicAdd(&st->hist[id[q]], 1);  // unset only for non-finite scores
+      ti[q] = id[n][q];
+      gt[q] = __fdiv_rn(sc[n][q], den);
+      if (id[n][q] >= 0 && id[n][q] < p.n_routed) atomicAdd(&st->hist[id[n][q]], 1);  // unset only if non-finite
     }
 #pragma unroll
     for (int q = 0; q < MOE_MAX_SHARED; ++q)
-      if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[q], den);
+      if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[n][q], den);
   }
 }
 
@@ -479,10 +513,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *reinterpret_cast<float4*>(zsum + (size_t)r_local * RED_LD + 4 * f) = acc;
       }
       named_bar_sync(1, 128);
-      // 2. route the rows: with only 128/S of them, one token per warp (all lanes busy)
-      for (int r = warp - 2; r < rows_per; r += 4) {
-        const int t = m0 + (int)crank * rows_per + r;
-        if (t < p.T) route_token_warp<K>(p, st, zsum + (size_t)r * RED_LD, t, lane);
+      // 2. route the rows: with only 128/S of them, 4 tokens per warp pass (all lanes busy)
+      const int t_first = m0 + (int)crank * rows_per;
+      for (int r = 4 * (warp - 2); r < rows_per; r += 16) {
+        const int n_valid = min(4, min(rows_per - r, p.T - (t_first + r)));
+        if (n_valid > 0) route_tokens_warp<K, 4>(p, st, zsum + (size_t)r * RED_LD, RED_LD, t_first + r, n_valid, lane);
       }
     }
     cluster_sync_all();  // no CTA leaves while another may still read its partial
