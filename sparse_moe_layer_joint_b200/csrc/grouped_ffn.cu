@@ -56,12 +56,12 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_NONE = 1;
 
-template <bool PAIR>
+template <bool PAIR, int ST>
 struct Cfg {
   static constexpr int TILE_M = PAIR ? 256 : 128;  // rows per tile (per pair, or per CTA)
   static constexpr int A_ROWS = 128;               // A rows held by one CTA
   static constexpr int B_ROWS = PAIR ? 128 : 256;  // B rows (output columns) held by one CTA
-  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int STAGES = ST;
   static constexpr int A_BYTES = A_ROWS * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -99,10 +99,10 @@ struct GroupTables {
   int prefix[MOE_MAX_GROUPS + 1];  // prefix[g] = row tiles of groups < g
 };
 
-template <bool PAIR>
+template <int ST>
 struct SmemTail {
-  uint64_t full[Cfg<PAIR>::STAGES];
-  uint64_t empty[Cfg<PAIR>::STAGES];
+  uint64_t full[ST];
+  uint64_t empty[ST];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -111,9 +111,9 @@ struct SmemTail {
   GroupTables gt;
 };
 
-template <bool PAIR>
+template <bool PAIR, int ST>
 constexpr size_t smem_bytes() {
-  return 1024 /* alignment slack */ + (size_t)Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + sizeof(SmemTail<PAIR>);
+  return 1024 /* alignment slack */ + (size_t)ST * Cfg<PAIR, ST>::STAGE_BYTES + sizeof(SmemTail<ST>);
 }
 
 struct Group {
@@ -196,16 +196,16 @@ __device__ __forceinline__ void build_tables(const Params& p, GroupTables& gt, i
   __syncthreads();
 }
 
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, int ST>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, ST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smemA = smem;
   uint8_t* smemB = smem + C::STAGES * C::A_BYTES;
-  SmemTail<PAIR>* st = reinterpret_cast<SmemTail<PAIR>*>(smem + C::STAGES * C::STAGE_BYTES);
+  SmemTail<ST>* st = reinterpret_cast<SmemTail<ST>*>(smem + C::STAGES * C::STAGE_BYTES);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -479,11 +479,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, int ST>
 int launch_one(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const Params& p, int grid,
                cudaStream_t stream) {
-  auto kfn = grouped_gemm_kernel<EPI, PAIR>;
-  constexpr size_t bytes = smem_bytes<PAIR>();
+  auto kfn = grouped_gemm_kernel<EPI, PAIR, ST>;
+  constexpr size_t bytes = smem_bytes<PAIR, ST>();
+  static_assert(bytes <= 232448, "shared memory per CTA");
   int rc = ensure_smem_attr((const void*)kfn, bytes);
   if (rc != MOE_OK) return rc;
   if (PAIR) {
@@ -529,9 +530,29 @@ bool choose_pair(long long rows, int groups) {
   return pair;
 }
 
+// Pipeline depth of the pair kernel (stages of 64-deep K slices in flight per CTA).  Six stages hide
+// more load latency and win on short launches.  Launches of several TFLOP run for milliseconds under
+// the board's power cap; there four stages win: with less prefetch the pairs that share A rows or
+// weight tiles stay closer together in K, so more of their loads hit L2 (at 65536 tokens, d 7168,
+// d_ff 2048 the first GEMM reads about 21 GB from DRAM with four stages against about 50 GB with six).
+// MOE_GEMM_STAGES="s1,s2" (each 4 or 6) forces the depth of GEMM1, GEMM2.
+constexpr double LONG_LAUNCH_FLOP = 4e12;
+
+int stages_for(bool pair, int which, double flop) {
+  if (!pair) return 4;
+  int st = flop >= LONG_LAUNCH_FLOP ? 4 : 6;
+  const char* env = getenv("MOE_GEMM_STAGES");
+  if (env && env[0] && env[1] == ',' && env[2] && env[3] == '\0') {
+    const char c = which == 1 ? env[0] : env[2];
+    if (c == '4') st = 4;
+    if (c == '6') st = 6;
+  }
+  return st;
+}
+
 template <int EPI>
-int run_gemm(const GemmSpec& g, bool pair, int sms, long long tiles_upper, cudaStream_t s) {
-  const uint32_t b_box = pair ? (uint32_t)Cfg<true>::B_ROWS : (uint32_t)Cfg<false>::B_ROWS;
+int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_upper, cudaStream_t s) {
+  const uint32_t b_box = pair ? (uint32_t)Cfg<true, 4>::B_ROWS : (uint32_t)Cfg<false, 4>::B_ROWS;
   CUtensorMap a0, a1, b;
   int rc;
   const uint64_t K = (uint64_t)g.p.K, N = (uint64_t)g.p.N;
@@ -546,9 +567,10 @@ int run_gemm(const GemmSpec& g, bool pair, int sms, long long tiles_upper, cudaS
   long long units = tiles_upper * g.p.n_tiles_n;
   if (pair) {
     long long pairs = units < sms / 2 ? units : sms / 2;
-    return launch_one<EPI, true>(a0, a1, b, g.p, (int)(2 * pairs), s);
+    if (stages == 6) return launch_one<EPI, true, 6>(a0, a1, b, g.p, (int)(2 * pairs), s);
+    return launch_one<EPI, true, 4>(a0, a1, b, g.p, (int)(2 * pairs), s);
   }
-  return launch_one<EPI, false>(a0, a1, b, g.p, (int)(units < sms ? units : sms), s);
+  return launch_one<EPI, false, 4>(a0, a1, b, g.p, (int)(units < sms ? units : sms), s);
 }
 
 }  // namespace gffn
@@ -581,7 +603,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   if (!status) return MOE_ERR_CUDA;
 
   const bool pair = choose_pair(h_rows, n_groups);
-  const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
+  const int tile_m = pair ? Cfg<true, 4>::TILE_M : Cfg<false, 4>::TILE_M;
   const long long tiles_upper = identity ? (long long)n_groups * ((n_rows + tile_m - 1) / tile_m)
                                          : (n_rows + tile_m - 1) / tile_m + n_groups;
 
@@ -610,7 +632,8 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g1.p.K = d;
   g1.p.n_tiles_n = (d_ff + BN - 1) / BN;
   g1.p.ldc = d_ff;
-  if ((rc = run_gemm<EPI_GELU>(g1, pair, sms, tiles_upper, s)) != MOE_OK) return rc;
+  const double flop = 2.0 * (double)h_rows * d * d_ff;  // per GEMM
+  if ((rc = run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s)) != MOE_OK) return rc;
 
   GemmSpec g2{};
   g2.a0 = h_scratch;
@@ -627,7 +650,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g2.p.K = d_ff;
   g2.p.n_tiles_n = (d + BN - 1) / BN;
   g2.p.ldc = d;
-  return run_gemm<EPI_NONE>(g2, pair, sms, tiles_upper, s);
+  return run_gemm<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
 }
 
 extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* row_token,
@@ -660,7 +683,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
 
   const int G = n_routed + n_shared;
   const bool pair = choose_pair(h_rows, G);
-  const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
+  const int tile_m = pair ? Cfg<true, 4>::TILE_M : Cfg<false, 4>::TILE_M;
   const long long tiles_upper =
       (R + tile_m - 1) / tile_m + n_routed + (long long)n_shared * ((T + tile_m - 1) / tile_m);
 
@@ -699,7 +722,8 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.p.K = d;
   g1.p.n_tiles_n = (d_ff + BN - 1) / BN;
   g1.p.ldc = d_ff;
-  if ((rc = run_gemm<EPI_GELU>(g1, pair, sms, tiles_upper, s)) != MOE_OK) return rc;
+  const double flop = 2.0 * (double)h_rows * d * d_ff;  // per GEMM
+  if ((rc = run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s)) != MOE_OK) return rc;
 
   // GEMM2: all A rows from H (map 0); routed outputs to y_perm, shared outputs to y_shared
   GemmSpec g2{};
@@ -720,5 +744,5 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g2.p.K = d_ff;
   g2.p.n_tiles_n = (d + BN - 1) / BN;
   g2.p.ldc = d;
-  return run_gemm<EPI_NONE>(g2, pair, sms, tiles_upper, s);
+  return run_gemm<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
 }

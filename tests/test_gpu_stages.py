@@ -204,10 +204,15 @@ def _ffn_weights(E, d, f, seed):
     return w1, w2
 
 
-@pytest.fixture(params=["pair", "single"])
+@pytest.fixture(params=["pair", "pair4", "single"])
 def gemm_variant(request, monkeypatch):
-    """Both grouped-GEMM kernels: CTA pairs (default) and single CTAs."""
+    """Every grouped-GEMM kernel: CTA pairs with six pipeline stages (short launches), with four
+    (long launches), and single CTAs."""
     monkeypatch.setenv("MOE_GEMM_CTA", "1" if request.param == "single" else "2")
+    if request.param == "pair4":
+        monkeypatch.setenv("MOE_GEMM_STAGES", "4,4")
+    else:
+        monkeypatch.delenv("MOE_GEMM_STAGES", raising=False)
     return request.param
 
 
