@@ -53,6 +53,10 @@ STREAM_TEST_TOPK = 10
 STREAM_TEST_ROWS = 11
 STREAM_TEST_GATES = 12
 STREAM_TEST_SHARED = 13
+# Streams of the Router Balance Lab workload.
+STREAM_LAB_CENTERS = 20
+STREAM_LAB_SPECIALTY = 21
+STREAM_LAB_JITTER = 22
 
 N_ROUTED = 256
 N_SHARED = 2
@@ -116,6 +120,45 @@ WORKLOADS = {
 }
 
 ZIPF_S = 1.1
+
+
+@dataclass(frozen=True)
+class LabWorkload:
+    """The Router Balance Lab ("Inkling, Dissected" §02g): a frozen router over 64
+    experts, top-6, embedding width 32, batches of 2048 tokens for 100 routing
+    steps, hard expert capacities of 1.25x the ideal load, tokens drawn from a
+    Zipf distribution over expert specialties (expert 0's home cluster about 30
+    times as common as expert 63's) and jittered.
+
+    Generator (this module's reading; the lab's own code is not on the page):
+    specialty centers c_i ~ N(0, I/d); router row i = alpha * c_i (bf16); token
+    t of step s has specialty e ~ P(e) proportional to (e + 1)^-zs with
+    64^zs = zipf_ratio, and x = c_e + sigma * N(0, I/d) (bf16).  alpha and sigma
+    were chosen so that, with no balancing, the hottest expert sits near twice
+    its fair share, as in the page's run."""
+    name: str = "lab"
+    T: int = 2048
+    d: int = 32
+    n_routed: int = 64
+    n_shared: int = 0
+    k: int = 6
+    steps: int = 100
+    capacity_factor: float = 1.25
+    zipf_ratio: float = 30.0
+    alpha: float = 4.0
+    sigma: float = 0.75
+    seed: int = 0
+    gammas: tuple = (0.0, 0.01, 0.05)
+    description: str = ("Router Balance Lab: 64 experts, top-6, d=32, 2048 tokens x 100 steps, "
+                        "Zipf-lumpy tokens, capacity 1.25x ideal")
+
+    @property
+    def n_experts(self) -> int:
+        return self.n_routed + self.n_shared
+
+
+LAB = LabWorkload()
+
 SKEW_BETA_PATH = os.path.join(_HERE, "skew_beta.json")
 
 
@@ -334,3 +377,38 @@ def torch_workload(w: Workload, device="cuda", with_weights: bool = True):
     off = host_logit_offset(w)
     out["logit_offset"] = None if off is None else torch.from_numpy(off).to(dev)
     return out
+
+
+# --------------------------------------------------------------------------
+# Router Balance Lab inputs (host side; the GPU path copies these bits)
+# --------------------------------------------------------------------------
+def lab_centers(w: LabWorkload) -> np.ndarray:
+    """Specialty centers c [n_routed, d] (float64), c_i ~ N(0, I/d)."""
+    return normal_f64(w.n_routed * w.d, w.seed, STREAM_LAB_CENTERS).reshape(w.n_routed, w.d) / math.sqrt(w.d)
+
+
+def lab_wr(w: LabWorkload) -> np.ndarray:
+    """Frozen router weight [n_routed, d] as bf16 bits: alpha * c."""
+    return f32_to_bf16_bits((w.alpha * lab_centers(w)).astype(np.float32))
+
+
+def lab_specialty(w: LabWorkload, step: int) -> np.ndarray:
+    """Each token's specialty at a step: inverse-CDF draw from P(e) ~ (e+1)^-zs."""
+    zs = math.log(w.zipf_ratio) / math.log(w.n_routed)
+    p = np.arange(1, w.n_routed + 1, dtype=np.float64) ** -zs
+    cdf = np.cumsum(p / p.sum())
+    u = (words(w.T, w.seed, STREAM_LAB_SPECIALTY, step * w.T).astype(np.float64) + 0.5) / 4294967296.0
+    return np.minimum(np.searchsorted(cdf, u, side="right"), w.n_routed - 1).astype(np.int64)
+
+
+def lab_x(w: LabWorkload, step: int) -> np.ndarray:
+    """Tokens [T, d] of a step as bf16 bits: c_e + sigma * N(0, I/d)."""
+    c = lab_centers(w)
+    jit = normal_f64(w.T * w.d, w.seed, STREAM_LAB_JITTER, step * w.T * w.d).reshape(w.T, w.d)
+    x = c[lab_specialty(w, step)] + w.sigma * jit / math.sqrt(w.d)
+    return f32_to_bf16_bits(x.astype(np.float32))
+
+
+def lab_x_all(w: LabWorkload) -> np.ndarray:
+    """Tokens of every step, [steps, T, d] bf16 bits."""
+    return np.stack([lab_x(w, s) for s in range(w.steps)])

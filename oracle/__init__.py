@@ -155,6 +155,77 @@ def bias_update(counts: np.ndarray, bias: np.ndarray, T: int, k: int, gamma: flo
 
 
 # ---------------------------------------------------------------------------
+# §02d: expert capacity -- assignments past an expert's capacity are dropped
+# ---------------------------------------------------------------------------
+def capacity_for(factor: float, T: int, k: int, n_routed: int) -> int:
+    """Capacity of every routed expert: ``factor`` times the ideal load k*T/n_routed,
+    rounded down to a whole number of tokens (the page gives 1.25x the ideal load
+    and no rounding; rounding down keeps the capacity at or below that bound).
+    The factor is taken as the decimal number it prints as, so 1.25 is 5/4 exactly."""
+    from fractions import Fraction
+    return int((Fraction(repr(float(factor))) * k * T) // n_routed)
+
+
+def capacity_keep(topk_idx: np.ndarray, capacity: int, n_routed: int) -> np.ndarray:
+    """keep[t, j]: whether the assignment of token t to expert topk_idx[t, j] is served.
+
+    Each expert serves at most ``capacity`` tokens per batch; its queue is filled
+    in token order, and the assignments that arrive once the queue is full are
+    the overflow, which is dropped (§02d).  A token never picks an expert twice,
+    so within one token the slot order does not matter."""
+    topk_idx = np.asarray(topk_idx)
+    T, k = topk_idx.shape
+    queued = [0] * n_routed
+    keep = np.zeros((T, k), dtype=bool)
+    for t in range(T):
+        for j in range(k):
+            e = int(topk_idx[t, j])
+            keep[t, j] = queued[e] < capacity
+            queued[e] += 1
+    return keep
+
+
+def load_metrics(counts: np.ndarray, capacity: Optional[int], T: int, k: int) -> Dict[str, float]:
+    """Balance metrics of one batch from the loads L_i (the demand: tokens that
+    selected expert i, dropped or not).  MaxVio = max_i L_i / Lbar - 1 with
+    Lbar = k*T/n_routed (the hottest expert's demand over the ideal, minus one);
+    dropped = sum_i max(0, L_i - capacity); drop_rate = dropped / (k*T), the share
+    of expert slots lost to overflow (§02g)."""
+    L = np.asarray(counts, dtype=np.int64)
+    n_routed = L.shape[0]
+    ideal = k * T / n_routed
+    dropped = int(np.maximum(L - capacity, 0).sum()) if capacity is not None else 0
+    return {"max_load": int(L.max()) if L.size else 0, "max_vio": float(L.max() / ideal - 1.0) if T else 0.0,
+            "dropped": dropped, "drop_rate": dropped / (k * T) if T else 0.0}
+
+
+def lab_run(w: "mi.LabWorkload", gamma: float, steps: Optional[int] = None,
+            bias0: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """The Router Balance Lab loop (§02g) for one balancing step size: per step,
+    score the step's tokens with the frozen router, take the biased top-k, count
+    the loads, apply the capacity, record MaxVio and the drop rate, then move the
+    bias (§02e).  gamma = 0 is the lab's no-balancing arm."""
+    steps = w.steps if steps is None else steps
+    wr = mi.lab_wr(w)
+    cap = capacity_for(w.capacity_factor, w.T, w.k, w.n_routed)
+    b = np.zeros(w.n_routed, dtype=np.float32) if bias0 is None else np.asarray(bias0, dtype=np.float32)
+    out = {"max_vio": [], "drop_rate": [], "dropped": [], "counts": [], "bias": [b.copy()], "capacity": cap}
+    for st in range(steps):
+        r = route(logits(mi.lab_x(w, st), wr), b, w.k, w.n_routed, w.n_shared)
+        L = load_counts(r["topk_idx"], w.n_routed)
+        m = load_metrics(L, cap, w.T, w.k)
+        out["max_vio"].append(m["max_vio"])
+        out["drop_rate"].append(m["drop_rate"])
+        out["dropped"].append(m["dropped"])
+        out["counts"].append(L)
+        b = bias_update(L, b, w.T, w.k, gamma)
+        out["bias"].append(b.copy())
+    for key in ("max_vio", "drop_rate", "dropped", "counts", "bias"):
+        out[key] = np.asarray(out[key])
+    return out
+
+
+# ---------------------------------------------------------------------------
 # dispatch (§02: every token goes to exactly its 6 routed experts)
 # ---------------------------------------------------------------------------
 def dispatch(topk_idx: np.ndarray, n_routed: int) -> Dict[str, np.ndarray]:
@@ -253,7 +324,8 @@ def route_workload(w: "mi.Workload", bias: np.ndarray, tokens: Optional[Sequence
 
 def forward_tokens(w: "mi.Workload", tokens: Sequence[int], bias: np.ndarray,
                    logit_offset: Optional[np.ndarray] = None, nthreads: int = 0,
-                   weights: Optional[Dict[str, np.ndarray]] = None) -> Dict[str, np.ndarray]:
+                   weights: Optional[Dict[str, np.ndarray]] = None,
+                   keep: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """The layer's forward for the given tokens of workload w, in fp64.
 
     Tokens are independent in this layer (each token's output depends only on
@@ -261,13 +333,20 @@ def forward_tokens(w: "mi.Workload", tokens: Sequence[int], bias: np.ndarray,
     layer's result on those tokens.  ``weights`` may hold host copies of
     w1 [E, f, d] and w2 [E, d, f]; otherwise each needed expert's matrices are
     generated on demand.
+
+    ``keep`` [len(tokens), k] (from ``capacity_keep`` over the whole batch, since
+    capacity couples the tokens): routed assignments marked False were dropped and
+    contribute nothing; the other gates are left as they are (§02d: a dropped
+    token simply does not get that expert's contribution).
     """
     tokens = np.asarray(tokens, dtype=np.int64)
     x = mi.host_x(w, tokens)
     r = route_workload(w, bias, tokens, logit_offset, x=x, nthreads=nthreads)
     n = len(tokens)
     contrib = r["contrib"]           # [n, k + n_shared] expert ids
-    gates = r["gates"]
+    gates = r["gates"].copy()
+    if keep is not None:
+        gates[:, :w.k] = np.where(np.asarray(keep, dtype=bool), gates[:, :w.k], 0.0)
     out = np.zeros((n, w.d), dtype=np.float64)
     for e in np.unique(contrib):
         rows, slots = np.nonzero(contrib == e)
