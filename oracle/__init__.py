@@ -228,23 +228,26 @@ def lab_run(w: "mi.LabWorkload", gamma: float, steps: Optional[int] = None,
 # ---------------------------------------------------------------------------
 # dispatch (§02: every token goes to exactly its 6 routed experts)
 # ---------------------------------------------------------------------------
-def dispatch(topk_idx: np.ndarray, n_routed: int) -> Dict[str, np.ndarray]:
+def dispatch(topk_idx: np.ndarray, n_routed: int, keep: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Group the T*k (token, slot) pairs by expert, each expert's rows in token order.
 
     offsets [n_routed + 1]: rows of expert e are offsets[e] .. offsets[e+1]-1;
-    row_token [T*k]: the token each row came from; token_row [T, k]: the row
-    each (token, slot) pair went to.
+    row_token [rows]: the token each row came from; token_row [T, k]: the row
+    each (token, slot) pair went to.  With ``keep`` (from ``capacity_keep``) only
+    the served pairs get rows and a dropped pair's token_row is -1.
     """
     topk_idx = np.asarray(topk_idx)
     T, k = topk_idx.shape
     flat = topk_idx.reshape(-1).astype(np.int64)
-    order = np.argsort(flat, kind="stable")  # by expert, then by (token, slot)
-    counts = np.bincount(flat, minlength=n_routed)
+    served = np.ones(T * k, dtype=bool) if keep is None else np.asarray(keep, dtype=bool).reshape(-1)
+    pairs = np.nonzero(served)[0]                              # served (token, slot) pairs, in token order
+    order = pairs[np.argsort(flat[pairs], kind="stable")]      # by expert, then by (token, slot)
+    counts = np.bincount(flat[pairs], minlength=n_routed)
     offsets = np.zeros(n_routed + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts)
     row_token = (order // k).astype(np.int32)
-    token_row = np.empty(T * k, dtype=np.int32)
-    token_row[order] = np.arange(T * k, dtype=np.int32)
+    token_row = np.full(T * k, -1, dtype=np.int32)
+    token_row[order] = np.arange(len(order), dtype=np.int32)
     return {"offsets": offsets.astype(np.int32), "row_token": row_token, "token_row": token_row.reshape(T, k)}
 
 

@@ -59,6 +59,32 @@ def test_keep_invariants():
     assert not oracle.capacity_keep(topk, 0, E).any()
 
 
+def test_dispatch_with_drops():
+    """Only served pairs get rows: expert e has min(L_e, C) rows, its earliest
+    tokens, in token order; dropped pairs point nowhere; with every pair served
+    the layout is the uncapped dispatch."""
+    g = json.load(open(os.path.join(GOLDEN, "capacity_example.json")))
+    topk = np.array(g["topk_idx"], dtype=np.int32)
+    keep = np.array(g["keep"])
+    r = oracle.dispatch(topk, g["n_routed"], keep)
+    assert r["offsets"].tolist() == [0, 2, 4, 6]
+    assert r["row_token"].tolist() == [0, 1, 0, 1, 2, 3]
+    assert r["token_row"].tolist() == [[0, 2], [3, 1], [-1, 4], [5, -1], [-1, -1]]
+    T, k, E = 700, 6, 32
+    topk = _distinct_topk(T, k, E, seed=11)
+    full = oracle.dispatch(topk, E)
+    same = oracle.dispatch(topk, E, np.ones((T, k), dtype=bool))
+    for key in full:
+        assert np.array_equal(full[key], same[key])
+    cap = 100
+    r = oracle.dispatch(topk, E, oracle.capacity_keep(topk, cap, E))
+    L = oracle.load_counts(topk, E)
+    assert np.array_equal(np.diff(r["offsets"]), np.minimum(L, cap))
+    for e in range(E):
+        rows = r["row_token"][r["offsets"][e]:r["offsets"][e + 1]]
+        assert np.array_equal(rows, np.nonzero((topk == e).any(axis=1))[0][:cap])
+
+
 def test_capacity_for():
     assert oracle.capacity_for(1.25, 2048, 6, 64) == 240      # lab: 1.25 x 192
     assert oracle.capacity_for(1.25, 65536, 6, 256) == 1920   # 1.25 x 1536
