@@ -88,7 +88,8 @@ typedef uint16_t moe_bf16;
  *   scores_out [T, n_routed + n_shared] fp32 or NULL: s_i for debugging
  * Logits are accumulated in fp32 from bf16 products (tcgen05 tensor cores);
  * s, s + b and the gates are fp32.
- * Limits: d % 64 == 0, 1 <= top_k <= min(MOE_MAX_TOP_K, n_routed),
+ * Limits: d % 8 == 0 (widths that are not a multiple of 64 are read as zeros
+ * past d), 1 <= top_k <= min(MOE_MAX_TOP_K, n_routed),
  * n_routed <= 256, n_shared <= 8, n_routed + n_shared <= 272.
  */
 int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const float* logit_offset,
@@ -120,6 +121,31 @@ size_t moe_permute_scratch_bytes(int T, int n_routed);
 int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d, int n_routed,
                 int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token, int32_t* token_row, void* scratch,
                 size_t scratch_bytes, void* stream);
+
+/*
+ * moe_permute_capped -- moe_permute with a hard expert capacity.
+ * "Inkling, Dissected" §02d: every expert can process at most a fixed number
+ * of tokens per batch; when more tokens select it, the overflow is dropped and
+ * those tokens get nothing from that expert (the layer output is made of what
+ * remains).  §02g: the capacity is 1.25x the ideal load k*T/n_routed.
+ *
+ * Arguments as moe_permute, plus
+ *   capacity   >= 0: rows each expert serves.  An expert's queue is filled in
+ *              token order; the (t, j) pair whose place in the queue of expert
+ *              topk_idx[t, j] is capacity or later is dropped: token_row[t, j]
+ *              = -1, no row is made for it (moe_combine then skips it, so the
+ *              token's other gates stay as they are).
+ *   offsets    rows of expert e are offsets[e] .. offsets[e+1]-1, with
+ *              offsets[e+1] - offsets[e] = min(L_e, capacity); rows past
+ *              offsets[n_routed] of x_perm and row_token are not written.
+ *   counts     (if given) still the demand L_e, dropped picks included.
+ * capacity >= max L_e gives exactly moe_permute's result.  Negative capacity:
+ * MOE_ERR_INVALID_ARG.  The capacity in tokens is the caller's to choose (the
+ * Python layer takes floor(factor * k*T / n_routed)).
+ */
+int moe_permute_capped(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                       int n_routed, int top_k, int capacity, int32_t* offsets, moe_bf16* x_perm,
+                       int32_t* row_token, int32_t* token_row, void* scratch, size_t scratch_bytes, void* stream);
 
 /*
  * moe_permute_noalloc -- moe_permute for callers that cannot allocate device
@@ -210,7 +236,8 @@ int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* ro
  * contributing experts) and §02b sketch (out += g_k * e_k(x)).
  *
  *   y_perm     [T*top_k, d] bf16 routed expert outputs in dispatch order
- *   token_row  [T, top_k] int32 (from moe_permute)
+ *   token_row  [T, top_k] int32 (from moe_permute or moe_permute_capped); an
+ *              entry of -1 (a dropped assignment) contributes nothing
  *   gates      [T, top_k + n_shared] fp32 (from moe_router_topk)
  *   y_shared   [n_shared, T, d] bf16 or NULL (then n_shared must be 0)
  *   out        [T, d] bf16: out[t] = sum_j g[t,j] y_perm[token_row[t,j]]
@@ -229,6 +256,20 @@ int moe_combine(const moe_bf16* y_perm, const int32_t* token_row, const float* g
  *   counts [n_routed] int32, bias [n_routed] fp32 (in/out).
  */
 int moe_bias_update(const int32_t* counts, int n_routed, int T, int top_k, float gamma, float* bias, void* stream);
+
+/*
+ * moe_load_stats -- the balance of one batch, from the loads alone.
+ * "Inkling, Dissected" §02g (the Router Balance Lab measures MaxVio, the
+ * hottest expert's load over the ideal minus one, and the share of expert
+ * slots dropped) and §02d (what overflows a capacity is dropped).
+ *   counts   [n_routed] int32: L_i (from moe_router_topk)
+ *   capacity >= 0 (tokens per expert)
+ *   stats    [2] int32 out (device): stats[0] = max_i L_i,
+ *            stats[1] = sum_i max(0, L_i - capacity), the dropped assignments.
+ * MaxVio = stats[0] * n_routed / (top_k * T) - 1 and drop rate =
+ * stats[1] / (top_k * T) are left to the caller.  Limits: n_routed <= 256.
+ */
+int moe_load_stats(const int32_t* counts, int n_routed, int capacity, int32_t* stats, void* stream);
 
 /* Human-readable text for a MOE_* return code. */
 const char* moe_status_string(int code);

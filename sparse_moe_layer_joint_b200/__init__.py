@@ -45,6 +45,8 @@ _lib.moe_router_topk.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i3
 _lib.moe_permute_scratch_bytes.argtypes = [_i32, _i32]
 _lib.moe_permute_scratch_bytes.restype = _sz
 _lib.moe_permute.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_permute_capped.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_load_stats.argtypes = [_vp, _i32, _i32, _vp, _vp]
 _lib.moe_permute_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_grouped_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
 _lib.moe_experts_ffn.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp,
@@ -56,7 +58,8 @@ _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_get_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.moe_set_wait_timeout_ns.argtypes = [_u64]
 _lib.moe_debug_bounded_wait.argtypes = [_u64, _vp]
-for _f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_experts_ffn", "moe_combine", "moe_bias_update", "moe_get_status",
+for _f in ("moe_router_topk", "moe_permute", "moe_permute_capped", "moe_permute_noalloc", "moe_grouped_ffn",
+           "moe_experts_ffn", "moe_combine", "moe_bias_update", "moe_load_stats", "moe_get_status",
            "moe_set_wait_timeout_ns", "moe_debug_bounded_wait"):
     getattr(_lib, _f).restype = _i32
 
@@ -128,6 +131,13 @@ def moe_permute(x, topk_idx, counts, T: int, d: int, n_routed: int, top_k: int, 
         _p(token_row), _p(scratch), scratch_bytes, _stream(stream)))
 
 
+def moe_permute_capped(x, topk_idx, counts, T: int, d: int, n_routed: int, top_k: int, capacity: int, offsets,
+                       x_perm, row_token, token_row, scratch, scratch_bytes: int, stream=None):
+    _check("moe_permute_capped", _lib.moe_permute_capped(
+        _p(x), _p(topk_idx), _p(counts), T, d, n_routed, top_k, capacity, _p(offsets), _p(x_perm), _p(row_token),
+        _p(token_row), _p(scratch), scratch_bytes, _stream(stream)))
+
+
 def moe_permute_noalloc(x, topk_idx, counts, T: int, d: int, n_routed: int, top_k: int, offsets, x_perm, row_token,
                         token_row, stream=None):
     """moe_permute without a scratch argument, for callers that cannot allocate
@@ -161,6 +171,17 @@ def moe_combine(y_perm, token_row, gates, y_shared, T: int, d: int, top_k: int, 
 
 def moe_bias_update(counts, n_routed: int, T: int, top_k: int, gamma: float, bias, stream=None):
     _check("moe_bias_update", _lib.moe_bias_update(_p(counts), n_routed, T, top_k, gamma, _p(bias), _stream(stream)))
+
+
+def moe_load_stats(counts, n_routed: int, capacity: int, stats, stream=None):
+    _check("moe_load_stats", _lib.moe_load_stats(_p(counts), n_routed, capacity, _p(stats), _stream(stream)))
+
+
+def capacity_for(factor: float, T: int, k: int, n_routed: int) -> int:
+    """Expert capacity in tokens: floor(factor * k*T / n_routed), with the factor
+    read as the decimal it prints as (1.25 = 5/4)."""
+    from fractions import Fraction
+    return int((Fraction(repr(float(factor))) * (k * T)) // n_routed)
 
 
 def moe_get_status(stream=None) -> int:
@@ -202,10 +223,13 @@ class MoELayer:
     bias [n_routed] fp32 (updated in place by ``bias_update``).
     """
 
-    def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True, gather_rows: bool = False):
+    def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True, gather_rows: bool = False,
+                 capacity_factor: Optional[float] = None):
         import torch
 
         self.shape = s = shape
+        # hard expert capacity (tokens per expert per batch); None: every assignment is served
+        self.capacity = None if capacity_factor is None else capacity_for(capacity_factor, s.T, s.top_k, s.n_routed)
         self.fused_experts = fused_experts
         # with the fused experts, GEMM1 can gather the routed rows from x itself (no x_perm copy);
         # measured slower on B200 at every workload here (32 row gathers per stage bound the TMA
@@ -229,6 +253,7 @@ class MoELayer:
         self.h_shared = torch.empty((max(s.n_shared, 1), s.T, s.d_ff), dtype=bf, device=dev)
         self.y_shared = torch.empty((max(s.n_shared, 1), s.T, s.d), dtype=bf, device=dev)
         self.out = torch.empty((s.T, s.d), dtype=bf, device=dev)
+        self.stats = torch.zeros((2,), dtype=torch.int32, device=dev)
         self.side = torch.cuda.Stream(device=dev)
         self.ev_start = torch.cuda.Event()
         self.ev_shared = torch.cuda.Event()
@@ -258,8 +283,12 @@ class MoELayer:
                             self.y_shared, stream=self.side)
             self.ev_shared.record(self.side)
         x_perm = None if self.gather_rows else self.x_perm
-        moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, x_perm, self.row_token,
-                    self.token_row, self.scratch, self.scratch_bytes, stream=main)
+        if self.capacity is None:
+            moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, x_perm, self.row_token,
+                        self.token_row, self.scratch, self.scratch_bytes, stream=main)
+        else:
+            moe_permute_capped(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.capacity, self.offsets,
+                               x_perm, self.row_token, self.token_row, self.scratch, self.scratch_bytes, stream=main)
         if ffn_events is not None:
             ffn_events[0].record(main)
         if self.fused_experts:
@@ -283,6 +312,19 @@ class MoELayer:
         experts = 2 if self.fused_experts else 4
         permute = 3 if self.gather_rows else 4
         return 1 + permute + experts + 1 + 1
+
+    def balance(self, stream=None) -> dict:
+        """MaxVio and drop rate of the last forward's loads (synchronises the stream)."""
+        import torch
+
+        s = self.shape
+        cap = self.capacity if self.capacity is not None else 2 ** 31 - 1
+        st = stream if stream is not None else torch.cuda.current_stream()
+        moe_load_stats(self.counts, s.n_routed, cap, self.stats, stream=st)
+        max_load, dropped = (int(v) for v in self.stats.cpu().tolist())
+        kT = s.top_k * s.T
+        return {"max_load": max_load, "dropped": dropped, "max_vio": max_load * s.n_routed / kT - 1.0 if kT else 0.0,
+                "drop_rate": dropped / kT if kT else 0.0}
 
     def bias_update(self, bias, gamma: float, stream=None, T_total: Optional[int] = None):
         """b += gamma * sign(Lbar - L) from this layer's counts; T_total: the batch's token

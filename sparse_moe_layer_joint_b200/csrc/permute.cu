@@ -5,12 +5,17 @@
 // Four launches, all deterministic (no atomics decide a position):
 //   1. chunk_hist   one CTA per 256-token chunk: hist[c][e] = picks of e in chunk c
 //   2. chunk_scan   one CTA: offsets[e] = exclusive scan over experts of the
-//                   per-expert totals; base[c][e] = offsets[e] + picks of e in
-//                   chunks before c; optional check of the caller's counts
+//                   rows each expert serves, min(picks, capacity);
+//                   base[c][e] = picks of e in chunks before c; optional check
+//                   of the caller's counts
 //   3. rank         one CTA per chunk: each warp takes 32 tokens; a per-warp
 //                   bitmask per expert (bit = lane) gives each pick its rank
 //                   among earlier lanes, a prefix over the 8 warps its rank
-//                   among earlier warps -> token_row, row_token
+//                   among earlier warps.  A pick whose rank in its expert's
+//                   queue (token order) reaches the capacity is dropped
+//                   (§02d: overflow tokens get nothing from that expert):
+//                   token_row = -1 and no row; otherwise row offsets[e] + rank
+//                   -> token_row, row_token
 //   4. copy_rows    grid-wide over (token, 256-vector slice) units: each x
 //                   slice is read once with 16-byte loads and written to the
 //                   token's k rows.
@@ -53,10 +58,10 @@ __global__ void __launch_bounds__(THREADS) chunk_hist_kernel(const int32_t* __re
 
 // One CTA of 256 threads; thread e owns expert e.
 __global__ void __launch_bounds__(THREADS) chunk_scan_kernel(const int32_t* __restrict__ hist, int n_chunks,
-                                                             int n_routed, const int32_t* __restrict__ counts,
+                                                             int n_routed, int capacity,
+                                                             const int32_t* __restrict__ counts,
                                                              int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ base, unsigned int* status) {
-  __shared__ int tot[MOE_MAX_ROUTED];
   __shared__ int warp_sum[WARPS];
   const int e = threadIdx.x;
   int total = 0;
@@ -64,9 +69,10 @@ __global__ void __launch_bounds__(THREADS) chunk_scan_kernel(const int32_t* __re
     for (int c = 0; c < n_chunks; ++c) total += hist[(size_t)c * n_routed + e];
     if (counts != nullptr && counts[e] != total) set_status(status, MOE_STATUS_COUNT_MISMATCH);
   }
-  // exclusive scan of totals over experts
+  const int served = total < capacity ? total : capacity;
+  // exclusive scan of the served rows over experts
   const int lane = e & 31, w = e >> 5;
-  int v = total;
+  int v = served;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     int u = __shfl_up_sync(0xffffffffu, v, o);
@@ -76,13 +82,11 @@ __global__ void __launch_bounds__(THREADS) chunk_scan_kernel(const int32_t* __re
   __syncthreads();
   int before = 0;
   for (int i = 0; i < w; ++i) before += warp_sum[i];
-  const int excl = before + v - total;
-  tot[e] = excl;
+  const int excl = before + v - served;
   if (e < n_routed) offsets[e] = excl;
-  if (e == n_routed - 1) offsets[n_routed] = excl + total;
-  __syncthreads();
+  if (e == n_routed - 1) offsets[n_routed] = excl + served;
   if (e < n_routed) {
-    int run = tot[e];
+    int run = 0;
     for (int c = 0; c < n_chunks; ++c) {
       base[(size_t)c * n_routed + e] = run;
       run += hist[(size_t)c * n_routed + e];
@@ -91,11 +95,13 @@ __global__ void __launch_bounds__(THREADS) chunk_scan_kernel(const int32_t* __re
 }
 
 __global__ void __launch_bounds__(THREADS) rank_kernel(const int32_t* __restrict__ topk_idx,
-                                                       const int32_t* __restrict__ base, int T, int k, int n_routed,
-                                                       int32_t* __restrict__ row_token,
+                                                       const int32_t* __restrict__ base,
+                                                       const int32_t* __restrict__ offsets, int T, int k,
+                                                       int n_routed, int capacity, int32_t* __restrict__ row_token,
                                                        int32_t* __restrict__ token_row) {
   __shared__ uint32_t mask[WARPS][MOE_MAX_ROUTED];
   __shared__ int pre[WARPS][MOE_MAX_ROUTED];
+  __shared__ int off[MOE_MAX_ROUTED];
   const int c = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < WARPS * MOE_MAX_ROUTED; i += THREADS) (&mask[0][0])[i] = 0u;
@@ -117,6 +123,7 @@ __global__ void __launch_bounds__(THREADS) rank_kernel(const int32_t* __restrict
   __syncthreads();
   // prefix over warps, per expert
   for (int e = threadIdx.x; e < n_routed; e += THREADS) {
+    off[e] = offsets[e];
     int run = base[(size_t)c * n_routed + e];
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) {
@@ -129,9 +136,10 @@ __global__ void __launch_bounds__(THREADS) rank_kernel(const int32_t* __restrict
 #pragma unroll
   for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
     if (ex[j] >= 0) {
-      const int pos = pre[warp][ex[j]] + __popc(mask[warp][ex[j]] & lt);
+      const int rank = pre[warp][ex[j]] + __popc(mask[warp][ex[j]] & lt);  // place in the expert's queue
+      const int pos = rank < capacity ? off[ex[j]] + rank : -1;
       token_row[(size_t)t * k + j] = pos;
-      row_token[pos] = t;
+      if (pos >= 0) row_token[pos] = t;
     } else if (j < k && valid) {
       token_row[(size_t)t * k + j] = -1;
     }
@@ -160,10 +168,10 @@ __global__ void __launch_bounds__(THREADS) copy_rows_kernel(const uint4* __restr
   }
 }
 
-// The launches shared by moe_permute and moe_permute_noalloc.
+// The launches shared by moe_permute, moe_permute_capped and moe_permute_noalloc.
 static int launch_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
-                          int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
-                          int32_t* token_row, void* scratch, cudaStream_t s) {
+                          int n_routed, int top_k, int capacity, int32_t* offsets, moe_bf16* x_perm,
+                          int32_t* row_token, int32_t* token_row, void* scratch, cudaStream_t s) {
   unsigned int* status = status_ptr();
   if (!status) return MOE_ERR_CUDA;
   int dev, sms;
@@ -173,8 +181,9 @@ static int launch_permute(const moe_bf16* x, const int32_t* topk_idx, const int3
   int32_t* hist = reinterpret_cast<int32_t*>(scratch);
   int32_t* base = hist + (size_t)n_chunks * n_routed;
   chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
-  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, counts, offsets, base, status);
-  rank_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, base, T, top_k, n_routed, row_token, token_row);
+  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, capacity, counts, offsets, base, status);
+  rank_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, base, offsets, T, top_k, n_routed, capacity, row_token,
+                                           token_row);
   if (x_perm == nullptr) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;  // indices only
   const int d_vec = d / 8;
   const long long units = (long long)T * ((d_vec + THREADS - 1) / THREADS);
@@ -195,11 +204,12 @@ extern "C" size_t moe_permute_scratch_bytes(int T, int n_routed) {
   return 2 * n_chunks * (size_t)n_routed * sizeof(int32_t) + 256;
 }
 
-extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
-                           int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
-                           int32_t* token_row, void* scratch, size_t scratch_bytes, void* stream) {
+static int permute_entry(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                         int n_routed, int top_k, int capacity, int32_t* offsets, moe_bf16* x_perm,
+                         int32_t* row_token, int32_t* token_row, void* scratch, size_t scratch_bytes,
+                         void* stream) {
   using namespace moe::perm;
-  if (T < 0 || d <= 0 || n_routed < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || d <= 0 || n_routed < 1 || top_k < 1 || capacity < 0) return MOE_ERR_INVALID_ARG;
   if (top_k > MOE_MAX_TOP_K || top_k > n_routed || n_routed > MOE_MAX_ROUTED) return MOE_ERR_INVALID_ARG;
   if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (!topk_idx || !offsets || !row_token || !token_row || !scratch || (x_perm && !x)) return MOE_ERR_INVALID_ARG;
@@ -213,8 +223,23 @@ extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int
     if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (n_routed + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  return launch_permute(x, topk_idx, counts, T, d, n_routed, top_k, offsets, x_perm, row_token, token_row, scratch,
-                        s);
+  return launch_permute(x, topk_idx, counts, T, d, n_routed, top_k, capacity, offsets, x_perm, row_token,
+                        token_row, scratch, s);
+}
+
+extern "C" int moe_permute(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                           int n_routed, int top_k, int32_t* offsets, moe_bf16* x_perm, int32_t* row_token,
+                           int32_t* token_row, void* scratch, size_t scratch_bytes, void* stream) {
+  return permute_entry(x, topk_idx, counts, T, d, n_routed, top_k, 0x7fffffff, offsets, x_perm, row_token,
+                       token_row, scratch, scratch_bytes, stream);
+}
+
+extern "C" int moe_permute_capped(const moe_bf16* x, const int32_t* topk_idx, const int32_t* counts, int T, int d,
+                                  int n_routed, int top_k, int capacity, int32_t* offsets, moe_bf16* x_perm,
+                                  int32_t* row_token, int32_t* token_row, void* scratch, size_t scratch_bytes,
+                                  void* stream) {
+  return permute_entry(x, topk_idx, counts, T, d, n_routed, top_k, capacity, offsets, x_perm, row_token,
+                       token_row, scratch, scratch_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -275,6 +300,6 @@ extern "C" int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, c
   }
   // Every part of the scratch that is read is written first in the same call
   // (hist by chunk_hist, base by chunk_scan), so nothing needs clearing.
-  return launch_permute(x, topk_idx, counts, T, d, n_routed, top_k, offsets, x_perm, row_token, token_row, scratch,
-                        s);
+  return launch_permute(x, topk_idx, counts, T, d, n_routed, top_k, 0x7fffffff, offsets, x_perm, row_token,
+                        token_row, scratch, s);
 }

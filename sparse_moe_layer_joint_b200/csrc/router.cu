@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int S = p.ksplit;
   const uint32_t crank = S > 1 ? cluster_ctarank() : 0u;
   const int m0 = (blockIdx.x / S) * BM;
-  const int kb_per = (p.d / BK) / S;
+  const int kb_per = ((p.d + BK - 1) / BK) / S;  // a last partial block is read as zeros past d
   const int kb0 = (int)crank * kb_per;
 
   if (tid == 0) {
@@ -590,7 +590,7 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   if (route_scale != 1.0f) return MOE_ERR_UNSUPPORTED;
   if (n_routed > MOE_MAX_ROUTED || n_shared > MOE_MAX_SHARED || n_routed + n_shared > B0_ROWS + B1_ROWS)
     return MOE_ERR_UNSUPPORTED;
-  if (d % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;  // 16-byte row pitch for the tensor map
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * n_routed, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (T == 0) return MOE_OK;
@@ -612,7 +612,7 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   p.d = d;
   p.n_routed = n_routed;
   p.n_shared = n_shared;
-  p.ksplit = choose_ksplit(n_mtiles, d / BK, sms);
+  p.ksplit = choose_ksplit(n_mtiles, (d + BK - 1) / BK, sms);
   p.topk_idx = topk_idx;
   p.gates = gates;
   p.counts = counts;

@@ -71,6 +71,8 @@ def test_router_worked_example(case):
 @pytest.mark.parametrize("T,d,n_routed,n_shared,k", [
     (1, 64, 256, 2, 6), (7, 128, 256, 2, 6), (300, 256, 256, 2, 6), (1000, 512, 256, 2, 6),
     (200, 64, 8, 2, 3), (130, 192, 64, 0, 2), (129, 128, 256, 8, 8), (256, 64, 16, 1, 1),
+    # widths that are not a multiple of 64 (the last K block is read as zeros past d)
+    (2048, 32, 64, 0, 6), (300, 96, 256, 2, 6), (129, 8, 16, 2, 4), (1000, 200, 256, 2, 6),
 ])
 def test_router_parity(T, d, n_routed, n_shared, k):
     E = n_routed + n_shared
