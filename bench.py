@@ -131,7 +131,7 @@ def run_ours(args, w, rank, world, local_rank):
         mi.gpu_normal_bf16(t["x"].data_ptr(), t["x"].numel(), w.seed, mi.STREAM_X, rank * w.T * w.d, w.std_x,
                            stream.cuda_stream)
     layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev,
-                         gather_rows=args.gather_rows)
+                         gather_rows=args.gather_rows, capacity_factor=args.capacity_factor)
     bias0 = t["bias"].clone()
     ffn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
@@ -172,11 +172,15 @@ def run_ours(args, w, rank, world, local_rank):
     # step touched: the expert GEMMs read only those experts' weights
     t["bias"].copy_(bias_at_start)
     local_counts = torch.empty((args.steps, w.n_routed), dtype=torch.int32, device=dev)
+    served = []
     for i in range(args.steps):
         layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
         local_counts[i].copy_(layer.counts)
+        if layer.capacity is not None:
+            served.append(w.T * w.k - layer.balance()["dropped"])
         dp.bias_step(layer, t["bias"], w.gamma)
     touched = (local_counts > 0).sum(dim=1).double().mean().item()
+    routed_rows = statistics.mean(served) if served else w.T * w.k   # rows the expert GEMMs compute
 
     # end to end through the public API: every step copies its x in from pinned host memory and
     # its output back to pinned host memory.  Like a serving loop, the copies of neighbouring steps
@@ -239,7 +243,7 @@ def run_ours(args, w, rank, world, local_rank):
     # touched routed experts and the shared experts + A rows read + hidden written and read
     # + outputs written (bf16)
     pk = peaks()
-    rows = w.T * (w.k + w.n_shared)
+    rows = routed_rows + w.T * w.n_shared
     ffn_flops = 2 * 2.0 * rows * w.d * w.f
     ffn_bytes = ((touched + w.n_shared) * 2 * w.d * w.f * 2
                  + rows * w.d * 2 + rows * w.f * 2 * 2 + rows * w.d * 2)
@@ -259,13 +263,17 @@ def run_ours(args, w, rank, world, local_rank):
                 "ms_per_launch_pair": round(ffn_ms, 4)}
     weight_bound = w.name in ("decode", "mid")
     roofline = hbm_roof if weight_bound else tensor_roof
-    roofline["layer_tflops"] = round(w.flops() / (ms * 1e-3) / 1e12, 1)
+    layer_flops = w.flops() - 2.0 * 2.0 * (w.T * w.k - routed_rows) * w.d * w.f
+    roofline["layer_tflops"] = round(layer_flops / (ms * 1e-3) / 1e12, 1)
     line = {
         "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox, random-init weights)",
         "config": dict(config_of(w, world), dispatch="rows gathered by GEMM1 (cp.async)" if args.gather_rows
-                       else "rows copied by moe_permute"), "clocks": clk,
+                       else "rows copied by moe_permute",
+                       **({"capacity_factor": args.capacity_factor, "capacity": layer.capacity,
+                           "served_routed_rows_mean": round(routed_rows, 1)} if layer.capacity is not None else {})),
+        "clocks": clk,
         "e2e": {"value": round(world * w.T / (e2e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": w.T * w.d * 2, "d2h_bytes_per_step": w.T * w.d * 2,
                 "ms_per_step": round(e2e_ms, 4),
@@ -276,6 +284,127 @@ def run_ours(args, w, rank, world, local_rank):
     }
     del bias0
     return line
+
+
+# ---------------------------------------------------------------------------
+# the Router Balance Lab loop ("Inkling, Dissected" §02g): routing only
+# ---------------------------------------------------------------------------
+LAB_METRIC = "Router Balance Lab routing step tokens/s on 1 B200 (router + capped dispatch + load stats + bias update)"
+
+
+def run_lab(args):
+    import torch
+
+    import sparse_moe_layer_joint_b200 as moe
+
+    w = mi.LAB
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    cap = moe.capacity_for(w.capacity_factor, w.T, w.k, w.n_routed)
+    x_host = torch.from_numpy(mi.lab_x_all(w).view(np.int16)).view(torch.bfloat16)   # [steps, T, d]
+    xs = x_host.to(dev)
+    wr = torch.from_numpy(mi.lab_wr(w).view(np.int16)).view(torch.bfloat16).to(dev)
+    b = torch.zeros(w.n_routed, dtype=torch.float32, device=dev)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
+    g = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
+    c = torch.empty(w.n_routed, dtype=torch.int32, device=dev)
+    off = torch.empty(w.n_routed + 1, dtype=torch.int32, device=dev)
+    rt = torch.empty(w.T * w.k, dtype=torch.int32, device=dev)
+    tr = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
+    nb = moe.moe_permute_scratch_bytes(w.T, w.n_routed)
+    scratch = torch.empty(nb, dtype=torch.uint8, device=dev)
+    n_steps = w.steps
+    stats = torch.empty((n_steps, 2), dtype=torch.int32, device=dev)
+
+    def step(i, x=None):
+        j = i % n_steps
+        moe.moe_router_topk(xs[j] if x is None else x, wr, b, None, w.T, w.d, w.n_routed, 0, w.k, 1.0, idx, g, c)
+        moe.moe_permute_capped(None, idx, c, w.T, w.d, w.n_routed, w.k, cap, off, None, rt, tr, scratch, nb)
+        moe.moe_load_stats(c, w.n_routed, cap, stats[j])
+        moe.moe_bias_update(c, w.n_routed, w.T, w.k, args.gamma, b)
+
+    # the balance of one full run from b = 0 (the lab's 100 steps), outside the timing
+    for i in range(n_steps):
+        step(i)
+    torch.cuda.synchronize()
+    st = stats.cpu().numpy().astype(np.float64)
+    kT = w.k * w.T
+    late = slice(n_steps // 2, None)
+    balance = {"gamma": args.gamma, "capacity": cap,
+               "max_vio_late_mean": round(float((st[late, 0] * w.n_routed / kT - 1).mean()), 4),
+               "drop_rate_late_mean": round(float((st[late, 1] / kT).mean()), 5),
+               "max_vio_first_step": round(float(st[0, 0] * w.n_routed / kT - 1), 4)}
+    b.zero_()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    # end to end: each step copies its tokens in from pinned host memory and reads its two load
+    # statistics back (the step's result a caller would log)
+    x_pin = x_host.pin_memory()
+    x_dev = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=dev)
+    st_host = torch.empty((2,), dtype=torch.int32).pin_memory()
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for i in range(args.steps):
+        x_dev.copy_(x_pin[i % n_steps], non_blocking=True)
+        step(i, x_dev)
+        st_host.copy_(stats[i % n_steps], non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e2.elapsed_time(e3) / args.steps
+    if moe.moe_get_status() != 0:
+        raise RuntimeError("device status after the lab run")
+    # algorithmic bytes of one step: x and W_r read, top-k/gates written, top-k read twice by the
+    # dispatch, its indices written (everything else is a few KB)
+    step_bytes = (w.T * w.d * 2 + w.n_routed * w.d * 2 + w.T * w.k * (4 + 4) + 2 * w.T * w.k * 4
+                  + w.T * w.k * 4 * 2)
+    pk = peaks()
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    return {
+        "metric": LAB_METRIC, "value": round(w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox: Zipf-lumpy jittered tokens, frozen random router)",
+        "config": lab_config(),
+        "clocks": clk,
+        "e2e": {"value": round(w.T / (e2e_ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": w.T * w.d * 2,
+                "d2h_bytes_per_step": 8, "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": 6 * args.steps,
+        "roofline": {"kernel": "whole routing step (6 launches)", "bound": "hbm", "achieved": round(gbs, 2),
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 6), "traffic": None,
+                     "note": "a 2048-token step moves ~0.4 MB: launch latency, not bandwidth, bounds it"},
+        "balance": balance,
+    }
+
+
+def lab_config():
+    w = mi.LAB
+    return {"workload": "lab", "description": w.description, "T": w.T, "d": w.d, "n_routed": w.n_routed,
+            "top_k": w.k, "capacity_factor": w.capacity_factor, "steps_per_run": w.steps,
+            "l2": "not flushed: the whole lab (13 MB of tokens) is L2-resident; latency-bound"}
+
+
+def lab_cpu(args, steps):
+    import oracle
+
+    w = mi.LAB
+    t0 = time.perf_counter()
+    r = oracle.lab_run(w, args.gamma, steps=steps)
+    dt = time.perf_counter() - t0
+    return dt, r
 
 
 # ---------------------------------------------------------------------------
@@ -410,7 +539,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS) + ["lab"])
+    ap.add_argument("--capacity-factor", type=float, default=None,
+                    help="hard expert capacity, as a multiple of the ideal load k*T/n_routed (overflow dropped)")
+    ap.add_argument("--gamma", type=float, default=0.01, help="bias step of the lab workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gather-rows", action="store_true",
@@ -423,6 +555,32 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload == "lab":
+        if rank == 0:
+            if args.impl == "reference":
+                k = max(1, min(args.steps, 20))
+                dt, _ = lab_cpu(args, k)
+                v = round(mi.LAB.T * k / dt, 1)
+                print(json.dumps({
+                    "impl": "reference", "metric": LAB_METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
+                    "steps": k, "warmup": 0, "ms_per_step": round(dt / k * 1e3, 3), "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                    "data": "synthetic (seeded Philox: Zipf-lumpy jittered tokens, frozen random router)",
+                    "config": lab_config(),
+                    "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                     "sample": f"{k} lab steps through the fp64 oracle"},
+                    "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+            else:
+                if world > 1:
+                    raise SystemExit("the lab workload runs on one GPU")
+                line = run_lab(args)
+                if not args.no_cpu_baseline:
+                    dt, _ = lab_cpu(args, 20)
+                    line["cpu_baseline"] = {"value": round(mi.LAB.T * 20 / dt, 1), "unit": UNIT, "cores": 1,
+                                            "kind": "oracle", "sample": f"20 lab steps through the fp64 oracle, "
+                                                                         f"wall {dt:.2f} s"}
+                print(json.dumps(line), flush=True)
+        return
     w = mi.WORKLOADS[args.workload]
 
     if args.kernel_case is not None:
