@@ -22,6 +22,8 @@ mid         4096    2048  768    b = 0
 skew        16384   4096  1024   Zipf(s=1.1)-ranked logit offset; 20 bias updates
 decode      64      7168  2048   b ~ U(-0.05, 0.05); weight-streaming bound
 prefill     65536   7168  2048   b ~ U(-0.05, 0.05); about 15 GB of expert weights
+inkling     65536   6144  3072   SwiGLU experts, route_scale 8; about 29 GB of weights
+inkling_decode 64   6144  3072   the same layer at decode scale
 =========  ======  ====  =====  ==================================================
 
 x ~ N(0, 1); router and first-layer expert weights ~ N(0, 1/d); second-layer
@@ -78,10 +80,21 @@ class Workload:
     bias_iters: int = 1
     skew: bool = False
     description: str = ""
+    activation: str = "gelu_tanh"   # or "swiglu": W1 holds the gate rows, then the up rows
+    route_scale: float = 1.0        # the released config's route_scale
+    global_scale: float = 1.0       # its learned scalar (no trained value here: 1)
 
     @property
     def n_experts(self) -> int:
         return self.n_routed + self.n_shared
+
+    @property
+    def w1_rows(self) -> int:
+        return 2 * self.f if self.activation == "swiglu" else self.f
+
+    @property
+    def gate_scale(self) -> float:
+        return self.route_scale * self.global_scale
 
     @property
     def std_x(self) -> float:
@@ -103,7 +116,8 @@ class Workload:
         """Algorithmic FLOPs of one layer forward: router GEMM + 2 expert GEMMs
         over the T*k routed and T*n_shared shared (token, expert) rows."""
         rows = self.T * (self.k + self.n_shared)
-        return 2.0 * self.T * self.d * self.n_experts + 2.0 * 2.0 * self.d * self.f * rows
+        mats = 3 if self.activation == "swiglu" else 2
+        return 2.0 * self.T * self.d * self.n_experts + 2.0 * mats * self.d * self.f * rows
 
 
 WORKLOADS = {
@@ -117,6 +131,15 @@ WORKLOADS = {
                        description="decode-scale: T=64, d=7168, d_ff=2048"),
     "prefill": Workload("prefill", 65536, 7168, 2048, b_half_width=0.05,
                         description="prefill-scale: T=65536, d=7168, d_ff=2048"),
+    # the released Inkling configuration ("Under the hood": hidden 6144, SwiGLU experts of
+    # intermediate 3072, route_scale 8 times a learned global_scale)
+    "inkling": Workload("inkling", 65536, 6144, 3072, b_half_width=0.05, activation="swiglu", route_scale=8.0,
+                        description="Inkling config, prefill-scale: T=65536, d=6144, SwiGLU d_ff=3072, "
+                                    "route_scale 8"),
+    "inkling_decode": Workload("inkling_decode", 64, 6144, 3072, b_half_width=0.05, activation="swiglu",
+                               route_scale=8.0,
+                               description="Inkling config, decode-scale: T=64, d=6144, SwiGLU d_ff=3072, "
+                                           "route_scale 8"),
 }
 
 ZIPF_S = 1.1
@@ -274,8 +297,10 @@ def host_wr(w: Workload) -> np.ndarray:
 
 
 def host_w1(w: Workload, e: int) -> np.ndarray:
-    """Expert e's first matrix [d_ff, d] (K-major), bf16 bits."""
-    return normal_bf16(w.f * w.d, w.seed, STREAM_W1, e * w.f * w.d, w.std_w1).reshape(w.f, w.d)
+    """Expert e's first matrix [d_ff, d] (K-major), bf16 bits; [2 d_ff, d] (gate rows,
+    then up rows) for SwiGLU experts."""
+    r = w.w1_rows
+    return normal_bf16(r * w.d, w.seed, STREAM_W1, e * r * w.d, w.std_w1).reshape(r, w.d)
 
 
 def host_w2(w: Workload, e: int) -> np.ndarray:
@@ -284,7 +309,8 @@ def host_w2(w: Workload, e: int) -> np.ndarray:
 
 
 def host_w1_all(w: Workload) -> np.ndarray:
-    return normal_bf16(w.n_experts * w.f * w.d, w.seed, STREAM_W1, 0, w.std_w1).reshape(w.n_experts, w.f, w.d)
+    r = w.w1_rows
+    return normal_bf16(w.n_experts * r * w.d, w.seed, STREAM_W1, 0, w.std_w1).reshape(w.n_experts, r, w.d)
 
 
 def host_w2_all(w: Workload) -> np.ndarray:
@@ -365,7 +391,7 @@ def torch_workload(w: Workload, device="cuda", with_weights: bool = True):
     gpu_normal_bf16(wr.data_ptr(), wr.numel(), w.seed, STREAM_WR, 0, w.std_wr, s)
     out["w_r"] = wr
     if with_weights:
-        w1 = torch.empty((w.n_experts, w.f, w.d), dtype=torch.bfloat16, device=dev)
+        w1 = torch.empty((w.n_experts, w.w1_rows, w.d), dtype=torch.bfloat16, device=dev)
         gpu_normal_bf16(w1.data_ptr(), w1.numel(), w.seed, STREAM_W1, 0, w.std_w1, s)
         w2 = torch.empty((w.n_experts, w.d, w.f), dtype=torch.bfloat16, device=dev)
         gpu_normal_bf16(w2.data_ptr(), w2.numel(), w.seed, STREAM_W2, 0, w.std_w2, s)

@@ -64,6 +64,9 @@ def lib():
         L.or_gelu_tanh.argtypes = [vp, i64, vp]
         L.or_expert_mlp.argtypes = [vp, i64, vp, vp, i64, i64, vp, i32]
         L.or_expert_mlp_f64.argtypes = [vp, i64, vp, vp, i64, i64, vp, i32]
+        L.or_silu.argtypes = [vp, i64, vp]
+        L.or_expert_swiglu.argtypes = [vp, i64, vp, vp, i64, i64, vp, i32]
+        L.or_expert_swiglu_f64.argtypes = [vp, i64, vp, vp, i64, i64, vp, i32]
         _lib = L
     return _lib
 
@@ -92,7 +95,7 @@ def sigmoid(z: np.ndarray) -> np.ndarray:
 
 
 def route(z: np.ndarray, bias: np.ndarray, k: int, n_routed: int, n_shared: int,
-          logit_offset: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+          logit_offset: Optional[np.ndarray] = None, route_scale: float = 1.0) -> Dict[str, np.ndarray]:
     """Biased top-k selection and joint gates from router logits.
 
     z [T, n_routed + n_shared] fp64 logits; bias [n_routed] (fp32 values).
@@ -103,6 +106,10 @@ def route(z: np.ndarray, bias: np.ndarray, k: int, n_routed: int, n_shared: int,
     index), gates [T, k + n_shared] fp64 (the k routed in topk order, then the
     shared experts in index order), s [T, E], sel [T, n_routed] = s + b and
     margin [T] = sel of the k-th minus sel of the (k+1)-th candidate.
+
+    ``route_scale``: the jointly normalised weights are multiplied by it ("Under
+    the hood", "The routing strategy", step 5: route_scale times the learned
+    global_scale; the caller passes the product).  1 leaves gates summing to 1.
     """
     z = np.array(z, dtype=np.float64)
     T, E = z.shape
@@ -127,7 +134,7 @@ def route(z: np.ndarray, bias: np.ndarray, k: int, n_routed: int, n_shared: int,
     # the denominator is a sum over a set: add its terms in ascending expert
     # index, so the gates depend on which experts are kept, not on their rank
     den = np.take_along_axis(s, np.sort(contrib, axis=1), axis=1).sum(axis=1, keepdims=True)
-    gates = s_c / den
+    gates = s_c / den * float(route_scale)
     return {"topk_idx": topk.astype(np.int32), "gates": gates, "s": s, "sel": sel, "margin": margin,
             "contrib": contrib.astype(np.int32)}
 
@@ -289,6 +296,47 @@ def expert_f64(xrows: np.ndarray, w1: np.ndarray, w2: np.ndarray, nthreads: int 
     return y
 
 
+def silu(u: np.ndarray) -> np.ndarray:
+    u = _c(u, np.float64)
+    out = np.empty_like(u)
+    lib().or_silu(u.ctypes.data, u.size, out.ctypes.data)
+    return out
+
+
+def expert_swiglu(xrows_bf16: np.ndarray, w1_bf16: np.ndarray, w2_bf16: np.ndarray, nthreads: int = 0) -> np.ndarray:
+    """The gated expert of the released configuration ("Under the hood", "MoE: the
+    expert configuration": SwiGLU experts), y[r] = W2 . (silu(Wg . x_r) * (Wu . x_r))
+    in fp64; W1 [2 d_ff, d] holds Wg (rows 0..d_ff-1) then Wu, W2 [d, d_ff] (bf16 bits)."""
+    x = _c(xrows_bf16, np.uint16)
+    w1 = _c(w1_bf16, np.uint16)
+    w2 = _c(w2_bf16, np.uint16)
+    n, d = x.shape
+    f = w2.shape[1]
+    assert w1.shape == (2 * f, d) and w2.shape == (d, f)
+    y = np.zeros((n, d), dtype=np.float64)
+    if n:
+        lib().or_expert_swiglu(x.ctypes.data, n, w1.ctypes.data, w2.ctypes.data, d, f, y.ctypes.data, nthreads)
+    return y
+
+
+def expert_swiglu_f64(xrows: np.ndarray, w1: np.ndarray, w2: np.ndarray, nthreads: int = 0) -> np.ndarray:
+    x = _c(xrows, np.float64)
+    w1 = _c(w1, np.float64)
+    w2 = _c(w2, np.float64)
+    n, d = x.shape
+    f = w2.shape[1]
+    assert w1.shape == (2 * f, d) and w2.shape == (d, f)
+    y = np.zeros((n, d), dtype=np.float64)
+    if n:
+        lib().or_expert_swiglu_f64(x.ctypes.data, n, w1.ctypes.data, w2.ctypes.data, d, f, y.ctypes.data, nthreads)
+    return y
+
+
+def expert_for(w: "mi.Workload"):
+    """The expert function of a workload's activation."""
+    return expert_swiglu if getattr(w, "activation", "gelu_tanh") == "swiglu" else expert
+
+
 # ---------------------------------------------------------------------------
 # combine (§02: weighted sum of the 8 contributors, honest gates)
 # ---------------------------------------------------------------------------
@@ -320,7 +368,7 @@ def route_workload(w: "mi.Workload", bias: np.ndarray, tokens: Optional[Sequence
     if wr is None:
         wr = mi.host_wr(w)
     z = logits(x, wr, nthreads)
-    r = route(z, bias, w.k, w.n_routed, w.n_shared, logit_offset)
+    r = route(z, bias, w.k, w.n_routed, w.n_shared, logit_offset, route_scale=w.gate_scale)
     r["z"] = z
     return r
 
@@ -357,7 +405,7 @@ def forward_tokens(w: "mi.Workload", tokens: Sequence[int], bias: np.ndarray,
             w1, w2 = weights["w1"][e], weights["w2"][e]
         else:
             w1, w2 = mi.host_w1(w, int(e)), mi.host_w2(w, int(e))
-        y = expert(x[rows], w1, w2, nthreads)
+        y = expert_for(w)(x[rows], w1, w2, nthreads)
         out[rows] += gates[rows, slots][:, None] * y
     r["out"] = out
     r["tokens"] = tokens
