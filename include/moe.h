@@ -61,6 +61,7 @@ typedef uint16_t moe_bf16;
 
 /* expert nonlinearity */
 #define MOE_ACT_GELU_TANH 0 /* gelu(u) = u/2 (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3))) */
+#define MOE_ACT_SWIGLU 1    /* h = silu(Wg x) * (Wu x), silu(u) = u / (1 + e^-u); W1 = [Wg; Wu] */
 
 /* limits */
 #define MOE_MAX_TOP_K 8
@@ -79,11 +80,14 @@ typedef uint16_t moe_bf16;
  *   bias       [n_routed] fp32      balancing bias b (selection only)
  *   logit_offset [n_routed] fp32 or NULL: added to the routed logits before the
  *              sigmoid (a workload input for skewed routing, not part of the method)
- *   route_scale must be 1.0 (gates sum to 1)
+ *   route_scale finite, > 0: the jointly normalised weights are multiplied by it
+ *              ("Under the hood", "The routing strategy", step 5: route_scale 8
+ *              times the learned global_scale; pass the product).  1: gates sum to 1
  *   topk_idx   [T, top_k] int32 out: kept routed experts, descending s_i + b_i,
  *              ties to the lower index
  *   gates      [T, top_k + n_shared] fp32 out: g of the kept experts in topk
- *              order, then the shared experts in index order; per token they sum to 1
+ *              order, then the shared experts in index order; per token they sum
+ *              to route_scale (each is fl32(fl32(s / sum) * route_scale))
  *   counts     [n_routed] int32 out: L_i; zeroed by this call, then accumulated
  *   scores_out [T, n_routed + n_shared] fp32 or NULL: s_i for debugging
  * Logits are accumulated in fp32 from bf16 products (tcgen05 tensor cores);
@@ -181,7 +185,10 @@ int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, const int32_
 /*
  * moe_grouped_ffn -- the expert MLPs, y = W2_e gelu(W1_e x), for groups of rows.
  * "Inkling, Dissected" §02: an expert is two matrix multiplies with a
- * nonlinearity between them (GELU, tanh form, here).
+ * nonlinearity between them (GELU, tanh form, here).  With MOE_ACT_SWIGLU the
+ * expert is the gated one of the released configuration ("Under the hood",
+ * "MoE: the expert configuration": SwiGLU experts), y = W2_e (silu(Wg_e x) *
+ * (Wu_e x)), three matrices.
  *
  *   rows       [n_rows, d] bf16 input rows
  *   offsets    [n_groups + 1] int32 or NULL.
@@ -190,10 +197,12 @@ int moe_permute_noalloc(const moe_bf16* x, const int32_t* topk_idx, const int32_
  *              is [n_rows, d_ff] and y is [n_rows, d].
  *              NULL: every group sees all n_rows rows (the shared experts);
  *              h_scratch is [n_groups, n_rows, d_ff] and y is [n_groups, n_rows, d].
- *   w1         [*, d_ff, d] bf16 all experts' first matrices (K-major)
+ *   w1         [*, d_ff, d] bf16 all experts' first matrices (K-major); for
+ *              MOE_ACT_SWIGLU [*, 2*d_ff, d]: rows 0..d_ff-1 the gate projection
+ *              Wg, rows d_ff..2*d_ff-1 the up projection Wu
  *   w2         [*, d, d_ff] bf16 all experts' second matrices (K-major)
  *   expert_base index of the first expert used (group g uses expert_base + g)
- *   activation MOE_ACT_GELU_TANH
+ *   activation MOE_ACT_GELU_TANH or MOE_ACT_SWIGLU
  *   h_scratch  bf16 hidden activations (caller-owned), written then read
  * Tensor cores (tcgen05, bf16 in, fp32 accumulate); h is rounded to bf16
  * between the two matmuls; y is bf16.
@@ -215,11 +224,14 @@ int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, 
  *              x_perm is NULL)
  *   x_perm     [T*top_k, d] bf16 (from moe_permute) or NULL: then the routed rows
  *              are gathered from x through row_token by the GEMM's own loads
- *              (TMA tile::gather4), and moe_permute need not copy rows
+ *              (cp.async row copies), and moe_permute need not copy rows
  *   row_token  [T*top_k] int32 (from moe_permute); used when x_perm is NULL
  *   offsets    [n_routed + 1] int32 (from moe_permute)
  *   w1, w2     [n_routed + n_shared, d_ff, d] and [n_routed + n_shared, d, d_ff]
- *              bf16: routed experts first, then the shared experts
+ *              bf16: routed experts first, then the shared experts; for
+ *              MOE_ACT_SWIGLU w1 is [n_routed + n_shared, 2*d_ff, d] (gate rows,
+ *              then up rows), as for moe_grouped_ffn
+ *   activation MOE_ACT_GELU_TANH or MOE_ACT_SWIGLU
  *   h_scratch  [T*top_k + n_shared*T, d_ff] bf16 (caller-owned)
  *   y_perm     [T*top_k, d] bf16 out (routed, dispatch order)
  *   y_shared   [n_shared, T, d] bf16 out

@@ -38,6 +38,7 @@ MOE_STATUS_TIMEOUT = 0x1
 MOE_STATUS_BAD_EXPERT = 0x2
 MOE_STATUS_COUNT_MISMATCH = 0x4
 MOE_ACT_GELU_TANH = 0
+MOE_ACT_SWIGLU = 1
 
 _vp, _i32, _u64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_float, ctypes.c_size_t
 
@@ -219,15 +220,22 @@ class MoELayer:
     """Device buffers for one layer shape and the call sequence of a forward.
 
     Weights are caller-owned torch tensors: w_router [n_routed + n_shared, d],
-    w1 [n_routed + n_shared, d_ff, d], w2 [n_routed + n_shared, d, d_ff] (bf16),
-    bias [n_routed] fp32 (updated in place by ``bias_update``).
+    w1 [n_routed + n_shared, d_ff, d] (``activation="swiglu"``: [n_routed + n_shared,
+    2*d_ff, d], gate rows then up rows), w2 [n_routed + n_shared, d, d_ff] (bf16),
+    bias [n_routed] fp32 (updated in place by ``bias_update``).  ``route_scale``
+    multiplies the joint routing weights (route_scale x global_scale of the released
+    configuration; 1 keeps them summing to 1).
     """
 
     def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True, gather_rows: bool = False,
-                 capacity_factor: Optional[float] = None):
+                 capacity_factor: Optional[float] = None, activation: str = "gelu_tanh", route_scale: float = 1.0):
         import torch
 
         self.shape = s = shape
+        # expert type: GELU MLP (w1 [E, d_ff, d]) or SwiGLU (w1 [E, 2*d_ff, d]: gate rows, then up rows)
+        self.activation = {"gelu_tanh": MOE_ACT_GELU_TANH, "swiglu": MOE_ACT_SWIGLU}[activation]
+        # multiplier of the joint routing weights (route_scale x global_scale of the released config)
+        self.route_scale = float(route_scale)
         # hard expert capacity (tokens per expert per batch); None: every assignment is served
         self.capacity = None if capacity_factor is None else capacity_for(capacity_factor, s.T, s.top_k, s.n_routed)
         self.fused_experts = fused_experts
@@ -273,13 +281,13 @@ class MoELayer:
         s = self.shape
         main = stream if stream is not None else torch.cuda.current_stream()
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
-        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, 1.0, self.topk_idx,
-                        self.gates, self.counts, scores_out, stream=main)
+        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, self.route_scale,
+                        self.topk_idx, self.gates, self.counts, scores_out, stream=main)
         side = s.n_shared > 0 and not self.fused_experts
         if side:
             self.ev_start.record(main)
             self.side.wait_event(self.ev_start)
-            moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, MOE_ACT_GELU_TANH, self.h_shared,
+            moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, self.activation, self.h_shared,
                             self.y_shared, stream=self.side)
             self.ev_shared.record(self.side)
         x_perm = None if self.gather_rows else self.x_perm
@@ -293,9 +301,9 @@ class MoELayer:
             ffn_events[0].record(main)
         if self.fused_experts:
             moe_experts_ffn(x, x_perm, self.row_token, self.offsets, T, s.n_routed, s.n_shared, k, w1, w2, d, f,
-                            MOE_ACT_GELU_TANH, self.h, self.y_perm, self.y_shared, stream=main)
+                            self.activation, self.h, self.y_perm, self.y_shared, stream=main)
         else:
-            moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, MOE_ACT_GELU_TANH,
+            moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, self.activation,
                             self.h, self.y_perm, stream=main)
         if ffn_events is not None:
             ffn_events[1].record(main)

@@ -55,6 +55,11 @@ constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_NONE = 1;
+// Gated first GEMM of SwiGLU experts: a tile's 256 accumulator columns are 128 gate
+// columns (weight rows 128*nt ..) then the 128 matching up columns (rows b_up_row +
+// 128*nt ..), and the epilogue writes silu(gate) * up into 128 output columns.
+constexpr int EPI_SWIGLU = 2;
+constexpr int SWIGLU_OUT = BN / 2;
 
 template <bool PAIR, int ST>
 struct Cfg {
@@ -88,6 +93,7 @@ struct Params {
   int c1_base, c1_stride, c1_limit;
   int N;  // output columns
   int K;  // reduction length
+  int b_up_row;  // EPI_SWIGLU: first weight row of the up projection (= d_ff)
   int n_tiles_n;
   int ldc;
   uint64_t timeout_ns;
@@ -281,7 +287,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Group gr = group_info(p, st->gt, ti.g);
       const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
       const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
-      const int b_row = ti.nt * BN + (int)rank * C::B_ROWS;
+      // weight rows of this CTA's share of the tile's 256 columns; for SwiGLU the first 128
+      // columns are gate rows and the other 128 the matching up rows
+      const int b_row = EPI == EPI_SWIGLU ? (rank == 0u ? ti.nt * SWIGLU_OUT : p.b_up_row + ti.nt * SWIGLU_OUT)
+                                          : ti.nt * BN + (int)rank * C::B_ROWS;
       const bool gather = gathering && ti.g < p.G_r;
       // gathered rows: copy instruction q moves rows 4q .. 4q+3 of the CTA's A tile, eight lanes per
       // row (lane l: row 4q + l/8, 16-byte chunk l%8), so each instruction reads four whole 128-byte
@@ -323,7 +332,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_3d_pair(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
           } else {
             if (!gather) tma_load_2d(a_dst, am, &st->full[stage], kb * BK, a_row);
-            tma_load_3d(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+            if (EPI == EPI_SWIGLU) {  // two 128-row boxes: gate rows, then up rows
+              uint8_t* b_dst = smemB + stage * C::B_BYTES;
+              tma_load_3d(b_dst, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+              tma_load_3d(b_dst + C::B_BYTES / 2, &tmB, &st->full[stage], kb * BK, p.b_up_row + ti.nt * SWIGLU_OUT,
+                          ti.g);
+            } else {
+              tma_load_3d(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+            }
           }
         }
         if (gathering) {
@@ -429,8 +445,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       __nv_bfloat16* crow = cbase + (size_t)c_row * p.ldc;
+      if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+        for (int ch = 0; ch < SWIGLU_OUT / 32; ++ch) {
+          const int col0 = ti.nt * SWIGLU_OUT + ch * 32;
+          if (col0 >= p.N) break;  // same for the whole warp
+          float g[32], u[32];
+          tmem_ld32(taddr + ch * 32, g);
+          tmem_ld32(taddr + SWIGLU_OUT + ch * 32, u);
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(silu_f32(g[2 * i]) * u[2 * i], silu_f32(g[2 * i + 1]) * u[2 * i + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+      }
+#pragma unroll 1
+      for (int ch = 0; ch < (EPI == EPI_SWIGLU ? 0 : BN / 32); ++ch) {
         const int col0 = ti.nt * BN + ch * 32;
         if (col0 >= p.N) break;  // same for the whole warp
         float v[32];
@@ -514,7 +549,8 @@ struct GemmSpec {
   uint32_t a0_box_rows;  // 128 for tiled A loads, 1 for row gathers
   const void* a1;  // may be null (then a0's map is passed twice)
   uint64_t a1_rows;
-  const void* b;   // weights of the launch's group 0: [G, N, K]
+  const void* b;   // weights of the launch's group 0: [G, b_rows, K]
+  uint64_t b_rows; // weight rows per group (0: N)
   Params p;
 };
 
@@ -552,10 +588,11 @@ int stages_for(bool pair, int which, double flop) {
 
 template <int EPI>
 int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_upper, cudaStream_t s) {
-  const uint32_t b_box = pair ? (uint32_t)Cfg<true, 4>::B_ROWS : (uint32_t)Cfg<false, 4>::B_ROWS;
+  // rows per weight box: a pair CTA loads 128; a single CTA 256, or 2 x 128 (gate, up) for SwiGLU
+  const uint32_t b_box = (pair || EPI == EPI_SWIGLU) ? (uint32_t)Cfg<true, 4>::B_ROWS : (uint32_t)Cfg<false, 4>::B_ROWS;
   CUtensorMap a0, a1, b;
   int rc;
-  const uint64_t K = (uint64_t)g.p.K, N = (uint64_t)g.p.N;
+  const uint64_t K = (uint64_t)g.p.K, N = g.b_rows ? g.b_rows : (uint64_t)g.p.N;
   if ((rc = encode_tmap_bf16(&a0, g.a0, 2, K, g.a0_rows, 1, BK, g.a0_box_rows ? g.a0_box_rows : 128)) != MOE_OK)
     return rc;
   if (g.a1) {
@@ -583,7 +620,9 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
                                int expert_base, const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff,
                                int activation, moe_bf16* h_scratch, moe_bf16* y, void* stream) {
   if (n_groups < 0 || n_rows < 0 || expert_base < 0 || d <= 0 || d_ff <= 0) return MOE_ERR_INVALID_ARG;
-  if (activation != MOE_ACT_GELU_TANH) return MOE_ERR_INVALID_ARG;
+  if (activation != MOE_ACT_GELU_TANH && activation != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  const bool swiglu = activation == MOE_ACT_SWIGLU;
+  const int w1_rows = swiglu ? 2 * d_ff : d_ff;  // SwiGLU: gate rows, then up rows
   if (!aligned16(rows) || !aligned16(w1) || !aligned16(w2) || !aligned16(h_scratch) || !aligned16(y))
     return MOE_ERR_INVALID_ARG;
   if (!rows || !w1 || !w2 || !h_scratch || !y) return MOE_ERR_INVALID_ARG;
@@ -620,7 +659,8 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   GemmSpec g1{};
   g1.a0 = rows;
   g1.a0_rows = (uint64_t)n_rows;
-  g1.b = reinterpret_cast<const __nv_bfloat16*>(w1) + (size_t)expert_base * d_ff * d;
+  g1.b = reinterpret_cast<const __nv_bfloat16*>(w1) + (size_t)expert_base * w1_rows * d;
+  g1.b_rows = (uint64_t)w1_rows;
   g1.p = p;
   g1.p.a_sh_base = 0;
   g1.p.a_sh_stride = 0;  // every shared group reads rows 0..n_rows-1
@@ -630,10 +670,13 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g1.p.c1_stride = n_rows;
   g1.p.N = d_ff;
   g1.p.K = d;
-  g1.p.n_tiles_n = (d_ff + BN - 1) / BN;
+  g1.p.n_tiles_n = swiglu ? (d_ff + SWIGLU_OUT - 1) / SWIGLU_OUT : (d_ff + BN - 1) / BN;
+  g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
-  const double flop = 2.0 * (double)h_rows * d * d_ff;  // per GEMM
-  if ((rc = run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s)) != MOE_OK) return rc;
+  const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
+  rc = swiglu ? run_gemm<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
+              : run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
+  if (rc != MOE_OK) return rc;
 
   GemmSpec g2{};
   g2.a0 = h_scratch;
@@ -658,7 +701,9 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
                                const moe_bf16* w1, const moe_bf16* w2, int d, int d_ff, int activation,
                                moe_bf16* h_scratch, moe_bf16* y_perm, moe_bf16* y_shared, void* stream) {
   if (T < 0 || n_routed < 0 || n_shared < 0 || top_k < 1 || d <= 0 || d_ff <= 0) return MOE_ERR_INVALID_ARG;
-  if (activation != MOE_ACT_GELU_TANH) return MOE_ERR_INVALID_ARG;
+  if (activation != MOE_ACT_GELU_TANH && activation != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  const bool swiglu = activation == MOE_ACT_SWIGLU;
+  const int w1_rows = swiglu ? 2 * d_ff : d_ff;  // SwiGLU: gate rows, then up rows
   if (n_routed + n_shared > MOE_MAX_GROUPS) return MOE_ERR_UNSUPPORTED;
   if (d % 64 != 0 || d_ff % 64 != 0) return MOE_ERR_UNSUPPORTED;
   if (!w1 || !w2 || !h_scratch || !aligned16(w1) || !aligned16(w2) || !aligned16(h_scratch))
@@ -706,6 +751,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.a1 = n_shared > 0 ? (const void*)x : nullptr;
   g1.a1_rows = (uint64_t)T;
   g1.b = w1;
+  g1.b_rows = (uint64_t)w1_rows;
   g1.p = p;
   g1.p.gather_rows = routed_gather ? row_token : nullptr;
   g1.p.gather_limit = T;
@@ -720,10 +766,13 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.p.c1_limit = (int)h_rows;
   g1.p.N = d_ff;
   g1.p.K = d;
-  g1.p.n_tiles_n = (d_ff + BN - 1) / BN;
+  g1.p.n_tiles_n = swiglu ? (d_ff + SWIGLU_OUT - 1) / SWIGLU_OUT : (d_ff + BN - 1) / BN;
+  g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
-  const double flop = 2.0 * (double)h_rows * d * d_ff;  // per GEMM
-  if ((rc = run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s)) != MOE_OK) return rc;
+  const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
+  rc = swiglu ? run_gemm<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
+              : run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
+  if (rc != MOE_OK) return rc;
 
   // GEMM2: all A rows from H (map 0); routed outputs to y_perm, shared outputs to y_shared
   GemmSpec g2{};

@@ -60,6 +60,7 @@ struct Params {
   int ksplit;           // CTAs (cluster size) sharing one 128-token tile: 1, 2, 4 or 8
   int32_t* topk_idx;
   float* gates;
+  float gate_scale;  // the joint weights are multiplied by it (route_scale x global_scale)
   int32_t* counts;
   float* scores;  // nullable
   uint64_t timeout_ns;
@@ -191,12 +192,12 @@ __device__ __forceinline__ void route_token(const Params& p, SmemTail* st, const
 #pragma unroll
   for (int q = 0; q < K; ++q) {
     ti[q] = id[q];
-    gt[q] = __fdiv_rn(sc[q], den);
+    gt[q] = __fmul_rn(__fdiv_rn(sc[q], den), p.gate_scale);
     if (id[q] >= 0 && id[q] < p.n_routed) atomicAdd(&st->hist[id[q]], 1);  // unset only for non-finite scores
   }
 #pragma unroll
   for (int q = 0; q < MOE_MAX_SHARED; ++q)
-    if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[q], den);
+    if (q < p.n_shared) gt[K + q] = __fmul_rn(__fdiv_rn(shv[q], den), p.gate_scale);
 }
 
 // Route NT tokens with one warp, their work interleaved so the latencies of the
@@ -326,12 +327,12 @@ __device__ __forceinline__ void route_tokens_warp(const Params& p, SmemTail* st,
 #pragma unroll
     for (int q = 0; q < K; ++q) {
       ti[q] = id[n][q];
-      gt[q] = __fdiv_rn(sc[n][q], den);
+      gt[q] = __fmul_rn(__fdiv_rn(sc[n][q], den), p.gate_scale);
       if (id[n][q] >= 0 && id[n][q] < p.n_routed) atomicAdd(&st->hist[id[n][q]], 1);  // unset only if non-finite
     }
 #pragma unroll
     for (int q = 0; q < MOE_MAX_SHARED; ++q)
-      if (q < p.n_shared) gt[K + q] = __fdiv_rn(shv[n][q], den);
+      if (q < p.n_shared) gt[K + q] = __fmul_rn(__fdiv_rn(shv[n][q], den), p.gate_scale);
   }
 }
 
@@ -587,7 +588,7 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
     return MOE_ERR_INVALID_ARG;
   if (T < 0 || d <= 0 || n_routed < 1 || n_shared < 0 || top_k < 1) return MOE_ERR_INVALID_ARG;
   if (top_k > MOE_MAX_TOP_K || top_k > n_routed) return MOE_ERR_INVALID_ARG;
-  if (route_scale != 1.0f) return MOE_ERR_UNSUPPORTED;
+  if (!(route_scale > 0.0f) || route_scale > 3.0e38f) return MOE_ERR_INVALID_ARG;  // finite, positive
   if (n_routed > MOE_MAX_ROUTED || n_shared > MOE_MAX_SHARED || n_routed + n_shared > B0_ROWS + B1_ROWS)
     return MOE_ERR_UNSUPPORTED;
   if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;  // 16-byte row pitch for the tensor map
@@ -615,6 +616,7 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   p.ksplit = choose_ksplit(n_mtiles, (d + BK - 1) / BK, sms);
   p.topk_idx = topk_idx;
   p.gates = gates;
+  p.gate_scale = route_scale;
   p.counts = counts;
   p.scores = scores_out;
   p.timeout_ns = wait_timeout_ns();

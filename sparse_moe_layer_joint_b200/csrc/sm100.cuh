@@ -225,6 +225,10 @@ __device__ __forceinline__ float gelu_tanh_f32(float u) {
   return 0.5f * u * (1.0f + tanh_approx(inner));
 }
 
+// SiLU (the swish of a SwiGLU gate), u * sigmoid(u) = u / (1 + e^-u), in fp32.
+// For very negative u, e^-u overflows to inf and the reciprocal to 0: silu -> -0.
+__device__ __forceinline__ float silu_f32(float u) { return u * __frcp_rn(1.0f + __expf(-u)); }
+
 }  // namespace moe
 
 namespace moe {

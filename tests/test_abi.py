@@ -57,7 +57,11 @@ def router(**kw):
     (dict(d=100), moe.MOE_ERR_UNSUPPORTED),
     (dict(nr=300), moe.MOE_ERR_UNSUPPORTED),
     (dict(ns=9), moe.MOE_ERR_UNSUPPORTED),
-    (dict(rs=8.0), moe.MOE_ERR_UNSUPPORTED),
+    (dict(d=36), moe.MOE_ERR_UNSUPPORTED),
+    (dict(rs=0.0), moe.MOE_ERR_INVALID_ARG),
+    (dict(rs=-8.0), moe.MOE_ERR_INVALID_ARG),
+    (dict(rs=float("nan")), moe.MOE_ERR_INVALID_ARG),
+    (dict(rs=float("inf")), moe.MOE_ERR_INVALID_ARG),
 ])
 def test_router_rejects(kw, code):
     assert router(**kw) == code
@@ -128,3 +132,21 @@ def test_wait_timeout_setting():
     assert L.moe_set_wait_timeout_ns(0) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_set_wait_timeout_ns(2_000_000_000) == moe.MOE_OK
     assert L.moe_debug_bounded_wait(0, NULL) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_ffn_rejects_unknown_activation():
+    for act in (2, -1, 99):
+        assert L.moe_grouped_ffn(A16, NULL, 2, 8, 0, A16, A16, 64, 64, act, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+        assert L.moe_experts_ffn(A16, A16, A16, A16, 8, 4, 2, 2, A16, A16, 64, 64, act, A16, A16, A16,
+                                 NULL) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_capacity_and_stats_reject():
+    assert L.moe_permute_capped(A16, A16, NULL, 8, 64, 256, 6, -1, A16, A16, A16, A16, A16, 1 << 20,
+                                NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_permute_capped(A16, A16, NULL, 8, 64, 256, 6, 5, A16, A16, A16, A16, A16, 16,
+                                NULL) == moe.MOE_ERR_SCRATCH
+    assert L.moe_load_stats(A16, 256, -3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(A16, 257, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(NULL, 256, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(0x10002, 256, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG

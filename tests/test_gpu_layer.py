@@ -20,7 +20,7 @@ if torch.cuda.is_available():
 def _layer(w, with_weights=True, fused=True, gather=False):
     t = mi.torch_workload(w, with_weights=with_weights)
     layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), fused_experts=fused,
-                         gather_rows=gather)
+                         gather_rows=gather, activation=w.activation, route_scale=w.gate_scale)
     return t, layer
 
 
@@ -60,7 +60,7 @@ def _run_and_check(name, tokens=None, check_all_routing=True, fused=True, gather
     if check_all_routing:
         ref = oracle.route_workload(w, b_host, logit_offset=off, x=x_bits)
         same = check_routing(layer.topk_idx.cpu().numpy(), layer.gates.cpu().numpy().astype(np.float64),
-                             layer.counts.cpu().numpy(), ref, w.k, w.n_routed, w.n_shared)
+                             layer.counts.cpu().numpy(), ref, w.k, w.n_routed, w.n_shared, w.gate_scale)
         # the bias update, bit-exact whenever the counts agree with the oracle's
         ref_counts = oracle.load_counts(ref["topk_idx"], w.n_routed)
         if (layer.counts.cpu().numpy() == ref_counts).all():
@@ -111,6 +111,17 @@ def test_layer_decode_sampled():
 def test_layer_prefill_sampled():
     w = mi.WORKLOADS["prefill"]
     _run_and_check("prefill", tokens=np.array([0, 1, 4095, 30000, 65535]), check_all_routing=False)
+
+
+def test_layer_inkling_decode_sampled():
+    """The released configuration (SwiGLU experts, d 6144, d_ff 3072, route_scale 8) at decode scale."""
+    _run_and_check("inkling_decode", tokens=np.arange(0, 64, 9))
+
+
+@pytest.mark.slow
+def test_layer_inkling_sampled():
+    """The released configuration at prefill scale (65536 tokens, about 29 GB of expert weights)."""
+    _run_and_check("inkling", tokens=np.array([0, 7, 40000, 65535]), check_all_routing=False)
 
 
 @pytest.mark.slow

@@ -315,6 +315,118 @@ def test_experts_ffn_parity(T, n_routed, n_shared, k, d, f, gemm_variant, gather
 
 
 # ---------------------------------------------------------------------------
+# SwiGLU experts (the released configuration: "Under the hood", SwiGLU FFNs)
+# ---------------------------------------------------------------------------
+def _swiglu_weights(E, d, f, seed):
+    w1 = mi.normal_bf16(E * 2 * f * d, seed, mi.STREAM_W1, std=1 / np.sqrt(d)).reshape(E, 2 * f, d)
+    w2 = mi.normal_bf16(E * d * f, seed, mi.STREAM_W2, std=1 / np.sqrt(f)).reshape(E, d, f)
+    return w1, w2
+
+
+@pytest.mark.parametrize("sizes,d,f", [
+    ([0, 1, 127, 128, 129, 300, 0, 5], 256, 128),
+    ([200, 37, 0, 513], 512, 192),          # d_ff not a multiple of 128: a half-width last tile
+    ([64] * 16, 128, 64),
+    ([1000], 1024, 512),
+    ([129, 255, 256, 257, 0, 511, 1], 256, 384),
+])
+def test_grouped_ffn_swiglu_parity(sizes, d, f, gemm_variant):
+    G = len(sizes)
+    n = int(sum(sizes))
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    rows = mi.normal_bf16(n * d, 14, mi.STREAM_TEST_ROWS).reshape(n, d)
+    base = 2
+    w1, w2 = _swiglu_weights(G + base, d, f, 14)
+    h = torch.full((n, f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((n, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    moe.moe_grouped_ffn(dev_bf16(rows), _i32(offsets), G, n, base, dev_bf16(w1), dev_bf16(w2), d, f,
+                        moe.MOE_ACT_SWIGLU, h, y)
+    assert moe.moe_get_status() == 0
+    yg = host_bf16_f64(y)
+    for g in range(G):
+        a, b = offsets[g], offsets[g + 1]
+        if a == b:
+            continue
+        ref = oracle.expert_swiglu(rows[a:b], w1[base + g], w2[base + g])
+        check_output(yg[a:b], ref, f"group {g}")
+
+
+def test_swiglu_special_weights(gemm_variant):
+    """Wg = I, Wu = I, W2 = I (d = d_ff): y = bf16(silu(x) * x); Wu = 0 gives exactly 0."""
+    n, d = 300, 128
+    rows = mi.normal_bf16(n * d, 15, mi.STREAM_TEST_ROWS).reshape(n, d)
+    eye = mi.f32_to_bf16_bits(np.eye(d, dtype=np.float32))
+    zero = np.zeros_like(eye)
+    w1 = np.stack([np.concatenate([eye, eye]), np.concatenate([eye, zero])])
+    w2 = np.stack([eye, eye])
+    off = _i32([0, 200, n])
+    h = torch.empty((n, d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((n, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_grouped_ffn(dev_bf16(rows), off, 2, n, 0, dev_bf16(w1), dev_bf16(w2), d, d, moe.MOE_ACT_SWIGLU, h, y)
+    yg = host_bf16_f64(y)
+    xr = mi.bf16_to_f64(rows[:200])
+    np.testing.assert_allclose(yg[:200], oracle.silu(xr) * xr, rtol=2 ** -6, atol=2e-3)
+    assert (yg[200:] == 0).all()
+
+
+@pytest.mark.parametrize("T,n_routed,n_shared,k,d,f", [
+    (300, 16, 2, 3, 256, 128), (64, 64, 2, 6, 384, 192), (700, 4, 0, 2, 128, 128), (129, 0, 2, 1, 128, 256),
+])
+def test_experts_ffn_swiglu_parity(T, n_routed, n_shared, k, d, f, gemm_variant):
+    E = n_routed + n_shared
+    x = mi.normal_bf16(T * d, 16, mi.STREAM_X).reshape(T, d)
+    w1, w2 = _swiglu_weights(E, d, f, 16)
+    R = T * k
+    h = torch.empty((R + n_shared * T, f), dtype=torch.bfloat16, device="cuda")
+    y_perm = torch.full((max(R, 1), d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y_sh = torch.full((max(n_shared, 1), T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    xp = None
+    if n_routed:
+        topk = _random_topk(T, k, n_routed, 17)
+        dp = oracle.dispatch(topk, n_routed)
+        xp = x[dp["row_token"]]
+        moe.moe_experts_ffn(dev_bf16(x), dev_bf16(xp), _i32(dp["row_token"]), _i32(dp["offsets"]), T, n_routed,
+                            n_shared, k, dev_bf16(w1), dev_bf16(w2), d, f, moe.MOE_ACT_SWIGLU, h, y_perm, y_sh)
+    else:
+        moe.moe_experts_ffn(dev_bf16(x), None, None, None, T, 0, n_shared, k, dev_bf16(w1), dev_bf16(w2), d, f,
+                            moe.MOE_ACT_SWIGLU, h, y_perm, y_sh)
+    assert moe.moe_get_status() == 0
+    if n_routed:
+        yp = host_bf16_f64(y_perm)
+        off = dp["offsets"]
+        for e in range(n_routed):
+            if off[e] < off[e + 1]:
+                check_output(yp[off[e]:off[e + 1]], oracle.expert_swiglu(xp[off[e]:off[e + 1]], w1[e], w2[e]),
+                             f"routed {e}")
+    ys = host_bf16_f64(y_sh)
+    for sidx in range(n_shared):
+        check_output(ys[sidx], oracle.expert_swiglu(x, w1[n_routed + sidx], w2[n_routed + sidx]), f"shared {sidx}")
+
+
+@pytest.mark.parametrize("scale", [8.0, 2.83])
+def test_router_route_scale(scale):
+    """Joint weights times route_scale x global_scale: sums equal the scale, values the
+    oracle's scaled weights, selection unchanged."""
+    T, d = 700, 256
+    x = mi.normal_bf16(T * d, 9, mi.STREAM_X).reshape(T, d)
+    wr = mi.normal_bf16(258 * d, 9, mi.STREAM_WR, std=1 / 16).reshape(258, d)
+    b = mi.uniform_f32(256, 9, mi.STREAM_B, -0.05, 0.05)
+    ref = oracle.route(oracle.logits(x, wr), b, 6, 256, 2, route_scale=scale)
+    xd, wd, bd = dev_bf16(x), dev_bf16(wr), _f32(b)
+    idx = torch.empty((T, 6), dtype=torch.int32, device="cuda")
+    g = torch.empty((T, 8), dtype=torch.float32, device="cuda")
+    c = torch.empty(256, dtype=torch.int32, device="cuda")
+    moe.moe_router_topk(xd, wd, bd, None, T, d, 256, 2, 6, scale, idx, g, c)
+    g1 = torch.empty_like(g)
+    moe.moe_router_topk(xd, wd, bd, None, T, d, 256, 2, 6, 1.0, idx, g1, c)
+    torch.cuda.synchronize()
+    check_routing(idx.cpu().numpy(), g.cpu().numpy().astype(np.float64), c.cpu().numpy(), ref, 6, 256, 2,
+                  gate_scale=scale)
+    # the scale is one fp32 multiply after the normalisation
+    np.testing.assert_array_equal(g.cpu().numpy(), (g1.cpu().numpy() * np.float32(scale)).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
 # combine
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("T,k,ns,d", [(1, 6, 2, 64), (333, 6, 2, 256), (1024, 2, 0, 128), (100, 8, 8, 72)])
