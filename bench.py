@@ -58,7 +58,7 @@ def peaks():
 def config_of(w, world):
     return {"workload": w.name, "description": w.description, "T_per_gpu": w.T, "global_tokens": w.T * world,
             "d": w.d, "d_ff": w.f, "n_routed": w.n_routed, "n_shared": w.n_shared, "top_k": w.k,
-            "activation": "gelu_tanh", "parallelism": f"dp{world} (replicas, counts all-reduced)" if world > 1
+            "activation": w.activation, "gate_scale": w.gate_scale, "parallelism": f"dp{world} (replicas, counts all-reduced)" if world > 1
             else "single GPU", "l2": "inputs larger than L2 (no flush)", "seed": w.seed}
 
 
@@ -131,7 +131,8 @@ def run_ours(args, w, rank, world, local_rank):
         mi.gpu_normal_bf16(t["x"].data_ptr(), t["x"].numel(), w.seed, mi.STREAM_X, rank * w.T * w.d, w.std_x,
                            stream.cuda_stream)
     layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev,
-                         gather_rows=args.gather_rows, capacity_factor=args.capacity_factor)
+                         gather_rows=args.gather_rows, capacity_factor=args.capacity_factor,
+                         activation=w.activation, route_scale=w.gate_scale)
     bias0 = t["bias"].clone()
     ffn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
@@ -244,12 +245,13 @@ def run_ours(args, w, rank, world, local_rank):
     # + outputs written (bf16)
     pk = peaks()
     rows = routed_rows + w.T * w.n_shared
-    ffn_flops = 2 * 2.0 * rows * w.d * w.f
-    ffn_bytes = ((touched + w.n_shared) * 2 * w.d * w.f * 2
+    mats = 3 if w.activation == "swiglu" else 2   # weight matrices per expert
+    ffn_flops = 2 * mats * rows * w.d * w.f
+    ffn_bytes = ((touched + w.n_shared) * mats * w.d * w.f * 2
                  + rows * w.d * 2 + rows * w.f * 2 * 2 + rows * w.d * 2)
     tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
     gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
-    kernel = "grouped_gemm_kernel x2 (all experts: GEMM1+GELU, GEMM2)"
+    kernel = f"grouped_gemm_kernel x2 (all experts: GEMM1+{'SwiGLU' if w.activation == 'swiglu' else 'GELU'}, GEMM2)"
     tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1),
                    "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                    "frac": round(tflops / pk["bf16_tflops_sustained"], 4),
@@ -261,9 +263,9 @@ def run_ours(args, w, rank, world, local_rank):
                 "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)", "traffic": None,
                 "bytes_per_launch_pair": round(ffn_bytes), "touched_routed_experts_mean": round(touched, 2),
                 "ms_per_launch_pair": round(ffn_ms, 4)}
-    weight_bound = w.name in ("decode", "mid")
+    weight_bound = w.name in ("decode", "mid", "inkling_decode")
     roofline = hbm_roof if weight_bound else tensor_roof
-    layer_flops = w.flops() - 2.0 * 2.0 * (w.T * w.k - routed_rows) * w.d * w.f
+    layer_flops = w.flops() - 2.0 * mats * (w.T * w.k - routed_rows) * w.d * w.f
     roofline["layer_tflops"] = round(layer_flops / (ms * 1e-3) / 1e12, 1)
     line = {
         "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
