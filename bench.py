@@ -42,6 +42,11 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
+# DRAM bytes (read + write) of one GEMM1 + GEMM2 launch pair, from one single-pass ncu capture of the
+# full-size layer (profiles/grouped_gemm_prefill_dram.md); workloads without a capture of the current
+# kernels report null
+TRAFFIC_PER_LAUNCH_PAIR = {"prefill": (20.84e9 + 2.14e9) + (12.84e9 + 7.48e9)}
+
 
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -252,15 +257,17 @@ def run_ours(args, w, rank, world, local_rank):
     tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
     gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
     kernel = f"grouped_gemm_kernel x2 (all experts: GEMM1+{'SwiGLU' if w.activation == 'swiglu' else 'GELU'}, GEMM2)"
+    traffic = TRAFFIC_PER_LAUNCH_PAIR.get(w.name) if args.capacity_factor is None and not args.gather_rows else None
     tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1),
                    "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                    "frac": round(tflops / pk["bf16_tflops_sustained"], 4),
                    "peak_source": f"{pk['src']} bf16 sustained (MEASURED_PEAKS.json)" if pk["src"] == "measured"
-                   else "fallback bf16 sustained", "traffic": None,
+                   else "fallback bf16 sustained", "traffic": traffic, "traffic_unit": "bytes per launch pair",
+                   "algorithmic_bytes_per_launch_pair": round(ffn_bytes),
                    "flop_per_launch_pair": ffn_flops, "ms_per_launch_pair": round(ffn_ms, 4)}
     hbm_roof = {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / pk["hbm_gbs"], 4),
-                "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)", "traffic": None,
+                "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)", "traffic": traffic,
                 "bytes_per_launch_pair": round(ffn_bytes), "touched_routed_experts_mean": round(touched, 2),
                 "ms_per_launch_pair": round(ffn_ms, 4)}
     weight_bound = w.name in ("decode", "mid", "inkling_decode")
