@@ -1,0 +1,111 @@
+"""Pins of the oracle's NVFP4 quantization ("Under the hood", "Quantization: BF16
+vs NVFP4": FP4 weights and activations, blocks of 16, FP8 block scales) to the
+OCP Microscaling format definitions, a library FP8 conversion, exact round
+trips and error bounds (no GPU)."""
+import numpy as np
+import pytest
+
+import moe_inputs as mi
+from oracle import nvfp4
+
+torch = pytest.importorskip("torch")
+
+
+def test_e2m1_table_and_round_trip():
+    mags = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    np.testing.assert_array_equal(nvfp4.e2m1_decode(np.arange(8)), mags)
+    np.testing.assert_array_equal(nvfp4.e2m1_decode(np.arange(8, 16)), [-m for m in mags])
+    codes = np.arange(16)
+    back = nvfp4.e2m1_encode(nvfp4.e2m1_decode(codes))
+    np.testing.assert_array_equal(back, np.where(codes == 8, 0, codes))   # -0 is written as +0
+
+
+@pytest.mark.parametrize("v,code", [
+    (0.25, 0), (0.2500001, 1), (0.75, 2), (0.7499, 1), (1.25, 2), (1.2501, 3), (1.75, 4), (2.5, 4), (2.51, 5),
+    (3.5, 6), (3.49, 5), (5.0, 6), (5.01, 7), (6.0, 7), (7.0, 7), (1e30, 7), (-0.1, 0), (-0.3, 9), (-5.0, 14),
+    (-9.0, 15),
+])
+def test_e2m1_ties_to_even_and_saturation(v, code):
+    assert int(nvfp4.e2m1_encode(np.array([v]))[0]) == code
+
+
+def test_e4m3_known_codes():
+    np.testing.assert_array_equal(nvfp4.e4m3_decode(np.array([0x38, 0x7E, 0x01, 0x08, 0x07, 0x77, 0x00])),
+                                  [1.0, 448.0, 2.0 ** -9, 2.0 ** -6, 0.875 * 2.0 ** -6, 240.0, 0.0])
+
+
+def test_e4m3_encoder_matches_torch_float8_cast():
+    """Round to nearest even on the E4M3 grid, against torch's float8_e4m3fn conversion:
+    a dense log-spaced sweep plus every exact midpoint between neighbouring values."""
+    table = nvfp4.e4m3_decode(np.arange(127))
+    mids = (table[:-1] + table[1:]) / 2
+    v = np.concatenate([np.geomspace(2.0 ** -12, 448.0, 20001), mids, table, [0.0, 2.0 ** -11, 447.9]])
+    v32 = v.astype(np.float32)
+    ref = torch.from_numpy(v32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(nvfp4.e4m3_encode_nonneg(v32), ref)
+    assert int(nvfp4.e4m3_encode_nonneg(np.array([1e9]))[0]) == 0x7E       # saturates
+
+
+def test_activation_round_trip_of_representable_blocks():
+    """Blocks built from E2M1 codes times an E4M3 scale, with a block maximum of
+    magnitude 6, are quantized back to exactly those codes and scales."""
+    rng_codes = mi.words(64 * 64, 3, mi.STREAM_TEST_ROWS) % 16
+    q = rng_codes.reshape(64, 64).astype(np.uint8)
+    q[:, ::16] = 7                                          # every block holds a +6
+    s = (mi.words(64 * 4, 4, mi.STREAM_TEST_ROWS) % 100 + 20).reshape(64, 4).astype(np.uint8)
+    x = nvfp4.dequantize(q, s).astype(np.float32)
+    q2, s2 = nvfp4.quantize_activation(x)
+    np.testing.assert_array_equal(s2, s)
+    np.testing.assert_array_equal(nvfp4.e2m1_decode(q2), nvfp4.e2m1_decode(q))
+
+
+def test_weight_round_trip_with_tensor_scale():
+    q = (mi.words(32 * 128, 5, mi.STREAM_TEST_ROWS) % 16).reshape(32, 128).astype(np.uint8)
+    q[:, ::16] = 7
+    s = (mi.words(32 * 8, 6, mi.STREAM_TEST_ROWS) % 90 + 30).reshape(32, 8).astype(np.uint8)
+    s[0, 0] = 0x7E                                          # the matrix maximum uses the largest scale
+    g = 2.0 ** -10
+    w = nvfp4.dequantize(q, s, g).astype(np.float32)
+    q2, s2, g2 = nvfp4.quantize_weight(w)
+    assert g2 == np.float32(g)
+    np.testing.assert_array_equal(s2, s)
+    np.testing.assert_array_equal(nvfp4.e2m1_decode(q2), nvfp4.e2m1_decode(q))
+
+
+def test_activation_codes_are_nearest_grid_points():
+    x = (mi.normal_f64(300 * 64, 7, mi.STREAM_TEST_ROWS).reshape(300, 64) * 3).astype(np.float32)
+    q, s = nvfp4.quantize_activation(x)
+    sd = nvfp4.e4m3_decode(s)
+    r = x.reshape(300, 4, 16) / sd[..., None]
+    got = nvfp4.e2m1_decode(q).reshape(300, 4, 16)
+    grid = np.concatenate([-nvfp4.E2M1_MAGNITUDE[::-1], nvfp4.E2M1_MAGNITUDE])
+    best = np.abs(r[..., None] - grid).min(axis=-1)
+    assert (np.abs(r - got) <= best + 1e-6).all()
+    # the block scale is amax/6 to within E4M3's half-step (relative 1/16), so the block maximum maps to 4 or 6
+    amax = np.abs(x.reshape(300, 4, 16)).max(axis=-1)
+    np.testing.assert_allclose(sd, amax / 6, rtol=1 / 16 + 1e-7)
+    assert set(np.unique(np.abs(got).max(axis=-1))) <= {4.0, 6.0}
+
+
+def test_scale_invariance_by_powers_of_two():
+    x = (mi.normal_f64(40 * 32, 8, mi.STREAM_TEST_ROWS).reshape(40, 32)).astype(np.float32)
+    q, s = nvfp4.quantize_activation(x)
+    q4, s4 = nvfp4.quantize_activation(x * np.float32(4))
+    np.testing.assert_array_equal(q4, q)
+    np.testing.assert_array_equal(s4.astype(int), s.astype(int) + 2 * 8)   # exponent field + 2
+
+
+def test_gemm_orientation():
+    """dq(A) dq(B)^T with B = c * identity reproduces c * dq(A): the weight rows
+    are the output features (a transposed operand fails).  c = 6 * 448 * 2^-10, so
+    the tensor scale is a power of two and c is exact."""
+    K = 64
+    x = mi.normal_f64(10 * K, 9, mi.STREAM_TEST_ROWS).reshape(10, K).astype(np.float32)
+    xq, xs = nvfp4.quantize_activation(x)
+    w = np.zeros((48, K), np.float32)
+    c = 6 * 448 * 2.0 ** -10
+    w[np.arange(48), np.arange(48)] = c                     # 48 outputs read the first 48 inputs
+    wq, ws, g = nvfp4.quantize_weight(w)
+    assert g == np.float32(2.0 ** -10)
+    np.testing.assert_allclose(nvfp4.gemm(xq, xs, wq, ws, g), c * nvfp4.dequantize(xq, xs)[:, :48],
+                               rtol=1e-14, atol=0)
