@@ -243,6 +243,84 @@ int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* ro
                     void* stream);
 
 /*
+ * NVFP4 routed experts (W4A4).  "Under the hood", "Quantization: BF16 vs NVFP4":
+ * the released NVFP4 checkpoint stores FP4 weights and activations in groups of
+ * 16 values, each with an FP8 scale ("group_size": 16, dynamic block scales),
+ * for Blackwell's FP4 tensor cores.  The router and the shared experts stay
+ * bf16.  Recipe (round to nearest even, saturating, in fp32):
+ *   weights      g = amax|W| / (6 * 448) per matrix; block scale
+ *                s = E4M3(fl(amax_b / 6) / g); codes E2M1(w / fl(s * g))
+ *   activations  s = E4M3(fl(amax_b / 6)) per block; codes E2M1(x / s)
+ * A block whose scale is 0 has codes 0.  E2M1 codes have no negative zero.
+ *
+ * Layouts:
+ *   codes   [rows, K/2] bytes, K-major; byte j of a row packs values 2j (bits
+ *           0-3) and 2j+1 (bits 4-7); E2M1 sign in bit 3
+ *   scales  atom-tiled, rows * K/16 bytes: 512-byte atoms of 128 rows x 64
+ *           values, the atoms of one 128-row block consecutive along K; the
+ *           scale of (row r, block b) is at byte
+ *             ((r/128) * (K/64) + b/4) * 512 + (r%32) * 16 + (r%128/32) * 4 + b%4
+ *   routed rows for the FP4 path: expert e's rows start at offsets_pad[e], a
+ *           multiple of 128 (offsets_pad[e+1] - offsets_pad[e] = the expert's
+ *           rows rounded up to 128); the rows of all experts fit in
+ *           moe_nvfp4_rows_capacity(T, n_routed, top_k) rows.
+ */
+#define MOE_NVFP4_EPI_GELU_FP4 0 /* out = FP4(gelu(g * acc)): codes + scales (the next GEMM's A) */
+#define MOE_NVFP4_EPI_BF16 1     /* out = bf16(g * acc) */
+
+/*
+ * moe_nvfp4_quantize_weights -- quantize G weight matrices [G, N, K] bf16 (K-major)
+ *   q       [G, N, K/2] bytes out; sf [G, N*K/16] bytes out (per matrix, atom-tiled)
+ *   gscale  [G] fp32 out: each matrix's tensor scale g
+ * Limits: N % 128 == 0, K % 256 == 0.  Run once per weight set.
+ */
+int moe_nvfp4_quantize_weights(const moe_bf16* w, int G, int N, int K, uint8_t* q, uint8_t* sf, float* gscale,
+                               void* stream);
+
+/* Rows (a multiple of 128) that the padded routed rows of one batch can need. */
+long long moe_nvfp4_rows_capacity(int T, int n_routed, int top_k);
+
+/*
+ * moe_nvfp4_dispatch -- the FP4 dispatch: each token's x row is quantized once
+ * (activation recipe) and written to the padded rows of its routed experts.
+ *   x          [T, d] bf16; topk_idx [T, top_k]; token_row [T, top_k] and
+ *              offsets [n_routed + 1] from moe_permute (or moe_permute_capped;
+ *              a token_row of -1 stays -1)
+ *   xq         [rows_cap, d/2] bytes out, xsf [rows_cap * d/16] bytes out
+ *              (rows_cap = moe_nvfp4_rows_capacity(T, n_routed, top_k)); rows
+ *              between experts (padding) are not written
+ *   token_row_pad [T, top_k] int32 out: the padded row of each (token, slot)
+ *   offsets_pad   [n_routed + 1] int32 out
+ * Limits: d % 256 == 0, n_routed <= 256, 1 <= top_k <= 8.
+ */
+int moe_nvfp4_dispatch(const moe_bf16* x, const int32_t* topk_idx, const int32_t* token_row, const int32_t* offsets,
+                       int T, int d, int n_routed, int top_k, uint8_t* xq, uint8_t* xsf, int32_t* token_row_pad,
+                       int32_t* offsets_pad, void* stream);
+
+/*
+ * moe_nvfp4_grouped_gemm -- out = g_e * (A_e x W_e^T) for every group e on FP4
+ * operands with block scales (tcgen05.mma kind::mxf4nvf4, block16 scales, fp32
+ * accumulation).  Group e: rows offsets_pad[e] .. offsets_pad[e+1]-1 of A,
+ * weight matrix e.
+ *   aq, asf    A codes [rows_cap, K/2] and scales (atom-tiled, K values a row)
+ *   wq, wsf, gscale   from moe_nvfp4_quantize_weights ([n_groups, N, K])
+ *   epilogue   MOE_NVFP4_EPI_GELU_FP4: out_q [rows_cap, N/2] and out_sf
+ *              (atom-tiled, N values a row) get FP4(gelu(.)) -- the expert's
+ *              hidden layer, ready as the second GEMM's A;
+ *              MOE_NVFP4_EPI_BF16: out [rows_cap, N] bf16 at the padded rows,
+ *              or, with offsets_out (e.g. moe_permute's offsets), group e's
+ *              i-th row to row offsets_out[e] + i of out [out_rows, N] for
+ *              i < offsets_out[e+1] - offsets_out[e] (padding rows dropped): the
+ *              y_perm layout moe_combine reads with moe_permute's token_row
+ * Padding rows are computed like any row (their FP4 outputs are not meaningful).
+ * Limits: N % 128 == 0, K % 256 == 0, rows_cap % 128 == 0, n_groups <= 256.
+ */
+int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, const int32_t* offsets_pad, int n_groups,
+                           long long rows_cap, const uint8_t* wq, const uint8_t* wsf, const float* gscale, int N,
+                           int K, int epilogue, uint8_t* out_q, uint8_t* out_sf, moe_bf16* out,
+                           const int32_t* offsets_out, long long out_rows, void* stream);
+
+/*
  * moe_combine -- gate-weighted sum of the contributors, back in token order.
  * "Inkling, Dissected" §02 (the layer output is the weighted sum of the 8
  * contributing experts) and §02b sketch (out += g_k * e_k(x)).

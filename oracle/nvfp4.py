@@ -160,3 +160,41 @@ def expert(x_f32: np.ndarray, w1: tuple, w2: tuple) -> dict:
     hq, hs = quantize_activation(h.astype(np.float32))
     y = gemm(hq, hs, *w2)
     return {"xq": xq, "xs": xs, "pre": pre, "h": h, "hq": hq, "hs": hs, "y": y}
+
+
+# ---------------------------------------------------------------------------
+# the layer with NVFP4 routed experts (router and shared experts in bf16)
+# ---------------------------------------------------------------------------
+def forward_tokens(w, tokens, bias, keep=None, cache=None) -> dict:
+    """The layer's forward for the given tokens of workload w with the routed
+    experts on NVFP4 operands (weights quantized by ``quantize_weight``, each
+    token's activations by ``quantize_activation``) and the shared experts as
+    in the bf16 layer; gates, routing and the combine as ``oracle.forward_tokens``.
+    ``cache`` (dict) keeps quantized expert weights between calls."""
+    import moe_inputs as mi
+    import oracle
+
+    cache = {} if cache is None else cache
+    tokens = np.asarray(tokens, dtype=np.int64)
+    x = mi.host_x(w, tokens)
+    r = oracle.route_workload(w, bias, tokens, mi.host_logit_offset(w), x=x)
+    contrib = r["contrib"]
+    gates = r["gates"].copy()
+    if keep is not None:
+        gates[:, :w.k] = np.where(np.asarray(keep, dtype=bool), gates[:, :w.k], 0.0)
+    xf = mi.bf16_to_f64(x).astype(np.float32)
+    out = np.zeros((len(tokens), w.d), dtype=np.float64)
+    for e in np.unique(contrib):
+        e = int(e)
+        rows, slots = np.nonzero(contrib == e)
+        if e < w.n_routed:
+            if e not in cache:
+                cache[e] = (quantize_weight(mi.bf16_to_f64(mi.host_w1(w, e)).astype(np.float32)),
+                            quantize_weight(mi.bf16_to_f64(mi.host_w2(w, e)).astype(np.float32)))
+            y = expert(xf[rows], *cache[e])["y"]
+        else:
+            y = oracle.expert(x[rows], mi.host_w1(w, e), mi.host_w2(w, e))
+        out[rows] += gates[rows, slots][:, None] * y
+    r["out"] = out
+    r["tokens"] = tokens
+    return r

@@ -39,6 +39,8 @@ MOE_STATUS_BAD_EXPERT = 0x2
 MOE_STATUS_COUNT_MISMATCH = 0x4
 MOE_ACT_GELU_TANH = 0
 MOE_ACT_SWIGLU = 1
+MOE_NVFP4_EPI_GELU_FP4 = 0
+MOE_NVFP4_EPI_BF16 = 1
 
 _vp, _i32, _u64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_float, ctypes.c_size_t
 
@@ -54,6 +56,13 @@ _lib.moe_experts_ffn.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp
                                  _vp, _vp]
 _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_bias_update.argtypes = [_vp, _i32, _i32, _i32, _f32, _vp, _vp]
+_i64 = ctypes.c_longlong
+_lib.moe_nvfp4_quantize_weights.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]
+_lib.moe_nvfp4_rows_capacity.argtypes = [_i32, _i32, _i32]
+_lib.moe_nvfp4_rows_capacity.restype = _i64
+_lib.moe_nvfp4_dispatch.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
+_lib.moe_nvfp4_grouped_gemm.argtypes = [_vp, _vp, _vp, _i32, _i64, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp,
+                                        _vp, _i64, _vp]
 _lib.moe_status_string.argtypes = [_i32]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_get_status.argtypes = [_vp, ctypes.POINTER(_i32)]
@@ -61,6 +70,7 @@ _lib.moe_set_wait_timeout_ns.argtypes = [_u64]
 _lib.moe_debug_bounded_wait.argtypes = [_u64, _vp]
 for _f in ("moe_router_topk", "moe_permute", "moe_permute_capped", "moe_permute_noalloc", "moe_grouped_ffn",
            "moe_experts_ffn", "moe_combine", "moe_bias_update", "moe_load_stats", "moe_get_status",
+           "moe_nvfp4_quantize_weights", "moe_nvfp4_dispatch", "moe_nvfp4_grouped_gemm",
            "moe_set_wait_timeout_ns", "moe_debug_bounded_wait"):
     getattr(_lib, _f).restype = _i32
 
@@ -178,6 +188,29 @@ def moe_load_stats(counts, n_routed: int, capacity: int, stats, stream=None):
     _check("moe_load_stats", _lib.moe_load_stats(_p(counts), n_routed, capacity, _p(stats), _stream(stream)))
 
 
+def moe_nvfp4_quantize_weights(w, G: int, N: int, K: int, q, sf, gscale, stream=None):
+    _check("moe_nvfp4_quantize_weights", _lib.moe_nvfp4_quantize_weights(
+        _p(w), G, N, K, _p(q), _p(sf), _p(gscale), _stream(stream)))
+
+
+def moe_nvfp4_rows_capacity(T: int, n_routed: int, top_k: int) -> int:
+    return int(_lib.moe_nvfp4_rows_capacity(T, n_routed, top_k))
+
+
+def moe_nvfp4_dispatch(x, topk_idx, token_row, offsets, T: int, d: int, n_routed: int, top_k: int, xq, xsf,
+                       token_row_pad, offsets_pad, stream=None):
+    _check("moe_nvfp4_dispatch", _lib.moe_nvfp4_dispatch(
+        _p(x), _p(topk_idx), _p(token_row), _p(offsets), T, d, n_routed, top_k, _p(xq), _p(xsf), _p(token_row_pad),
+        _p(offsets_pad), _stream(stream)))
+
+
+def moe_nvfp4_grouped_gemm(aq, asf, offsets_pad, n_groups: int, rows_cap: int, wq, wsf, gscale, N: int, K: int,
+                           epilogue: int, out_q, out_sf, out, offsets_out, out_rows: int, stream=None):
+    _check("moe_nvfp4_grouped_gemm", _lib.moe_nvfp4_grouped_gemm(
+        _p(aq), _p(asf), _p(offsets_pad), n_groups, rows_cap, _p(wq), _p(wsf), _p(gscale), N, K, epilogue,
+        _p(out_q), _p(out_sf), _p(out), _p(offsets_out), out_rows, _stream(stream)))
+
+
 def capacity_for(factor: float, T: int, k: int, n_routed: int) -> int:
     """Expert capacity in tokens: floor(factor * k*T / n_routed), with the factor
     read as the decimal it prints as (1.25 = 5/4)."""
@@ -228,10 +261,16 @@ class MoELayer:
     """
 
     def __init__(self, shape: LayerShape, device="cuda", fused_experts: bool = True, gather_rows: bool = False,
-                 capacity_factor: Optional[float] = None, activation: str = "gelu_tanh", route_scale: float = 1.0):
+                 capacity_factor: Optional[float] = None, activation: str = "gelu_tanh", route_scale: float = 1.0,
+                 precision: str = "bf16"):
         import torch
 
         self.shape = s = shape
+        # "nvfp4": the routed experts in NVFP4 (W4A4, quantized weights set by set_nvfp4_weights);
+        # the router and the shared experts stay bf16
+        if precision not in ("bf16", "nvfp4"):
+            raise ValueError(precision)
+        self.nvfp4 = precision == "nvfp4"
         # expert type: GELU MLP (w1 [E, d_ff, d]) or SwiGLU (w1 [E, 2*d_ff, d]: gate rows, then up rows)
         self.activation = {"gelu_tanh": MOE_ACT_GELU_TANH, "swiglu": MOE_ACT_SWIGLU}[activation]
         # multiplier of the joint routing weights (route_scale x global_scale of the released config)
@@ -262,9 +301,54 @@ class MoELayer:
         self.y_shared = torch.empty((max(s.n_shared, 1), s.T, s.d), dtype=bf, device=dev)
         self.out = torch.empty((s.T, s.d), dtype=bf, device=dev)
         self.stats = torch.zeros((2,), dtype=torch.int32, device=dev)
+        if self.nvfp4:
+            if self.activation != MOE_ACT_GELU_TANH:
+                raise ValueError("the NVFP4 experts are GELU experts")
+            self.rows_cap = moe_nvfp4_rows_capacity(s.T, s.n_routed, s.top_k)
+            u8 = torch.uint8
+            self.xq = torch.empty((self.rows_cap, s.d // 2), dtype=u8, device=dev)
+            self.xsf = torch.empty((self.rows_cap * s.d // 16,), dtype=u8, device=dev)
+            self.hq = torch.empty((self.rows_cap, s.d_ff // 2), dtype=u8, device=dev)
+            self.hsf = torch.empty((self.rows_cap * s.d_ff // 16,), dtype=u8, device=dev)
+            self.token_row_pad = torch.empty((s.T, s.top_k), dtype=torch.int32, device=dev)
+            self.offsets_pad = torch.empty((s.n_routed + 1,), dtype=torch.int32, device=dev)
+            self.w1q = self.w1sf = self.g1 = self.w2q = self.w2sf = self.g2 = None
         self.side = torch.cuda.Stream(device=dev)
         self.ev_start = torch.cuda.Event()
         self.ev_shared = torch.cuda.Event()
+
+    def set_nvfp4_weights(self, w1, w2, stream=None):
+        """Quantize the routed experts' weights (the first n_routed of w1 [E, d_ff, d] and
+        w2 [E, d, d_ff]) to NVFP4 on the device; the shared experts keep using w1, w2."""
+        import torch
+
+        s = self.shape
+        dev = w1.device
+        E, f, d = s.n_routed, s.d_ff, s.d
+        self.w1q = torch.empty((E, f, d // 2), dtype=torch.uint8, device=dev)
+        self.w1sf = torch.empty((E, f * d // 16), dtype=torch.uint8, device=dev)
+        self.g1 = torch.empty((E,), dtype=torch.float32, device=dev)
+        self.w2q = torch.empty((E, d, f // 2), dtype=torch.uint8, device=dev)
+        self.w2sf = torch.empty((E, d * f // 16), dtype=torch.uint8, device=dev)
+        self.g2 = torch.empty((E,), dtype=torch.float32, device=dev)
+        moe_nvfp4_quantize_weights(w1, E, f, d, self.w1q, self.w1sf, self.g1, stream=stream)
+        moe_nvfp4_quantize_weights(w2, E, d, f, self.w2q, self.w2sf, self.g2, stream=stream)
+
+    def _forward_nvfp4(self, x, w1, w2, main):
+        s = self.shape
+        T, d, f, k = s.T, s.d, s.d_ff, s.top_k
+        if self.w1q is None:
+            raise RuntimeError("set_nvfp4_weights() first")
+        moe_nvfp4_dispatch(x, self.topk_idx, self.token_row, self.offsets, T, d, s.n_routed, k, self.xq, self.xsf,
+                           self.token_row_pad, self.offsets_pad, stream=main)
+        moe_nvfp4_grouped_gemm(self.xq, self.xsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w1q, self.w1sf,
+                               self.g1, f, d, MOE_NVFP4_EPI_GELU_FP4, self.hq, self.hsf, None, None, 0, stream=main)
+        moe_nvfp4_grouped_gemm(self.hq, self.hsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w2q, self.w2sf,
+                               self.g2, d, f, MOE_NVFP4_EPI_BF16, None, None, self.y_perm, self.offsets, T * k,
+                               stream=main)
+        if s.n_shared > 0:
+            moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, self.activation, self.h_shared,
+                            self.y_shared, stream=main)
 
     def forward(self, x, w_router, w1, w2, bias, logit_offset=None, stream=None, scores_out=None,
                 ffn_events=None, out=None):
@@ -283,14 +367,14 @@ class MoELayer:
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
         moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, self.route_scale,
                         self.topk_idx, self.gates, self.counts, scores_out, stream=main)
-        side = s.n_shared > 0 and not self.fused_experts
+        side = s.n_shared > 0 and not self.fused_experts and not self.nvfp4
         if side:
             self.ev_start.record(main)
             self.side.wait_event(self.ev_start)
             moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, self.activation, self.h_shared,
                             self.y_shared, stream=self.side)
             self.ev_shared.record(self.side)
-        x_perm = None if self.gather_rows else self.x_perm
+        x_perm = None if (self.gather_rows or self.nvfp4) else self.x_perm
         if self.capacity is None:
             moe_permute(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.offsets, x_perm, self.row_token,
                         self.token_row, self.scratch, self.scratch_bytes, stream=main)
@@ -299,7 +383,9 @@ class MoELayer:
                                x_perm, self.row_token, self.token_row, self.scratch, self.scratch_bytes, stream=main)
         if ffn_events is not None:
             ffn_events[0].record(main)
-        if self.fused_experts:
+        if self.nvfp4:
+            self._forward_nvfp4(x, w1, w2, main)
+        elif self.fused_experts:
             moe_experts_ffn(x, x_perm, self.row_token, self.offsets, T, s.n_routed, s.n_shared, k, w1, w2, d, f,
                             self.activation, self.h, self.y_perm, self.y_shared, stream=main)
         else:
@@ -317,6 +403,8 @@ class MoELayer:
     # kernels of libmoe launched by one forward + bias update
     def launches_per_step(self) -> int:
         """libmoe kernels one forward + bias update launches."""
+        if self.nvfp4:  # permute (indices) 3, FP4 dispatch 1, FP4 GEMMs 2, shared bf16 GEMMs 2
+            return 1 + 3 + 1 + 2 + 2 + 1 + 1
         experts = 2 if self.fused_experts else 4
         permute = 3 if self.gather_rows else 4
         return 1 + permute + experts + 1 + 1

@@ -95,11 +95,12 @@ namespace {
 struct TmapKey {
   const void* base;
   int rank;
+  int elem_bytes;  // 2: bf16, 1: bytes (packed FP4 pairs)
   uint64_t dim0, dim1, dim2;
   uint32_t box0, box1;
   bool operator==(const TmapKey& o) const {
-    return base == o.base && rank == o.rank && dim0 == o.dim0 && dim1 == o.dim1 && dim2 == o.dim2 &&
-           box0 == o.box0 && box1 == o.box1;
+    return base == o.base && rank == o.rank && elem_bytes == o.elem_bytes && dim0 == o.dim0 && dim1 == o.dim1 &&
+           dim2 == o.dim2 && box0 == o.box0 && box1 == o.box1;
   }
 };
 
@@ -115,9 +116,9 @@ std::mutex g_tmap_mu;
 
 }  // namespace
 
-int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
-                     uint32_t box0, uint32_t box1) {
-  const TmapKey key{base, rank, dim0, dim1, rank == 3 ? dim2 : 1, box0, box1};
+static int encode_tmap(CUtensorMap* map, const void* base, int elem_bytes, int rank, uint64_t dim0, uint64_t dim1,
+                       uint64_t dim2, uint32_t box0, uint32_t box1) {
+  const TmapKey key{base, rank, elem_bytes, dim0, dim1, rank == 3 ? dim2 : 1, box0, box1};
   {
     std::lock_guard<std::mutex> lk(g_tmap_mu);
     for (int i = 0; i < kTmapCacheSize; ++i) {
@@ -130,11 +131,11 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return MOE_ERR_CUDA;
   cuuint64_t dims[3] = {dim0, dim1, dim2};
-  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  cuuint64_t strides[2] = {dim0 * elem_bytes, dim0 * dim1 * elem_bytes};
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   memset(map, 0, sizeof(*map));
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
@@ -145,6 +146,16 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0
   e.key = key;
   e.map = *map;
   return MOE_OK;
+}
+
+int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                     uint32_t box0, uint32_t box1) {
+  return encode_tmap(map, base, 2, rank, dim0, dim1, dim2, box0, box1);
+}
+
+int encode_tmap_u8(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                   uint32_t box0, uint32_t box1) {
+  return encode_tmap(map, base, 1, rank, dim0, dim1, dim2, box0, box1);
 }
 
 namespace {

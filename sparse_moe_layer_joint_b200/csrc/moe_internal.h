@@ -24,6 +24,10 @@ int ensure_smem_attr(const void* kernel, size_t bytes);
 int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                      uint32_t box0, uint32_t box1);
 
+// The same for a byte tensor (dims and box in bytes; packed FP4 pairs).
+int encode_tmap_u8(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                   uint32_t box0, uint32_t box1);
+
 // Limit on device-side waits for kernels launched from now on.
 uint64_t wait_timeout_ns();
 

@@ -1,0 +1,645 @@
+// nvfp4.cu -- the routed experts in NVFP4 (W4A4): FP4 (E2M1) weights and
+// activations in blocks of 16 values, each block with an FP8 (E4M3) scale, on
+// the tcgen05 block-scaled tensor-core path ("Under the hood", "Quantization:
+// BF16 vs NVFP4": FP4 weights and activations, group size 16, FP8 scale
+// metadata, dynamic block scales, for Blackwell FP4 tensor cores).
+//
+// Recipe (every conversion rounds to nearest, ties to even, and saturates):
+//   weights      one fp32 scale per matrix, g = amax|W| / (6 * 448); per block
+//                s = E4M3(fl(amax_b / 6) / g); codes E2M1(w / fl(s * g))
+//   activations  per block s = E4M3(fl(amax_b / 6)); codes E2M1(x / s)
+// A block whose scale rounds to zero has all codes zero.
+//
+// Layouts (device memory, all caller-owned):
+//   codes        [rows, K/2] bytes, K-major; byte j of a row holds values 2j
+//                (bits 0-3) and 2j+1 (bits 4-7)
+//   scales       atom-tiled: atoms of 128 rows x 64 values (4 scales a row),
+//                512 bytes, the atoms of one 128-row block consecutive along K;
+//                inside an atom the scale of (row r, block b) is at byte
+//                (r % 32) * 16 + (r % 128 / 32) * 4 + b % 4 -- one 32 x 16-byte
+//                block that tcgen05.cp copies to TMEM as the MMA reads it
+//   routed rows  each expert's rows start at a multiple of 128 ("padded"
+//                offsets), so every 128-row tile owns whole scale atoms
+//
+// Kernels:
+//   weight_amax / weight_quant / weight_scale   weights, once
+//   dispatch_quant   x rows quantized once per token and written to the padded
+//                    rows of its k experts (the FP4 dispatch)
+//   fp4_gemm_kernel<EPI>   persistent grouped GEMM, one CTA per 128 x 128 tile:
+//                    warp 0 loads code tiles (TMA, 128-byte swizzle) and scale
+//                    atoms (bulk copies), warp 1 copies the scales to TMEM
+//                    (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4 with
+//                    block16 scales, warps 2-5 drain the accumulator: x the
+//                    weight matrix's g, then GELU and FP4 re-quantization
+//                    (GEMM1) or bf16 (GEMM2)
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace fp4 {
+
+constexpr int ATOM_ROWS = 128;
+constexpr int ATOM_K = 64;
+constexpr int ATOM_BYTES = 512;
+constexpr float E2M1_MAX = 6.0f;
+constexpr float E4M3_MAX = 448.0f;
+
+// Byte offset of the scale of (row r, 16-value block b) in the atom-tiled
+// layout of a matrix with K values per row.
+__host__ __device__ __forceinline__ size_t sf_offset(long long r, int b, int K) {
+  const long long atoms_k = K / ATOM_K;
+  return (size_t)(((r / ATOM_ROWS) * atoms_k + (b >> 2)) * ATOM_BYTES + (r & 31) * 16 + ((r & 127) >> 5) * 4 +
+                  (b & 3));
+}
+
+// Nearest E2M1 value (ties to the even code), saturating at +-6; no negative zero.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float m = fabsf(v);
+  uint32_t c = m <= 0.25f ? 0u
+               : m < 0.75f ? 1u
+               : m <= 1.25f ? 2u
+               : m < 1.75f ? 3u
+               : m <= 2.5f ? 4u
+               : m < 3.5f ? 5u
+               : m <= 5.0f ? 6u
+                           : 7u;
+  if (c != 0u && v < 0.0f) c |= 8u;
+  return c;
+}
+
+__device__ __forceinline__ uint32_t e4m3_code(float s) {  // s >= 0
+  return (uint32_t)__nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  return e == 0u ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// 16 values with one scale (already chosen): packed codes, 4 bits each, value i at bits 4i of word i/8.
+__device__ __forceinline__ uint2 pack16(const float* v, float denom) {
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t c = denom > 0.0f ? e2m1_code(__fdiv_rn(v[i], denom)) : 0u;
+    w[i >> 3] |= c << (4 * (i & 7));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// Activation block: dynamic scale, no tensor scale.
+__device__ __forceinline__ uint2 quant16_act(const float* v, uint32_t& sf) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  sf = e4m3_code(__fdiv_rn(amax, E2M1_MAX));
+  return pack16(v, e4m3_value(sf));
+}
+
+__device__ __forceinline__ void bf16x8_to_float(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// GELU, tanh form, with the accurate tanh: its output decides FP4 codes, so it
+// is kept as close as the fp32 arithmetic allows.
+__device__ __forceinline__ float gelu_tanh_accurate(float u) {
+  const float k0 = 0.7978845608028654f;
+  const float k1 = 0.044715f;
+  return 0.5f * u * (1.0f + tanhf(k0 * (u + k1 * u * u * u)));
+}
+
+// ---------------------------------------------------------------------------
+// weights
+// ---------------------------------------------------------------------------
+__global__ void weight_amax_kernel(const uint4* __restrict__ w, long long vec_per_matrix,
+                                   unsigned int* __restrict__ amax_bits) {
+  const int g = blockIdx.y;
+  const uint4* src = w + (size_t)g * vec_per_matrix;
+  float m = 0.0f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < vec_per_matrix;
+       i += (long long)gridDim.x * blockDim.x) {
+    float f[8];
+    bf16x8_to_float(__ldg(src + i), f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(f[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits + g, __float_as_uint(m));  // m >= 0: bits order as values
+}
+
+// One thread per 16-value block of one row of one matrix.
+__global__ void weight_quant_kernel(const uint4* __restrict__ w, int G, int N, int K,
+                                    const unsigned int* __restrict__ amax_bits, uint8_t* __restrict__ q,
+                                    uint8_t* __restrict__ sf) {
+  const int nb = K / 16;
+  const long long units = (long long)G * N * nb;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int b = (int)(u % nb);
+    const long long rowg = u / nb;  // g * N + n
+    const int g = (int)(rowg / N);
+    const int n = (int)(rowg - (long long)g * N);
+    const float gs = __fdiv_rn(__uint_as_float(amax_bits[g]), E2M1_MAX * E4M3_MAX);
+    float v[16];
+    const uint4* src = w + rowg * (K / 8) + 2 * b;
+    bf16x8_to_float(__ldg(src), v);
+    bf16x8_to_float(__ldg(src + 1), v + 8);
+    uint32_t s = 0u;
+    float denom = 0.0f;
+    if (gs > 0.0f) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      s = e4m3_code(__fdiv_rn(__fdiv_rn(amax, E2M1_MAX), gs));
+      denom = __fmul_rn(e4m3_value(s), gs);
+    }
+    *reinterpret_cast<uint2*>(q + rowg * (K / 2) + 8 * b) = pack16(v, denom);
+    sf[(size_t)g * N * nb + sf_offset(n, b, K)] = (uint8_t)s;
+  }
+}
+
+__global__ void weight_scale_kernel(unsigned int* amax_bits_to_scale, int G) {
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g < G) {
+    const float s = __fdiv_rn(__uint_as_float(amax_bits_to_scale[g]), E2M1_MAX * E4M3_MAX);
+    amax_bits_to_scale[g] = __float_as_uint(s);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dispatch: quantize each token's x once, write it to its k padded rows
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) dispatch_quant_kernel(const uint4* __restrict__ x,
+                                                             const int32_t* __restrict__ topk_idx,
+                                                             const int32_t* __restrict__ token_row,
+                                                             const int32_t* __restrict__ offsets, int T, int d,
+                                                             int n_routed, int k, long long rows_cap,
+                                                             uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf,
+                                                             int32_t* __restrict__ token_row_pad,
+                                                             int32_t* __restrict__ offsets_pad) {
+  __shared__ int off[MOE_MAX_ROUTED + 1], offp[MOE_MAX_ROUTED + 1];
+  __shared__ int wsum[8];
+  // padded offsets: every expert's rows start at a multiple of 128
+  {
+    const int e = threadIdx.x;
+    int n = 0;
+    if (e < n_routed) {
+      off[e] = offsets[e];
+      n = offsets[e + 1] - offsets[e];
+      n = n < 0 ? 0 : n;
+    }
+    if (e == n_routed - 1) off[n_routed] = offsets[n_routed];
+    int v = (n + ATOM_ROWS - 1) / ATOM_ROWS * ATOM_ROWS;
+    const int own = v;
+    const int lane = e & 31, w = e >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    if (lane == 31) wsum[w] = v;
+    __syncthreads();
+    int before = 0;
+    for (int i = 0; i < w; ++i) before += wsum[i];
+    if (e < n_routed) offp[e] = before + v - own;
+    if (e == n_routed - 1) offp[n_routed] = before + v;
+    __syncthreads();
+    if (blockIdx.x == 0 && e < n_routed) offsets_pad[e] = offp[e];
+    if (blockIdx.x == 0 && e == 0) offsets_pad[n_routed] = offp[n_routed];  // n_routed may equal the block size
+  }
+  const int nb = d / 16;
+  const long long units = (long long)T * nb;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(u / nb);
+    const int b = (int)(u - (long long)t * nb);
+    float v[16];
+    const uint4* src = x + (size_t)t * (d / 8) + 2 * b;
+    bf16x8_to_float(__ldg(src), v);
+    bf16x8_to_float(__ldg(src + 1), v + 8);
+    uint32_t s;
+    const uint2 packed = quant16_act(v, s);
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(topk_idx + (size_t)t * k + j);
+      const int r = __ldg(token_row + (size_t)t * k + j);
+      long long rp = -1;
+      if (e >= 0 && e < n_routed && r >= off[e] && r < off[e + 1]) rp = (long long)r - off[e] + offp[e];
+      if (rp >= rows_cap) rp = -1;
+      if (b == 0) token_row_pad[(size_t)t * k + j] = (int32_t)rp;
+      if (rp < 0) continue;
+      *reinterpret_cast<uint2*>(xq + rp * (d / 2) + 8 * b) = packed;
+      xsf[sf_offset(rp, b, d)] = (uint8_t)s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// grouped GEMM on NVFP4 operands
+// ---------------------------------------------------------------------------
+constexpr int NUM_THREADS = 192;
+constexpr int TM = 128;           // rows per tile
+constexpr int TN = 128;           // output columns per tile (MMA N)
+constexpr int ROW_BYTES = 128;    // code bytes per row per stage: 256 values
+constexpr int KV_STAGE = 256;     // values along K per stage
+constexpr int STAGES = 5;
+constexpr int A_BYTES = TM * ROW_BYTES;
+constexpr int B_BYTES = TN * ROW_BYTES;
+constexpr int SF_BYTES = (KV_STAGE / ATOM_K) * ATOM_BYTES;  // 4 atoms = 2 KB per operand per stage
+constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + 2 * SF_BYTES;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SFA_COL = 256;  // 16 columns: 4 K-chunks x 4
+constexpr uint32_t SFB_COL = 320;
+constexpr int EPI_GELU_FP4 = 0;   // GEMM1: x g1, GELU, FP4 out (the next GEMM's A)
+constexpr int EPI_BF16 = 1;       // GEMM2: x g2, bf16 out
+
+struct Params {
+  const int* offsets_pad;  // [G + 1] group row starts, multiples of 128
+  int G;
+  long long rows_cap;      // rows of A / of the outputs
+  const uint8_t* a_sf;     // atom-tiled scales of A [rows_cap, K]
+  const uint8_t* b_sf;     // atom-tiled scales of the weights, per group b_sf_stride bytes
+  long long b_sf_stride;
+  const float* gscale;     // [G] weight tensor scales
+  int N, K, n_tiles_n;
+  uint8_t* out_q;          // EPI_GELU_FP4: codes [rows_cap, N/2] and atom-tiled scales
+  uint8_t* out_sf;
+  __nv_bfloat16* out;      // EPI_BF16: [rows_cap, N], or [out_rows, N] through offsets_out
+  const int* offsets_out;  // EPI_BF16, nullable: group e's row i goes to row offsets_out[e] + i (i < its count)
+  long long out_rows;
+  uint64_t timeout_ns;
+  unsigned int* status;
+};
+
+struct Tables {
+  int off[MOE_MAX_ROUTED + 1];
+  int prefix[MOE_MAX_ROUTED + 1];  // row tiles of groups < g
+  int off_out[MOE_MAX_ROUTED + 1];
+};
+
+struct SmemTail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  Tables t;
+};
+
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + 2 * SF_BYTES) + sizeof(SmemTail);
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sSFA = sB + STAGES * B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * SF_BYTES;
+  SmemTail* st = reinterpret_cast<SmemTail*>(sSFB + STAGES * SF_BYTES);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&st->full[s], 1);
+      mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&st->tfull[a], 1);
+      mbar_init(&st->tempty[a], 4);
+    }
+    mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    fence_barrier_init();
+  }
+  // group tables: clamped padded offsets and the row-tile prefix
+  for (int i = tid; i <= p.G; i += NUM_THREADS) {
+    long long v = p.offsets_pad[i];
+    v = v < 0 ? 0 : (v > p.rows_cap ? p.rows_cap : v);
+    st->t.off[i] = (int)v;
+    if (p.offsets_out != nullptr) {
+      long long o = p.offsets_out[i];
+      st->t.off_out[i] = (int)(o < 0 ? 0 : (o > p.out_rows ? p.out_rows : o));
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int g = 0; g < p.G; ++g) {
+      st->t.prefix[g] = run;
+      const int rows = st->t.off[g + 1] - st->t.off[g];
+      run += rows > 0 ? (rows + TM - 1) / TM : 0;
+    }
+    st->t.prefix[p.G] = run;
+  }
+  __syncthreads();
+  const int total_tiles = st->t.prefix[p.G] * p.n_tiles_n;
+  if ((int)blockIdx.x >= total_tiles) return;
+
+  if (warp == 1) tmem_alloc(&st->tmem_base, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = st->tmem_base;
+  const int num_kb = p.K / KV_STAGE;
+  const int atoms_k = p.K / ATOM_K;
+  volatile int* abort_flag = &st->abort_flag;
+
+  auto tile_of = [&](int tile, int& g, int& m, int& nt) {
+    const int mt = tile / p.n_tiles_n;
+    nt = tile - mt * p.n_tiles_n;
+    int lo = 0, hi = p.G;  // largest g with prefix[g] <= mt
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (st->t.prefix[mid] <= mt)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    g = lo;
+    m = mt - st->t.prefix[lo];
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        int g, m, nt;
+        tile_of(tile, g, m, nt);
+        const int a_row = st->t.off[g] + m * TM;
+        const int n0 = nt * TN;
+        const uint8_t* sfa = p.a_sf + ((size_t)(a_row / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
+        const uint8_t* sfb = p.b_sf + (size_t)g * p.b_sf_stride + ((size_t)(n0 / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
+          if (!ok) break;
+          uint64_t* bar = &st->full[stage];
+          mbar_arrive_expect_tx(bar, STAGE_TX);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
+          tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
+          bulk_load(sSFA + stage * SF_BYTES, sfa + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+          bulk_load(sSFB + stage * SF_BYTES, sfb + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // wind down: let the copies already issued land before the CTA exits
+        int zero = 0;
+        for (long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+          mbar_wait(&st->full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.timeout_ns, &zero, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_nvf4(TM, TN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&st->full[stage], phase, p.timeout_ns, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+          const uint32_t sfa_addr = smem_u32(sSFA + stage * SF_BYTES);
+          const uint32_t sfb_addr = smem_u32(sSFB + stage * SF_BYTES);
+#pragma unroll
+          for (int j = 0; j < KV_STAGE / ATOM_K; ++j) {
+            tmem_cp_sf(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
+            tmem_cp_sf(tmem_base + SFB_COL + 4 * j, make_desc_sf(sfb_addr + j * ATOM_BYTES));
+          }
+#pragma unroll
+          for (int j = 0; j < KV_STAGE / ATOM_K; ++j)
+            mma_nvf4_ss(d_tmem, make_desc_sw128(a_addr + j * 32), make_desc_sw128(b_addr + j * 32), idesc,
+                        tmem_base + SFA_COL + 4 * j, tmem_base + SFB_COL + 4 * j, (kb | j) != 0 ? 1u : 0u);
+          mma_commit(&st->empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&st->tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      int zero = 0;
+      mma_commit(&st->drain);
+      mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, one tile row per thread
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int g, m, nt;
+      tile_of(tile, g, m, nt);
+      const int in_group = m * TM + quarter * 32 + lane;  // row within the group
+      const long long r = (long long)st->t.off[g] + in_group;
+      bool valid = r < p.rows_cap;
+      long long r_out = r;  // output row
+      if (EPI == EPI_BF16 && p.offsets_out != nullptr) {
+        r_out = (long long)st->t.off_out[g] + in_group;
+        valid = in_group < st->t.off_out[g + 1] - st->t.off_out[g] && r_out < p.out_rows;
+      }
+      const float gs = __ldg(p.gscale + g);
+      if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TN);
+#pragma unroll 1
+      for (int ch = 0; ch < TN / 32; ++ch) {
+        const int col0 = nt * TN + ch * 32;
+        if (col0 >= p.N) break;  // same for the whole warp
+        float v[32];
+        tmem_ld32(taddr + ch * 32, v);
+        if (!valid) continue;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], gs);
+        if (EPI == EPI_GELU_FP4) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_accurate(v[i]);
+          uint32_t s0, s1;
+          const uint2 q0 = quant16_act(v, s0);
+          const uint2 q1 = quant16_act(v + 16, s1);
+          *reinterpret_cast<uint4*>(p.out_q + r * (p.N / 2) + col0 / 2) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+          const size_t so = sf_offset(r, col0 / 16, p.N);  // the two blocks share an atom line (b even)
+          p.out_sf[so] = (uint8_t)s0;
+          p.out_sf[so + 1] = (uint8_t)s1;
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + r_out * p.N + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&st->tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace fp4
+}  // namespace moe
+
+using namespace moe;
+using namespace moe::fp4;
+
+extern "C" int moe_nvfp4_quantize_weights(const moe_bf16* w, int G, int N, int K, uint8_t* q, uint8_t* sf,
+                                          float* gscale, void* stream) {
+  if (!w || !q || !sf || !gscale || G < 0 || N < 0 || K < 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(q) || !aligned16(sf) || !aligned4(gscale)) return MOE_ERR_INVALID_ARG;
+  if (N % ATOM_ROWS != 0 || K % KV_STAGE != 0) return MOE_ERR_UNSUPPORTED;
+  if (G == 0 || N == 0 || K == 0) return MOE_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  int dev, sms;
+  int rc = device_info(&dev, &sms);
+  if (rc != MOE_OK) return rc;
+  unsigned int* amax = reinterpret_cast<unsigned int*>(gscale);  // amax first, then the scale, in place
+  if (cudaMemsetAsync(amax, 0, sizeof(float) * G, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const long long vec = (long long)N * K / 8;
+  const int bx = (int)((vec + 256 * 8 - 1) / (256 * 8) < 64 ? (vec + 256 * 8 - 1) / (256 * 8) : 64);
+  weight_amax_kernel<<<dim3(bx, G), 256, 0, s>>>(reinterpret_cast<const uint4*>(w), vec, amax);
+  const long long units = (long long)G * N * (K / 16);
+  const int grid = (int)(units / 256 + 1 < (long long)sms * 16 ? units / 256 + 1 : (long long)sms * 16);
+  weight_quant_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(w), G, N, K, amax, q, sf);
+  weight_scale_kernel<<<(G + 255) / 256, 256, 0, s>>>(amax, G);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" long long moe_nvfp4_rows_capacity(int T, int n_routed, int top_k) {
+  if (T < 0 || n_routed < 1 || top_k < 1) return 0;
+  const long long r = (long long)T * top_k + (long long)n_routed * (ATOM_ROWS - 1);
+  return (r + ATOM_ROWS - 1) / ATOM_ROWS * ATOM_ROWS;
+}
+
+extern "C" int moe_nvfp4_dispatch(const moe_bf16* x, const int32_t* topk_idx, const int32_t* token_row,
+                                  const int32_t* offsets, int T, int d, int n_routed, int top_k, uint8_t* xq,
+                                  uint8_t* xsf, int32_t* token_row_pad, int32_t* offsets_pad, void* stream) {
+  if (!x || !topk_idx || !token_row || !offsets || !xq || !xsf || !token_row_pad || !offsets_pad)
+    return MOE_ERR_INVALID_ARG;
+  if (T < 0 || d <= 0 || n_routed < 1 || n_routed > MOE_MAX_ROUTED || top_k < 1 || top_k > MOE_MAX_TOP_K)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(xsf) || !aligned4(topk_idx) || !aligned4(token_row) ||
+      !aligned4(offsets) || !aligned4(token_row_pad) || !aligned4(offsets_pad))
+    return MOE_ERR_INVALID_ARG;
+  if (d % KV_STAGE != 0) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  int dev, sms;
+  int rc = device_info(&dev, &sms);
+  if (rc != MOE_OK) return rc;
+  const long long units = (long long)T * (d / 16);
+  long long grid = (units + 255) / 256;
+  if (grid > (long long)sms * 8) grid = (long long)sms * 8;
+  if (grid < 1) grid = 1;  // the offsets are written even with no tokens
+  dispatch_quant_kernel<<<(int)grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), topk_idx, token_row, offsets,
+                                                 T, d, n_routed, top_k, moe_nvfp4_rows_capacity(T, n_routed, top_k),
+                                                 xq, xsf, token_row_pad, offsets_pad);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, const int32_t* offsets_pad,
+                                      int n_groups, long long rows_cap, const uint8_t* wq, const uint8_t* wsf,
+                                      const float* gscale, int N, int K, int epilogue, uint8_t* out_q,
+                                      uint8_t* out_sf, moe_bf16* out, const int32_t* offsets_out,
+                                      long long out_rows, void* stream) {
+  if (!aq || !asf || !offsets_pad || !wq || !wsf || !gscale || n_groups < 0 || rows_cap < 0 || N <= 0 || K <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (n_groups > MOE_MAX_ROUTED) return MOE_ERR_UNSUPPORTED;
+  if (epilogue != MOE_NVFP4_EPI_GELU_FP4 && epilogue != MOE_NVFP4_EPI_BF16) return MOE_ERR_INVALID_ARG;
+  if (epilogue == MOE_NVFP4_EPI_GELU_FP4 && (!out_q || !out_sf || !aligned16(out_q))) return MOE_ERR_INVALID_ARG;
+  if (epilogue == MOE_NVFP4_EPI_BF16 && (!out || !aligned16(out))) return MOE_ERR_INVALID_ARG;
+  if (offsets_out != nullptr && (!aligned4(offsets_out) || out_rows < 0 || out_rows > 0x7fffffffLL))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(aq) || !aligned16(asf) || !aligned16(wq) || !aligned16(wsf) || !aligned4(gscale) ||
+      !aligned4(offsets_pad))
+    return MOE_ERR_INVALID_ARG;
+  if (N % TN != 0 || K % KV_STAGE != 0 || rows_cap % ATOM_ROWS != 0) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (n_groups == 0 || rows_cap == 0) return MOE_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  int dev, sms;
+  int rc = device_info(&dev, &sms);
+  if (rc != MOE_OK) return rc;
+  unsigned int* status = status_ptr();
+  if (!status) return MOE_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if ((rc = encode_tmap_u8(&ta, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, TM)) != MOE_OK) return rc;
+  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, (uint64_t)N, (uint64_t)n_groups, ROW_BYTES, TN)) != MOE_OK)
+    return rc;
+  Params p{};
+  p.offsets_pad = offsets_pad;
+  p.G = n_groups;
+  p.rows_cap = rows_cap;
+  p.a_sf = asf;
+  p.b_sf = wsf;
+  p.b_sf_stride = (long long)N * (K / 16);
+  p.gscale = gscale;
+  p.N = N;
+  p.K = K;
+  p.n_tiles_n = N / TN;
+  p.out_q = out_q;
+  p.out_sf = out_sf;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.offsets_out = epilogue == MOE_NVFP4_EPI_BF16 ? offsets_out : nullptr;
+  p.out_rows = out_rows;
+  p.timeout_ns = wait_timeout_ns();
+  p.status = status;
+  const long long tiles_upper = (rows_cap / TM) * p.n_tiles_n;
+  const int grid = (int)(tiles_upper < sms ? tiles_upper : sms);
+  if (epilogue == MOE_NVFP4_EPI_GELU_FP4) {
+    auto kfn = fp4_gemm_kernel<EPI_GELU_FP4>;
+    if ((rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES)) != MOE_OK) return rc;
+    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+  } else {
+    auto kfn = fp4_gemm_kernel<EPI_BF16>;
+    if ((rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES)) != MOE_OK) return rc;
+    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

@@ -225,6 +225,56 @@ __device__ __forceinline__ float gelu_tanh_f32(float u) {
   return 0.5f * u * (1.0f + tanh_approx(inner));
 }
 
+// ----------------------------------------------------------------------------
+// NVFP4 (block-scaled FP4) operands
+// ----------------------------------------------------------------------------
+// Untiled bulk copy global -> this CTA's shared memory, completing on an
+// mbarrier (both addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte scale-factor block stored as
+// 512 contiguous bytes (no swizzle; 8-row core matrices of 128 B, 128 B apart).
+__device__ __forceinline__ uint64_t make_desc_sf(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)(128u >> 4) << 16;          // leading byte offset (one core matrix along K)
+  d |= (uint64_t)(128u >> 4) << 32;          // stride byte offset: next 8 rows
+  d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
+  return d;                                   // layout type 0: no swizzle
+}
+
+// Copy one 32 x 128-bit scale-factor block from shared memory into TMEM columns
+// [taddr, taddr + 4), the same data into the lanes of all four warps' quarters.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor, kind::mxf4nvf4 with block16 scales: packed E2M1 A and
+// B (K-major), E4M3 scale factors, fp32 accumulator, K = 64 per instruction.
+__host__ __device__ constexpr uint32_t make_idesc_nvf4(int M, int N) {
+  return (1u << 7)                        // A format: E2M1
+         | (1u << 10)                     // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | (0u << 23)                     // scale format: E4M3
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= (A * SFA)[smem] x (B * SFB)[smem]^T over K = 64, SFA / SFB in TMEM.
+__device__ __forceinline__ void mma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+
 // SiLU (the swish of a SwiGLU gate), u * sigmoid(u) = u / (1 + e^-u), in fp32.
 // For very negative u, e^-u overflows to inf and the reciprocal to 0: silu -> -0.
 __device__ __forceinline__ float silu_f32(float u) { return u * __frcp_rn(1.0f + __expf(-u)); }

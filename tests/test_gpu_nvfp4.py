@@ -1,0 +1,219 @@
+"""NVFP4 routed experts on the GPU ("Under the hood", "Quantization: BF16 vs
+NVFP4": FP4 weights and activations, blocks of 16, FP8 scales) against the
+oracle: weight and activation quantization bit-exact, the block-scaled grouped
+GEMM on the oracle's quantized operands, and the layer with NVFP4 experts."""
+import numpy as np
+import pytest
+
+import moe_inputs as mi
+import oracle
+from oracle import nvfp4
+from parity import check_output, check_routing, dev_bf16, host_bf16_bits, host_bf16_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if torch.cuda.is_available():
+    import sparse_moe_layer_joint_b200 as moe
+
+
+# the documented device layouts, written out for the tests
+def _unpack_codes(b):
+    b = np.asarray(b, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = b & 15
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def _pack_codes(c):
+    c = np.asarray(c, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def _sf_index(R, K):
+    r = np.arange(R)[:, None]
+    b = np.arange(K // 16)[None, :]
+    return (((r // 128) * (K // 64) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4)
+
+
+def _sf_logical(buf, R, K):
+    return np.asarray(buf, dtype=np.uint8).reshape(-1)[_sf_index(R, K)]
+
+
+def _sf_tiled(s, R, K):
+    out = np.zeros(R * K // 16, dtype=np.uint8)
+    out[_sf_index(R, K)] = s
+    return out
+
+
+def _u8(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
+def _i32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+@pytest.mark.parametrize("G,N,K,std", [(3, 256, 512, 0.05), (2, 128, 256, 30.0), (1, 384, 768, 1e-3)])
+def test_quantize_weights_bit_exact(G, N, K, std):
+    w = mi.normal_bf16(G * N * K, 21, mi.STREAM_W1, std=std).reshape(G, N, K)
+    if G > 1:
+        w[1] = 0                                              # an all-zero matrix: g = 0, codes 0
+    q = torch.empty((G, N, K // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((G, N * K // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(G, dtype=torch.float32, device="cuda")
+    moe.moe_nvfp4_quantize_weights(dev_bf16(w), G, N, K, q, sf, g)
+    assert moe.moe_get_status() == 0
+    qh, sfh, gh = q.cpu().numpy(), sf.cpu().numpy(), g.cpu().numpy()
+    for i in range(G):
+        rq, rs, rg = nvfp4.quantize_weight(mi.bf16_to_f64(w[i]).astype(np.float32))
+        assert gh[i] == rg
+        np.testing.assert_array_equal(_unpack_codes(qh[i]), rq)
+        np.testing.assert_array_equal(_sf_logical(sfh[i], N, K), rs)
+
+
+def _dispatch(T, k, E, d, seed, cap=None):
+    x = mi.normal_bf16(T * d, seed, mi.STREAM_X).reshape(T, d)
+    u = mi.words(T * E, seed, mi.STREAM_TEST_TOPK).reshape(T, E).astype(np.float64)
+    topk = np.argsort(-(u - 2e9 * np.log1p(np.arange(E))[None, :] / 10), axis=1, kind="stable")[:, :k].astype(np.int32)
+    keep = oracle.capacity_keep(topk, cap, E) if cap is not None else None
+    dp = oracle.dispatch(topk, E, keep)
+    rows_cap = moe.moe_nvfp4_rows_capacity(T, E, k)
+    xq = torch.zeros((rows_cap, d // 2), dtype=torch.uint8, device="cuda")
+    xsf = torch.zeros((rows_cap * d // 16,), dtype=torch.uint8, device="cuda")
+    trp = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    offp = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    moe.moe_nvfp4_dispatch(dev_bf16(x), _i32(topk), _i32(dp["token_row"]), _i32(dp["offsets"]), T, d, E, k, xq, xsf,
+                           trp, offp)
+    assert moe.moe_get_status() == 0
+    return x, topk, dp, rows_cap, xq, xsf, trp, offp
+
+
+@pytest.mark.parametrize("T,k,E,d,cap", [(300, 6, 16, 512, None), (1, 6, 256, 256, None), (1000, 2, 64, 768, 40),
+                                         (513, 8, 8, 256, None)])
+def test_dispatch_quant_bit_exact(T, k, E, d, cap):
+    x, topk, dp, rows_cap, xq, xsf, trp, offp = _dispatch(T, k, E, d, T + E, cap)
+    counts = np.diff(dp["offsets"])
+    off_pad = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)])
+    np.testing.assert_array_equal(offp.cpu().numpy(), off_pad)
+    # the padded row of (t, j): same place in its expert's rows as in the unpadded layout
+    tr = dp["token_row"]
+    e_of = topk.astype(np.int64)
+    expect = np.where(tr >= 0, tr - dp["offsets"][e_of] + off_pad[e_of], -1)
+    np.testing.assert_array_equal(trp.cpu().numpy(), expect)
+    q_ref, s_ref = nvfp4.quantize_activation(mi.bf16_to_f64(x).astype(np.float32))
+    codes = _unpack_codes(xq.cpu().numpy())
+    sfs = _sf_logical(xsf.cpu().numpy(), rows_cap, d)
+    t_idx, j_idx = np.nonzero(expect >= 0)
+    rows = expect[t_idx, j_idx]
+    np.testing.assert_array_equal(codes[rows], q_ref[t_idx])
+    np.testing.assert_array_equal(sfs[rows], s_ref[t_idx])
+
+
+def _gemm_inputs(sizes, N, K, seed):
+    """A (activations) and W quantized by the oracle, laid out as the device expects."""
+    G = len(sizes)
+    off_pad = np.concatenate([[0], np.cumsum([(n + 127) // 128 * 128 for n in sizes])]).astype(np.int32)
+    rows_cap = max(int(off_pad[-1]), 128)
+    a = (mi.normal_f64(rows_cap * K, seed, mi.STREAM_TEST_ROWS).reshape(rows_cap, K)).astype(np.float32)
+    aq, as_ = nvfp4.quantize_activation(a)
+    w = mi.normal_bf16(G * N * K, seed, mi.STREAM_W1, std=K ** -0.5).reshape(G, N, K)
+    wq = [nvfp4.quantize_weight(mi.bf16_to_f64(w[g]).astype(np.float32)) for g in range(G)]
+    dev = {
+        "aq": _u8(_pack_codes(aq)), "asf": _u8(_sf_tiled(as_, rows_cap, K)), "off_pad": _i32(off_pad),
+        "wq": _u8(np.stack([_pack_codes(q) for q, _, _ in wq])),
+        "wsf": _u8(np.stack([_sf_tiled(s, N, K) for _, s, _ in wq])),
+        "g": torch.tensor([gg for _, _, gg in wq], dtype=torch.float32, device="cuda"),
+    }
+    return aq, as_, wq, off_pad, rows_cap, dev
+
+
+@pytest.mark.parametrize("sizes,N,K", [([130, 0, 1, 300], 256, 512), ([128] * 3, 128, 256), ([700], 384, 1024),
+                                       ([5, 260, 17, 0, 129, 64, 1, 1], 128, 768)])
+def test_gemm_bf16_out_matches_oracle(sizes, N, K):
+    aq, as_, wq, off_pad, rows_cap, dev = _gemm_inputs(sizes, N, K, len(sizes) + N)
+    G = len(sizes)
+    # unpadded output rows through offsets_out
+    off_out = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R = int(off_out[-1])
+    out = torch.full((max(R, 1), N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    moe.moe_nvfp4_grouped_gemm(dev["aq"], dev["asf"], dev["off_pad"], G, rows_cap, dev["wq"], dev["wsf"], dev["g"],
+                               N, K, moe.MOE_NVFP4_EPI_BF16, None, None, out, _i32(off_out), R)
+    assert moe.moe_get_status() == 0
+    got = host_bf16_f64(out)
+    for g in range(G):
+        if sizes[g] == 0:
+            continue
+        a0 = off_pad[g]
+        ref = nvfp4.gemm(aq[a0:a0 + sizes[g]], as_[a0:a0 + sizes[g]], *wq[g])
+        check_output(got[off_out[g]:off_out[g + 1]], ref, f"group {g}")
+        np.testing.assert_allclose(got[off_out[g]:off_out[g + 1]], ref, rtol=2 ** -7, atol=1e-3 * np.abs(ref).max())
+
+
+def test_gemm_gelu_fp4_out_matches_oracle():
+    """GEMM1's epilogue: g * acc, GELU, FP4 re-quantization.  The codes decide on
+    fp32 values that differ from the oracle's by the accumulation order, so a code
+    or scale may sit on the other side of a rounding boundary: at most 0.1% may
+    differ, and the dequantized hidden rows agree to the usual tolerance."""
+    sizes, N, K = [300, 77, 128], 512, 768
+    aq, as_, wq, off_pad, rows_cap, dev = _gemm_inputs(sizes, N, K, 5)
+    G = len(sizes)
+    hq = torch.zeros((rows_cap, N // 2), dtype=torch.uint8, device="cuda")
+    hsf = torch.zeros((rows_cap * N // 16,), dtype=torch.uint8, device="cuda")
+    moe.moe_nvfp4_grouped_gemm(dev["aq"], dev["asf"], dev["off_pad"], G, rows_cap, dev["wq"], dev["wsf"], dev["g"],
+                               N, K, moe.MOE_NVFP4_EPI_GELU_FP4, hq, hsf, None, None, 0)
+    assert moe.moe_get_status() == 0
+    codes = _unpack_codes(hq.cpu().numpy())
+    sfs = _sf_logical(hsf.cpu().numpy(), rows_cap, N)
+    n_code = n_sf = 0
+    for g in range(G):
+        a0, n = off_pad[g], sizes[g]
+        pre = nvfp4.gemm(aq[a0:a0 + n], as_[a0:a0 + n], *wq[g])
+        h = oracle.gelu_tanh(pre)
+        rq, rs = nvfp4.quantize_activation(h.astype(np.float32))
+        n_code += int((codes[a0:a0 + n] != rq).sum())
+        n_sf += int((sfs[a0:a0 + n] != rs).sum())
+        check_output(nvfp4.dequantize(codes[a0:a0 + n], sfs[a0:a0 + n]), nvfp4.dequantize(rq, rs), f"h {g}")
+    total = sum(sizes) * N
+    assert n_code <= 1e-3 * total and n_sf <= 1e-3 * total / 16, (n_code, n_sf)
+
+
+def _nvfp4_layer(name, tokens, cap=None):
+    w = mi.WORKLOADS[name]
+    t = mi.torch_workload(w)
+    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), precision="nvfp4",
+                         capacity_factor=cap)
+    layer.set_nvfp4_weights(t["w1"], t["w2"])
+    b_host = t["bias"].cpu().numpy()
+    out = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    gpu_idx = layer.topk_idx.cpu().numpy()
+    keep = None
+    if cap is not None:
+        keep = oracle.capacity_keep(gpu_idx, layer.capacity, w.n_routed)[tokens]
+    r = nvfp4.forward_tokens(w, tokens, b_host, keep=keep)
+    same = np.array([list(a) == list(b) for a, b in zip(gpu_idx[tokens], r["topk_idx"])])
+    assert same.mean() > 0.8
+    got = host_bf16_f64(out[torch.from_numpy(np.asarray(tokens)).cuda()])
+    check_output(got[same], r["out"][same], f"{name} nvfp4")
+    # the cost of the format: the bf16 layer's output on the same tokens, for the record
+    ref_bf16 = oracle.forward_tokens(w, tokens, b_host, mi.host_logit_offset(w), keep=keep)["out"]
+    rel = np.linalg.norm(got[same] - ref_bf16[same]) / np.linalg.norm(ref_bf16[same])
+    assert rel < 0.25
+    return rel
+
+
+def test_layer_nvfp4_mid_sampled():
+    _nvfp4_layer("mid", np.arange(0, 4096, 211))
+
+
+@pytest.mark.slow
+def test_layer_nvfp4_decode_sampled():
+    _nvfp4_layer("decode", np.array([0, 31, 63]))
+
+
+@pytest.mark.slow
+def test_layer_nvfp4_mid_with_capacity():
+    _nvfp4_layer("mid", np.arange(0, 4096, 301), cap=1.0)
