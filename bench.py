@@ -137,7 +137,10 @@ def run_ours(args, w, rank, world, local_rank):
                            stream.cuda_stream)
     layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev,
                          gather_rows=args.gather_rows, capacity_factor=args.capacity_factor,
-                         activation=w.activation, route_scale=w.gate_scale)
+                         activation=w.activation, route_scale=w.gate_scale, precision=args.precision)
+    if args.precision == "nvfp4":
+        layer.set_nvfp4_weights(t["w1"], t["w2"])
+        torch.cuda.synchronize()
     bias0 = t["bias"].clone()
     ffn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
@@ -249,6 +252,8 @@ def run_ours(args, w, rank, world, local_rank):
     # touched routed experts and the shared experts + A rows read + hidden written and read
     # + outputs written (bf16)
     pk = peaks()
+    if args.precision == "nvfp4":
+        return nvfp4_line(args, w, world, layer, ms, e2e_ms, ffn_ms, clk, touched, routed_rows, pk)
     rows = routed_rows + w.T * w.n_shared
     mats = 3 if w.activation == "swiglu" else 2   # weight matrices per expert
     ffn_flops = 2 * mats * rows * w.d * w.f
@@ -293,6 +298,45 @@ def run_ours(args, w, rank, world, local_rank):
     }
     del bias0
     return line
+
+
+def nvfp4_line(args, w, world, layer, ms, e2e_ms, ffn_ms, clk, touched, routed_rows, pk):
+    """Bench line of the layer with NVFP4 routed experts; the roofline kernel is the pair of
+    FP4 grouped GEMMs (routed rows only: the shared experts run in bf16 outside the window)."""
+    rows = routed_rows
+    ffn_flops = 2 * 2.0 * rows * w.d * w.f
+    fp4_matrix = w.d * w.f // 2 + w.d * w.f // 16            # codes + block scales of one matrix
+    ffn_bytes = (touched * 2 * fp4_matrix                     # the touched routed experts' weights
+                 + rows * (w.d // 2 + w.d // 16)              # A codes and scales
+                 + 2 * rows * (w.f // 2 + w.f // 16)          # hidden codes and scales, written and read
+                 + rows * w.d * 2)                            # y rows (bf16)
+    tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
+    gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
+    fp4_peak = 4.0 * pk["bf16_tflops_sustained"]              # nominal dense FP4 / BF16 = 9 / 2.25
+    kernel = "fp4_gemm_kernel x2 (routed experts: GEMM1+GELU+FP4 requantization, GEMM2)"
+    tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1), "peak": round(fp4_peak, 1),
+                   "unit": "TFLOP/s", "frac": round(tflops / fp4_peak, 4),
+                   "peak_source": "measured bf16 sustained x 4 (nominal dense FP4/BF16 ratio)", "traffic": None,
+                   "flop_per_launch_pair": ffn_flops, "ms_per_launch_pair": round(ffn_ms, 4)}
+    hbm_roof = {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / pk["hbm_gbs"], 4), "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)",
+                "traffic": None, "bytes_per_launch_pair": round(ffn_bytes),
+                "touched_routed_experts_mean": round(touched, 2), "ms_per_launch_pair": round(ffn_ms, 4)}
+    weight_bound = w.T * w.k < 16 * w.n_routed
+    roofline = hbm_roof if weight_bound else tensor_roof
+    return {
+        "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block-16 scales, fp32 acc) routed "
+                                                      "experts; bf16 router and shared experts",
+        "data": "synthetic (seeded Philox, random-init weights)",
+        "config": dict(config_of(w, world), precision="nvfp4 routed experts (W4A4)"), "clocks": clk,
+        "e2e": {"value": round(world * w.T / (e2e_ms * 1e-3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": w.T * w.d * 2, "d2h_bytes_per_step": w.T * w.d * 2,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": layer.launches_per_step() * args.steps,
+        "roofline": roofline, "roofline_other": tensor_roof if weight_bound else hbm_roof,
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -450,6 +494,24 @@ def cpu_baseline(w, n_tokens=4):
                       "before timing"}
 
 
+def cpu_baseline_nvfp4(w, n_tokens=2):
+    """The NVFP4 oracle (routed experts on FP4 operands, fp64 sums) on a bounded sample; the
+    touched experts' weights are generated and quantized before timing."""
+    from oracle import nvfp4
+
+    tokens = (np.arange(n_tokens) * 7919) % w.T
+    b = mi.host_bias(w)
+    cache = {}
+    nvfp4.forward_tokens(w, tokens, b, cache=cache)       # fills the cache (untimed)
+    t0 = time.perf_counter()
+    nvfp4.forward_tokens(w, tokens, b, cache=cache)
+    dt = time.perf_counter() - t0
+    return {"value": round(len(tokens) / dt, 4), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{len(tokens)} tokens of the {w.name} workload through the NVFP4 oracle (FP4 activation "
+                      f"quantization, fp64 sums over dequantized operands), wall {dt:.2f} s; weights quantized "
+                      "before timing"}
+
+
 def run_reference(args, w):
     tokens, b, off, weights = oracle_sample(w, 2)
     per_step = 1
@@ -508,6 +570,34 @@ def run_kernel_case(args):
     elif args.kernel_case == "grouped_ffn":
         def call():
             moe.moe_grouped_ffn(rows, offsets, G, n, 0, w1, w2, d, f, moe.MOE_ACT_GELU_TANH, h, y)
+    elif args.kernel_case == "nvfp4_ffn":
+        # the same slice with NVFP4 operands: rows quantized once by the FP4 dispatch (one expert
+        # per row, groups of 1536 = 12 x 128 rows, so no padding), then GEMM1 + GELU + FP4 and GEMM2
+        u8 = torch.uint8
+        w1q = torch.empty((G, f, d // 2), dtype=u8, device=dev)
+        w1sf = torch.empty((G, f * d // 16), dtype=u8, device=dev)
+        g1 = torch.empty(G, dtype=torch.float32, device=dev)
+        w2q = torch.empty((G, d, f // 2), dtype=u8, device=dev)
+        w2sf = torch.empty((G, d * f // 16), dtype=u8, device=dev)
+        g2 = torch.empty(G, dtype=torch.float32, device=dev)
+        moe.moe_nvfp4_quantize_weights(w1, G, f, d, w1q, w1sf, g1)
+        moe.moe_nvfp4_quantize_weights(w2, G, d, f, w2q, w2sf, g2)
+        rows_cap = moe.moe_nvfp4_rows_capacity(n, G, 1)
+        xq = torch.empty((rows_cap, d // 2), dtype=u8, device=dev)
+        xsf = torch.empty((rows_cap * d // 16,), dtype=u8, device=dev)
+        hq = torch.empty((rows_cap, f // 2), dtype=u8, device=dev)
+        hsf = torch.empty((rows_cap * f // 16,), dtype=u8, device=dev)
+        topk = (torch.arange(n, device=dev, dtype=torch.int32) // per).reshape(n, 1)
+        trow = torch.arange(n, device=dev, dtype=torch.int32).reshape(n, 1)
+        trp = torch.empty_like(trow)
+        offp = torch.empty(G + 1, dtype=torch.int32, device=dev)
+        moe.moe_nvfp4_dispatch(rows, topk, trow, offsets, n, d, G, 1, xq, xsf, trp, offp)
+
+        def call():
+            moe.moe_nvfp4_grouped_gemm(xq, xsf, offp, G, rows_cap, w1q, w1sf, g1, f, d, moe.MOE_NVFP4_EPI_GELU_FP4,
+                                       hq, hsf, None, None, 0)
+            moe.moe_nvfp4_grouped_gemm(hq, hsf, offp, G, rows_cap, w2q, w2sf, g2, d, f, moe.MOE_NVFP4_EPI_BF16,
+                                       None, None, y, offsets, n)
     else:
         # comparison only (not the product path): the same two GEMMs per expert through cuBLAS
         xr, hr, yr = rows.view(G, per, d), h.view(G, per, f), y.view(G, per, d)
@@ -552,11 +642,14 @@ def main():
     ap.add_argument("--capacity-factor", type=float, default=None,
                     help="hard expert capacity, as a multiple of the ideal load k*T/n_routed (overflow dropped)")
     ap.add_argument("--gamma", type=float, default=0.01, help="bias step of the lab workload")
+    ap.add_argument("--precision", choices=["bf16", "nvfp4"], default="bf16",
+                    help="nvfp4: the routed experts in NVFP4 (W4A4); router and shared experts stay bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gather-rows", action="store_true",
                     help="GEMM1 gathers the routed rows from x (cp.async) instead of reading rows copied by dispatch")
-    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "router"], default=None,
+    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "nvfp4_ffn", "router"],
+                    default=None,
                     help="time one kernel alone on a small profiling case instead of the layer")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -614,7 +707,7 @@ def main():
         line = run_ours(args, w, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(w)
+                line["cpu_baseline"] = cpu_baseline_nvfp4(w) if args.precision == "nvfp4" else cpu_baseline(w)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

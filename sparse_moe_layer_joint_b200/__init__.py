@@ -334,18 +334,22 @@ class MoELayer:
         moe_nvfp4_quantize_weights(w1, E, f, d, self.w1q, self.w1sf, self.g1, stream=stream)
         moe_nvfp4_quantize_weights(w2, E, d, f, self.w2q, self.w2sf, self.g2, stream=stream)
 
-    def _forward_nvfp4(self, x, w1, w2, main):
+    def _forward_nvfp4(self, x, w1, w2, main, ffn_events=None):
         s = self.shape
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
         if self.w1q is None:
             raise RuntimeError("set_nvfp4_weights() first")
         moe_nvfp4_dispatch(x, self.topk_idx, self.token_row, self.offsets, T, d, s.n_routed, k, self.xq, self.xsf,
                            self.token_row_pad, self.offsets_pad, stream=main)
+        if ffn_events is not None:
+            ffn_events[0].record(main)
         moe_nvfp4_grouped_gemm(self.xq, self.xsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w1q, self.w1sf,
                                self.g1, f, d, MOE_NVFP4_EPI_GELU_FP4, self.hq, self.hsf, None, None, 0, stream=main)
         moe_nvfp4_grouped_gemm(self.hq, self.hsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w2q, self.w2sf,
                                self.g2, d, f, MOE_NVFP4_EPI_BF16, None, None, self.y_perm, self.offsets, T * k,
                                stream=main)
+        if ffn_events is not None:
+            ffn_events[1].record(main)
         if s.n_shared > 0:
             moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, self.activation, self.h_shared,
                             self.y_shared, stream=main)
@@ -381,17 +385,17 @@ class MoELayer:
         else:
             moe_permute_capped(x, self.topk_idx, self.counts, T, d, s.n_routed, k, self.capacity, self.offsets,
                                x_perm, self.row_token, self.token_row, self.scratch, self.scratch_bytes, stream=main)
-        if ffn_events is not None:
+        if ffn_events is not None and not self.nvfp4:
             ffn_events[0].record(main)
-        if self.nvfp4:
-            self._forward_nvfp4(x, w1, w2, main)
+        if self.nvfp4:  # its events bracket the two FP4 GEMMs alone
+            self._forward_nvfp4(x, w1, w2, main, ffn_events)
         elif self.fused_experts:
             moe_experts_ffn(x, x_perm, self.row_token, self.offsets, T, s.n_routed, s.n_shared, k, w1, w2, d, f,
                             self.activation, self.h, self.y_perm, self.y_shared, stream=main)
         else:
             moe_grouped_ffn(self.x_perm, self.offsets, s.n_routed, T * k, 0, w1, w2, d, f, self.activation,
                             self.h, self.y_perm, stream=main)
-        if ffn_events is not None:
+        if ffn_events is not None and not self.nvfp4:
             ffn_events[1].record(main)
         if side:
             main.wait_event(self.ev_shared)
