@@ -312,6 +312,11 @@ int moe_nvfp4_dispatch(const moe_bf16* x, const int32_t* topk_idx, const int32_t
  *              i-th row to row offsets_out[e] + i of out [out_rows, N] for
  *              i < offsets_out[e+1] - offsets_out[e] (padding rows dropped): the
  *              y_perm layout moe_combine reads with moe_permute's token_row
+ *   offsets_out [n_groups + 1] int32 or NULL; values clamped to [0, out_rows].
+ *              With either epilogue it also gives each group's real row count:
+ *              rows past it are padding and are not loaded (their outputs are
+ *              not meaningful), which saves most of the A traffic when groups
+ *              have few rows (decode)
  * Padding rows are computed like any row (their FP4 outputs are not meaningful).
  * Limits: N % 128 == 0, K % 256 == 0, rows_cap % 128 == 0, n_groups <= 256.
  */

@@ -344,7 +344,8 @@ class MoELayer:
         if ffn_events is not None:
             ffn_events[0].record(main)
         moe_nvfp4_grouped_gemm(self.xq, self.xsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w1q, self.w1sf,
-                               self.g1, f, d, MOE_NVFP4_EPI_GELU_FP4, self.hq, self.hsf, None, None, 0, stream=main)
+                               self.g1, f, d, MOE_NVFP4_EPI_GELU_FP4, self.hq, self.hsf, None, self.offsets, T * k,
+                               stream=main)
         moe_nvfp4_grouped_gemm(self.hq, self.hsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w2q, self.w2sf,
                                self.g2, d, f, MOE_NVFP4_EPI_BF16, None, None, self.y_perm, self.offsets, T * k,
                                stream=main)

@@ -280,7 +280,9 @@ struct Params {
   uint8_t* out_q;          // EPI_GELU_FP4: codes [rows_cap, N/2] and atom-tiled scales
   uint8_t* out_sf;
   __nv_bfloat16* out;      // EPI_BF16: [rows_cap, N], or [out_rows, N] through offsets_out
-  const int* offsets_out;  // EPI_BF16, nullable: group e's row i goes to row offsets_out[e] + i (i < its count)
+  const int* offsets_out;  // nullable: the groups' real rows (offsets_out[e+1] - offsets_out[e] of them); with
+                           // EPI_BF16 group e's row i goes to row offsets_out[e] + i.  Rows past a group's
+                           // real count are not loaded (their outputs are not meaningful)
   long long out_rows;
   uint64_t timeout_ns;
   unsigned int* status;
@@ -308,7 +310,8 @@ static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
+                    const __grid_constant__ CUtensorMap tmB, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -382,6 +385,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmA32);
       tma_prefetch_desc(&tmB);
       int stage = 0;
       uint32_t phase = 0;
@@ -392,14 +396,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_of(tile, g, m, nt);
         const int a_row = st->t.off[g] + m * TM;
         const int n0 = nt * TN;
+        // A rows to load: the group's real rows in this tile, in 32-row boxes (few-row groups at small
+        // T would otherwise fill three quarters of every A stage with padding)
+        int a_boxes = 4;
+        if (p.offsets_out != nullptr) {
+          const int real = st->t.off_out[g + 1] - st->t.off_out[g] - m * TM;
+          a_boxes = real >= TM ? 4 : (real <= 0 ? 1 : (real + 31) / 32);
+        }
+        const uint32_t tx = STAGE_TX - (uint32_t)(4 - a_boxes) * (A_BYTES / 4);
         const uint8_t* sfa = p.a_sf + ((size_t)(a_row / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
         const uint8_t* sfb = p.b_sf + (size_t)g * p.b_sf_stride + ((size_t)(n0 / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
         for (int kb = 0; kb < num_kb; ++kb) {
           ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
           if (!ok) break;
           uint64_t* bar = &st->full[stage];
-          mbar_arrive_expect_tx(bar, STAGE_TX);
-          tma_load_2d(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
+          mbar_arrive_expect_tx(bar, tx);
+          if (a_boxes == 4) {
+            tma_load_2d(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
+          } else {
+            for (int i = 0; i < a_boxes; ++i)
+              tma_load_2d(sA + stage * A_BYTES + i * (A_BYTES / 4), &tmA32, bar, kb * ROW_BYTES, a_row + 32 * i);
+          }
           tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
           bulk_load(sSFA + stage * SF_BYTES, sfa + (size_t)kb * SF_BYTES, SF_BYTES, bar);
           bulk_load(sSFB + stage * SF_BYTES, sfb + (size_t)kb * SF_BYTES, SF_BYTES, bar);
@@ -612,8 +629,9 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (rc != MOE_OK) return rc;
   unsigned int* status = status_ptr();
   if (!status) return MOE_ERR_CUDA;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, ta32, tb;
   if ((rc = encode_tmap_u8(&ta, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, TM)) != MOE_OK) return rc;
+  if ((rc = encode_tmap_u8(&ta32, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, 32)) != MOE_OK) return rc;
   if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, (uint64_t)N, (uint64_t)n_groups, ROW_BYTES, TN)) != MOE_OK)
     return rc;
   Params p{};
@@ -630,7 +648,7 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   p.out_q = out_q;
   p.out_sf = out_sf;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
-  p.offsets_out = epilogue == MOE_NVFP4_EPI_BF16 ? offsets_out : nullptr;
+  p.offsets_out = offsets_out;
   p.out_rows = out_rows;
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
@@ -639,11 +657,11 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (epilogue == MOE_NVFP4_EPI_GELU_FP4) {
     auto kfn = fp4_gemm_kernel<EPI_GELU_FP4>;
     if ((rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES)) != MOE_OK) return rc;
-    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, ta32, tb, p);
   } else {
     auto kfn = fp4_gemm_kernel<EPI_BF16>;
     if ((rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES)) != MOE_OK) return rc;
-    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, ta32, tb, p);
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -199,3 +199,29 @@ def test_layer_identical_experts_give_that_expert():
     out = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"])
     ref = oracle.expert(mi.host_x(w), mi.host_w1(w, 0), mi.host_w2(w, 0))
     check_output(host_bf16_f64(out), ref, "identical experts")
+
+
+def test_layer_step_replays_as_cuda_graph():
+    """The whole step (router -> ... -> combine -> bias update) captured as one CUDA graph
+    replays bit-identically to the eager calls (no host work, allocation or sync inside)."""
+    w = mi.WORKLOADS["tiny"]
+    t, layer = _layer(w)
+    b0 = t["bias"].clone()
+    outs = []
+    for _ in range(2):
+        layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
+        layer.bias_update(t["bias"], w.gamma)
+        outs.append((layer.out.clone(), t["bias"].clone()))
+    torch.cuda.synchronize()
+    t["bias"].copy_(b0)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
+        layer.bias_update(t["bias"], w.gamma)
+    t["bias"].copy_(b0)  # capture ran nothing; start the replays from the same bias
+    for out, bias in outs:
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(layer.out, out)
+        assert torch.equal(t["bias"], bias)
+    assert moe.moe_get_status() == 0

@@ -151,18 +151,23 @@ def test_gemm_bf16_out_matches_oracle(sizes, N, K):
         np.testing.assert_allclose(got[off_out[g]:off_out[g + 1]], ref, rtol=2 ** -7, atol=1e-3 * np.abs(ref).max())
 
 
-def test_gemm_gelu_fp4_out_matches_oracle():
+@pytest.mark.parametrize("sizes,real_rows", [([300, 77, 128], False), ([1, 5, 33, 64, 100, 129, 0, 2], True)])
+def test_gemm_gelu_fp4_out_matches_oracle(sizes, real_rows):
     """GEMM1's epilogue: g * acc, GELU, FP4 re-quantization.  The codes decide on
     fp32 values that differ from the oracle's by the accumulation order, so a code
     or scale may sit on the other side of a rounding boundary: at most 0.1% may
-    differ, and the dequantized hidden rows agree to the usual tolerance."""
-    sizes, N, K = [300, 77, 128], 512, 768
+    differ, and the dequantized hidden rows agree to the usual tolerance.  With the
+    groups' real row counts given, only those rows are loaded (padding rows are
+    then not meaningful and not compared)."""
+    N, K = 512, 768
     aq, as_, wq, off_pad, rows_cap, dev = _gemm_inputs(sizes, N, K, 5)
     G = len(sizes)
     hq = torch.zeros((rows_cap, N // 2), dtype=torch.uint8, device="cuda")
     hsf = torch.zeros((rows_cap * N // 16,), dtype=torch.uint8, device="cuda")
+    off_real = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     moe.moe_nvfp4_grouped_gemm(dev["aq"], dev["asf"], dev["off_pad"], G, rows_cap, dev["wq"], dev["wsf"], dev["g"],
-                               N, K, moe.MOE_NVFP4_EPI_GELU_FP4, hq, hsf, None, None, 0)
+                               N, K, moe.MOE_NVFP4_EPI_GELU_FP4, hq, hsf, None,
+                               _i32(off_real) if real_rows else None, int(off_real[-1]) if real_rows else 0)
     assert moe.moe_get_status() == 0
     codes = _unpack_codes(hq.cpu().numpy())
     sfs = _sf_logical(hsf.cpu().numpy(), rows_cap, N)
