@@ -289,13 +289,15 @@ class MoELayer:
         self.gates = torch.empty((s.T, s.top_k + s.n_shared), dtype=torch.float32, device=dev)
         self.counts = torch.empty((s.n_routed,), dtype=torch.int32, device=dev)
         self.offsets = torch.empty((s.n_routed + 1,), dtype=torch.int32, device=dev)
-        self.x_perm = torch.empty((max(R, 1), s.d), dtype=bf, device=dev)
+        # the bf16 path's copied rows and hidden rows (the NVFP4 path keeps its own FP4 buffers)
+        R_bf16 = 1 if self.nvfp4 else max(R, 1)
+        self.x_perm = torch.empty((R_bf16, s.d), dtype=bf, device=dev)
         self.row_token = torch.empty((max(R, 1),), dtype=torch.int32, device=dev)
         self.token_row = torch.empty((s.T, s.top_k), dtype=torch.int32, device=dev)
         self.scratch_bytes = moe_permute_scratch_bytes(s.T, s.n_routed)
         self.scratch = torch.empty((self.scratch_bytes,), dtype=torch.uint8, device=dev)
         # hidden rows: routed rows, then (fused path) the shared experts' rows
-        self.h = torch.empty((max(R + s.n_shared * s.T, 1), s.d_ff), dtype=bf, device=dev)
+        self.h = torch.empty((1 if self.nvfp4 else max(R + s.n_shared * s.T, 1), s.d_ff), dtype=bf, device=dev)
         self.y_perm = torch.empty((max(R, 1), s.d), dtype=bf, device=dev)
         self.h_shared = torch.empty((max(s.n_shared, 1), s.T, s.d_ff), dtype=bf, device=dev)
         self.y_shared = torch.empty((max(s.n_shared, 1), s.T, s.d), dtype=bf, device=dev)

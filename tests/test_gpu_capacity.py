@@ -206,3 +206,24 @@ def test_lab_loop_per_step(gamma):
     late = slice(50, None)
     assert abs(np.mean(max_vio[late]) - ref_run["max_vio"][late].mean()) < 0.05
     assert abs(np.mean(drop_rate[late]) - ref_run["drop_rate"][late].mean()) < 0.005
+
+
+@pytest.mark.slow
+def test_layer_inkling_decode_with_capacity():
+    """Capacity with the released configuration (SwiGLU experts, route_scale 8) at decode scale."""
+    w = mi.WORKLOADS["inkling_decode"]
+    t = mi.torch_workload(w)
+    layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), capacity_factor=1.0,
+                         activation=w.activation, route_scale=w.gate_scale)
+    b_host = t["bias"].cpu().numpy()
+    out = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    gpu_idx = layer.topk_idx.cpu().numpy()
+    keep = oracle.capacity_keep(gpu_idx, layer.capacity, w.n_routed)
+    assert layer.capacity == 1 and (~keep).any()        # 64 * 6 / 256 = 1.5 -> 1 token per expert
+    tokens = np.array([0, 5, 63])
+    r = oracle.forward_tokens(w, tokens, b_host, keep=keep[tokens])
+    same = np.array([list(a) == list(b) for a, b in zip(gpu_idx[tokens], r["topk_idx"])])
+    got = host_bf16_f64(out[torch.from_numpy(tokens).cuda()])
+    check_output(got[same], r["out"][same], "inkling_decode capacity")

@@ -222,3 +222,35 @@ def test_layer_nvfp4_decode_sampled():
 @pytest.mark.slow
 def test_layer_nvfp4_mid_with_capacity():
     _nvfp4_layer("mid", np.arange(0, 4096, 301), cap=1.0)
+
+
+@pytest.mark.slow
+def test_layer_nvfp4_prefill_sampled():
+    """Full prefill size (65536 tokens, 256 experts of d 7168 / d_ff 2048) with NVFP4 experts."""
+    _nvfp4_layer("prefill", np.array([0, 40000, 65535]))
+
+
+def test_nvfp4_zero_tokens_and_empty_experts():
+    """T = 0: the dispatch still writes the (all-zero) padded offsets; the GEMMs then have no tiles."""
+    E, d, k = 16, 256, 2
+    x = torch.zeros((1, d), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((1, k), dtype=torch.int32, device="cuda")
+    off = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
+    xq = torch.zeros((128, d // 2), dtype=torch.uint8, device="cuda")
+    xsf = torch.zeros((128 * d // 16,), dtype=torch.uint8, device="cuda")
+    trp = torch.zeros((1, k), dtype=torch.int32, device="cuda")
+    offp = torch.full((E + 1,), -3, dtype=torch.int32, device="cuda")
+    moe.moe_nvfp4_dispatch(x, idx, idx, off, 0, d, E, k, xq, xsf, trp, offp)
+    assert (offp.cpu().numpy() == 0).all()
+    w = torch.zeros((E, 128, d), dtype=torch.bfloat16, device="cuda")
+    wq = torch.zeros((E, 128, d // 2), dtype=torch.uint8, device="cuda")
+    wsf = torch.zeros((E, 128 * d // 16), dtype=torch.uint8, device="cuda")
+    g = torch.zeros(E, dtype=torch.float32, device="cuda")
+    moe.moe_nvfp4_quantize_weights(w, E, 128, d, wq, wsf, g)
+    y = torch.full((1, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_nvfp4_grouped_gemm(xq, xsf, offp, E, 128, wq, wsf, g, 128, d, moe.MOE_NVFP4_EPI_BF16, None, None, y,
+                               off, 0)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    assert (y.float().cpu().numpy() == 7.0).all()      # nothing written
+    assert (g.cpu().numpy() == 0).all()                 # all-zero weights: tensor scale 0
