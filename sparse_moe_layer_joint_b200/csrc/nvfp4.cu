@@ -254,17 +254,28 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(const uint4* __rest
 // ---------------------------------------------------------------------------
 constexpr int NUM_THREADS = 192;
 constexpr int TM = 128;           // rows per tile
-constexpr int TN = 128;           // output columns per tile (MMA N)
 constexpr int ROW_BYTES = 128;    // code bytes per row per stage: 256 values
 constexpr int KV_STAGE = 256;     // values along K per stage
-constexpr int STAGES = 6;  // 36 KB each: as many bytes in flight as fit (weight streaming at small T)
 constexpr int A_BYTES = TM * ROW_BYTES;
-constexpr int B_BYTES = TN * ROW_BYTES;
-constexpr int SF_BYTES = (KV_STAGE / ATOM_K) * ATOM_BYTES;  // 4 atoms = 2 KB per operand per stage
-constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + 2 * SF_BYTES;
+constexpr int SF_BYTES = (KV_STAGE / ATOM_K) * ATOM_BYTES;  // 4 atoms = 2 KB per 128 rows per stage
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SFA_COL = 256;  // 16 columns: 4 K-chunks x 4
-constexpr uint32_t SFB_COL = 320;
+
+// Tile width (MMA N).  128 (default): two accumulators (double-buffered epilogue), six 36 KB stages.
+// 256: twice the MMA work per stage, but two 256-column accumulators leave no TMEM for the scales, so one
+// accumulator (the next tile's MMAs wait for the epilogue) and four 54 KB stages -- measured slower.
+template <int TN_>
+struct FCfg {
+  static constexpr int TN = TN_;
+  static constexpr int ACC_BUFS = TN == 256 ? 1 : 2;
+  static constexpr int STAGES = TN == 256 ? 4 : 6;
+  static constexpr int B_BYTES = TN * ROW_BYTES;
+  static constexpr int SFB_BYTES = (TN / ATOM_ROWS) * SF_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
+  static constexpr uint32_t STAGE_TX = (uint32_t)STAGE_BYTES;
+  static constexpr uint32_t SFA_COL = 256;  // 16 columns: 4 K-chunks x 4
+  static constexpr uint32_t SFB_COL = 320;  // 4 K-chunks x TN/32 columns
+  static_assert(ACC_BUFS * TN <= (int)SFA_COL && SFB_COL + 4 * (TN / 32) <= TMEM_COLS, "TMEM columns");
+};
 constexpr int EPI_GELU_FP4 = 0;   // GEMM1: x g1, GELU, FP4 out (the next GEMM's A)
 constexpr int EPI_BF16 = 1;       // GEMM2: x g2, bf16 out
 
@@ -294,6 +305,7 @@ struct Tables {
   int off_out[MOE_MAX_ROUTED + 1];
 };
 
+template <int STAGES>
 struct SmemTail {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -305,20 +317,29 @@ struct SmemTail {
   Tables t;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + 2 * SF_BYTES) + sizeof(SmemTail);
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+template <int TN>
+constexpr size_t smem_bytes() {
+  using C = FCfg<TN>;
+  return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + sizeof(SmemTail<C::STAGES>);
+}
+static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448, "shared memory per CTA");
 
-template <int EPI>
+template <int EPI, int TN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
                     const __grid_constant__ CUtensorMap tmB, const Params p) {
+  using C = FCfg<TN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int B_BYTES = C::B_BYTES;
+  constexpr int SFB_BYTES = C::SFB_BYTES;
+  constexpr uint32_t SFA_COL = C::SFA_COL, SFB_COL = C::SFB_COL;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSFA = sB + STAGES * B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * SF_BYTES;
-  SmemTail* st = reinterpret_cast<SmemTail*>(sSFB + STAGES * SF_BYTES);
+  SmemTail<STAGES>* st = reinterpret_cast<SmemTail<STAGES>*>(sSFB + STAGES * SFB_BYTES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -403,7 +424,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int real = st->t.off_out[g + 1] - st->t.off_out[g] - m * TM;
           a_boxes = real >= TM ? 4 : (real <= 0 ? 1 : (real + 31) / 32);
         }
-        const uint32_t tx = STAGE_TX - (uint32_t)(4 - a_boxes) * (A_BYTES / 4);
+        const uint32_t tx = C::STAGE_TX - (uint32_t)(4 - a_boxes) * (A_BYTES / 4);
         const uint8_t* sfa = p.a_sf + ((size_t)(a_row / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
         const uint8_t* sfb = p.b_sf + (size_t)g * p.b_sf_stride + ((size_t)(n0 / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
         for (int kb = 0; kb < num_kb; ++kb) {
@@ -419,7 +440,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
           bulk_load(sSFA + stage * SF_BYTES, sfa + (size_t)kb * SF_BYTES, SF_BYTES, bar);
-          bulk_load(sSFB + stage * SF_BYTES, sfb + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+#pragma unroll
+          for (int rb = 0; rb < TN / ATOM_ROWS; ++rb)  // the weight rows' 128-row blocks
+            bulk_load(sSFB + stage * SFB_BYTES + rb * SF_BYTES,
+                      sfb + ((size_t)rb * atoms_k) * ATOM_BYTES + (size_t)kb * SF_BYTES, SF_BYTES, bar);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -455,16 +479,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
           const uint32_t sfa_addr = smem_u32(sSFA + stage * SF_BYTES);
-          const uint32_t sfb_addr = smem_u32(sSFB + stage * SF_BYTES);
+          const uint32_t sfb_addr = smem_u32(sSFB + stage * SFB_BYTES);
+          // K-chunk j's scales: A's 128 rows in 4 columns; the weights' TN rows in TN/32 columns, 4 per
+          // 128-row block (the layout the MMA reads: row r at lane r % 32, column r / 32)
 #pragma unroll
           for (int j = 0; j < KV_STAGE / ATOM_K; ++j) {
             tmem_cp_sf(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
-            tmem_cp_sf(tmem_base + SFB_COL + 4 * j, make_desc_sf(sfb_addr + j * ATOM_BYTES));
+#pragma unroll
+            for (int rb = 0; rb < TN / ATOM_ROWS; ++rb)
+              tmem_cp_sf(tmem_base + SFB_COL + (TN / 32) * j + 4 * rb,
+                         make_desc_sf(sfb_addr + rb * SF_BYTES + j * ATOM_BYTES));
           }
 #pragma unroll
           for (int j = 0; j < KV_STAGE / ATOM_K; ++j)
             mma_nvf4_ss(d_tmem, make_desc_sw128(a_addr + j * 32), make_desc_sw128(b_addr + j * 32), idesc,
-                        tmem_base + SFA_COL + 4 * j, tmem_base + SFB_COL + 4 * j, (kb | j) != 0 ? 1u : 0u);
+                        tmem_base + SFA_COL + 4 * j, tmem_base + SFB_COL + (TN / 32) * j, (kb | j) != 0 ? 1u : 0u);
           mma_commit(&st->empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -473,8 +502,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         mma_commit(&st->tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       int zero = 0;
       mma_commit(&st->drain);
@@ -531,8 +562,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&st->tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -543,6 +576,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+}
+
+template <int EPI, int TN>
+int launch_fp4(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const Params& p, int grid,
+               cudaStream_t s) {
+  auto kfn = fp4_gemm_kernel<EPI, TN>;
+  constexpr size_t bytes = smem_bytes<TN>();
+  const int rc = ensure_smem_attr((const void*)kfn, bytes);
+  if (rc != MOE_OK) return rc;
+  kfn<<<grid, NUM_THREADS, bytes, s>>>(ta, ta32, tb, p);
+  return MOE_OK;
 }
 
 }  // namespace fp4
@@ -620,7 +664,14 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (!aligned16(aq) || !aligned16(asf) || !aligned16(wq) || !aligned16(wsf) || !aligned4(gscale) ||
       !aligned4(offsets_pad))
     return MOE_ERR_INVALID_ARG;
-  if (N % TN != 0 || K % KV_STAGE != 0 || rows_cap % ATOM_ROWS != 0) return MOE_ERR_UNSUPPORTED;
+  if (N % 128 != 0 || K % KV_STAGE != 0 || rows_cap % ATOM_ROWS != 0) return MOE_ERR_UNSUPPORTED;
+  // tile width: 128 (measured faster at every size here: 1.87 against 2.19 ms on a prefill-shaped slice,
+  // 3.50 against 3.13 TB/s at decode); MOE_FP4_TN=256 selects the single-accumulator 256-wide tiles
+  int tn = 128;
+  if (const char* env = getenv("MOE_FP4_TN")) {
+    if (env[0] == '1' && env[1] == '2' && env[2] == '8' && env[3] == '\0') tn = 128;
+    if (env[0] == '2' && env[1] == '5' && env[2] == '6' && env[3] == '\0' && N % 256 == 0) tn = 256;
+  }
   if (rows_cap > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if (n_groups == 0 || rows_cap == 0) return MOE_OK;
   cudaStream_t s = (cudaStream_t)stream;
@@ -632,7 +683,7 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   CUtensorMap ta, ta32, tb;
   if ((rc = encode_tmap_u8(&ta, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, TM)) != MOE_OK) return rc;
   if ((rc = encode_tmap_u8(&ta32, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, 32)) != MOE_OK) return rc;
-  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, (uint64_t)N, (uint64_t)n_groups, ROW_BYTES, TN)) != MOE_OK)
+  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, (uint64_t)N, (uint64_t)n_groups, ROW_BYTES, tn)) != MOE_OK)
     return rc;
   Params p{};
   p.offsets_pad = offsets_pad;
@@ -644,7 +695,7 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   p.gscale = gscale;
   p.N = N;
   p.K = K;
-  p.n_tiles_n = N / TN;
+  p.n_tiles_n = N / tn;
   p.out_q = out_q;
   p.out_sf = out_sf;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
@@ -654,14 +705,12 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   p.status = status;
   const long long tiles_upper = (rows_cap / TM) * p.n_tiles_n;
   const int grid = (int)(tiles_upper < sms ? tiles_upper : sms);
-  if (epilogue == MOE_NVFP4_EPI_GELU_FP4) {
-    auto kfn = fp4_gemm_kernel<EPI_GELU_FP4>;
-    if ((rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES)) != MOE_OK) return rc;
-    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, ta32, tb, p);
-  } else {
-    auto kfn = fp4_gemm_kernel<EPI_BF16>;
-    if ((rc = ensure_smem_attr((const void*)kfn, SMEM_BYTES)) != MOE_OK) return rc;
-    kfn<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, ta32, tb, p);
-  }
+  if (epilogue == MOE_NVFP4_EPI_GELU_FP4)
+    rc = tn == 256 ? launch_fp4<EPI_GELU_FP4, 256>(ta, ta32, tb, p, grid, s)
+                   : launch_fp4<EPI_GELU_FP4, 128>(ta, ta32, tb, p, grid, s);
+  else
+    rc = tn == 256 ? launch_fp4<EPI_BF16, 256>(ta, ta32, tb, p, grid, s)
+                   : launch_fp4<EPI_BF16, 128>(ta, ta32, tb, p, grid, s);
+  if (rc != MOE_OK) return rc;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -111,6 +111,13 @@ def test_dispatch_quant_bit_exact(T, k, E, d, cap):
     np.testing.assert_array_equal(sfs[rows], s_ref[t_idx])
 
 
+@pytest.fixture(params=["tn128", "tn256"])
+def fp4_tile(request, monkeypatch):
+    """Both FP4 GEMM tile widths (128, the default, and 256 where N is a multiple of 256)."""
+    monkeypatch.setenv("MOE_FP4_TN", request.param[2:])
+    return request.param
+
+
 def _gemm_inputs(sizes, N, K, seed):
     """A (activations) and W quantized by the oracle, laid out as the device expects."""
     G = len(sizes)
@@ -131,7 +138,7 @@ def _gemm_inputs(sizes, N, K, seed):
 
 @pytest.mark.parametrize("sizes,N,K", [([130, 0, 1, 300], 256, 512), ([128] * 3, 128, 256), ([700], 384, 1024),
                                        ([5, 260, 17, 0, 129, 64, 1, 1], 128, 768)])
-def test_gemm_bf16_out_matches_oracle(sizes, N, K):
+def test_gemm_bf16_out_matches_oracle(sizes, N, K, fp4_tile):
     aq, as_, wq, off_pad, rows_cap, dev = _gemm_inputs(sizes, N, K, len(sizes) + N)
     G = len(sizes)
     # unpadded output rows through offsets_out
@@ -152,7 +159,7 @@ def test_gemm_bf16_out_matches_oracle(sizes, N, K):
 
 
 @pytest.mark.parametrize("sizes,real_rows", [([300, 77, 128], False), ([1, 5, 33, 64, 100, 129, 0, 2], True)])
-def test_gemm_gelu_fp4_out_matches_oracle(sizes, real_rows):
+def test_gemm_gelu_fp4_out_matches_oracle(sizes, real_rows, fp4_tile):
     """GEMM1's epilogue: g * acc, GELU, FP4 re-quantization.  The codes decide on
     fp32 values that differ from the oracle's by the accumulation order, so a code
     or scale may sit on the other side of a rounding boundary: at most 0.1% may
