@@ -109,3 +109,34 @@ def test_gemm_orientation():
     assert g == np.float32(2.0 ** -10)
     np.testing.assert_allclose(nvfp4.gemm(xq, xs, wq, ws, g), c * nvfp4.dequantize(xq, xs)[:, :48],
                                rtol=1e-14, atol=0)
+
+
+def test_layer_composition_with_identical_experts():
+    """All routed experts equal (and both shared experts equal): every routed
+    contributor gives the same NVFP4 expert output Y4 and every shared one the same
+    bf16 output Y, so out = (sum of routed gates) * Y4 + (sum of shared gates) * Y."""
+    import oracle
+
+    w = mi.Workload("pin", 12, 256, 256, b_half_width=0.1)
+    tokens = np.arange(12)
+    w1r, w2r = mi.host_w1(w, 3), mi.host_w2(w, 3)
+    w1s, w2s = mi.host_w1(w, 256), mi.host_w2(w, 256)
+
+    import moe_inputs
+
+    orig = (moe_inputs.host_w1, moe_inputs.host_w2)
+    try:
+        moe_inputs.host_w1 = lambda ww, e: w1r if e < ww.n_routed else w1s
+        moe_inputs.host_w2 = lambda ww, e: w2r if e < ww.n_routed else w2s
+        bias = mi.host_bias(w)
+        r = nvfp4.forward_tokens(w, tokens, bias)
+    finally:
+        moe_inputs.host_w1, moe_inputs.host_w2 = orig
+    x = mi.host_x(w, tokens)
+    wq1 = nvfp4.quantize_weight(mi.bf16_to_f64(w1r).astype(np.float32))
+    wq2 = nvfp4.quantize_weight(mi.bf16_to_f64(w2r).astype(np.float32))
+    y4 = nvfp4.expert(mi.bf16_to_f64(x).astype(np.float32), wq1, wq2)["y"]
+    ybf = oracle.expert(x, w1s, w2s)
+    g = r["gates"]
+    expect = g[:, :w.k].sum(axis=1, keepdims=True) * y4 + g[:, w.k:].sum(axis=1, keepdims=True) * ybf
+    np.testing.assert_allclose(r["out"], expect, rtol=1e-12, atol=1e-12)
