@@ -150,3 +150,39 @@ def test_capacity_and_stats_reject():
     assert L.moe_load_stats(A16, 257, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_load_stats(NULL, 256, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_load_stats(0x10002, 256, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_nvfp4_entry_points_reject():
+    E = moe.MOE_ERR_INVALID_ARG
+    U = moe.MOE_ERR_UNSUPPORTED
+    qw = L.moe_nvfp4_quantize_weights
+    assert qw(A16, 2, 100, 256, A16, A16, A16, NULL) == U            # N not a multiple of 128
+    assert qw(A16, 2, 128, 200, A16, A16, A16, NULL) == U            # K not a multiple of 256
+    assert qw(NULL, 2, 128, 256, A16, A16, A16, NULL) == E
+    assert qw(MIS, 2, 128, 256, A16, A16, A16, NULL) == E
+    assert qw(A16, 0, 128, 256, A16, A16, A16, NULL) == moe.MOE_OK  # nothing to do
+    dsp = L.moe_nvfp4_dispatch
+    assert dsp(A16, A16, A16, A16, 8, 128, 16, 2, A16, A16, A16, A16, NULL) == U      # d % 256
+    assert dsp(A16, A16, A16, A16, 8, 256, 300, 2, A16, A16, A16, A16, NULL) == E     # n_routed > 256
+    assert dsp(A16, A16, A16, A16, 8, 256, 16, 9, A16, A16, A16, A16, NULL) == E      # top_k > 8
+    assert dsp(A16, A16, A16, 0x10002, 8, 256, 16, 2, A16, A16, A16, A16, NULL) == E  # misaligned offsets
+    gm = L.moe_nvfp4_grouped_gemm
+    args = [A16, A16, A16, 4, 1024, A16, A16, A16, 256, 512, 1, NULL, NULL, A16, NULL, 0, NULL]
+
+    def call(**kw):
+        a = list(args)
+        names = ["aq", "asf", "offp", "G", "rows", "wq", "wsf", "g", "N", "K", "epi", "oq", "osf", "out", "offo",
+                 "orows", "s"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return gm(*a)
+
+    assert call(N=200) == U
+    assert call(K=300) == U
+    assert call(rows=1000) == U                                      # rows_cap % 128
+    assert call(G=300) == U
+    assert call(epi=5) == E
+    assert call(epi=0) == E                                          # FP4 out needs out_q / out_sf
+    assert call(out=NULL) == E                                       # bf16 out needs out
+    assert call(offo=0x10002) == E
+    assert call(G=0) == moe.MOE_OK
