@@ -16,6 +16,14 @@
  * "Under the hood" (huggingface.co blog), "The routing strategy", adds that the
  * shared experts join the normalisation but are never top-k candidates.
  *
+ * Beyond that core path the library also covers: hard expert capacities with
+ * token dropping and per-batch balance statistics (§02d, §02g:
+ * moe_permute_capped, moe_load_stats); the released configuration's SwiGLU
+ * experts and routing-weight scale ("Under the hood", "MoE: the expert
+ * configuration", "The routing strategy": MOE_ACT_SWIGLU, route_scale); and
+ * NVFP4 W4A4 routed experts on the block-scaled tensor cores ("Under the hood",
+ * "Quantization: BF16 vs NVFP4": moe_nvfp4_*).
+ *
  * Conventions for every call
  * --------------------------
  *  - All tensor pointers are DEVICE pointers to caller-owned memory, row-major,
