@@ -26,7 +26,7 @@ Sources (all on "Inkling, Dissected", engineermaxxing.com, unless noted):
   after adding the correction bias, shared experts join the normalisation but
   are never candidates.
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
 ties in the top-k go to the lower expert index; the output order of the top-k
 is descending biased score; sign(0) = 0; Lbar = k*T/n_routed compared in
 integers; only routed experts are counted; the bias update follows the forward
