@@ -279,7 +279,8 @@ int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* ro
 /*
  * moe_nvfp4_quantize_weights -- quantize G weight matrices [G, N, K] bf16 (K-major)
  *   q       [G, N, K/2] bytes out; sf [G, N*K/16] bytes out (per matrix, atom-tiled)
- *   gscale  [G] fp32 out: each matrix's tensor scale g
+ *   gscale  [G] fp32 out: each matrix's tensor scale g (the call also uses it as
+ *           scratch for the matrices' amax before writing g)
  * Limits: N % 128 == 0, K % 256 == 0.  Run once per weight set.
  */
 int moe_nvfp4_quantize_weights(const moe_bf16* w, int G, int N, int K, uint8_t* q, uint8_t* sf, float* gscale,
