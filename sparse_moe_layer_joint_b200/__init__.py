@@ -417,7 +417,9 @@ class MoELayer:
         return 1 + permute + experts + 1 + 1
 
     def balance(self, stream=None) -> dict:
-        """MaxVio and drop rate of the last forward's loads (synchronises the stream)."""
+        """MaxVio and drop rate of the last forward's loads (synchronises the stream).  With
+        data-parallel replicas call it before ``dp.bias_step``, which sums the counts over the
+        ranks in place: it describes this rank's batch."""
         import torch
 
         s = self.shape
