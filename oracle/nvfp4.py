@@ -152,6 +152,22 @@ def gemm(a_q, a_s, b_q, b_s, g_b) -> np.ndarray:
     return dequantize(a_q, a_s) @ dequantize(b_q, b_s).T * float(g_b)
 
 
+def expert_swiglu(x_f32: np.ndarray, w1: tuple, w2: tuple) -> dict:
+    """One SwiGLU expert ("Under the hood", "MoE: the expert configuration") on NVFP4
+    operands: W1 [2 d_ff, d] (gate rows, then up rows) is one quantized matrix (one
+    tensor scale g1); h = silu(g1 * sum(dq(x) dq(Wg))) * (g1 * sum(dq(x) dq(Wu))),
+    quantized like any activation; y = g2 * sum(dq(h) dq(W2))."""
+    q1, s1, g1 = w1
+    f = q1.shape[0] // 2
+    xq, xs = quantize_activation(x_f32)
+    pre = gemm(xq, xs, q1, s1, g1)          # [n, 2 d_ff]: gate columns, then up columns
+    gate, up = pre[:, :f], pre[:, f:]
+    h = gate / (1.0 + np.exp(-gate)) * up
+    hq, hs = quantize_activation(h.astype(np.float32))
+    y = gemm(hq, hs, *w2)
+    return {"xq": xq, "xs": xs, "pre": pre, "h": h, "hq": hq, "hs": hs, "y": y}
+
+
 def expert(x_f32: np.ndarray, w1: tuple, w2: tuple) -> dict:
     """One GELU expert on NVFP4 operands.  x_f32 [n, d] (the bf16 inputs as fp32);
     w1 = (q [f, d], s, g), w2 = (q [d, f], s, g) from ``quantize_weight``.
@@ -195,9 +211,10 @@ def forward_tokens(w, tokens, bias, keep=None, cache=None) -> dict:
             if e not in cache:
                 cache[e] = (quantize_weight(mi.bf16_to_f64(mi.host_w1(w, e)).astype(np.float32)),
                             quantize_weight(mi.bf16_to_f64(mi.host_w2(w, e)).astype(np.float32)))
-            y = expert(xf[rows], *cache[e])["y"]
+            fn = expert_swiglu if getattr(w, "activation", "gelu_tanh") == "swiglu" else expert
+            y = fn(xf[rows], *cache[e])["y"]
         else:
-            y = oracle.expert(x[rows], mi.host_w1(w, e), mi.host_w2(w, e))
+            y = oracle.expert_for(w)(x[rows], mi.host_w1(w, e), mi.host_w2(w, e))
         out[rows] += gates[rows, slots][:, None] * y
     r["out"] = out
     r["tokens"] = tokens

@@ -140,3 +140,25 @@ def test_layer_composition_with_identical_experts():
     g = r["gates"]
     expect = g[:, :w.k].sum(axis=1, keepdims=True) * y4 + g[:, w.k:].sum(axis=1, keepdims=True) * ybf
     np.testing.assert_allclose(r["out"], expect, rtol=1e-12, atol=1e-12)
+
+
+def test_swiglu_expert_special_case():
+    """Representable operands: x a block of +-3 and +-2, Wg = c * I and Wu = c/4 * I (c = 6 * 448 *
+    2^-10, so the tensor scale is a power of two), W2 = c * I: the hidden layer is
+    silu(c x) * (c x / 4) exactly before its own quantization (the gate rows come first: swapped
+    halves give silu(c x / 4) * c x), and y = c * dq(quantize(h))."""
+    from scipy.special import expit
+
+    d = 64
+    x = np.tile(np.array([6.0, -4.0, 4.0, -6.0] * 4, np.float32), (3, 4))[:, :d] * np.float32(0.5)
+    c = 6 * 448 * 2.0 ** -10
+    eye = np.eye(d, dtype=np.float32) * np.float32(c)
+    w1 = nvfp4.quantize_weight(np.concatenate([eye, eye / np.float32(4)]))
+    assert w1[2] == np.float32(2.0 ** -10)
+    w2 = nvfp4.quantize_weight(eye)
+    r = nvfp4.expert_swiglu(x, w1, w2)
+    z = c * x.astype(np.float64)
+    h = z * expit(z) * (z / 4)
+    np.testing.assert_allclose(r["h"], h, rtol=1e-12)
+    hq, hs = nvfp4.quantize_activation(h.astype(np.float32))
+    np.testing.assert_allclose(r["y"], c * nvfp4.dequantize(hq, hs), rtol=1e-12)
