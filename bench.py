@@ -328,16 +328,18 @@ def nvfp4_line(args, w, world, layer, ms, e2e_ms, ffn_ms, clk, touched, routed_r
     """Bench line of the layer with NVFP4 routed experts; the roofline kernel is the pair of
     FP4 grouped GEMMs (routed rows only: the shared experts run in bf16 outside the window)."""
     rows = routed_rows
-    ffn_flops = 2 * 2.0 * rows * w.d * w.f
+    mats = 3 if w.activation == "swiglu" else 2               # d x d_ff matrices per expert
+    ffn_flops = 2 * mats * rows * w.d * w.f
     fp4_matrix = w.d * w.f // 2 + w.d * w.f // 16            # codes + block scales of one matrix
-    ffn_bytes = (touched * 2 * fp4_matrix                     # the touched routed experts' weights
+    ffn_bytes = (touched * mats * fp4_matrix                  # the touched routed experts' weights
                  + rows * (w.d // 2 + w.d // 16)              # A codes and scales
                  + 2 * rows * (w.f // 2 + w.f // 16)          # hidden codes and scales, written and read
                  + rows * w.d * 2)                            # y rows (bf16)
     tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
     gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
     fp4_peak = 4.0 * pk["bf16_tflops_sustained"]              # nominal dense FP4 / BF16 = 9 / 2.25
-    kernel = "fp4_gemm_kernel x2 (routed experts: GEMM1+GELU+FP4 requantization, GEMM2)"
+    act = "SwiGLU" if w.activation == "swiglu" else "GELU"
+    kernel = f"fp4_gemm_kernel x2 (routed experts: GEMM1+{act}+FP4 requantization, GEMM2)"
     tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1), "peak": round(fp4_peak, 1),
                    "unit": "TFLOP/s", "frac": round(tflops / fp4_peak, 4),
                    "peak_source": "measured bf16 sustained x 4 (nominal dense FP4/BF16 ratio)", "traffic": None,

@@ -275,6 +275,8 @@ int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* ro
  */
 #define MOE_NVFP4_EPI_GELU_FP4 0 /* out = FP4(gelu(g * acc)): codes + scales (the next GEMM's A) */
 #define MOE_NVFP4_EPI_BF16 1     /* out = bf16(g * acc) */
+#define MOE_NVFP4_EPI_SWIGLU_FP4 2 /* SwiGLU GEMM1: weights [n_groups, 2N, K] (gate rows, then up rows);
+                                      out = FP4(silu(g * acc_gate) * (g * acc_up)), N output columns */
 
 /*
  * moe_nvfp4_quantize_weights -- quantize G weight matrices [G, N, K] bf16 (K-major)
@@ -313,7 +315,10 @@ int moe_nvfp4_dispatch(const moe_bf16* x, const int32_t* topk_idx, const int32_t
  * weight matrix e.
  *   aq, asf    A codes [rows_cap, K/2] and scales (atom-tiled, K values a row)
  *   wq, wsf, gscale   from moe_nvfp4_quantize_weights ([n_groups, N, K])
- *   epilogue   MOE_NVFP4_EPI_GELU_FP4: out_q [rows_cap, N/2] and out_sf
+ *   epilogue   MOE_NVFP4_EPI_SWIGLU_FP4: as GELU_FP4 for a SwiGLU expert's first
+ *              GEMM: wq / wsf / gscale quantize [n_groups, 2N, K] (gate rows, then
+ *              up rows, one matrix per group), out = FP4(silu(gate) * up), N columns;
+ *              MOE_NVFP4_EPI_GELU_FP4: out_q [rows_cap, N/2] and out_sf
  *              (atom-tiled, N values a row) get FP4(gelu(.)) -- the expert's
  *              hidden layer, ready as the second GEMM's A;
  *              MOE_NVFP4_EPI_BF16: out [rows_cap, N] bf16 at the padded rows,

@@ -41,6 +41,7 @@ MOE_ACT_GELU_TANH = 0
 MOE_ACT_SWIGLU = 1
 MOE_NVFP4_EPI_GELU_FP4 = 0
 MOE_NVFP4_EPI_BF16 = 1
+MOE_NVFP4_EPI_SWIGLU_FP4 = 2
 
 _vp, _i32, _u64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_float, ctypes.c_size_t
 
@@ -304,8 +305,6 @@ class MoELayer:
         self.out = torch.empty((s.T, s.d), dtype=bf, device=dev)
         self.stats = torch.zeros((2,), dtype=torch.int32, device=dev)
         if self.nvfp4:
-            if self.activation != MOE_ACT_GELU_TANH:
-                raise ValueError("the NVFP4 experts are GELU experts")
             self.rows_cap = moe_nvfp4_rows_capacity(s.T, s.n_routed, s.top_k)
             u8 = torch.uint8
             self.xq = torch.empty((self.rows_cap, s.d // 2), dtype=u8, device=dev)
@@ -320,20 +319,22 @@ class MoELayer:
         self.ev_shared = torch.cuda.Event()
 
     def set_nvfp4_weights(self, w1, w2, stream=None):
-        """Quantize the routed experts' weights (the first n_routed of w1 [E, d_ff, d] and
-        w2 [E, d, d_ff]) to NVFP4 on the device; the shared experts keep using w1, w2."""
+        """Quantize the routed experts' weights (the first n_routed of w1 [E, d_ff, d] -- [E, 2*d_ff, d]
+        for SwiGLU, one quantized matrix per expert -- and w2 [E, d, d_ff]) to NVFP4 on the device; the
+        shared experts keep using w1, w2."""
         import torch
 
         s = self.shape
         dev = w1.device
         E, f, d = s.n_routed, s.d_ff, s.d
-        self.w1q = torch.empty((E, f, d // 2), dtype=torch.uint8, device=dev)
-        self.w1sf = torch.empty((E, f * d // 16), dtype=torch.uint8, device=dev)
+        f1 = 2 * f if self.activation == MOE_ACT_SWIGLU else f  # rows of each W1
+        self.w1q = torch.empty((E, f1, d // 2), dtype=torch.uint8, device=dev)
+        self.w1sf = torch.empty((E, f1 * d // 16), dtype=torch.uint8, device=dev)
         self.g1 = torch.empty((E,), dtype=torch.float32, device=dev)
         self.w2q = torch.empty((E, d, f // 2), dtype=torch.uint8, device=dev)
         self.w2sf = torch.empty((E, d * f // 16), dtype=torch.uint8, device=dev)
         self.g2 = torch.empty((E,), dtype=torch.float32, device=dev)
-        moe_nvfp4_quantize_weights(w1, E, f, d, self.w1q, self.w1sf, self.g1, stream=stream)
+        moe_nvfp4_quantize_weights(w1, E, f1, d, self.w1q, self.w1sf, self.g1, stream=stream)
         moe_nvfp4_quantize_weights(w2, E, d, f, self.w2q, self.w2sf, self.g2, stream=stream)
 
     def _forward_nvfp4(self, x, w1, w2, main, ffn_events=None):
@@ -345,9 +346,9 @@ class MoELayer:
                            self.token_row_pad, self.offsets_pad, stream=main)
         if ffn_events is not None:
             ffn_events[0].record(main)
+        epi1 = MOE_NVFP4_EPI_SWIGLU_FP4 if self.activation == MOE_ACT_SWIGLU else MOE_NVFP4_EPI_GELU_FP4
         moe_nvfp4_grouped_gemm(self.xq, self.xsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w1q, self.w1sf,
-                               self.g1, f, d, MOE_NVFP4_EPI_GELU_FP4, self.hq, self.hsf, None, self.offsets, T * k,
-                               stream=main)
+                               self.g1, f, d, epi1, self.hq, self.hsf, None, self.offsets, T * k, stream=main)
         moe_nvfp4_grouped_gemm(self.hq, self.hsf, self.offsets_pad, s.n_routed, self.rows_cap, self.w2q, self.w2sf,
                                self.g2, d, f, MOE_NVFP4_EPI_BF16, None, None, self.y_perm, self.offsets, T * k,
                                stream=main)

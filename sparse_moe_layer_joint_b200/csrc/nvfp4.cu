@@ -278,6 +278,8 @@ struct FCfg {
 };
 constexpr int EPI_GELU_FP4 = 0;   // GEMM1: x g1, GELU, FP4 out (the next GEMM's A)
 constexpr int EPI_BF16 = 1;       // GEMM2: x g2, bf16 out
+constexpr int EPI_SWIGLU_FP4 = 2; // GEMM1 of SwiGLU experts (256-wide tiles: 128 gate + the 128 matching up
+                                  // columns), silu(g1 gate) * (g1 up), FP4 out
 
 struct Params {
   const int* offsets_pad;  // [G + 1] group row starts, multiples of 128
@@ -287,7 +289,8 @@ struct Params {
   const uint8_t* b_sf;     // atom-tiled scales of the weights, per group b_sf_stride bytes
   long long b_sf_stride;
   const float* gscale;     // [G] weight tensor scales
-  int N, K, n_tiles_n;
+  int N, K, n_tiles_n;    // N: output columns
+  int b_up_row;            // EPI_SWIGLU_FP4: first weight row of the up projection (= N)
   uint8_t* out_q;          // EPI_GELU_FP4: codes [rows_cap, N/2] and atom-tiled scales
   uint8_t* out_sf;
   __nv_bfloat16* out;      // EPI_BF16: [rows_cap, N], or [out_rows, N] through offsets_out
@@ -329,6 +332,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
                     const __grid_constant__ CUtensorMap tmB, const Params p) {
   using C = FCfg<TN>;
+  static_assert(EPI != EPI_SWIGLU_FP4 || TN == 256, "SwiGLU tiles hold gate and up columns side by side");
+  constexpr int OUT_W = EPI == EPI_SWIGLU_FP4 ? TN / 2 : TN;  // output columns per tile
   constexpr int STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int SFB_BYTES = C::SFB_BYTES;
@@ -416,7 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int g, m, nt;
         tile_of(tile, g, m, nt);
         const int a_row = st->t.off[g] + m * TM;
-        const int n0 = nt * TN;
+        const int n0 = nt * OUT_W;  // first output column; for SwiGLU also the first gate row
         // A rows to load: the group's real rows in this tile, in 32-row boxes (few-row groups at small
         // T would otherwise fill three quarters of every A stage with padding)
         int a_boxes = 4;
@@ -426,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const uint32_t tx = C::STAGE_TX - (uint32_t)(4 - a_boxes) * (A_BYTES / 4);
         const uint8_t* sfa = p.a_sf + ((size_t)(a_row / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
-        const uint8_t* sfb = p.b_sf + (size_t)g * p.b_sf_stride + ((size_t)(n0 / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
+        const uint8_t* sfb_g = p.b_sf + (size_t)g * p.b_sf_stride;
         for (int kb = 0; kb < num_kb; ++kb) {
           ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
           if (!ok) break;
@@ -438,12 +443,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < a_boxes; ++i)
               tma_load_2d(sA + stage * A_BYTES + i * (A_BYTES / 4), &tmA32, bar, kb * ROW_BYTES, a_row + 32 * i);
           }
-          tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
+          if (EPI == EPI_SWIGLU_FP4) {  // gate rows, then the matching up rows (128-row boxes)
+            tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
+            tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &tmB, bar, kb * ROW_BYTES, p.b_up_row + n0, g);
+          } else {
+            tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
+          }
           bulk_load(sSFA + stage * SF_BYTES, sfa + (size_t)kb * SF_BYTES, SF_BYTES, bar);
 #pragma unroll
-          for (int rb = 0; rb < TN / ATOM_ROWS; ++rb)  // the weight rows' 128-row blocks
+          for (int rb = 0; rb < TN / ATOM_ROWS; ++rb) {  // the weight rows' 128-row blocks
+            const int blk = (EPI == EPI_SWIGLU_FP4 && rb == 1) ? (p.b_up_row + n0) / ATOM_ROWS : n0 / ATOM_ROWS + rb;
             bulk_load(sSFB + stage * SFB_BYTES + rb * SF_BYTES,
-                      sfb + ((size_t)rb * atoms_k) * ATOM_BYTES + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+                      sfb_g + ((size_t)blk * atoms_k) * ATOM_BYTES + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -532,11 +544,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TN);
 #pragma unroll 1
-      for (int ch = 0; ch < TN / 32; ++ch) {
-        const int col0 = nt * TN + ch * 32;
+      for (int ch = 0; ch < OUT_W / 32; ++ch) {
+        const int col0 = nt * OUT_W + ch * 32;
         if (col0 >= p.N) break;  // same for the whole warp
         float v[32];
         tmem_ld32(taddr + ch * 32, v);
+        if (EPI == EPI_SWIGLU_FP4) {
+          float u[32];
+          tmem_ld32(taddr + OUT_W + ch * 32, u);
+          if (!valid) continue;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gate = __fmul_rn(v[i], gs);
+            v[i] = __fmul_rn(__fmul_rn(gate, __frcp_rn(1.0f + __expf(-gate))), __fmul_rn(u[i], gs));
+          }
+          uint32_t s0, s1;
+          const uint2 q0 = quant16_act(v, s0);
+          const uint2 q1 = quant16_act(v + 16, s1);
+          *reinterpret_cast<uint4*>(p.out_q + r * (p.N / 2) + col0 / 2) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+          const size_t so = sf_offset(r, col0 / 16, p.N);
+          p.out_sf[so] = (uint8_t)s0;
+          p.out_sf[so + 1] = (uint8_t)s1;
+          continue;
+        }
         if (!valid) continue;
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], gs);
@@ -656,8 +686,11 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (!aq || !asf || !offsets_pad || !wq || !wsf || !gscale || n_groups < 0 || rows_cap < 0 || N <= 0 || K <= 0)
     return MOE_ERR_INVALID_ARG;
   if (n_groups > MOE_MAX_ROUTED) return MOE_ERR_UNSUPPORTED;
-  if (epilogue != MOE_NVFP4_EPI_GELU_FP4 && epilogue != MOE_NVFP4_EPI_BF16) return MOE_ERR_INVALID_ARG;
-  if (epilogue == MOE_NVFP4_EPI_GELU_FP4 && (!out_q || !out_sf || !aligned16(out_q))) return MOE_ERR_INVALID_ARG;
+  if (epilogue != MOE_NVFP4_EPI_GELU_FP4 && epilogue != MOE_NVFP4_EPI_BF16 && epilogue != MOE_NVFP4_EPI_SWIGLU_FP4)
+    return MOE_ERR_INVALID_ARG;
+  const bool fp4_out = epilogue != MOE_NVFP4_EPI_BF16;
+  const bool swiglu = epilogue == MOE_NVFP4_EPI_SWIGLU_FP4;
+  if (fp4_out && (!out_q || !out_sf || !aligned16(out_q))) return MOE_ERR_INVALID_ARG;
   if (epilogue == MOE_NVFP4_EPI_BF16 && (!out || !aligned16(out))) return MOE_ERR_INVALID_ARG;
   if (offsets_out != nullptr && (!aligned4(offsets_out) || out_rows < 0 || out_rows > 0x7fffffffLL))
     return MOE_ERR_INVALID_ARG;
@@ -672,6 +705,8 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
     if (env[0] == '1' && env[1] == '2' && env[2] == '8' && env[3] == '\0') tn = 128;
     if (env[0] == '2' && env[1] == '5' && env[2] == '6' && env[3] == '\0' && N % 256 == 0) tn = 256;
   }
+  if (swiglu) tn = 256;  // 128 gate + 128 up columns a tile
+  const uint64_t b_rows = swiglu ? 2ull * N : (uint64_t)N;  // weight rows per group
   if (rows_cap > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if (n_groups == 0 || rows_cap == 0) return MOE_OK;
   cudaStream_t s = (cudaStream_t)stream;
@@ -683,7 +718,8 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   CUtensorMap ta, ta32, tb;
   if ((rc = encode_tmap_u8(&ta, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, TM)) != MOE_OK) return rc;
   if ((rc = encode_tmap_u8(&ta32, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, 32)) != MOE_OK) return rc;
-  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, (uint64_t)N, (uint64_t)n_groups, ROW_BYTES, tn)) != MOE_OK)
+  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, b_rows, (uint64_t)n_groups, ROW_BYTES, swiglu ? 128 : tn)) !=
+      MOE_OK)
     return rc;
   Params p{};
   p.offsets_pad = offsets_pad;
@@ -691,11 +727,12 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   p.rows_cap = rows_cap;
   p.a_sf = asf;
   p.b_sf = wsf;
-  p.b_sf_stride = (long long)N * (K / 16);
+  p.b_sf_stride = (long long)b_rows * (K / 16);
   p.gscale = gscale;
   p.N = N;
   p.K = K;
-  p.n_tiles_n = N / tn;
+  p.n_tiles_n = swiglu ? N / 128 : N / tn;
+  p.b_up_row = N;
   p.out_q = out_q;
   p.out_sf = out_sf;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
@@ -705,7 +742,9 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   p.status = status;
   const long long tiles_upper = (rows_cap / TM) * p.n_tiles_n;
   const int grid = (int)(tiles_upper < sms ? tiles_upper : sms);
-  if (epilogue == MOE_NVFP4_EPI_GELU_FP4)
+  if (swiglu)
+    rc = launch_fp4<EPI_SWIGLU_FP4, 256>(ta, ta32, tb, p, grid, s);
+  else if (epilogue == MOE_NVFP4_EPI_GELU_FP4)
     rc = tn == 256 ? launch_fp4<EPI_GELU_FP4, 256>(ta, ta32, tb, p, grid, s)
                    : launch_fp4<EPI_GELU_FP4, 128>(ta, ta32, tb, p, grid, s);
   else
