@@ -558,24 +558,48 @@ def cpu_baseline_nvfp4(w, n_tokens=2):
 
 
 def run_reference(args, w):
-    tokens, b, off, weights = oracle_sample(w, 2)
+    """The oracle on the host cores, one token a step (a bounded sample of the same workload): the fp64
+    layer, or with --precision nvfp4 the NVFP4 oracle (expert weights quantized before timing)."""
+    if args.precision == "nvfp4":
+        from oracle import nvfp4
+
+        tokens = (np.arange(2) * 7919) % w.T
+        b = mi.host_bias(w)
+        cache = {}
+        nvfp4.forward_tokens(w, tokens, b, cache=cache)  # quantizes the touched experts (untimed)
+
+        def one(tok):
+            t0 = time.perf_counter()
+            nvfp4.forward_tokens(w, tok, b, cache=cache)
+            return time.perf_counter() - t0
+        what = "the NVFP4 oracle (FP4 activation quantization, fp64 sums over dequantized operands)"
+    else:
+        tokens, b, off, weights = oracle_sample(w, 2)
+
+        def one(tok):
+            return oracle_forward_timed(w, tok, b, off, weights)
+        what = "the fp64 oracle (router + 8 expert MLPs + combine)"
     per_step = 1
     for i in range(args.warmup):
-        oracle_forward_timed(w, tokens[i % len(tokens):i % len(tokens) + per_step], b, off, weights)
+        one(tokens[i % len(tokens):i % len(tokens) + per_step])
     total = 0.0
     for i in range(args.steps):
         j = i % len(tokens)
-        total += oracle_forward_timed(w, tokens[j:j + per_step], b, off, weights)
+        total += one(tokens[j:j + per_step])
     ms = total / args.steps * 1e3
     v = round(per_step / (ms * 1e-3), 4)
+    config = dict(config_of(w, 1), dispatch="rows gathered by GEMM1 (cp.async)" if args.gather_rows
+                  else "rows copied by moe_permute")
+    if args.precision == "nvfp4":
+        config["precision"] = "nvfp4 routed experts (W4A4)"
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, random-init weights)",
-        "config": config_of(w, 1),
+        "config": config,
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"each step: {per_step} token of the {w.name} workload through the fp64 oracle "
-                                   "(router + 8 expert MLPs + combine), weights generated before timing"},
+                         "sample": f"each step: {per_step} token of the {w.name} workload through {what}, "
+                                   "weights generated before timing"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
