@@ -81,3 +81,22 @@ def test_workload_flop_counts():
     w = mi.WORKLOADS["prefill"]
     assert w.flops() == pytest.approx(31.03e12, rel=1e-3)
     assert w.flops() / w.T == pytest.approx(473.5e6, rel=1e-3)
+
+
+def test_lab_generator_recipe():
+    """The Router Balance Lab inputs follow their stated recipe: specialties Zipf-distributed with
+    expert 0 about 30 times as common as expert 63, tokens at their specialty's center plus
+    N(0, sigma^2 / d) jitter, router rows alpha * center."""
+    w = mi.LAB
+    spec = np.concatenate([mi.lab_specialty(w, s) for s in range(w.steps)])
+    counts = np.bincount(spec, minlength=w.n_routed)
+    assert 30 * 0.8 < counts[0] / counts[-1] < 30 * 1.25
+    assert (np.diff(counts[:8]) < 0).all()                  # the most common specialties in Zipf order
+    c = mi.lab_centers(w)
+    np.testing.assert_array_equal(mi.lab_wr(w), mi.f32_to_bf16_bits((w.alpha * c).astype(np.float32)))
+    x = mi.bf16_to_f64(mi.lab_x(w, 7))
+    jit = x - c[mi.lab_specialty(w, 7)]
+    assert abs(jit.mean()) < 0.005
+    np.testing.assert_allclose(jit.std(), w.sigma / np.sqrt(w.d), rtol=0.03)
+    # steps draw fresh batches
+    assert not np.array_equal(mi.lab_x(w, 0), mi.lab_x(w, 1))
