@@ -358,3 +358,16 @@ def test_skew_offset_calibration():
     r = oracle.route_workload(w, np.zeros(256, np.float32), logit_offset=mi.host_logit_offset(w))
     c = np.sort(oracle.load_counts(r["topk_idx"], 256))[::-1]
     assert abs(c[:8].sum() / c.sum() - 0.30) <= 0.005
+
+
+@pytest.mark.parametrize("T,d,E", [(1, 64, 258), (37, 256, 258), (5, 7168, 9), (300, 32, 64)])
+def test_logits_against_numpy_matmul(T, d, E):
+    """The router logits z = x W_r^T (§02b) against numpy's fp64 matrix product of the same
+    exactly widened bf16 values; and a hand case with one-hot rows picks out W_r's columns."""
+    x = mi.normal_bf16(T * d, 12, mi.STREAM_X).reshape(T, d)
+    wr = mi.normal_bf16(E * d, 12, mi.STREAM_WR, std=d ** -0.5).reshape(E, d)
+    z = oracle.logits(x, wr)
+    ref = mi.bf16_to_f64(x) @ mi.bf16_to_f64(wr).T
+    np.testing.assert_allclose(z, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    onehot = mi.f32_to_bf16_bits(np.eye(min(d, 8), d, dtype=np.float32))
+    np.testing.assert_array_equal(oracle.logits(onehot, wr), mi.bf16_to_f64(wr)[:, :min(d, 8)].T)
