@@ -91,7 +91,19 @@ def header_functions() -> list:
     with open(HEADER_PATH) as fh:
         text = fh.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(moe_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:[a-z_0-9]+\s+)*[a-z_0-9]+\s*\*?\s*(moe_[a-z_0-9]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def header_arity() -> dict:
+    """Number of parameters of each function include/moe.h declares."""
+    with open(HEADER_PATH) as fh:
+        text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"(moe_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
 
 
 def status_string(code: int) -> str:

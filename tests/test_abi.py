@@ -186,3 +186,13 @@ def test_nvfp4_entry_points_reject():
     assert call(out=NULL) == E                                       # bf16 out needs out
     assert call(offo=0x10002) == E
     assert call(G=0) == moe.MOE_OK
+
+
+def test_binding_arity_matches_the_header():
+    """Every function the header declares has a ctypes signature with as many arguments."""
+    arity = moe.header_arity()
+    assert set(arity) == set(moe.header_functions())
+    for name, n in arity.items():
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
