@@ -70,3 +70,47 @@ def test_single_process_is_a_no_op():
     assert dp.world_size() == 1
     assert dp.global_counts(c) is c and c.tolist() == [0, 1, 2, 3]
     assert dp.total_tokens(100) == 100
+
+
+def _lab_worker(rank, world, port, out_dir, steps, gamma):
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+
+    import moe_inputs as mi
+    import oracle
+    from sparse_moe_layer_joint_b200 import dp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = mi.LAB
+        half = w.T // world
+        wr = mi.lab_wr(w)
+        b = np.zeros(w.n_routed, np.float32)
+        for s in range(steps):
+            x = mi.lab_x(w, s)[rank * half:(rank + 1) * half]      # this rank's share of the step's batch
+            r = oracle.route(oracle.logits(x, wr), b, w.k, w.n_routed, 0)
+            counts = torch.from_numpy(oracle.load_counts(r["topk_idx"], w.n_routed).astype(np.int32))
+            dp.global_counts(counts)
+            b = oracle.bias_update(counts.numpy(), b, dp.total_tokens(half), w.k, gamma)
+        np.save(os.path.join(out_dir, f"lab_bias_{rank}.npy"), b)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_run_the_lab_like_one(tmp_path):
+    """The Router Balance Lab split over two data-parallel ranks (each routes half of every
+    step's batch; the loads are summed before each update) ends with the bias of the
+    single-process run on whole batches, bit for bit."""
+    import moe_inputs as mi
+    import oracle
+
+    steps, gamma = 12, 0.01
+    mp.start_processes(_lab_worker, args=(2, _free_port(), str(tmp_path), steps, gamma), nprocs=2,
+                       start_method="spawn")
+    ref = oracle.lab_run(mi.LAB, gamma, steps=steps)["bias"][-1]
+    for rank in range(2):
+        np.testing.assert_array_equal(np.load(tmp_path / f"lab_bias_{rank}.npy").view(np.uint32), ref.view(np.uint32))
