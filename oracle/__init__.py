@@ -36,7 +36,11 @@ nonlinearity is GELU (tanh form); experts have no biases; no residual is added.
 The functions follow the pages' order: ``route`` (scores, biased top-k, joint
 gates), ``load_counts``, ``bias_update``, ``dispatch`` (grouping of the
 (token, expert) pairs by expert), ``expert`` (one expert MLP), ``combine`` and
-``forward_tokens`` (all of it for a set of tokens).
+``forward_tokens`` (all of it for a set of tokens).  Further: expert capacity
+and its metrics (``capacity_for``, ``capacity_keep``, ``load_metrics``, §02d),
+the Router Balance Lab loop (``lab_run``, §02g), the SwiGLU expert of the
+released configuration (``expert_swiglu``, "Under the hood") and, in
+``oracle/nvfp4.py``, the NVFP4 quantization and experts.
 """
 from __future__ import annotations
 
