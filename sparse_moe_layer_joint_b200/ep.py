@@ -1,0 +1,136 @@
+"""Expert parallelism across ranks (one process per GPU).
+
+"Inkling, Dissected" §02d: each expert can serve only so many tokens per batch,
+"set by memory and the all-to-all communication schedule" -- the experts live on
+different GPUs and every token's rows travel to the GPUs of its experts and back.
+Here rank r holds the routed experts [r*E/W, (r+1)*E/W) (E = n_routed, W ranks,
+W dividing E) and a replica of the shared experts.  One step on rank r:
+
+1. route its own tokens (router kernel) and group the (token, slot) pairs by
+   expert (moe_permute): the experts of each destination rank are then one
+   contiguous block of rows;
+2. exchange the per-expert row counts, then the rows (two all-to-alls);
+3. run the owned experts on the rows received from every source rank
+   (moe_grouped_ffn once per source chunk, whose rows are grouped by expert);
+4. send the results back (all-to-all): they land in the sender's dispatch order,
+   so the combine is the one-GPU combine (moe_combine through token_row);
+5. the bias update uses the loads summed over ranks (as in ``dp``).
+
+The plan and exchange functions below are device-agnostic (torch tensors, any
+backend that implements all_to_all_single); ``ExpertParallelLayer`` runs the
+GPU step with the library's kernels and NCCL.
+"""
+from __future__ import annotations
+
+from typing import List, Sequence, Tuple
+
+import numpy as np
+
+
+def expert_range(n_routed: int, world: int, rank: int) -> Tuple[int, int]:
+    """Routed experts [lo, hi) held by ``rank``."""
+    if n_routed % world != 0:
+        raise ValueError(f"{n_routed} routed experts do not split over {world} ranks")
+    per = n_routed // world
+    return rank * per, (rank + 1) * per
+
+
+def send_counts(offsets: Sequence[int], n_routed: int, world: int) -> List[int]:
+    """Rows this rank sends to each rank: the dispatch offsets at the experts blocks' bounds."""
+    off = np.asarray(offsets, dtype=np.int64)
+    per = n_routed // world
+    return [int(off[(q + 1) * per] - off[q * per]) for q in range(world)]
+
+
+def exchange_counts(counts_by_expert, world: int, group=None):
+    """All-to-all of per-expert row counts: ``counts_by_expert`` [n_routed] int32 (this rank's
+    dispatch); returns [world, n_routed/world]: row s = the rows source s sends for each of
+    this rank's experts."""
+    import torch
+    import torch.distributed as dist
+
+    per = counts_by_expert.numel() // world
+    out = torch.empty((world * per,), dtype=counts_by_expert.dtype, device=counts_by_expert.device)
+    dist.all_to_all_single(out, counts_by_expert.contiguous(), group=group)
+    return out.view(world, per)
+
+
+def exchange_rows(rows, send: Sequence[int], recv: Sequence[int], group=None, out=None):
+    """All-to-all of row blocks: ``rows`` [sum(send), ...] ordered by destination rank; returns
+    [sum(recv), ...] ordered by source rank (in ``out`` when given)."""
+    import torch
+    import torch.distributed as dist
+
+    n = int(sum(recv))
+    if out is None:
+        out = torch.empty((n,) + tuple(rows.shape[1:]), dtype=rows.dtype, device=rows.device)
+    else:
+        out = out[:n]
+    dist.all_to_all_single(out, rows.contiguous(), output_split_sizes=[int(v) for v in recv],
+                           input_split_sizes=[int(v) for v in send], group=group)
+    return out
+
+
+def chunk_offsets(recv_by_expert: np.ndarray) -> List[np.ndarray]:
+    """Per source rank, the group offsets of its received chunk (rows grouped by this rank's
+    experts, in expert order), relative to the chunk's first row."""
+    return [np.concatenate([[0], np.cumsum(row)]).astype(np.int32) for row in np.asarray(recv_by_expert)]
+
+
+class ExpertParallelLayer:
+    """One layer step with the routed experts split over ranks (bf16, GELU or SwiGLU experts).
+
+    Not exercised on GPUs in this repository's tests: every run here has one GPU.  Its
+    compute is the library's kernels (router, permute, grouped FFN, combine, bias update);
+    its exchange is NCCL all-to-all of the dispatched rows and of the expert outputs.
+    Weights: ``w_router`` and the shared experts' matrices as on one GPU; ``w1_local`` /
+    ``w2_local`` hold only this rank's routed experts, followed by the shared experts.
+    """
+
+    def __init__(self, shape, rank: int, world: int, device="cuda", group=None, activation: str = "gelu_tanh",
+                 route_scale: float = 1.0):
+        import torch
+
+        from sparse_moe_layer_joint_b200 import MoELayer
+
+        self.rank, self.world, self.group = rank, world, group
+        self.lo, self.hi = expert_range(shape.n_routed, world, rank)
+        self.local = MoELayer(shape, device=device, activation=activation, route_scale=route_scale)
+        self.dev = torch.device(device)
+
+    def forward(self, x, w_router, w1_local, w2_local, bias, logit_offset=None):
+        import torch
+
+        import sparse_moe_layer_joint_b200 as moe
+
+        L, s = self.local, self.local.shape
+        T, d, f, k = s.T, s.d, s.d_ff, s.top_k
+        E_loc = self.hi - self.lo
+        moe.moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, L.route_scale,
+                            L.topk_idx, L.gates, L.counts, None)
+        moe.moe_permute(x, L.topk_idx, L.counts, T, d, s.n_routed, k, L.offsets, L.x_perm, L.row_token,
+                        L.token_row, L.scratch, L.scratch_bytes)
+        # shared experts on this rank's tokens while the exchange runs
+        if s.n_shared > 0:
+            moe.moe_grouped_ffn(x, None, s.n_shared, T, E_loc, w1_local, w2_local, d, f, L.activation,
+                                L.h_shared, L.y_shared)
+        offsets = L.offsets.cpu().numpy()                      # split sizes for the exchange (1 KB)
+        send = send_counts(offsets, s.n_routed, self.world)
+        by_expert = torch.from_numpy(np.diff(offsets).astype(np.int32)).to(self.dev)
+        recv_by_expert = exchange_counts(by_expert, self.world, self.group).cpu().numpy()
+        recv = recv_by_expert.sum(axis=1)
+        x_recv = exchange_rows(L.x_perm[:int(offsets[-1])], send, recv, self.group)
+        y_recv = torch.empty_like(x_recv)
+        h = torch.empty((max(x_recv.shape[0], 1), f), dtype=x_recv.dtype, device=self.dev)
+        start = 0
+        for src, off in enumerate(chunk_offsets(recv_by_expert)):
+            n = int(off[-1])
+            if n:
+                off_dev = torch.from_numpy(off).to(self.dev)
+                moe.moe_grouped_ffn(x_recv[start:start + n], off_dev, E_loc, n, 0, w1_local, w2_local, d, f,
+                                    L.activation, h[:n], y_recv[start:start + n])
+            start += n
+        exchange_rows(y_recv, recv, send, self.group, out=L.y_perm)   # back in this rank's dispatch order
+        moe.moe_combine(L.y_perm, L.token_row, L.gates, L.y_shared if s.n_shared > 0 else None, T, d, k,
+                        s.n_shared, L.out)
+        return L.out

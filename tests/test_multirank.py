@@ -114,3 +114,75 @@ def test_two_ranks_run_the_lab_like_one(tmp_path):
     ref = oracle.lab_run(mi.LAB, gamma, steps=steps)["bias"][-1]
     for rank in range(2):
         np.testing.assert_array_equal(np.load(tmp_path / f"lab_bias_{rank}.npy").view(np.uint32), ref.view(np.uint32))
+
+
+def _ep_worker(rank, world, port, out_dir):
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+
+    import moe_inputs as mi
+    import oracle
+    from sparse_moe_layer_joint_b200 import ep
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = mi.WORKLOADS["tiny"]
+        T_local = w.T // world
+        tokens = np.arange(rank * T_local, (rank + 1) * T_local)
+        b = mi.host_bias(w)
+        x = mi.host_x(w, tokens)
+        r = oracle.route_workload(w, b, tokens, x=x)
+        dp = oracle.dispatch(r["topk_idx"], w.n_routed)
+        x_perm = torch.from_numpy(mi.bf16_to_f64(x)[dp["row_token"]])
+        send = ep.send_counts(dp["offsets"], w.n_routed, world)
+        by_expert = torch.from_numpy(np.diff(dp["offsets"]).astype(np.int32))
+        recv_by_expert = ep.exchange_counts(by_expert, world).numpy()
+        recv = recv_by_expert.sum(axis=1)
+        x_recv = ep.exchange_rows(x_perm, send, recv)
+        lo, hi = ep.expert_range(w.n_routed, world, rank)
+        # this rank's experts on the rows from every source (the oracle stands in for the GPU kernels)
+        y_recv = np.zeros_like(x_recv.numpy())
+        start = 0
+        for off in ep.chunk_offsets(recv_by_expert):
+            for j in range(hi - lo):
+                a0, a1 = start + off[j], start + off[j + 1]
+                if a1 > a0:
+                    rows = mi.f32_to_bf16_bits(x_recv.numpy()[a0:a1].astype(np.float32))
+                    y_recv[a0:a1] = oracle.expert(rows, mi.host_w1(w, lo + j), mi.host_w2(w, lo + j))
+            start += int(off[-1])
+        y_perm = ep.exchange_rows(torch.from_numpy(y_recv), recv, send).numpy()
+        y_sh = np.stack([oracle.expert(x, mi.host_w1(w, e), mi.host_w2(w, e))
+                         for e in range(w.n_routed, w.n_experts)])
+        out = oracle.combine(y_perm, dp["token_row"], r["gates"], y_sh)
+        np.save(os.path.join(out_dir, f"ep_out_{rank}.npy"), out)
+        np.save(os.path.join(out_dir, f"ep_recv_{rank}.npy"), recv_by_expert)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_exchange_matches_one_process(tmp_path, world):
+    """Experts split over ranks (rank r holds 256/W routed experts): the rows each token sends
+    to its experts' ranks come back in dispatch order, and the combined output equals the
+    single-process layer on the same tokens (every expert row computed the same way in fp64;
+    only the order of the gate-weighted sum differs, so to fp64 rounding)."""
+    import moe_inputs as mi
+    import oracle
+
+    mp.start_processes(_ep_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    w = mi.WORKLOADS["tiny"]
+    b = mi.host_bias(w)
+    full = oracle.forward_tokens(w, np.arange(w.T), b)
+    T_local = w.T // world
+    counts = np.zeros(w.n_routed, np.int64)
+    for rank in range(world):
+        got = np.load(tmp_path / f"ep_out_{rank}.npy")
+        np.testing.assert_allclose(got, full["out"][rank * T_local:(rank + 1) * T_local], rtol=1e-12, atol=1e-14)
+        counts[rank * (w.n_routed // world):(rank + 1) * (w.n_routed // world)] = \
+            np.load(tmp_path / f"ep_recv_{rank}.npy").sum(axis=0)
+    # every (token, slot) pair reached the rank of its expert exactly once
+    np.testing.assert_array_equal(counts, oracle.load_counts(full["topk_idx"], w.n_routed))
