@@ -212,6 +212,8 @@ def run_ours(args, w, rank, world, local_rank):
         dp.bias_step(layer, t["bias"], w.gamma)
     touched = (local_counts > 0).sum(dim=1).double().mean().item()
     routed_rows = statistics.mean(served) if served else w.T * w.k   # rows the expert GEMMs compute
+    if args.log_balance and rank == 0:
+        write_balance_log(args.log_balance, local_counts.cpu().numpy(), w.T, w.k, layer.capacity)
 
     # end to end through the public API: every step copies its x in from pinned host memory and
     # its output back to pinned host memory.  Like a serving loop, the copies of neighbouring steps
@@ -409,6 +411,13 @@ def run_lab(args):
     torch.cuda.synchronize()
     st = stats.cpu().numpy().astype(np.float64)
     kT = w.k * w.T
+    if args.log_balance:
+        with open(args.log_balance, "w") as fh:
+            for i in range(n_steps):
+                fh.write(json.dumps({"step": i, "max_load": int(st[i, 0]),
+                                     "max_vio": round(float(st[i, 0] * w.n_routed / kT - 1), 6),
+                                     "capacity": cap, "dropped": int(st[i, 1]),
+                                     "drop_rate": round(float(st[i, 1] / kT), 8)}) + "\n")
     late = slice(n_steps // 2, None)
     balance = {"gamma": args.gamma, "capacity": cap,
                "max_vio_late_mean": round(float((st[late, 0] * w.n_routed / kT - 1).mean()), 4),
@@ -486,6 +495,19 @@ def run_lab(args):
                      "note": "a 2048-token step moves ~0.4 MB: launch latency, not bandwidth, bounds it"},
         "balance": balance,
     }
+
+
+def write_balance_log(path, counts, T, k, capacity):
+    """One JSON line per step: the largest load, MaxVio (largest load over the ideal k*T/E, minus one)
+    and, with a capacity, the assignments dropped and their share of the k*T slots."""
+    with open(path, "w") as fh:
+        for step, L in enumerate(np.asarray(counts, dtype=np.int64)):
+            rec = {"step": step, "max_load": int(L.max()), "max_vio": round(float(L.max() * len(L) / (k * T) - 1), 6),
+                   "mean_load": round(float(L.mean()), 3)}
+            if capacity is not None:
+                dropped = int(np.maximum(L - capacity, 0).sum())
+                rec.update(capacity=int(capacity), dropped=dropped, drop_rate=round(dropped / (k * T), 8))
+            fh.write(json.dumps(rec) + "\n")
 
 
 def lab_config():
@@ -711,6 +733,8 @@ def main():
     ap.add_argument("--capacity-factor", type=float, default=None,
                     help="hard expert capacity, as a multiple of the ideal load k*T/n_routed (overflow dropped)")
     ap.add_argument("--gamma", type=float, default=0.01, help="bias step of the lab workload")
+    ap.add_argument("--log-balance", default=None, metavar="PATH",
+                    help="write one JSON line per step (largest load, MaxVio, drops) to PATH")
     ap.add_argument("--graph", action="store_true",
                     help="time the step as one replayed CUDA graph (one GPU; for the launch-bound sizes)")
     ap.add_argument("--precision", choices=["bf16", "nvfp4"], default="bf16",

@@ -132,6 +132,20 @@ def _stream(stream) -> Optional[int]:
 def _check(fn: str, rc: int):
     if rc != MOE_OK:
         raise MoEError(fn, rc)
+    if _DEBUG_SYNC:
+        _debug_sync(fn)
+
+
+# MOE_DEBUG_SYNC=1: after every call, synchronise and read the device status word, so a
+# device-side error is reported at the call that caused it (slow; off by default).
+_DEBUG_SYNC = os.environ.get("MOE_DEBUG_SYNC") == "1"
+
+
+def _debug_sync(fn: str):
+    v = _i32(0)
+    rc = _lib.moe_get_status(None, ctypes.byref(v))
+    if rc != MOE_OK or v.value != 0:
+        raise MoEError(f"{fn} (device status {v.value:#x})", rc if rc != MOE_OK else MOE_ERR_DEVICE)
 
 
 # ---------------------------------------------------------------------------
@@ -450,3 +464,26 @@ class MoELayer:
         s = self.shape
         moe_bias_update(self.counts, s.n_routed, s.T if T_total is None else T_total, s.top_k, gamma, bias,
                         stream=stream)
+
+
+# MOE_NVTX=1: every moe_* call above is bracketed by an NVTX range named after it (for timelines
+# in a profiler; off by default, when the functions are left untouched).
+def _nvtx_wrap(fn):
+    import functools
+
+    import torch
+
+    @functools.wraps(fn)
+    def wrapped(*args, **kwargs):
+        torch.cuda.nvtx.range_push(fn.__name__)
+        try:
+            return fn(*args, **kwargs)
+        finally:
+            torch.cuda.nvtx.range_pop()
+
+    return wrapped
+
+
+if os.environ.get("MOE_NVTX") == "1":
+    for _name in [n for n in list(globals()) if n.startswith("moe_") and callable(globals()[n])]:
+        globals()[_name] = _nvtx_wrap(globals()[_name])
