@@ -13,13 +13,9 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: takes more than a few seconds")
     # build the in-tree libraries if stale (no-op when up to date), before the
     # test modules import them
-    import moe_inputs.build
-    import oracle.build
-    import sparse_moe_layer_joint_b200.build as moe_build
+    import __graft_entry__
 
-    moe_inputs.build.build()
-    oracle.build.build()
-    moe_build.build()
+    __graft_entry__.build()
 
 
 def cuda_ok():
