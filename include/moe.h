@@ -259,7 +259,9 @@ int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* ro
  *   weights      g = amax|W| / (6 * 448) per matrix; block scale
  *                s = E4M3(fl(amax_b / 6) / g); codes E2M1(w / fl(s * g))
  *   activations  s = E4M3(fl(amax_b / 6)) per block; codes E2M1(x / s)
- * A block whose scale is 0 has codes 0.  E2M1 codes have no negative zero.
+ * Each quotient (w / fl(s * g), x / s) is correctly rounded to fp32 before its
+ * E2M1 rounding, so an exact midpoint takes the even code.  A block whose scale
+ * is 0 has codes 0.  E2M1 codes have no negative zero.
  *
  * Layouts:
  *   codes   [rows, K/2] bytes, K-major; byte j of a row packs values 2j (bits

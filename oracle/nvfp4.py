@@ -17,12 +17,13 @@ Recipe (this oracle's reading; the page gives only the block size and the FP8
 scales): every conversion rounds to nearest, ties to even, and saturates to the
 largest finite value.  A weight matrix W gets one fp32 scale g = amax|W| / (6 * 448)
 and per 16-block scales s_b = E4M3(fl32(amax_b / 6) / g); its codes are
-q = E2M1(fl32(w * fl32(1 / fl32(s_b * g)))).  An activation block (dynamic, no
-tensor scale) gets s_b = E4M3(fl32(amax_b / 6)) and q = E2M1(fl32(x * fl32(1 / s_b))).
-Values are scaled by the reciprocal of the block scale (one reciprocal a block,
-as a kernel does it, rather than a division per value).  A block whose scale
-rounds to 0 has all codes 0.  The quantities that decide a code or a scale are
-computed in fp32, in the order written, as the kernels compute them.
+q = E2M1(fl32(w / fl32(s_b * g))).  An activation block (dynamic, no tensor
+scale) gets s_b = E4M3(fl32(amax_b / 6)) and q = E2M1(fl32(x / s_b)).  A value
+is divided by its block's scale, as the format's definition puts it (an element
+stands for its code times the scale, so the code is the value over the scale),
+each division correctly rounded to fp32.  A block whose scale rounds to 0 has
+all codes 0.  Every quantity that decides a code or a scale is one fp32 operation
+on fp32 operands, in the order written.
 
 The expert (§02 of "Inkling, Dissected": two matmuls with a nonlinearity, GELU
 tanh form here) on quantized operands: h = gelu(g1 * sum(dq(x) dq(W1))),
@@ -113,8 +114,7 @@ def quantize_activation(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     s_code = e4m3_encode_nonneg((amax / np.float32(6.0)).astype(np.float32))
     s = e4m3_decode(s_code).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        inv = (np.float32(1.0) / s).astype(np.float32)
-        r = (b * inv[..., None]).astype(np.float32)
+        r = (b / s[..., None]).astype(np.float32)
     q = np.where(s[..., None] > 0, e2m1_encode(r), 0).astype(np.uint8)
     return q.reshape(np.shape(x)), s_code
 
@@ -131,8 +131,7 @@ def quantize_weight(w: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.float32]:
     s_code = e4m3_encode_nonneg(((amax / np.float32(6.0)).astype(np.float32) / g).astype(np.float32))
     denom = (e4m3_decode(s_code).astype(np.float32) * g).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        inv = (np.float32(1.0) / denom).astype(np.float32)
-        r = (b * inv[..., None]).astype(np.float32)
+        r = (b / denom[..., None]).astype(np.float32)
     q = np.where(denom[..., None] > 0, e2m1_encode(r), 0).astype(np.uint8)
     return q.reshape(w.shape), s_code, g
 

@@ -83,12 +83,13 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
 }
 
 // 16 values with one scale (already chosen): packed codes, 4 bits each, value i at bits 4i of word i/8.
+// A code is the E2M1 rounding of the value over its scale, the quotient correctly rounded to fp32
+// (a product with the scale's reciprocal would land past an exact tie, e.g. 1.25 * 0.9375 / 0.9375).
 __device__ __forceinline__ uint2 pack16(const float* v, float denom) {
   uint32_t w[2] = {0u, 0u};
   if (denom > 0.0f) {
-    const float inv = __frcp_rn(denom);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
+    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code(__fdiv_rn(v[i], denom)) << (4 * (i & 7));
   }
   return make_uint2(w[0], w[1]);
 }

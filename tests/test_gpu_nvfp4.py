@@ -111,6 +111,57 @@ def test_dispatch_quant_bit_exact(T, k, E, d, cap):
     np.testing.assert_array_equal(sfs[rows], s_ref[t_idx])
 
 
+def _tie_rows(n_rows, K):
+    """Rows of K values made of blocks whose quotients x / s are exact E2M1 midpoints
+    (bf16-exact; see the oracle pin of the same name): scales 15/16 * 2^e."""
+    out = np.zeros((n_rows, K), dtype=np.float32)
+    for r in range(n_rows):
+        for b in range(K // 16):
+            s = 0.9375 * 2.0 ** ((r + 3 * b) % 9 - 5)
+            v = np.array([6, 1.25, 2.5, 5, -1.25, -2.5, -5, 0.25, 1.75, 3.5, 0.75, 0, 0, 0, 0, 0]) * s
+            out[r, 16 * b:16 * b + 16] = np.roll(v, (r + b) % 16)
+    bits = out.view(np.uint32)
+    assert ((bits & 0xFFFF) == 0).all()                      # every value is a bf16
+    return (bits >> 16).astype(np.uint16)
+
+
+def test_quantize_at_exact_ties_divides():
+    """Weights and the FP4 dispatch on blocks whose values over their scale are exact
+    E2M1 midpoints: the codes are the even ones, as the oracle's division gives."""
+    N, K = 128, 256
+    w = _tie_rows(N, K)
+    w[5, 7] = np.uint16(np.float32(448 * 6 * 2.0 ** -4).view(np.uint32) >> 16)   # g = 2^-4
+    q = torch.empty((1, N, K // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((1, N * K // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    moe.moe_nvfp4_quantize_weights(dev_bf16(w[None]), 1, N, K, q, sf, g)
+    assert moe.moe_get_status() == 0
+    rq, rs, rg = nvfp4.quantize_weight(mi.bf16_to_f64(w).astype(np.float32))
+    assert g.cpu().numpy()[0] == rg
+    np.testing.assert_array_equal(_unpack_codes(q.cpu().numpy()[0]), rq)
+    np.testing.assert_array_equal(_sf_logical(sf.cpu().numpy()[0], N, K), rs)
+
+    T, k, E = 64, 2, 4
+    x = _tie_rows(T, K)
+    topk = np.stack([np.arange(T) % E, (np.arange(T) + 1) % E], axis=1).astype(np.int32)
+    dp = oracle.dispatch(topk, E)
+    rows_cap = moe.moe_nvfp4_rows_capacity(T, E, k)
+    xq = torch.zeros((rows_cap, K // 2), dtype=torch.uint8, device="cuda")
+    xsf = torch.zeros((rows_cap * K // 16,), dtype=torch.uint8, device="cuda")
+    trp = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    offp = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    moe.moe_nvfp4_dispatch(dev_bf16(x), _i32(topk), _i32(dp["token_row"]), _i32(dp["offsets"]), T, K, E, k, xq, xsf,
+                           trp, offp)
+    assert moe.moe_get_status() == 0
+    q_ref, s_ref = nvfp4.quantize_activation(mi.bf16_to_f64(x).astype(np.float32))
+    rows = trp.cpu().numpy()
+    codes = _unpack_codes(xq.cpu().numpy())
+    sfs = _sf_logical(xsf.cpu().numpy(), rows_cap, K)
+    for j in range(k):
+        np.testing.assert_array_equal(codes[rows[:, j]], q_ref)
+        np.testing.assert_array_equal(sfs[rows[:, j]], s_ref)
+
+
 @pytest.fixture(params=["tn128", "tn256"])
 def fp4_tile(request, monkeypatch):
     """Both FP4 GEMM tile widths (128, the default, and 256 where N is a multiple of 256)."""

@@ -87,6 +87,61 @@ def test_activation_codes_are_nearest_grid_points():
     assert set(np.unique(np.abs(got).max(axis=-1))) <= {4.0, 6.0}
 
 
+def _tie_blocks():
+    """Blocks whose quotients x / s are exact E2M1 midpoints.  Each block's first
+    value is 6 s, so its scale is s = E4M3(6 s / 6); the others are m s for the
+    midpoints m in {1.25, 2.5, 5}, which round to the lower, even code (1, 2, 4).
+    With s = 15/16 * 2^e the fp32 reciprocal of s is inexact, and m s times it
+    rounds to just above m, which would give the upper code."""
+    scales = [0.9375 * 2.0 ** e for e in (-5, -2, 0, 1, 3)]
+    blocks = []
+    for s in scales:
+        b = np.zeros(16, dtype=np.float64)
+        b[0] = 6 * s
+        b[1:4] = [1.25 * s, 2.5 * s, 5 * s]
+        b[4:7] = [-1.25 * s, -2.5 * s, -5 * s]
+        b[7:10] = [0.25 * s, 1.75 * s, 3.5 * s]      # ties that go up (0.75, 1.75, 3.5) or to 0
+        b[10] = 0.75 * s
+        blocks.append(b)
+    return np.array(scales), np.array(blocks).astype(np.float32)
+
+
+TIE_CODES = [7, 2, 4, 6, 10, 12, 14, 0, 4, 6, 2, 0, 0, 0, 0, 0]
+
+
+def test_codes_are_rounded_quotients_at_exact_ties():
+    """A code is the E2M1 rounding (ties to even) of the exact quotient x / s: at a
+    midpoint the even code wins.  Checked on blocks where a product with the fp32
+    reciprocal of s lands just past the midpoint."""
+    scales, x = _tie_blocks()
+    inv = (np.float32(1) / scales.astype(np.float32)).astype(np.float32)
+    assert (((x[:, 1] * inv).astype(np.float32)) > np.float32(1.25)).all()   # the reciprocal form would round up
+    q, s = nvfp4.quantize_activation(x)
+    np.testing.assert_array_equal(nvfp4.e4m3_decode(s)[:, 0], scales)
+    np.testing.assert_array_equal(q, np.tile(TIE_CODES, (len(scales), 1)))
+    # weights: the same blocks with a power-of-two tensor scale (the quotient is unchanged)
+    w = np.concatenate([x, np.full((1, 16), 448 * 6 * 2.0 ** -4, np.float32)])
+    qw, sw, g = nvfp4.quantize_weight(w)
+    assert g == np.float32(2.0 ** -4)
+    np.testing.assert_array_equal(qw[:-1], np.tile(TIE_CODES, (len(scales), 1)))
+
+
+def test_codes_equal_fp64_quotients_rounded_to_fp32():
+    """The fp32 quotient equals the fp64 quotient of the same fp32 operands rounded
+    to fp32 (a correctly rounded division, by the double-rounding bound for
+    division); the codes then follow from the E2M1 rounding of that value."""
+    x = (mi.normal_f64(500 * 64, 9, mi.STREAM_TEST_ROWS).reshape(500, 64) * 2).astype(np.float32)
+    q, s = nvfp4.quantize_activation(x)
+    sd = nvfp4.e4m3_decode(s)
+    r = (x.reshape(500, 4, 16).astype(np.float64) / sd[..., None]).astype(np.float32)
+    np.testing.assert_array_equal(q.reshape(500, 4, 16), np.where(sd[..., None] > 0, nvfp4.e2m1_encode(r), 0))
+    w = (mi.normal_f64(64 * 256, 10, mi.STREAM_TEST_ROWS).reshape(64, 256) * 0.02).astype(np.float32)
+    qw, sw, g = nvfp4.quantize_weight(w)
+    den = (nvfp4.e4m3_decode(sw).astype(np.float32) * g).astype(np.float32)
+    rw = (w.reshape(64, 16, 16).astype(np.float64) / den[..., None]).astype(np.float32)
+    np.testing.assert_array_equal(qw.reshape(64, 16, 16), np.where(den[..., None] > 0, nvfp4.e2m1_encode(rw), 0))
+
+
 def test_scale_invariance_by_powers_of_two():
     x = (mi.normal_f64(40 * 32, 8, mi.STREAM_TEST_ROWS).reshape(40, 32)).astype(np.float32)
     q, s = nvfp4.quantize_activation(x)
