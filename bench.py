@@ -15,12 +15,17 @@ T tokens (data-parallel replicas of the same weights: weak scaling); the load
 counts are summed over ranks with one NCCL all-reduce (256 int32) before the
 bias update, so every replica keeps the same bias.
 
+The default (prefill) run also measures the decode-scale layer (T 64, d 7168,
+weight-streaming bound) after the prefill steps, on its own clock, and reports
+it under "decode" in the same line (--no-decode skips it).
+
 --impl reference times the CPU oracle (fp64, the layer's plain definition) on
 the host cores on a bounded sample of the same workload; rank 0 only.
 """
 from __future__ import annotations
 
 import argparse
+import copy
 import json
 import os
 import statistics
@@ -45,6 +50,10 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 # DRAM bytes (read + write) of one GEMM1 + GEMM2 launch pair, from one single-pass ncu capture of the
 # full-size layer (profiles/grouped_gemm_prefill_dram.md); workloads without a capture of the current
 # kernels report null
+# the decode record of the default run times this many decode steps per prefill step (a decode
+# step is ~2 ms, a prefill step ~30 ms)
+DECODE_STEPS_PER_STEP = 10
+
 TRAFFIC_PER_LAUNCH_PAIR = {"prefill": (20.84e9 + 2.14e9) + (12.84e9 + 7.48e9)}
 
 
@@ -121,7 +130,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm: the CUDA path through libmoe
 # ---------------------------------------------------------------------------
-def run_ours(args, w, rank, world, local_rank):
+def run_ours(args, w, rank, world, local_rank, want_cpu=False):
     import torch
     import torch.distributed as dist
 
@@ -277,7 +286,10 @@ def run_ours(args, w, rank, world, local_rank):
     # + outputs written (bf16)
     pk = peaks()
     if args.precision == "nvfp4":
-        return nvfp4_line(args, w, world, layer, ms, e2e_ms, ffn_ms, clk, touched, routed_rows, pk)
+        line = nvfp4_line(args, w, world, layer, ms, e2e_ms, ffn_ms, clk, touched, routed_rows, pk)
+        if want_cpu:
+            line["cpu_baseline"] = cpu_baseline_nvfp4(w)
+        return line
     rows = routed_rows + w.T * w.n_shared
     mats = 3 if w.activation == "swiglu" else 2   # weight matrices per expert
     ffn_flops = 2 * mats * rows * w.d * w.f
@@ -323,6 +335,8 @@ def run_ours(args, w, rank, world, local_rank):
         "roofline_other": tensor_roof if weight_bound else hbm_roof,
     }
     del bias0
+    if want_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, t)
     return line
 
 
@@ -402,7 +416,7 @@ def run_lab(args):
         j = i % n_steps
         moe.moe_router_topk(xs[j] if x is None else x, wr, b, None, w.T, w.d, w.n_routed, 0, w.k, 1.0, idx, g, c)
         moe.moe_permute_capped(None, idx, c, w.T, w.d, w.n_routed, w.k, cap, off, None, rt, tr, scratch, nb)
-        moe.moe_load_stats(c, w.n_routed, cap, stats[j])
+        moe.moe_load_stats(c, w.n_routed, w.T, w.k, cap, stats[j])
         moe.moe_bias_update(c, w.n_routed, w.T, w.k, args.gamma, b)
 
     # the balance of one full run from b = 0 (the lab's 100 steps), outside the timing
@@ -552,13 +566,46 @@ def oracle_forward_timed(w, tokens, b, off, weights):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, n_tokens=4):
-    tokens, b, off, weights = oracle_sample(w, n_tokens)
-    dt = oracle_forward_timed(w, tokens, b, off, weights)
-    return {"value": round(len(tokens) / dt, 4), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{len(tokens)} tokens of the {w.name} workload (full layer: fp64 router over 258 experts, "
-                      f"top-{w.k}, joint gates, 8 expert MLPs each), wall {dt:.2f} s; expert weights generated "
-                      "before timing"}
+def cpu_baseline(w, t=None, n_sample=32):
+    """The oracle as it stands, on the host cores, priced for the whole batch: the fp64 routing
+    (logits over 258 experts, biased top-k, joint gates) of every token of the batch, then the whole
+    layer (routing, the 8 expert MLPs of each token, combine) on a seeded sample of tokens.  Tokens
+    are independent, so the sample's time per token plus the routing time per token prices the
+    batch.  ``t``: the workload's device tensors; the sample's expert weights are copied from them
+    before timing (the device and host generators give the same bits), which avoids regenerating
+    hundreds of weight matrices on the host."""
+    import oracle
+
+    b = mi.host_bias(w)
+    off = mi.host_logit_offset(w)
+    x_all = None
+    if t is not None:
+        import torch
+
+        x_all = t["x"].view(torch.int16).cpu().numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    oracle.route_workload(w, b, logit_offset=off, x=x_all)
+    t_route = time.perf_counter() - t0
+    n_sample = min(n_sample, w.T)
+    tokens = (np.arange(n_sample) * 7919) % w.T
+    r = oracle.route_workload(w, b, tokens, off)
+    experts = sorted(set(int(e) for e in np.unique(r["contrib"])))
+    if t is not None:
+        import torch
+
+        def bits(a):
+            return a.view(torch.int16).cpu().numpy().view(np.uint16)
+        weights = {"w1": {e: bits(t["w1"][e]) for e in experts}, "w2": {e: bits(t["w2"][e]) for e in experts}}
+    else:
+        weights = {"w1": {e: mi.host_w1(w, e) for e in experts}, "w2": {e: mi.host_w2(w, e) for e in experts}}
+    t_layer = oracle_forward_timed(w, tokens, b, off, weights)
+    per_token = t_route / w.T + t_layer / n_sample
+    return {"value": round(1.0 / per_token, 4), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"routing of all {w.T} tokens of the {w.name} workload (fp64 logits over 258 experts, top-{w.k}, "
+                      f"joint gates; {t_route:.2f} s on all cores) + the whole layer on a {n_sample}-token sample "
+                      f"(routing, 8 expert MLPs per token, combine; {t_layer:.2f} s, one thread per row of an "
+                      f"expert's group); value = 1 / (route s / {w.T} + layer s / {n_sample}); expert weights "
+                      "prepared before timing"}
 
 
 def cpu_baseline_nvfp4(w, n_tokens=2):
@@ -741,6 +788,8 @@ def main():
                     help="nvfp4: the routed experts in NVFP4 (W4A4); router and shared experts stay bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="prefill workload: skip the decode-scale record measured after the prefill steps")
     ap.add_argument("--gather-rows", action="store_true",
                     help="GEMM1 gathers the routed rows from x (cp.async) instead of reading rows copied by dispatch")
     ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "nvfp4_ffn", "router"],
@@ -799,10 +848,20 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, w, rank, world, local_rank)
+        line = run_ours(args, w, rank, world, local_rank,
+                        want_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
+        if (args.workload == "prefill" and not args.no_decode and args.precision == "bf16" and not args.graph
+                and args.capacity_factor is None and not args.gather_rows):
+            # the decode-scale layer (T 64, d 7168), weight-streaming bound, measured in the same run
+            # on its own clock: each step reads the touched experts' weights from HBM
+            dargs = copy.copy(args)
+            dargs.steps = args.steps * DECODE_STEPS_PER_STEP
+            dargs.log_balance = None
+            dec = run_ours(dargs, mi.WORKLOADS["decode"], rank, world, local_rank)
+            line["decode"] = {k: dec[k] for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
+                                                  "ms_per_step", "config", "clocks", "e2e", "gpu_launches",
+                                                  "roofline")}
         if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline_nvfp4(w) if args.precision == "nvfp4" else cpu_baseline(w)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

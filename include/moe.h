@@ -373,14 +373,32 @@ int moe_bias_update(const int32_t* counts, int n_routed, int T, int top_k, float
  * "Inkling, Dissected" §02g (the Router Balance Lab measures MaxVio, the
  * hottest expert's load over the ideal minus one, and the share of expert
  * slots dropped) and §02d (what overflows a capacity is dropped).
- *   counts   [n_routed] int32: L_i (from moe_router_topk)
- *   capacity >= 0 (tokens per expert)
+ *   counts   [n_routed] int32: L_i (from moe_router_topk), the demand of the
+ *            batch of T tokens with top_k choices each
+ *   capacity >= 0 (tokens per expert; INT_MAX when no capacity applies)
  *   stats    [2] int32 out (device): stats[0] = max_i L_i,
- *            stats[1] = sum_i max(0, L_i - capacity), the dropped assignments.
- * MaxVio = stats[0] * n_routed / (top_k * T) - 1 and drop rate =
- * stats[1] / (top_k * T) are left to the caller.  Limits: n_routed <= 256.
+ *            stats[1] = sum_i max(0, L_i - capacity), the dropped assignments
+ *   metrics  [2] fp32 out (device) or NULL: metrics[0] = MaxVio =
+ *            max_i L_i * n_routed / (top_k * T) - 1, metrics[1] = drop rate =
+ *            stats[1] / (top_k * T); each quotient is formed in fp64 from the
+ *            exact integers and rounded once to fp32 (both 0 when T = 0).
+ * Limits: n_routed <= 256.  Errors: MOE_ERR_INVALID_ARG (null counts or stats,
+ * a pointer not 4-byte aligned, capacity < 0, T < 0, top_k < 1).
  */
-int moe_load_stats(const int32_t* counts, int n_routed, int capacity, int32_t* stats, void* stream);
+int moe_load_stats(const int32_t* counts, int n_routed, int T, int top_k, int capacity, int32_t* stats,
+                   float* metrics, void* stream);
+
+/*
+ * moe_capacity_for -- the expert capacity of "Inkling, Dissected" §02d ("1.25x
+ * the ideal load", the setting §02g's lab uses): floor(factor * top_k * T /
+ * n_routed) tokens, with factor = factor_num / factor_den given exactly (1.25 as
+ * 5/4), so no binary rounding of the factor moves the result.  Rounding down
+ * keeps the capacity at or below the stated multiple of the ideal load.
+ * Returns the capacity (clamped to INT_MAX), or MOE_ERR_INVALID_ARG for
+ * factor_num < 0, factor_den < 1, T < 0, top_k < 1 or n_routed < 1.  Host only,
+ * no device work.
+ */
+long long moe_capacity_for(long long factor_num, long long factor_den, int T, int top_k, int n_routed);
 
 /* Human-readable text for a MOE_* return code. */
 const char* moe_status_string(int code);

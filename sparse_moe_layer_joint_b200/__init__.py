@@ -50,7 +50,9 @@ _lib.moe_permute_scratch_bytes.argtypes = [_i32, _i32]
 _lib.moe_permute_scratch_bytes.restype = _sz
 _lib.moe_permute.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_permute_capped.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
-_lib.moe_load_stats.argtypes = [_vp, _i32, _i32, _vp, _vp]
+_lib.moe_load_stats.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.moe_capacity_for.argtypes = [ctypes.c_longlong, ctypes.c_longlong, _i32, _i32, _i32]
+_lib.moe_capacity_for.restype = ctypes.c_longlong
 _lib.moe_permute_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_grouped_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
 _lib.moe_experts_ffn.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp,
@@ -136,12 +138,17 @@ def _check(fn: str, rc: int):
         _debug_sync(fn)
 
 
-# MOE_DEBUG_SYNC=1: after every call, synchronise and read the device status word, so a
-# device-side error is reported at the call that caused it (slow; off by default).
+# MOE_DEBUG_SYNC=1: after every call, synchronise the device and read the device status word, so
+# a device-side error is reported at the call that caused it (slow; off by default).
 _DEBUG_SYNC = os.environ.get("MOE_DEBUG_SYNC") == "1"
 
 
 def _debug_sync(fn: str):
+    import torch
+
+    # the call may have run on any stream (MoELayer uses a side stream too): wait for the whole
+    # device, so the status read sees this call's kernels and its reset races no running kernel
+    torch.cuda.synchronize()
     v = _i32(0)
     rc = _lib.moe_get_status(None, ctypes.byref(v))
     if rc != MOE_OK or v.value != 0:
@@ -211,8 +218,16 @@ def moe_bias_update(counts, n_routed: int, T: int, top_k: int, gamma: float, bia
     _check("moe_bias_update", _lib.moe_bias_update(_p(counts), n_routed, T, top_k, gamma, _p(bias), _stream(stream)))
 
 
-def moe_load_stats(counts, n_routed: int, capacity: int, stats, stream=None):
-    _check("moe_load_stats", _lib.moe_load_stats(_p(counts), n_routed, capacity, _p(stats), _stream(stream)))
+def moe_load_stats(counts, n_routed: int, T: int, top_k: int, capacity: int, stats, metrics=None, stream=None):
+    _check("moe_load_stats", _lib.moe_load_stats(_p(counts), n_routed, T, top_k, capacity, _p(stats), _p(metrics),
+                                                 _stream(stream)))
+
+
+def moe_capacity_for(factor_num: int, factor_den: int, T: int, top_k: int, n_routed: int) -> int:
+    c = int(_lib.moe_capacity_for(int(factor_num), int(factor_den), T, top_k, n_routed))
+    if c < 0:
+        raise MoEError("moe_capacity_for", c)
+    return c
 
 
 def moe_nvfp4_quantize_weights(w, G: int, N: int, K: int, q, sf, gscale, stream=None):
@@ -239,10 +254,11 @@ def moe_nvfp4_grouped_gemm(aq, asf, offsets_pad, n_groups: int, rows_cap: int, w
 
 
 def capacity_for(factor: float, T: int, k: int, n_routed: int) -> int:
-    """Expert capacity in tokens: floor(factor * k*T / n_routed), with the factor
-    read as the decimal it prints as (1.25 = 5/4)."""
+    """Expert capacity in tokens (moe_capacity_for), the Python float factor passed
+    as the exact fraction of the decimal it prints as (1.25 -> 5/4)."""
     from fractions import Fraction
-    return int((Fraction(repr(float(factor))) * (k * T)) // n_routed)
+    q = Fraction(repr(float(factor)))
+    return moe_capacity_for(q.numerator, q.denominator, T, k, n_routed)
 
 
 def moe_get_status(stream=None) -> int:
@@ -329,7 +345,8 @@ class MoELayer:
         self.h_shared = torch.empty((max(s.n_shared, 1), s.T, s.d_ff), dtype=bf, device=dev)
         self.y_shared = torch.empty((max(s.n_shared, 1), s.T, s.d), dtype=bf, device=dev)
         self.out = torch.empty((s.T, s.d), dtype=bf, device=dev)
-        self.stats = torch.zeros((2,), dtype=torch.int32, device=dev)
+        # moe_load_stats output: max load and dropped assignments (int32), then MaxVio and the drop rate (fp32 bits)
+        self.stats = torch.zeros((4,), dtype=torch.int32, device=dev)
         if self.nvfp4:
             self.rows_cap = moe_nvfp4_rows_capacity(s.T, s.n_routed, s.top_k)
             u8 = torch.uint8
@@ -452,11 +469,12 @@ class MoELayer:
         s = self.shape
         cap = self.capacity if self.capacity is not None else 2 ** 31 - 1
         st = stream if stream is not None else torch.cuda.current_stream()
-        moe_load_stats(self.counts, s.n_routed, cap, self.stats, stream=st)
-        max_load, dropped = (int(v) for v in self.stats.cpu().tolist())
-        kT = s.top_k * s.T
-        return {"max_load": max_load, "dropped": dropped, "max_vio": max_load * s.n_routed / kT - 1.0 if kT else 0.0,
-                "drop_rate": dropped / kT if kT else 0.0}
+        moe_load_stats(self.counts, s.n_routed, s.T, s.top_k, cap, self.stats[:2], self.stats[2:].view(torch.float32),
+                       stream=st)
+        host = self.stats.cpu()
+        max_load, dropped = (int(v) for v in host[:2].tolist())
+        max_vio, drop_rate = (float(v) for v in host[2:].view(torch.float32).tolist())
+        return {"max_load": max_load, "dropped": dropped, "max_vio": max_vio, "drop_rate": drop_rate}
 
     def bias_update(self, bias, gamma: float, stream=None, T_total: Optional[int] = None):
         """b += gamma * sign(Lbar - L) from this layer's counts; T_total: the batch's token

@@ -5,7 +5,11 @@
 // gamma * (+1, 0 or -1), which is exact before rounding.
 //
 // load_stats -- the balance of one batch from the same loads (§02d, §02g):
-// the largest load and the assignments past the experts' capacity.
+// the largest load and the assignments past the experts' capacity, and from
+// them MaxVio and the drop rate.
+//
+// capacity_for -- the capacity of §02d/§02g ("1.25x the ideal load"):
+// floor(factor * k*T / n_routed), the factor given as an exact fraction.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,8 +29,8 @@ __global__ void bias_update_kernel(const int32_t* __restrict__ counts, int n_rou
 }
 
 // One CTA of 256 threads; thread i owns expert i (n_routed <= 256).
-__global__ void load_stats_kernel(const int32_t* __restrict__ counts, int n_routed, int capacity,
-                                  int32_t* __restrict__ stats) {
+__global__ void load_stats_kernel(const int32_t* __restrict__ counts, int n_routed, long long kT, int capacity,
+                                  int32_t* __restrict__ stats, float* __restrict__ metrics) {
   __shared__ int wmax[8], wdrop[8];
   const int i = threadIdx.x;
   const int L = i < n_routed ? counts[i] : 0;
@@ -49,6 +53,12 @@ __global__ void load_stats_kernel(const int32_t* __restrict__ counts, int n_rout
     }
     stats[0] = mx;
     stats[1] = dr;
+    if (metrics != nullptr) {
+      // MaxVio = max_i L_i / Lbar - 1 with Lbar = k*T / n_routed; drop rate = dropped / (k*T).
+      // Both quotients are formed in fp64 from the exact integers and rounded once to fp32.
+      metrics[0] = kT > 0 ? (float)((double)mx * (double)n_routed / (double)kT - 1.0) : 0.0f;
+      metrics[1] = kT > 0 ? (float)((double)dr / (double)kT) : 0.0f;
+    }
   }
 }
 
@@ -64,9 +74,22 @@ extern "C" int moe_bias_update(const int32_t* counts, int n_routed, int T, int t
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-extern "C" int moe_load_stats(const int32_t* counts, int n_routed, int capacity, int32_t* stats, void* stream) {
-  if (!counts || !stats || n_routed < 1 || n_routed > MOE_MAX_ROUTED || capacity < 0) return MOE_ERR_INVALID_ARG;
-  if (!moe::aligned4(counts) || !moe::aligned4(stats)) return MOE_ERR_INVALID_ARG;
-  moe::load_stats_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(counts, n_routed, capacity, stats);
+extern "C" int moe_load_stats(const int32_t* counts, int n_routed, int T, int top_k, int capacity, int32_t* stats,
+                              float* metrics, void* stream) {
+  if (!counts || !stats || n_routed < 1 || n_routed > MOE_MAX_ROUTED || capacity < 0 || T < 0 || top_k < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (!moe::aligned4(counts) || !moe::aligned4(stats) || (metrics && !moe::aligned4(metrics)))
+    return MOE_ERR_INVALID_ARG;
+  moe::load_stats_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(counts, n_routed, (long long)top_k * T, capacity, stats,
+                                                              metrics);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" long long moe_capacity_for(long long factor_num, long long factor_den, int T, int top_k, int n_routed) {
+  if (factor_num < 0 || factor_den < 1 || T < 0 || top_k < 1 || n_routed < 1) return MOE_ERR_INVALID_ARG;
+  // floor(factor * k*T / n_routed) in exact integer arithmetic (128-bit: no intermediate can overflow)
+  const unsigned __int128 num = (unsigned __int128)factor_num * (unsigned __int128)top_k * (unsigned __int128)T;
+  const unsigned __int128 den = (unsigned __int128)factor_den * (unsigned __int128)n_routed;
+  const unsigned __int128 c = num / den;
+  return c > (unsigned __int128)0x7fffffff ? (long long)0x7fffffff : (long long)c;
 }

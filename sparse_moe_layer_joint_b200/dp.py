@@ -11,6 +11,19 @@ the same number of tokens.
 from __future__ import annotations
 
 
+def _all_reduce_sum(t, group=None):
+    """All-reduce (sum); gloo has no CUDA all-reduce path here, so CUDA tensors go through a host copy."""
+    import torch.distributed as dist
+
+    if t.is_cuda and dist.get_backend(group) == "gloo":
+        h = t.cpu()
+        dist.all_reduce(h, op=dist.ReduceOp.SUM, group=group)
+        t.copy_(h)
+        return t
+    dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return t
+
+
 def world_size(group=None) -> int:
     import torch.distributed as dist
 
@@ -19,10 +32,8 @@ def world_size(group=None) -> int:
 
 def global_counts(counts, group=None):
     """Sum the per-expert load counts over all ranks, in place (no-op on one rank)."""
-    import torch.distributed as dist
-
     if world_size(group) > 1:
-        dist.all_reduce(counts, op=dist.ReduceOp.SUM, group=group)
+        _all_reduce_sum(counts, group)
     return counts
 
 

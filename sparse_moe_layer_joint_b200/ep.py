@@ -9,16 +9,21 @@ W dividing E) and a replica of the shared experts.  One step on rank r:
 1. route its own tokens (router kernel) and group the (token, slot) pairs by
    expert (moe_permute): the experts of each destination rank are then one
    contiguous block of rows;
-2. exchange the per-expert row counts, then the rows (two all-to-alls);
+2. exchange the per-expert row counts, then the rows (two all-to-alls); the
+   shared experts run on a second stream meanwhile;
 3. run the owned experts on the rows received from every source rank
    (moe_grouped_ffn once per source chunk, whose rows are grouped by expert);
 4. send the results back (all-to-all): they land in the sender's dispatch order,
    so the combine is the one-GPU combine (moe_combine through token_row);
-5. the bias update uses the loads summed over ranks (as in ``dp``).
+5. ``bias_update``: the loads summed over ranks (one all-reduce, as in ``dp``),
+   then the update with the whole batch's token count on every rank.
+
+No capacity is applied in this mode: every (token, slot) pair is served.
 
 The plan and exchange functions below are device-agnostic (torch tensors, any
-backend that implements all_to_all_single); ``ExpertParallelLayer`` runs the
-GPU step with the library's kernels and NCCL.
+backend that implements all_to_all_single; with gloo, CUDA tensors are staged
+through host memory).  ``ExpertParallelLayer`` runs the GPU step with the
+library's kernels and NCCL (or gloo).
 """
 from __future__ import annotations
 
@@ -42,16 +47,29 @@ def send_counts(offsets: Sequence[int], n_routed: int, world: int) -> List[int]:
     return [int(off[(q + 1) * per] - off[q * per]) for q in range(world)]
 
 
+def _all_to_all(out, inp, out_splits=None, in_splits=None, group=None):
+    """all_to_all_single; gloo has no CUDA all-to-all, so there CUDA tensors go through host copies."""
+    import torch.distributed as dist
+
+    if inp.is_cuda and dist.get_backend(group) == "gloo":
+        host_out = out.new_empty(out.shape, device="cpu")
+        dist.all_to_all_single(host_out, inp.cpu(), output_split_sizes=out_splits, input_split_sizes=in_splits,
+                               group=group)
+        out.copy_(host_out)
+        return out
+    dist.all_to_all_single(out, inp, output_split_sizes=out_splits, input_split_sizes=in_splits, group=group)
+    return out
+
+
 def exchange_counts(counts_by_expert, world: int, group=None):
     """All-to-all of per-expert row counts: ``counts_by_expert`` [n_routed] int32 (this rank's
     dispatch); returns [world, n_routed/world]: row s = the rows source s sends for each of
     this rank's experts."""
     import torch
-    import torch.distributed as dist
 
     per = counts_by_expert.numel() // world
     out = torch.empty((world * per,), dtype=counts_by_expert.dtype, device=counts_by_expert.device)
-    dist.all_to_all_single(out, counts_by_expert.contiguous(), group=group)
+    _all_to_all(out, counts_by_expert.contiguous(), group=group)
     return out.view(world, per)
 
 
@@ -59,16 +77,13 @@ def exchange_rows(rows, send: Sequence[int], recv: Sequence[int], group=None, ou
     """All-to-all of row blocks: ``rows`` [sum(send), ...] ordered by destination rank; returns
     [sum(recv), ...] ordered by source rank (in ``out`` when given)."""
     import torch
-    import torch.distributed as dist
 
     n = int(sum(recv))
     if out is None:
         out = torch.empty((n,) + tuple(rows.shape[1:]), dtype=rows.dtype, device=rows.device)
     else:
         out = out[:n]
-    dist.all_to_all_single(out, rows.contiguous(), output_split_sizes=[int(v) for v in recv],
-                           input_split_sizes=[int(v) for v in send], group=group)
-    return out
+    return _all_to_all(out, rows.contiguous(), [int(v) for v in recv], [int(v) for v in send], group)
 
 
 def chunk_offsets(recv_by_expert: np.ndarray) -> List[np.ndarray]:
@@ -80,11 +95,13 @@ def chunk_offsets(recv_by_expert: np.ndarray) -> List[np.ndarray]:
 class ExpertParallelLayer:
     """One layer step with the routed experts split over ranks (bf16, GELU or SwiGLU experts).
 
-    Not exercised on GPUs in this repository's tests: every run here has one GPU.  Its
-    compute is the library's kernels (router, permute, grouped FFN, combine, bias update);
-    its exchange is NCCL all-to-all of the dispatched rows and of the expert outputs.
-    Weights: ``w_router`` and the shared experts' matrices as on one GPU; ``w1_local`` /
-    ``w2_local`` hold only this rank's routed experts, followed by the shared experts.
+    Its compute is the library's kernels (router, permute, grouped FFN, combine, bias update);
+    its exchange is an all-to-all of the dispatched rows and of the expert outputs (NCCL, or
+    gloo through host copies).  Weights: ``w_router`` and the shared experts' matrices as on one
+    GPU; ``w1_local`` / ``w2_local`` hold only this rank's routed experts, followed by the
+    shared experts.  The tests run it at one rank (NCCL) and at two ranks sharing one GPU (gloo:
+    the ranks' kernels never wait on each other, the exchange is on the host); across several
+    GPUs it is not measured here.
     """
 
     def __init__(self, shape, rank: int, world: int, device="cuda", group=None, activation: str = "gelu_tanh",
@@ -97,6 +114,10 @@ class ExpertParallelLayer:
         self.lo, self.hi = expert_range(shape.n_routed, world, rank)
         self.local = MoELayer(shape, device=device, activation=activation, route_scale=route_scale)
         self.dev = torch.device(device)
+        self.offsets_host = torch.empty((shape.n_routed + 1,), dtype=torch.int32).pin_memory()
+        self.ev_offsets = torch.cuda.Event()
+        self.ev_routed = torch.cuda.Event()
+        self.ev_shared = torch.cuda.Event()
 
     def forward(self, x, w_router, w1_local, w2_local, bias, logit_offset=None):
         import torch
@@ -106,18 +127,27 @@ class ExpertParallelLayer:
         L, s = self.local, self.local.shape
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
         E_loc = self.hi - self.lo
+        main = torch.cuda.current_stream(self.dev)
         moe.moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, L.route_scale,
-                            L.topk_idx, L.gates, L.counts, None)
-        moe.moe_permute(x, L.topk_idx, L.counts, T, d, s.n_routed, k, L.offsets, L.x_perm, L.row_token,
-                        L.token_row, L.scratch, L.scratch_bytes)
-        # shared experts on this rank's tokens while the exchange runs
+                            L.topk_idx, L.gates, L.counts, None, stream=main)
+        # shared experts on this rank's tokens, on the side stream while the exchange runs
         if s.n_shared > 0:
+            self.ev_routed.record(main)
+            L.side.wait_event(self.ev_routed)
             moe.moe_grouped_ffn(x, None, s.n_shared, T, E_loc, w1_local, w2_local, d, f, L.activation,
-                                L.h_shared, L.y_shared)
-        offsets = L.offsets.cpu().numpy()                      # split sizes for the exchange (1 KB)
+                                L.h_shared, L.y_shared, stream=L.side)
+            self.ev_shared.record(L.side)
+        moe.moe_permute(x, L.topk_idx, L.counts, T, d, s.n_routed, k, L.offsets, L.x_perm, L.row_token,
+                        L.token_row, L.scratch, L.scratch_bytes, stream=main)
+        # the split sizes of the exchange are host values: copy the 257 offsets (1 KB) and wait for
+        # that copy alone (the event is on the main stream; the side stream keeps running)
+        self.offsets_host.copy_(L.offsets, non_blocking=True)
+        self.ev_offsets.record(main)
+        self.ev_offsets.synchronize()
+        offsets = self.offsets_host.numpy().astype(np.int64)
         send = send_counts(offsets, s.n_routed, self.world)
-        by_expert = torch.from_numpy(np.diff(offsets).astype(np.int32)).to(self.dev)
-        recv_by_expert = exchange_counts(by_expert, self.world, self.group).cpu().numpy()
+        # rows per expert = the router's counts (no capacity in this mode)
+        recv_by_expert = exchange_counts(L.counts, self.world, self.group).cpu().numpy()
         recv = recv_by_expert.sum(axis=1)
         x_recv = exchange_rows(L.x_perm[:int(offsets[-1])], send, recv, self.group)
         y_recv = torch.empty_like(x_recv)
@@ -128,9 +158,18 @@ class ExpertParallelLayer:
             if n:
                 off_dev = torch.from_numpy(off).to(self.dev)
                 moe.moe_grouped_ffn(x_recv[start:start + n], off_dev, E_loc, n, 0, w1_local, w2_local, d, f,
-                                    L.activation, h[:n], y_recv[start:start + n])
+                                    L.activation, h[:n], y_recv[start:start + n], stream=main)
             start += n
         exchange_rows(y_recv, recv, send, self.group, out=L.y_perm)   # back in this rank's dispatch order
+        if s.n_shared > 0:
+            main.wait_event(self.ev_shared)
         moe.moe_combine(L.y_perm, L.token_row, L.gates, L.y_shared if s.n_shared > 0 else None, T, d, k,
-                        s.n_shared, L.out)
+                        s.n_shared, L.out, stream=main)
         return L.out
+
+    def bias_update(self, bias, gamma: float):
+        """§02e after the step: this rank's loads summed over all ranks (in place, one all-reduce of
+        n_routed int32), then b += gamma * sign(Lbar - L) with the whole batch's token count."""
+        from sparse_moe_layer_joint_b200 import dp
+
+        dp.bias_step(self.local, bias, gamma, group=self.group)

@@ -5,6 +5,7 @@ import ctypes
 
 import pytest
 
+import oracle
 import sparse_moe_layer_joint_b200 as moe
 
 NULL = None
@@ -146,10 +147,32 @@ def test_capacity_and_stats_reject():
                                 NULL) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_permute_capped(A16, A16, NULL, 8, 64, 256, 6, 5, A16, A16, A16, A16, A16, 16,
                                 NULL) == moe.MOE_ERR_SCRATCH
-    assert L.moe_load_stats(A16, 256, -3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
-    assert L.moe_load_stats(A16, 257, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
-    assert L.moe_load_stats(NULL, 256, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
-    assert L.moe_load_stats(0x10002, 256, 3, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(A16, 256, 64, 6, -3, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(A16, 257, 64, 6, 3, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(NULL, 256, 64, 6, 3, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(0x10002, 256, 64, 6, 3, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(A16, 256, -1, 6, 3, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(A16, 256, 64, 0, 3, A16, A16, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_load_stats(A16, 256, 64, 6, 3, A16, 0x10002, NULL) == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("factor,T,k,E", [(1.25, 2048, 6, 64), (1.25, 65536, 6, 256), (1.25, 100, 6, 64),
+                                          (1.0, 256, 6, 256), (1.1, 1000, 1, 10), (0.0, 500, 6, 256),
+                                          (2.5, 1, 6, 256), (1.3333, 4096, 8, 7)])
+def test_capacity_for_matches_the_oracle(factor, T, k, E):
+    """moe_capacity_for (exact integer floor of factor * k*T / n_routed) against the oracle's
+    definition, with the Python float factor passed as the fraction of its decimal form."""
+    assert moe.capacity_for(factor, T, k, E) == oracle.capacity_for(factor, T, k, E)
+
+
+def test_capacity_for_rejects_and_clamps():
+    assert L.moe_capacity_for(5, 0, 10, 6, 64) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_capacity_for(-1, 4, 10, 6, 64) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_capacity_for(5, 4, -1, 6, 64) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_capacity_for(5, 4, 10, 0, 64) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_capacity_for(5, 4, 10, 6, 0) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_capacity_for(10 ** 12, 1, 2 ** 31 - 1, 8, 1) == 2 ** 31 - 1      # clamped, no overflow
+    assert L.moe_capacity_for(5, 4, 0, 6, 64) == 0
 
 
 def test_nvfp4_entry_points_reject():

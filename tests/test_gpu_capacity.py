@@ -82,10 +82,13 @@ def test_load_stats_exact(E, cap, skew):
     topk = _topk(T, k, E, E + 3, skew)
     L = oracle.load_counts(topk, E)
     st = torch.full((2,), -1, dtype=torch.int32, device="cuda")
-    moe.moe_load_stats(_i32(L), E, cap, st)
+    mt = torch.full((2,), -1, dtype=torch.float32, device="cuda")
+    moe.moe_load_stats(_i32(L), E, T, k, cap, st, mt)
     got = st.cpu().numpy()
     m = oracle.load_metrics(L, cap, T, k)
     assert got[0] == m["max_load"] and got[1] == m["dropped"]
+    # MaxVio and the drop rate: the oracle's fp64 values rounded once to fp32
+    np.testing.assert_array_equal(mt.cpu().numpy(), np.array([m["max_vio"], m["drop_rate"]], dtype=np.float32))
 
 
 def _layer_with_capacity(name, factor, tokens):
@@ -107,6 +110,7 @@ def _layer_with_capacity(name, factor, tokens):
     bal = layer.balance()
     m = oracle.load_metrics(layer.counts.cpu().numpy(), cap, w.T, w.k)
     assert bal["dropped"] == m["dropped"] == int((~keep).sum()) and bal["max_load"] == m["max_load"]
+    assert bal["max_vio"] == np.float32(m["max_vio"]) and bal["drop_rate"] == np.float32(m["drop_rate"])
     assert m["dropped"] > 0
     # the routing itself, and the output with the drops applied, against the oracle
     off = mi.host_logit_offset(w)
@@ -166,7 +170,7 @@ def _gpu_lab(w, gamma):
     for s in range(w.steps):
         moe.moe_router_topk(xs[s], wr, b, None, w.T, w.d, w.n_routed, 0, w.k, 1.0, idx, g, c)
         moe.moe_permute_capped(None, idx, c, w.T, w.d, w.n_routed, w.k, cap, off, None, rt, tr, scratch, nb)
-        moe.moe_load_stats(c, w.n_routed, cap, st)
+        moe.moe_load_stats(c, w.n_routed, w.T, w.k, cap, st)
         moe.moe_bias_update(c, w.n_routed, w.T, w.k, gamma, b)
         res["topk"].append(idx.cpu().numpy())
         res["counts"].append(c.cpu().numpy())

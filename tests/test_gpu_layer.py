@@ -45,7 +45,29 @@ def _check_dispatch_properties(layer, x_bits, T, k, n_routed):
         np.testing.assert_array_equal(xp, x_bits[rt[sample]])
 
 
-def _run_and_check(name, tokens=None, check_all_routing=True, fused=True, gather=False):
+def _check_expert_groups(w, layer, t, x_bits, experts, shared_tokens=None):
+    """Whole row groups of the expert GEMMs at full size: every y_perm row of each
+    listed expert (its ragged last tile included) against the oracle's expert on
+    the token that row holds; optionally the shared experts' rows of some tokens."""
+    off = layer.offsets.cpu().numpy().astype(np.int64)
+    rt = layer.row_token.cpu().numpy()
+    fn = oracle.expert_for(w)
+    for e in experts:
+        lo, hi = int(off[e]), int(off[e + 1])
+        assert hi > lo
+        got = host_bf16_f64(layer.y_perm[lo:hi])
+        ref = fn(x_bits[rt[lo:hi]], host_bf16_bits(t["w1"][e]), host_bf16_bits(t["w2"][e]))
+        check_output(got, ref, f"{w.name} expert {e} rows {lo}..{hi}")
+    if shared_tokens is not None:
+        for s_i in range(w.n_shared):
+            e = w.n_routed + s_i
+            got = host_bf16_f64(layer.y_shared[s_i][torch.from_numpy(shared_tokens).cuda()])
+            ref = fn(x_bits[shared_tokens], host_bf16_bits(t["w1"][e]), host_bf16_bits(t["w2"][e]))
+            check_output(got, ref, f"{w.name} shared expert {e}")
+
+
+def _run_and_check(name, tokens=None, check_all_routing=True, fused=True, gather=False, expert_groups=None,
+                   shared_tokens=None):
     w = mi.WORKLOADS[name]
     t, layer = _layer(w, fused=fused, gather=gather)
     bias0 = t["bias"].clone()
@@ -67,6 +89,8 @@ def _run_and_check(name, tokens=None, check_all_routing=True, fused=True, gather
             nb = oracle.bias_update(ref_counts, b_host, w.T, w.k, w.gamma)
             np.testing.assert_array_equal(t["bias"].cpu().numpy().view(np.uint32), nb.view(np.uint32))
     _check_dispatch_properties(layer, x_bits, w.T, w.k, w.n_routed)
+    if expert_groups is not None:
+        _check_expert_groups(w, layer, t, x_bits, expert_groups, shared_tokens)
     # layer output on the sampled tokens
     if tokens is None:
         tokens = np.arange(w.T)
@@ -108,9 +132,13 @@ def test_layer_decode_sampled():
 
 
 @pytest.mark.slow
-def test_layer_prefill_sampled():
-    w = mi.WORKLOADS["prefill"]
-    _run_and_check("prefill", tokens=np.array([0, 1, 4095, 30000, 65535]), check_all_routing=False)
+def test_layer_prefill_full_routing_and_groups():
+    """Prefill size (65536 tokens, d 7168): every token's routing and gates, the counts
+    and the bias update against the oracle; the complete row groups of the first, a
+    middle and the last routed expert, and 512 tokens of both shared experts, from the
+    full-size GEMM launches; the layer output on sampled tokens."""
+    _run_and_check("prefill", tokens=np.array([0, 1, 4095, 30000, 65535]), expert_groups=[0, 128, 255],
+                   shared_tokens=np.arange(65536 - 512, 65536))
 
 
 def test_layer_inkling_decode_sampled():
@@ -119,9 +147,12 @@ def test_layer_inkling_decode_sampled():
 
 
 @pytest.mark.slow
-def test_layer_inkling_sampled():
-    """The released configuration at prefill scale (65536 tokens, about 29 GB of expert weights)."""
-    _run_and_check("inkling", tokens=np.array([0, 7, 40000, 65535]), check_all_routing=False)
+def test_layer_inkling_full_routing_and_groups():
+    """The released configuration at prefill scale (65536 tokens, about 29 GB of expert
+    weights): all tokens' routing (route_scale 8), counts and bias update; whole row
+    groups of three routed experts and 256 tokens of the shared experts."""
+    _run_and_check("inkling", tokens=np.array([0, 7, 40000, 65535]), expert_groups=[0, 131, 255],
+                   shared_tokens=np.arange(0, 65536, 256))
 
 
 @pytest.mark.slow

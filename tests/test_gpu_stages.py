@@ -478,6 +478,19 @@ def test_bounded_wait_times_out_and_reports():
     assert counts.sum() == 64 * 6
 
 
+def test_debug_sync_reports_the_failing_call(monkeypatch):
+    """With the debug-sync check on, a device-side timeout raises at the call that timed out,
+    also when that call ran on a stream other than the current one."""
+    assert moe.moe_get_status() == 0
+    monkeypatch.setattr(moe, "_DEBUG_SYNC", True)
+    side = torch.cuda.Stream()
+    with pytest.raises(moe.MoEError) as err:
+        moe.moe_debug_bounded_wait(20_000_000, stream=side)
+    assert "moe_debug_bounded_wait" in str(err.value) and err.value.code == moe.MOE_ERR_TIMEOUT
+    moe.moe_permute_scratch_bytes(64, 256)          # a call that does not check the status
+    assert moe.moe_get_status() == 0                 # the debug check read and cleared the bit
+
+
 def test_generator_device_matches_host():
     """The device generator writes the same bits as the host generator."""
     w = mi.WORKLOADS["tiny"]
