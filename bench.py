@@ -299,16 +299,19 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
     gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
     kernel = f"grouped_gemm_kernel x2 (all experts: GEMM1+{'SwiGLU' if w.activation == 'swiglu' else 'GELU'}, GEMM2)"
     traffic = TRAFFIC_PER_LAUNCH_PAIR.get(w.name) if args.capacity_factor is None and not args.gather_rows else None
+    # the expert launches are timed inside a step of tens of ms, not a seconds-long loop: the burst peak
     tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1),
-                   "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                   "frac": round(tflops / pk["bf16_tflops_sustained"], 4),
-                   "peak_source": f"{pk['src']} bf16 sustained (MEASURED_PEAKS.json)" if pk["src"] == "measured"
-                   else "fallback bf16 sustained", "traffic": traffic, "traffic_unit": "bytes per launch pair",
+                   "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                   "frac": round(tflops / pk["bf16_tflops"], 4),
+                   "frac_of_sustained": round(tflops / pk["bf16_tflops_sustained"], 4),
+                   "peak_source": f"{pk['src']} bf16 burst (MEASURED_PEAKS.json)" if pk["src"] == "measured"
+                   else "fallback bf16 burst (1.59 PFLOP/s)", "traffic": traffic, "traffic_unit": "bytes per launch pair",
                    "algorithmic_bytes_per_launch_pair": round(ffn_bytes),
                    "flop_per_launch_pair": ffn_flops, "ms_per_launch_pair": round(ffn_ms, 4)}
     hbm_roof = {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / pk["hbm_gbs"], 4),
-                "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)", "traffic": traffic,
+                "peak_source": f"{pk['src']} HBM copy (MEASURED_PEAKS.json)" if pk["src"] == "measured"
+                else "fallback HBM copy (6.65 TB/s)", "traffic": traffic,
                 "bytes_per_launch_pair": round(ffn_bytes), "touched_routed_experts_mean": round(touched, 2),
                 "ms_per_launch_pair": round(ffn_ms, 4)}
     weight_bound = w.name in ("decode", "mid", "inkling_decode")
