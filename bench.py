@@ -322,7 +322,7 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
         "metric": METRIC, "value": round(world * w.T / (ms * 1e-3), 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox, random-init weights)",
-        "config": dict(config_of(w, world), dispatch="rows gathered by GEMM1 (cp.async)" if args.gather_rows
+        "config": dict(config_of(w, world), dispatch="rows gathered by GEMM1 (TMA gather4)" if args.gather_rows
                        else "rows copied by moe_permute",
                        **({"cuda_graph": True, "ms_per_step_without_graph": round(eager_ms, 4)}
                           if eager_ms is not None else {}),
@@ -660,7 +660,7 @@ def run_reference(args, w):
         total += one(tokens[j:j + per_step])
     ms = total / args.steps * 1e3
     v = round(per_step / (ms * 1e-3), 4)
-    config = dict(config_of(w, 1), dispatch="rows gathered by GEMM1 (cp.async)" if args.gather_rows
+    config = dict(config_of(w, 1), dispatch="rows gathered by GEMM1 (TMA gather4)" if args.gather_rows
                   else "rows copied by moe_permute")
     if args.precision == "nvfp4":
         config["precision"] = "nvfp4 routed experts (W4A4)"
@@ -794,7 +794,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true",
                     help="prefill workload: skip the decode-scale record measured after the prefill steps")
     ap.add_argument("--gather-rows", action="store_true",
-                    help="GEMM1 gathers the routed rows from x (cp.async) instead of reading rows copied by dispatch")
+                    help="GEMM1 gathers the routed rows from x (TMA tile::gather4) instead of reading rows copied "
+                         "by dispatch")
     ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "nvfp4_ffn", "router"],
                     default=None,
                     help="time one kernel alone on a small profiling case instead of the layer")

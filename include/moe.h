@@ -232,7 +232,9 @@ int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int n_groups, 
  *              x_perm is NULL)
  *   x_perm     [T*top_k, d] bf16 (from moe_permute) or NULL: then the routed rows
  *              are gathered from x through row_token by the GEMM's own loads
- *              (cp.async row copies), and moe_permute need not copy rows
+ *              (TMA tile::gather4, four rows an instruction), and moe_permute
+ *              need not copy rows (on B200 this is slower than copied rows:
+ *              the gathers bound the TMA unit)
  *   row_token  [T*top_k] int32 (from moe_permute); used when x_perm is NULL
  *   offsets    [n_routed + 1] int32 (from moe_permute)
  *   w1, w2     [n_routed + n_shared, d_ff, d] and [n_routed + n_shared, d, d_ff]

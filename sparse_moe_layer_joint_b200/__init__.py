@@ -321,9 +321,10 @@ class MoELayer:
         # hard expert capacity (tokens per expert per batch); None: every assignment is served
         self.capacity = None if capacity_factor is None else capacity_for(capacity_factor, s.T, s.top_k, s.n_routed)
         self.fused_experts = fused_experts
-        # with the fused experts, GEMM1 can gather the routed rows from x itself (no x_perm copy);
-        # measured slower on B200 at every workload here (32 row gathers per stage bound the TMA
-        # unit), so the default copies the rows in moe_permute and loads tiles
+        # with the fused experts, GEMM1 can gather the routed rows from x itself (TMA tile::gather4
+        # loads, no x_perm copy); measured slower on B200 (at prefill size GEMM1 took 1.65x as long:
+        # 32 four-row gathers per stage bound the TMA unit), so the default copies the rows in
+        # moe_permute and loads whole tiles
         self.gather_rows = gather_rows and fused_experts
         dev = torch.device(device)
         R = s.T * s.top_k

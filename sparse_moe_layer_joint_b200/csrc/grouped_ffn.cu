@@ -15,7 +15,9 @@
 //
 // Per CTA (persistent, static round-robin over tiles):
 //   warp 0      TMA producer into a shared-memory ring of A and B tiles
-//               (128-byte swizzle, full/empty mbarriers)
+//               (128-byte swizzle, full/empty mbarriers); in gathering launches
+//               the routed A rows come from the token rows through the row
+//               indices, one tile::gather4 load (four rows) per lane and stage
 //   warp 1      TMEM owner + MMA issuer (one thread): tcgen05.mma kind::f16,
 //               bf16 in, fp32 accumulators in TMEM, two 256-column
 //               accumulator buffers so the epilogue of tile i overlaps the
@@ -33,6 +35,10 @@
 //                 CTAs' barriers, both epilogues release the accumulator on
 //                 the leader.  Per CTA this halves the B operand's shared-
 //                 memory traffic (6-stage ring of 32 KB).
+//   WIDE          pair tiles of 256 x 512 (see Cfg): 25% fewer L2 bytes per FLOP,
+//                 but one accumulator (the epilogue is not overlapped); measured
+//                 no faster than 256 x 256 on B200 at the prefill size, so off by
+//                 default (MOE_GEMM_WIDE=1).
 // Ragged groups: a tile's A rows may run past its group (into the next
 // group's rows, or past the tensor where TMA fills zeros); the epilogue writes
 // only the group's own rows.
@@ -51,7 +57,6 @@ namespace gffn {
 
 constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 64;   // reduction depth per stage (one 128-byte swizzle atom)
-constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_NONE = 1;
@@ -61,26 +66,37 @@ constexpr int EPI_NONE = 1;
 constexpr int EPI_SWIGLU = 2;
 constexpr int SWIGLU_OUT = BN / 2;
 
-template <bool PAIR, int ST>
+// WIDE (pairs only): a tile is 256 x 512, two 256-column halves that share the A stage; each CTA
+// holds 128 A rows and 2 x 128 weight rows per stage, so a K step moves 48 KB per CTA for twice
+// the MMA work of a 256 x 256 tile (32 KB): 25% fewer L2 -> shared-memory bytes per FLOP.  Its
+// 512-column accumulator fills TMEM, so there is one accumulator, drained by eight epilogue warps
+// (two per TMEM lane quarter, one per column half) before the next tile's MMAs start.
+template <bool PAIR, int ST, bool WIDE = false>
 struct Cfg {
+  static_assert(!WIDE || PAIR, "wide tiles are pair tiles");
+  static constexpr int NH = WIDE ? 2 : 1;          // 256-column halves per tile
+  static constexpr int TILE_N = BN * NH;           // output columns per tile
   static constexpr int TILE_M = PAIR ? 256 : 128;  // rows per tile (per pair, or per CTA)
   static constexpr int A_ROWS = 128;               // A rows held by one CTA
-  static constexpr int B_ROWS = PAIR ? 128 : 256;  // B rows (output columns) held by one CTA
+  static constexpr int B_HALF_ROWS = PAIR ? 128 : 256;  // weight rows of one column half held by one CTA
+  static constexpr int B_ROWS = B_HALF_ROWS * NH;  // B rows (output columns) held by one CTA
   static constexpr int STAGES = ST;
   static constexpr int A_BYTES = A_ROWS * BK * 2;
+  static constexpr int B_HALF_BYTES = B_HALF_ROWS * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARPS = 4 * NH;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int ACC_BUFS = WIDE ? 1 : 2;   // accumulators of 256 * NH columns in TMEM
   static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // bytes landing on the (leader's) full barrier
-  static constexpr uint32_t TX_B_BYTES = (PAIR ? 2 : 1) * B_BYTES;     // when A rows arrive by cp.async instead
-  static constexpr int GATHER_LAG = STAGES - 2;  // stages of row copies a producer lane keeps in flight
-  static constexpr int GATHER_ARRIVALS = 32 * (PAIR ? 2 : 1);  // producer lanes arriving per stage
+  static_assert(A_ROWS == 4 * 32, "one gather4 load per producer lane covers the CTA's A rows");
 };
 
 struct Params {
   const int* offsets;  // [G_r + 1] routed group row offsets (device); unused when G_r == 0
-  const int* gather_rows;  // non-null: routed A rows are gathered, row r of group g = gather_rows[off[g] + r]
+  const int* gather_rows;  // non-null: routed A rows are gathered through map A0 (one-row boxes),
+                           // row r of group g = gather_rows[off[g] + r]
   int gather_limit;        // gathered row indices are clamped to [0, gather_limit)
-  const __nv_bfloat16* gather_src;  // rows gathered from here (row stride K)
   int G_r;             // routed groups
   int G_s;             // shared groups
   int routed_rows;     // offsets are clamped to [0, routed_rows]
@@ -96,9 +112,15 @@ struct Params {
   int b_up_row;  // EPI_SWIGLU: first weight row of the up projection (= d_ff)
   int n_tiles_n;
   int ldc;
+  int hints;  // L2 policies: HINT_B_KEEP weight tiles evict_last, HINT_C_STREAM outputs evict_first,
+              // HINT_A_STREAM A tiles evict_first
   uint64_t timeout_ns;
   unsigned int* status;
 };
+
+constexpr int HINT_B_KEEP = 1;
+constexpr int HINT_C_STREAM = 2;
+constexpr int HINT_A_STREAM = 4;
 
 struct GroupTables {
   int off[MOE_MAX_GROUPS + 1];
@@ -117,9 +139,9 @@ struct SmemTail {
   GroupTables gt;
 };
 
-template <bool PAIR, int ST>
+template <bool PAIR, int ST, bool WIDE = false>
 constexpr size_t smem_bytes() {
-  return 1024 /* alignment slack */ + (size_t)ST * Cfg<PAIR, ST>::STAGE_BYTES + sizeof(SmemTail<ST>);
+  return 1024 /* alignment slack */ + (size_t)ST * Cfg<PAIR, ST, WIDE>::STAGE_BYTES + sizeof(SmemTail<ST>);
 }
 
 struct Group {
@@ -171,9 +193,9 @@ __device__ __forceinline__ TileInfo tile_info(int tile, const int* prefix, int n
 }
 
 // Load the routed offsets and build the row-tile prefix over all groups.
-template <int TILE_M>
+template <int TILE_M, int THREADS>
 __device__ __forceinline__ void build_tables(const Params& p, GroupTables& gt, int tid, int warp, int lane) {
-  for (int i = tid; i <= p.G_r && p.G_r > 0; i += NUM_THREADS) {
+  for (int i = tid; i <= p.G_r && p.G_r > 0; i += THREADS) {
     int v = p.offsets[i];
     gt.off[i] = v < 0 ? 0 : (v > p.routed_rows ? p.routed_rows : v);
   }
@@ -202,11 +224,12 @@ __device__ __forceinline__ void build_tables(const Params& p, GroupTables& gt, i
   __syncthreads();
 }
 
-template <int EPI, bool PAIR, int ST>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int EPI, bool PAIR, int ST, bool WIDE>
+__global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using C = Cfg<PAIR, ST>;
+  using C = Cfg<PAIR, ST, WIDE>;
+  static_assert(!WIDE || EPI != EPI_SWIGLU, "SwiGLU tiles pair gate and up halves within 256 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smemA = smem;
@@ -222,21 +245,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (tid == 0) {
-    // gathering launches: the producer lanes of both CTAs also arrive once per stage
-    const uint32_t full_count = 1u + (p.gather_rows != nullptr ? (uint32_t)C::GATHER_ARRIVALS : 0u);
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&st->full[s], full_count);
+      mbar_init(&st->full[s], 1);
       mbar_init(&st->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&st->tfull[a], 1);
-      mbar_init(&st->tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
+      mbar_init(&st->tempty[a], (PAIR ? 2 : 1) * C::EPI_WARPS);  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(&st->drain, 1);
     st->abort_flag = 0;
     fence_barrier_init();
   }
-  build_tables<C::TILE_M>(p, st->gt, tid, warp, lane);
+  build_tables<C::TILE_M, C::THREADS>(p, st->gt, tid, warp, lane);
   const int G = p.G_r + p.G_s;
   const int total_tiles = st->gt.prefix[G] * p.n_tiles_n;
   if (unit >= total_tiles) return;  // uniform across the CTA (and the pair), before TMEM is taken
@@ -258,11 +279,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = &st->abort_flag;
 
   if (warp == 0) {
-    // ================= producer (whole warp) =================
-    // Tiles arrive by TMA (lane 0).  In gathering launches the routed groups' A rows are instead
-    // copied by the lanes with cp.async, in 16-byte chunks placed in the 128-byte swizzled layout;
-    // every lane commits one copy group per stage and, GATHER_LAG stages later, once that group has
-    // landed, arrives on the stage's full barrier (the pair leader's).
+    // ================= producer =================
+    // Tiles arrive by TMA.  Tiled loads are issued by lane 0.  In gathering launches the routed
+    // groups' A rows are instead gathered from the source rows through the row indices with
+    // tile::gather4 loads, one per lane and stage: lane l brings rows 4l .. 4l+3 of the CTA's
+    // 128-row A tile, so the whole warp runs the loop.
     const bool gathering = p.gather_rows != nullptr;
     if (lane == 0) {
       tma_prefetch_desc(&tmA0);
@@ -274,14 +295,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     long issued = 0;
     bool ok = true;
     const bool active = gathering || lane == 0;  // without gathers, lane 0 alone produces
-    auto lane_arrive = [&](long it) {  // this lane's arrival for stage iteration `it`
-      fence_proxy_async_smem();
-      uint64_t* bar = &st->full[it % C::STAGES];
-      if (PAIR)
-        mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
-      else
-        mbar_arrive(bar);
-    };
+    const uint64_t pol_last = l2_policy_evict_last();
+    const uint64_t pol_first = l2_policy_evict_first();
     for (int tile = unit; active && tile < total_tiles && ok; tile += n_units) {
       const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
       const Group gr = group_info(p, st->gt, ti.g);
@@ -289,47 +304,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
       // weight rows of this CTA's share of the tile's 256 columns; for SwiGLU the first 128
       // columns are gate rows and the other 128 the matching up rows
+      // (a wide tile's second half: b_row + 256)
       const int b_row = EPI == EPI_SWIGLU ? (rank == 0u ? ti.nt * SWIGLU_OUT : p.b_up_row + ti.nt * SWIGLU_OUT)
-                                          : ti.nt * BN + (int)rank * C::B_ROWS;
+                                          : ti.nt * C::TILE_N + (int)rank * C::B_HALF_ROWS;
       const bool gather = gathering && ti.g < p.G_r;
-      // gathered rows: copy instruction q moves rows 4q .. 4q+3 of the CTA's A tile, eight lanes per
-      // row (lane l: row 4q + l/8, 16-byte chunk l%8), so each instruction reads four whole 128-byte
-      // row pieces; this lane's 32 source rows are kept as indices
-      int srow_idx[32];
+      int src[4] = {0, 0, 0, 0};  // this lane's four source rows (rows past the group: row 0, masked later)
       if (gather) {
-        const int r_base = ti.m * C::TILE_M + (int)rank * C::A_ROWS;  // tile row 0 within the group
+        const int r0 = ti.m * C::TILE_M + (int)rank * C::A_ROWS + 4 * lane;  // row within the group
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int r = r_base + 4 * q + (lane >> 3);
-          int v = 0;  // rows past the group: any valid row, masked in the epilogue
-          if (r < gr.rows) {
-            v = __ldg(p.gather_rows + gr.a_base + r);
-            v = v < 0 ? 0 : (v >= p.gather_limit ? p.gather_limit - 1 : v);
+        for (int i = 0; i < 4; ++i) {
+          if (r0 + i < gr.rows) {
+            const int v = __ldg(p.gather_rows + gr.a_base + r0 + i);
+            src[i] = v < 0 ? 0 : (v >= p.gather_limit ? p.gather_limit - 1 : v);
           }
-          srow_idx[q] = v;
         }
       }
       for (int kb = 0; kb < num_kb; ++kb) {
         if (lane == 0) ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
         if (gathering) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        if (lane == 0 && leader) mbar_arrive_expect_tx(&st->full[stage], gather ? C::TX_B_BYTES : C::TX_BYTES);
-        if (gathering) __syncwarp();
+        if (lane == 0 && leader) mbar_arrive_expect_tx(&st->full[stage], C::TX_BYTES);
         uint8_t* a_dst = smemA + stage * C::A_BYTES;
         if (gather) {
-          const uint32_t a_base = smem_u32(a_dst);
-          const int c = lane & 7;
-          const __nv_bfloat16* src = p.gather_src + kb * BK + c * 8;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int row = 4 * q + (lane >> 3);
-            cp_async_16(a_base + row * 128 + ((c ^ (row & 7)) << 4), src + (size_t)srow_idx[q] * p.K);
-          }
+          __syncwarp();
+          uint8_t* dst = a_dst + lane * 4 * (BK * 2);
+          if (PAIR)
+            tma_gather4_pair(dst, &tmA0, &st->full[stage], kb * BK, src[0], src[1], src[2], src[3]);
+          else
+            tma_gather4(dst, &tmA0, &st->full[stage], kb * BK, src[0], src[1], src[2], src[3]);
         }
         if (lane == 0) {
           if (PAIR) {
-            if (!gather) tma_load_2d_pair(a_dst, am, &st->full[stage], kb * BK, a_row);
-            tma_load_3d_pair(smemB + stage * C::B_BYTES, &tmB, &st->full[stage], kb * BK, b_row, ti.g);
+            if (!gather) {
+              if (p.hints & HINT_A_STREAM)
+                tma_load_2d_pair_hint(a_dst, am, &st->full[stage], kb * BK, a_row, pol_first);
+              else
+                tma_load_2d_pair(a_dst, am, &st->full[stage], kb * BK, a_row);
+            }
+#pragma unroll
+            for (int h = 0; h < C::NH; ++h) {
+              uint8_t* b_dst = smemB + stage * C::B_BYTES + h * C::B_HALF_BYTES;
+              if (p.hints & HINT_B_KEEP)
+                tma_load_3d_pair_hint(b_dst, &tmB, &st->full[stage], kb * BK, b_row + h * BN, ti.g, pol_last);
+              else
+                tma_load_3d_pair(b_dst, &tmB, &st->full[stage], kb * BK, b_row + h * BN, ti.g);
+            }
           } else {
             if (!gather) tma_load_2d(a_dst, am, &st->full[stage], kb * BK, a_row);
             if (EPI == EPI_SWIGLU) {  // two 128-row boxes: gate rows, then up rows
@@ -342,13 +361,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        if (gathering) {
-          cp_async_commit();  // one group per stage (empty for TMA-loaded tiles)
-          if (issued >= C::GATHER_LAG) {
-            cp_async_wait<C::GATHER_LAG>();
-            lane_arrive(issued - C::GATHER_LAG);
-          }
-        }
         ++issued;
         if (++stage == C::STAGES) {
           stage = 0;
@@ -356,13 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-    if (gathering) {
-      // the last stages' copies: wait for all of them, then arrive for each
-      cp_async_wait<0>();
-      if (ok)
-        for (long it = issued > C::GATHER_LAG ? issued - C::GATHER_LAG : 0; it < issued; ++it) lane_arrive(it);
-    }
-    if (!ok && !PAIR && lane == 0 && !gathering) {
+    if (!ok && !PAIR && lane == 0) {
       // wind down: let the copies already issued land before the CTA exits
       int zero = 0;
       for (long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
@@ -371,7 +377,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ================= MMA issuer (the pair's leader) =================
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc_bf16(C::TILE_M, BN);
+      constexpr uint32_t idesc = make_idesc_bf16(C::TILE_M, BN);  // one MMA per 256-column half
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -380,25 +386,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
         if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::TILE_N);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&st->full[stage], phase, p.timeout_ns, abort_flag, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // rows copied by cp.async (generic proxy) are read by the tensor core (async proxy)
-          if (p.gather_rows != nullptr) fence_proxy_async_smem();
           const uint32_t a_addr = smem_u32(smemA + stage * C::A_BYTES);
           const uint32_t b_addr = smem_u32(smemB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = make_desc_sw128(a_addr + k * 32);
-            const uint64_t bd = make_desc_sw128(b_addr + k * 32);
-            if (PAIR)
-              mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-            else
-              mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < C::NH; ++h) {
+              const uint64_t bd = make_desc_sw128(b_addr + h * C::B_HALF_BYTES + k * 32);
+              if (PAIR)
+                mma_bf16_ss_pair(d_tmem + h * BN, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+              else
+                mma_bf16_ss(d_tmem + h * BN, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
           }
           if (PAIR)
             mma_commit_pair(&st->empty[stage], 0x3);
@@ -414,8 +421,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mma_commit_pair(&st->tfull[acc], 0x3);
         else
           mma_commit(&st->tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       // no MMA may still be running when TMEM is released
       int zero = 0;
@@ -426,13 +435,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
     }
   } else {
-    // ================= epilogue (warps 2..5) =================
+    // ================= epilogue (warps 2 .. 2 + EPI_WARPS - 1) =================
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;  // the 256-column half of the tile this warp drains
     const int row_in_tile = (int)rank * C::A_ROWS + quarter * 32 + lane;
     const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(&st->tempty[0]), 0) : 0u;
     const uint32_t tempty1 = PAIR ? mapa_shared(smem_u32(&st->tempty[1]), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
+    const bool c_stream = (p.hints & HINT_C_STREAM) != 0;
+    const uint64_t pol_c = l2_policy_evict_first();
+    auto store16 = [&](uint4* dst, const uint32_t* pk) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        if (c_stream)
+          st_global_v4_hint(dst + q, v, pol_c);
+        else
+          dst[q] = v;
+      }
+    };
     for (int tile = unit; tile < total_tiles; tile += n_units) {
       const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
       const Group gr = group_info(p, st->gt, ti.g);
@@ -443,7 +465,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool valid = (r < gr.rows) && (c_row < climit);
       if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t taddr =
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::TILE_N + half * BN);
       __nv_bfloat16* crow = cbase + (size_t)c_row * p.ldc;
       if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
@@ -458,15 +481,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(silu_f32(g[2 * i]) * u[2 * i], silu_f32(g[2 * i + 1]) * u[2 * i + 1]);
-            uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            store16(reinterpret_cast<uint4*>(crow + col0), pk);
           }
         }
       }
 #pragma unroll 1
       for (int ch = 0; ch < (EPI == EPI_SWIGLU ? 0 : BN / 32); ++ch) {
-        const int col0 = ti.nt * BN + ch * 32;
+        const int col0 = ti.nt * C::TILE_N + half * BN + ch * 32;
         if (col0 >= p.N) break;  // same for the whole warp
         float v[32];
         tmem_ld32(taddr + ch * 32, v);
@@ -481,9 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             pk[i] = pack_bf16x2(a, b);
           }
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          store16(reinterpret_cast<uint4*>(crow + col0), pk);
         }
       }
       tc_fence_before();
@@ -494,8 +513,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else
           mbar_arrive(&st->tempty[acc]);
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -514,11 +535,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EPI, bool PAIR, int ST>
+template <int EPI, bool PAIR, int ST, bool WIDE = false>
 int launch_one(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const Params& p, int grid,
                cudaStream_t stream) {
-  auto kfn = grouped_gemm_kernel<EPI, PAIR, ST>;
-  constexpr size_t bytes = smem_bytes<PAIR, ST>();
+  auto kfn = grouped_gemm_kernel<EPI, PAIR, ST, WIDE>;
+  constexpr size_t bytes = smem_bytes<PAIR, ST, WIDE>();
+  constexpr int NUM_THREADS = Cfg<PAIR, ST, WIDE>::THREADS;
   static_assert(bytes <= 232448, "shared memory per CTA");
   int rc = ensure_smem_attr((const void*)kfn, bytes);
   if (rc != MOE_OK) return rc;
@@ -581,15 +603,38 @@ int stages_for(bool pair, int which, double flop) {
   if (env && env[0] && env[1] == ',' && env[2] && env[3] == '\0') {
     const char c = which == 1 ? env[0] : env[2];
     if (c == '4') st = 4;
+    if (c == '5') st = 5;
     if (c == '6') st = 6;
   }
   return st;
 }
 
+// L2 policies of a launch (HINT_* bits).  MOE_GEMM_HINTS=<0..7> overrides.
+int hints_for() {
+  int h = 0;
+  const char* env = getenv("MOE_GEMM_HINTS");
+  if (env && env[0] >= '0' && env[0] <= '7' && env[1] == '\0') h = env[0] - '0';
+  return h;
+}
+
+// Wide 256 x 512 pair tiles (GELU and plain epilogues).  MOE_GEMM_WIDE=0 or =1 forces them off or on.
+bool wide_for(bool pair, int epi) {
+  bool wide = false;
+  const char* env = getenv("MOE_GEMM_WIDE");
+  if (env && env[0] == '1' && env[1] == '\0') wide = true;
+  if (env && env[0] == '0' && env[1] == '\0') wide = false;
+  return wide && pair && epi != EPI_SWIGLU;
+}
+
 template <int EPI>
 int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_upper, cudaStream_t s) {
-  // rows per weight box: a pair CTA loads 128; a single CTA 256, or 2 x 128 (gate, up) for SwiGLU
-  const uint32_t b_box = (pair || EPI == EPI_SWIGLU) ? (uint32_t)Cfg<true, 4>::B_ROWS : (uint32_t)Cfg<false, 4>::B_ROWS;
+  // rows per weight box: a pair CTA loads 128 (per column half); a single CTA 256, or 2 x 128 (gate,
+  // up) for SwiGLU
+  const uint32_t b_box = (pair || EPI == EPI_SWIGLU) ? (uint32_t)Cfg<true, 4>::B_HALF_ROWS
+                                                     : (uint32_t)Cfg<false, 4>::B_HALF_ROWS;
+  const bool wide = wide_for(pair, EPI);
+  Params p = g.p;
+  if (wide) p.n_tiles_n = (p.N + Cfg<true, 4, true>::TILE_N - 1) / Cfg<true, 4, true>::TILE_N;
   CUtensorMap a0, a1, b;
   int rc;
   const uint64_t K = (uint64_t)g.p.K, N = g.b_rows ? g.b_rows : (uint64_t)g.p.N;
@@ -601,13 +646,17 @@ int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_
     a1 = a0;
   }
   if ((rc = encode_tmap_bf16(&b, g.b, 3, K, N, (uint64_t)(g.p.G_r + g.p.G_s), BK, b_box)) != MOE_OK) return rc;
-  long long units = tiles_upper * g.p.n_tiles_n;
+  long long units = tiles_upper * p.n_tiles_n;
   if (pair) {
     long long pairs = units < sms / 2 ? units : sms / 2;
-    if (stages == 6) return launch_one<EPI, true, 6>(a0, a1, b, g.p, (int)(2 * pairs), s);
-    return launch_one<EPI, true, 4>(a0, a1, b, g.p, (int)(2 * pairs), s);
+    if (wide) {
+      if constexpr (EPI != EPI_SWIGLU) return launch_one<EPI, true, 4, true>(a0, a1, b, p, (int)(2 * pairs), s);
+    }
+    if (stages == 6) return launch_one<EPI, true, 6>(a0, a1, b, p, (int)(2 * pairs), s);
+    if (stages == 5) return launch_one<EPI, true, 5>(a0, a1, b, p, (int)(2 * pairs), s);
+    return launch_one<EPI, true, 4>(a0, a1, b, p, (int)(2 * pairs), s);
   }
-  return launch_one<EPI, false, 4>(a0, a1, b, g.p, (int)(units < sms ? units : sms), s);
+  return launch_one<EPI, false, 4>(a0, a1, b, p, (int)(units < sms ? units : sms), s);
 }
 
 }  // namespace gffn
@@ -655,6 +704,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   p.a_sh_map = 0;
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
+  p.hints = hints_for();
 
   GemmSpec g1{};
   g1.a0 = rows;
@@ -740,6 +790,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   p.shared_rows = T;
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
+  p.hints = hints_for();
 
   // GEMM1: routed rows from x_perm, or gathered from x through row_token (map 0), shared rows from x
   // (map 1); H = [routed rows | shared s rows]
@@ -747,7 +798,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   const bool routed_gather = n_routed > 0 && gather;
   g1.a0 = (n_routed > 0 && !gather) ? (const void*)x_perm : (const void*)x;
   g1.a0_rows = (n_routed > 0 && !gather) ? (uint64_t)R : (uint64_t)T;
-  g1.a0_box_rows = 128u;
+  g1.a0_box_rows = routed_gather ? 1u : 128u;  // gather4 loads take a tensor map whose box is one row
   g1.a1 = n_shared > 0 ? (const void*)x : nullptr;
   g1.a1_rows = (uint64_t)T;
   g1.b = w1;
@@ -755,7 +806,6 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.p = p;
   g1.p.gather_rows = routed_gather ? row_token : nullptr;
   g1.p.gather_limit = T;
-  g1.p.gather_src = reinterpret_cast<const __nv_bfloat16*>(x);
   g1.p.a_sh_map = (n_routed > 0 || n_shared == 0) ? 1 : 0;
   g1.p.a_sh_base = 0;
   g1.p.a_sh_stride = 0;

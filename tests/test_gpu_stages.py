@@ -206,15 +206,17 @@ def _ffn_weights(E, d, f, seed):
     return w1, w2
 
 
-@pytest.fixture(params=["pair", "pair4", "single"])
+@pytest.fixture(params=["pair", "pair4", "wide", "single"])
 def gemm_variant(request, monkeypatch):
     """Every grouped-GEMM kernel: CTA pairs with six pipeline stages (short launches), with four
-    (long launches), and single CTAs."""
+    (long launches), pairs on 256 x 512 tiles (GELU and plain epilogues; SwiGLU launches keep
+    256-wide tiles), and single CTAs."""
     monkeypatch.setenv("MOE_GEMM_CTA", "1" if request.param == "single" else "2")
     if request.param == "pair4":
         monkeypatch.setenv("MOE_GEMM_STAGES", "4,4")
     else:
         monkeypatch.delenv("MOE_GEMM_STAGES", raising=False)
+    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if request.param == "wide" else "0")
     return request.param
 
 
