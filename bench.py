@@ -47,14 +47,18 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
-# DRAM bytes (read + write) of one GEMM1 + GEMM2 launch pair, from one single-pass ncu capture of the
-# full-size layer (profiles/grouped_gemm_prefill_dram.md); workloads without a capture of the current
-# kernels report null
 # the decode record of the default run times this many decode steps per prefill step (a decode
 # step is ~2 ms, a prefill step ~30 ms)
 DECODE_STEPS_PER_STEP = 10
 
-TRAFFIC_PER_LAUNCH_PAIR = {"prefill": (20.84e9 + 2.14e9) + (12.84e9 + 7.48e9)}
+# DRAM bytes (read + write) of one GEMM1 + GEMM2 launch pair, from one single-pass ncu capture of the
+# full-size layer (profiles/grouped_gemm_prefill_dram.md: the mean of the two timed launch pairs);
+# workloads without a capture of the current kernels report null
+TRAFFIC_PER_LAUNCH_PAIR = {"prefill": ((20.85e9 + 2.14e9 + 12.57e9 + 7.48e9) + (21.05e9 + 2.14e9 + 12.99e9 + 7.48e9)) / 2}
+# Weight-streaming launches read what their tokens touch, which drifts as the bias moves the loads, so the
+# capture gives DRAM bytes over algorithmic bytes at the captured launches (profiles/launches_decode.md),
+# applied to the timed launches' algorithmic bytes
+TRAFFIC_RATIO = {"decode": 1.0}
 
 
 def peaks():
@@ -107,7 +111,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, smax, reasons = [], [], set()
+        sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as fh:
             for line in fh:
@@ -119,12 +123,17 @@ class ClockSampler:
                     smax.append(float(parts[2]))
                 except ValueError:
                     continue
+                try:
+                    power.append(float(parts[3]))
+                except ValueError:
+                    pass
                 for n, v in zip(names, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(n)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": statistics.median(power) if power else None}
 
 
 # ---------------------------------------------------------------------------
@@ -298,7 +307,12 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
     tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
     gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
     kernel = f"grouped_gemm_kernel x2 (all experts: GEMM1+{'SwiGLU' if w.activation == 'swiglu' else 'GELU'}, GEMM2)"
-    traffic = TRAFFIC_PER_LAUNCH_PAIR.get(w.name) if args.capacity_factor is None and not args.gather_rows else None
+    traffic = None
+    if args.capacity_factor is None and not args.gather_rows:
+        if w.name in TRAFFIC_PER_LAUNCH_PAIR:
+            traffic = TRAFFIC_PER_LAUNCH_PAIR[w.name]
+        elif w.name in TRAFFIC_RATIO:
+            traffic = round(TRAFFIC_RATIO[w.name] * ffn_bytes)
     # the expert launches are timed inside a step of tens of ms, not a seconds-long loop: the burst peak
     tensor_roof = {"kernel": kernel, "bound": "tensor", "achieved": round(tflops, 1),
                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -792,7 +806,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
-                    help="prefill workload: skip the decode-scale record measured after the prefill steps")
+                    help="prefill workload: skip the decode-scale record measured in the same run")
+    ap.add_argument("--decode-first", action="store_true",
+                    help="prefill workload: measure the decode-scale record before the prefill steps")
     ap.add_argument("--gather-rows", action="store_true",
                     help="GEMM1 gathers the routed rows from x (TMA tile::gather4) instead of reading rows copied "
                          "by dispatch")
@@ -852,19 +868,25 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, w, rank, world, local_rank,
-                        want_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
-        if (args.workload == "prefill" and not args.no_decode and args.precision == "bf16" and not args.graph
-                and args.capacity_factor is None and not args.gather_rows):
+        want_decode = (args.workload == "prefill" and not args.no_decode and args.precision == "bf16"
+                       and not args.graph and args.capacity_factor is None and not args.gather_rows)
+
+        def decode_record():
             # the decode-scale layer (T 64, d 7168), weight-streaming bound, measured in the same run
             # on its own clock: each step reads the touched experts' weights from HBM
             dargs = copy.copy(args)
             dargs.steps = args.steps * DECODE_STEPS_PER_STEP
             dargs.log_balance = None
             dec = run_ours(dargs, mi.WORKLOADS["decode"], rank, world, local_rank)
-            line["decode"] = {k: dec[k] for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
-                                                  "ms_per_step", "config", "clocks", "e2e", "gpu_launches",
-                                                  "roofline")}
+            return {k: dec[k] for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                                        "config", "clocks", "e2e", "gpu_launches", "roofline")}
+
+        dec = decode_record() if want_decode and args.decode_first else None
+        line = run_ours(args, w, rank, world, local_rank,
+                        want_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
+        if want_decode:
+            line["decode"] = dec if dec is not None else decode_record()
+            line["decode"]["measured"] = "before the prefill steps" if args.decode_first else "after the prefill steps"
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -66,6 +66,8 @@ typedef uint16_t moe_bf16;
 #define MOE_STATUS_TIMEOUT 0x1u        /* a bounded mbarrier wait gave up          */
 #define MOE_STATUS_BAD_EXPERT 0x2u     /* permute saw an expert id outside [0,n)   */
 #define MOE_STATUS_COUNT_MISMATCH 0x4u /* permute's counts differ from topk_idx    */
+#define MOE_STATUS_RECV_OVERFLOW 0x8u  /* expert-parallel dispatch/combine: a row's place
+                                          in the owner's receive buffer is outside it */
 
 /* expert nonlinearity */
 #define MOE_ACT_GELU_TANH 0 /* gelu(u) = u/2 (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3))) */
@@ -76,6 +78,7 @@ typedef uint16_t moe_bf16;
 #define MOE_MAX_ROUTED 256
 #define MOE_MAX_SHARED 8
 #define MOE_MAX_GROUPS 1024
+#define MOE_EP_MAX_WORLD 64 /* ranks of an expert-parallel group */
 
 /*
  * moe_router_topk -- router scores, biased top-k, joint gates, load counts.
@@ -404,6 +407,68 @@ long long moe_capacity_for(long long factor_num, long long factor_den, int T, in
 
 /* Human-readable text for a MOE_* return code. */
 const char* moe_status_string(int code);
+
+/*
+ * Expert parallelism over peer memory.  "Inkling, Dissected" §02d: the experts
+ * live on different GPUs and every token's rows travel to its experts' GPUs and
+ * back (the all-to-all schedule that bounds an expert's capacity).  Rank q of a
+ * group of W ranks owns the routed experts [q*E/W, (q+1)*E/W) (E = n_routed, W
+ * dividing E) and keeps, in its own device memory, a receive buffer recv_x
+ * [recv_rows, d] and an output buffer recv_y [recv_rows, d] (bf16).  Its rows are
+ * grouped by its experts and, within an expert, by source rank, so the owner runs
+ * one moe_grouped_ffn over all of them (groups recv_offsets, expert_base 0, its
+ * experts' weights).  A step on rank r:
+ *   1. moe_router_topk, moe_permute (x_perm may be NULL) on its T tokens;
+ *   2. the caller all-gathers the per-expert counts: counts_all [W, E] int32;
+ *   3. moe_ep_plan -> send_base [E] (where this rank's rows of expert e start in
+ *      the owner's buffer) and recv_offsets [E/W + 1] (the groups of this rank's
+ *      buffer);
+ *   4. moe_ep_dispatch: every routed (token, slot) row is stored straight into its
+ *      owner's recv_x at send_base[e] + (its place among this rank's rows of e);
+ *   5. the caller orders the ranks (a collective or barrier: every rank's
+ *      dispatch is complete before any owner reads), the owner runs
+ *      moe_grouped_ffn(recv_x, recv_offsets, E/W, recv_rows, 0, ...) -> recv_y,
+ *      then the caller orders the ranks again;
+ *   6. moe_ep_combine gathers each token's outputs from the owners' recv_y and
+ *      adds the shared experts' rows, in the order and arithmetic of moe_combine
+ *      (one rank gives results bit-identical to moe_combine);
+ *   7. the bias update with the counts summed over the ranks and the whole batch's
+ *      token count.
+ * recv_x / recv_y are arrays of W device pointers, in device memory (8-byte
+ * aligned), entry q addressing rank q's buffer: this rank's own, and the peers'
+ * as mapped into this process (moe_ipc_open, or any peer-accessible mapping).
+ * Rows whose place falls outside [0, recv_rows) are skipped and set
+ * MOE_STATUS_RECV_OVERFLOW; an expert id outside [0, E) sets
+ * MOE_STATUS_BAD_EXPERT.  Errors: MOE_ERR_INVALID_ARG (null or misaligned
+ * pointers, W not dividing E, W > MOE_EP_MAX_WORLD, rank outside [0, W)),
+ * MOE_ERR_UNSUPPORTED (d % 8 != 0).  Asynchronous on the stream; allocates nothing.
+ */
+int moe_ep_plan(const int32_t* counts_all, int rank, int world, int n_routed, int32_t* send_base,
+                int32_t* recv_offsets, void* stream);
+int moe_ep_dispatch(const moe_bf16* x, const int32_t* topk_idx, const int32_t* token_row, const int32_t* offsets,
+                    const int32_t* send_base, int T, int d, int n_routed, int top_k, int world,
+                    moe_bf16* const* recv_x, long long recv_rows, void* stream);
+int moe_ep_combine(const moe_bf16* const* recv_y, const int32_t* topk_idx, const int32_t* token_row,
+                   const int32_t* offsets, const int32_t* send_base, const float* gates, const moe_bf16* y_shared,
+                   int T, int d, int n_routed, int top_k, int n_shared, int world, long long recv_rows,
+                   moe_bf16* out, void* stream);
+
+/*
+ * Peer mappings of device buffers between processes (CUDA IPC), for the
+ * expert-parallel buffers above.  moe_ipc_get_handle writes the handle of the
+ * device allocation that holds dev_ptr into moe_ipc_handle_bytes() bytes of host
+ * memory, and dev_ptr's byte offset in that allocation into *offset (both to be
+ * sent to the other ranks: a pointer from a caching allocator is often inside a
+ * larger allocation).  moe_ipc_open maps a peer's handle into this process (peer
+ * access enabled on demand) and returns the mapped allocation's address plus
+ * offset; moe_ipc_close unmaps the allocation that holds a pointer moe_ipc_open
+ * returned.  A handle cannot be opened in the process that made it.  Host calls;
+ * errors: MOE_ERR_INVALID_ARG (null pointers), MOE_ERR_CUDA (the runtime refused).
+ */
+int moe_ipc_handle_bytes(void);
+int moe_ipc_get_handle(const void* dev_ptr, void* handle, unsigned long long* offset);
+int moe_ipc_open(const void* handle, unsigned long long offset, void** dev_ptr);
+int moe_ipc_close(void* dev_ptr);
 
 /*
  * moe_get_status -- synchronise `stream`, then read and clear this device's

@@ -37,6 +37,7 @@ MOE_ERR_SCRATCH = -6
 MOE_STATUS_TIMEOUT = 0x1
 MOE_STATUS_BAD_EXPERT = 0x2
 MOE_STATUS_COUNT_MISMATCH = 0x4
+MOE_STATUS_RECV_OVERFLOW = 0x8
 MOE_ACT_GELU_TANH = 0
 MOE_ACT_SWIGLU = 1
 MOE_NVFP4_EPI_GELU_FP4 = 0
@@ -66,6 +67,14 @@ _lib.moe_nvfp4_rows_capacity.restype = _i64
 _lib.moe_nvfp4_dispatch.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_nvfp4_grouped_gemm.argtypes = [_vp, _vp, _vp, _i32, _i64, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp,
                                         _vp, _i64, _vp]
+_lib.moe_ep_plan.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.moe_ep_dispatch.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp]
+_lib.moe_ep_combine.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp,
+                                _vp]
+_lib.moe_ipc_handle_bytes.argtypes = []
+_lib.moe_ipc_get_handle.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_ulonglong)]
+_lib.moe_ipc_open.argtypes = [_vp, ctypes.c_ulonglong, ctypes.POINTER(_vp)]
+_lib.moe_ipc_close.argtypes = [_vp]
 _lib.moe_status_string.argtypes = [_i32]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_get_status.argtypes = [_vp, ctypes.POINTER(_i32)]
@@ -74,7 +83,8 @@ _lib.moe_debug_bounded_wait.argtypes = [_u64, _vp]
 for _f in ("moe_router_topk", "moe_permute", "moe_permute_capped", "moe_permute_noalloc", "moe_grouped_ffn",
            "moe_experts_ffn", "moe_combine", "moe_bias_update", "moe_load_stats", "moe_get_status",
            "moe_nvfp4_quantize_weights", "moe_nvfp4_dispatch", "moe_nvfp4_grouped_gemm",
-           "moe_set_wait_timeout_ns", "moe_debug_bounded_wait"):
+           "moe_set_wait_timeout_ns", "moe_debug_bounded_wait", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine",
+           "moe_ipc_handle_bytes", "moe_ipc_get_handle", "moe_ipc_open", "moe_ipc_close"):
     getattr(_lib, _f).restype = _i32
 
 
@@ -251,6 +261,51 @@ def moe_nvfp4_grouped_gemm(aq, asf, offsets_pad, n_groups: int, rows_cap: int, w
     _check("moe_nvfp4_grouped_gemm", _lib.moe_nvfp4_grouped_gemm(
         _p(aq), _p(asf), _p(offsets_pad), n_groups, rows_cap, _p(wq), _p(wsf), _p(gscale), N, K, epilogue,
         _p(out_q), _p(out_sf), _p(out), _p(offsets_out), out_rows, _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# expert parallelism over peer memory (moe_ep_*) and the peer mappings (moe_ipc_*)
+# ---------------------------------------------------------------------------
+def moe_ep_plan(counts_all, rank: int, world: int, n_routed: int, send_base, recv_offsets, stream=None):
+    _check("moe_ep_plan", _lib.moe_ep_plan(_p(counts_all), rank, world, n_routed, _p(send_base), _p(recv_offsets),
+                                           _stream(stream)))
+
+
+def moe_ep_dispatch(x, topk_idx, token_row, offsets, send_base, T: int, d: int, n_routed: int, top_k: int,
+                    world: int, recv_x, recv_rows: int, stream=None):
+    """recv_x: a device tensor of ``world`` int64 device addresses (rank q's receive buffer)."""
+    _check("moe_ep_dispatch", _lib.moe_ep_dispatch(
+        _p(x), _p(topk_idx), _p(token_row), _p(offsets), _p(send_base), T, d, n_routed, top_k, world, _p(recv_x),
+        int(recv_rows), _stream(stream)))
+
+
+def moe_ep_combine(recv_y, topk_idx, token_row, offsets, send_base, gates, y_shared, T: int, d: int, n_routed: int,
+                   top_k: int, n_shared: int, world: int, recv_rows: int, out, stream=None):
+    """recv_y: a device tensor of ``world`` int64 device addresses (rank q's output buffer)."""
+    _check("moe_ep_combine", _lib.moe_ep_combine(
+        _p(recv_y), _p(topk_idx), _p(token_row), _p(offsets), _p(send_base), _p(gates), _p(y_shared), T, d, n_routed,
+        top_k, n_shared, world, int(recv_rows), _p(out), _stream(stream)))
+
+
+def moe_ipc_get_handle(t):
+    """(handle bytes, byte offset) of the device allocation holding tensor t's data."""
+    n = int(_lib.moe_ipc_handle_bytes())
+    buf = ctypes.create_string_buffer(n)
+    off = ctypes.c_ulonglong(0)
+    _check("moe_ipc_get_handle", _lib.moe_ipc_get_handle(_p(t), buf, ctypes.byref(off)))
+    return buf.raw, int(off.value)
+
+
+def moe_ipc_open(handle: bytes, offset: int) -> int:
+    """Map a peer process's allocation; returns the device address of its data in this process."""
+    ptr = _vp()
+    buf = ctypes.create_string_buffer(bytes(handle), len(handle))
+    _check("moe_ipc_open", _lib.moe_ipc_open(buf, int(offset), ctypes.byref(ptr)))
+    return int(ptr.value)
+
+
+def moe_ipc_close(ptr: int):
+    _check("moe_ipc_close", _lib.moe_ipc_close(int(ptr)))
 
 
 def capacity_for(factor: float, T: int, k: int, n_routed: int) -> int:

@@ -78,13 +78,15 @@ int ensure_smem_attr(const void* kernel, size_t bytes) {
   int dev;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   static std::mutex mu;
-  static std::unordered_map<const void*, uint64_t> done;  // kernel -> bitmask of devices
+  // (kernel, device) -> the limit set so far; a kernel whose shared memory depends on its
+  // arguments raises it again when a call needs more
+  static std::unordered_map<const void*, std::unordered_map<int, size_t>> done;
   std::lock_guard<std::mutex> lk(mu);
-  uint64_t& mask = done[kernel];
-  if (dev < 64 && (mask >> dev) & 1u) return MOE_OK;
+  size_t& have = done[kernel][dev];
+  if (have >= bytes) return MOE_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (dev < 64) mask |= (1ull << dev);
+  have = bytes;
   return MOE_OK;
 }
 

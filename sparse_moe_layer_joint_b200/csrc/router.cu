@@ -29,6 +29,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "moe.h"
 #include "moe_internal.h"
@@ -209,8 +210,8 @@ __device__ __forceinline__ void route_token(const Params& p, SmemTail* st, const
 // pick each token's experts in descending order.  Lane n then forms token n's
 // joint gates (denominator summed over the contributors in ascending expert
 // index) and writes its outputs.
-template <int K, int NT>
-__device__ __forceinline__ void route_tokens_warp(const Params& p, SmemTail* st, const float* z, int ld, int t0,
+template <int K, int NT, class ST>
+__device__ __forceinline__ void route_tokens_warp(const Params& p, ST* st, const float* z, int ld, int t0,
                                                   int n_valid, int lane) {
   const int E = p.n_routed + p.n_shared;
   float s[NT][8], sel[NT][8];
@@ -540,6 +541,208 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Small batches (T <= SMALL_T_MAX): the tensor-core router's fixed cost (TMEM
+// allocation, the TMA pipeline, a 128-row tile for a few tokens) dominates, and
+// a few CTAs route every token.  Here the logits are CUDA-core dot products
+// spread over many CTAs instead: a cluster of SMALL_CL CTAs takes TB tokens,
+// CTA c computes the logits of experts c*EPS .. (c+1)*EPS-1 for them (fp32
+// FMAs over 16-byte vectors of x staged in shared memory and of W_r from
+// global memory; each lane sums a fixed set of K positions, then a fixed
+// shuffle tree, so the result does not depend on timing) and stores them in
+// the cluster leader's shared memory; after a cluster barrier the leader routes
+// the TB tokens with the warp-level top-k above.
+// ---------------------------------------------------------------------------
+constexpr int SMALL_T_MAX = 256;
+constexpr int SMALL_D_MAX = 2048;  // wider rows: the tensor-core router is faster (measured at d 6144, 7168)
+constexpr int SMALL_CL = 8;        // CTAs per cluster: the experts are split into this many slices
+constexpr int SMALL_THREADS = 256;
+constexpr int SMALL_TB_MAX = 16;
+constexpr int SMALL_U = 4;         // experts a warp works on at once
+constexpr size_t SMALL_X_BUDGET = 160 * 1024;  // bytes of staged x rows per CTA
+
+struct SmallTail {
+  alignas(16) float bias[MOE_MAX_ROUTED];
+  alignas(16) float off[MOE_MAX_ROUTED];
+  int hist[MOE_MAX_ROUTED];
+};
+
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Sum TB per-lane partial sums over the warp, scattering the results: at each of
+// log2(TB) steps a lane keeps half of its values and adds the partner's copies of
+// them (offsets 16, 8, ...), then the last values are summed over the remaining
+// lanes.  Lane l ends with the total of token l >> (5 - log2 TB); 2 TB - 1 + ...
+// shuffles instead of 5 TB.  The order of the additions is fixed.
+template <int TB>
+__device__ __forceinline__ float warp_sum_scatter(const float (&acc)[TB], int lane) {
+  constexpr int LOG = TB == 1 ? 0 : TB == 2 ? 1 : TB == 4 ? 2 : TB == 8 ? 3 : 4;
+  static_assert((1 << LOG) == TB && TB <= 16, "TB: a power of two up to 16");
+  float v[TB];
+#pragma unroll
+  for (int i = 0; i < TB; ++i) v[i] = acc[i];
+#pragma unroll
+  for (int st = 0; st < LOG; ++st) {
+    const int half = TB >> (st + 1);
+    const int off = 16 >> st;
+    const bool hi = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = hi ? v[i] : v[i + half];
+      const float keep = hi ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int off = 16 >> LOG; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+  return r;
+}
+
+// Dynamic shared memory: x rows [TB][d] bf16, logits [TB][RED_LD] fp32 (the
+// leader's are filled by the whole cluster), then the bias / offset / histogram.
+template <int TB>
+size_t small_smem_bytes(int d) {
+  return (size_t)TB * d * 2 + (size_t)TB * RED_LD * 4 + sizeof(SmallTail) + 16;
+}
+
+template <int K, int TB>
+__global__ void __launch_bounds__(SMALL_THREADS, 1)
+    router_small_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
+  const int d = p.d;
+  uint4* xs = reinterpret_cast<uint4*>(smem);                        // [TB][d/8]
+  float* logits = reinterpret_cast<float*>(smem + (size_t)TB * d * 2);  // [TB][RED_LD]
+  SmallTail* st = reinterpret_cast<SmallTail*>(smem + (size_t)TB * d * 2 + (size_t)TB * RED_LD * 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t crank = cluster_ctarank();
+  const int t0 = (int)(blockIdx.x / SMALL_CL) * TB;
+  const int E = p.n_routed + p.n_shared;
+  const int eps = (E + SMALL_CL - 1) / SMALL_CL;
+  const int e_lo = (int)crank * eps;
+  const int e_hi = min(E, e_lo + eps);
+  const int nv = d / 8;  // 16-byte vectors per row
+
+  // stage this block's token rows (rows past T are zero) and the routing inputs
+  for (int i = tid; i < TB * nv; i += SMALL_THREADS) {
+    const int r = i / nv, v = i - r * nv;
+    xs[i] = t0 + r < p.T ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d) + v) : make_uint4(0, 0, 0, 0);
+  }
+  if (crank == 0) {
+    for (int i = tid; i < MOE_MAX_ROUTED; i += SMALL_THREADS) {
+      st->bias[i] = i < p.n_routed ? p.bias[i] : 0.0f;
+      st->off[i] = (p.offset != nullptr && i < p.n_routed) ? p.offset[i] : 0.0f;
+      st->hist[i] = 0;
+    }
+    for (int i = tid; i < TB * RED_LD; i += SMALL_THREADS) logits[i] = 0.0f;
+  }
+  __syncthreads();
+  cluster_sync_all();  // the leader's logit rows are zeroed before any CTA writes into them
+
+  // logits of this CTA's experts: a warp takes SMALL_U experts at a time (their weight loads in flight
+  // together), lane l sums vectors l, l + 32, ... of each
+  const uint32_t lead_logits = mapa_shared(smem_u32(logits), 0);
+  constexpr int SHIFT = 5 - (TB == 1 ? 0 : TB == 2 ? 1 : TB == 4 ? 2 : TB == 8 ? 3 : 4);
+  for (int e0 = e_lo + warp * SMALL_U; e0 < e_hi; e0 += (SMALL_THREADS / 32) * SMALL_U) {
+    float acc[SMALL_U][TB];
+#pragma unroll
+    for (int u = 0; u < SMALL_U; ++u)
+#pragma unroll
+      for (int t = 0; t < TB; ++t) acc[u][t] = 0.0f;
+    for (int v = lane; v < nv; v += 32) {
+      float wf[SMALL_U][8];
+#pragma unroll
+      for (int u = 0; u < SMALL_U; ++u) {
+        const int e = min(e0 + u, e_hi - 1);  // past the slice: a valid row, result not stored
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(w + (size_t)e * d) + v), wf[u]);
+      }
+#pragma unroll
+      for (int t = 0; t < TB; ++t) {
+        float xf[8];
+        bf16x8_to_f32(xs[t * nv + v], xf);
+#pragma unroll
+        for (int u = 0; u < SMALL_U; ++u)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[u][t] = fmaf(xf[j], wf[u][j], acc[u][t]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < SMALL_U; ++u) {
+      const float v = warp_sum_scatter<TB>(acc[u], lane);
+      if (e0 + u < e_hi && (lane & ((1 << SHIFT) - 1)) == 0)
+        st_dsmem_f32(lead_logits + (uint32_t)(((lane >> SHIFT) * RED_LD + e0 + u) * 4), v);
+    }
+  }
+  cluster_sync_all();  // every logit of the block is in the leader's shared memory
+  if (crank != 0) return;
+
+  // route: warp w takes tokens 2w, 2w + 1 (TB <= 16)
+  const int r = 2 * warp;
+  const int n_valid = min(2, min(TB - r, p.T - (t0 + r)));
+  if (n_valid > 0) route_tokens_warp<K, 2>(p, st, logits + (size_t)r * RED_LD, RED_LD, t0 + r, n_valid, lane);
+  __syncthreads();
+  for (int e = tid; e < p.n_routed; e += SMALL_THREADS) {
+    const int c = st->hist[e];
+    if (c) atomicAdd(&p.counts[e], c);
+  }
+}
+
+template <int K, int TB>
+int launch_small(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p, cudaStream_t s) {
+  auto kfn = router_small_kernel<K, TB>;
+  const size_t bytes = small_smem_bytes<TB>(p.d);
+  int rc = ensure_smem_attr((const void*)kfn, bytes);
+  if (rc != MOE_OK) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(((p.T + TB - 1) / TB) * SMALL_CL), 1, 1);
+  cfg.blockDim = dim3(SMALL_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = SMALL_CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kfn, x, w, p) != cudaSuccess) return MOE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Tokens per cluster: about 128 CTAs in flight for the batch, at most 16 tokens, and the
+// staged rows within the shared-memory budget.  0: the small path does not apply.
+int small_tb(int T, int d) {
+  if (T > SMALL_T_MAX || d > SMALL_D_MAX) return 0;
+  int tb = 1;
+  while (tb < SMALL_TB_MAX && (long long)((T + 2 * tb - 1) / (2 * tb)) * SMALL_CL >= 128) tb *= 2;
+  while (tb > 1 && (size_t)tb * d * 2 > SMALL_X_BUDGET) tb /= 2;
+  if ((size_t)tb * d * 2 > SMALL_X_BUDGET) return 0;
+  return tb;
+}
+
+template <int K>
+int launch_small_k(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p, int tb, cudaStream_t s) {
+  switch (tb) {
+    case 1: return launch_small<K, 1>(x, w, p, s);
+    case 2: return launch_small<K, 2>(x, w, p, s);
+    case 4: return launch_small<K, 4>(x, w, p, s);
+    case 8: return launch_small<K, 8>(x, w, p, s);
+    default: return launch_small<K, 16>(x, w, p, s);
+  }
+}
+
 template <int K>
 int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const Params& p, int grid,
            cudaStream_t s) {
@@ -598,6 +801,47 @@ extern "C" int moe_router_topk(const moe_bf16* x, const moe_bf16* w_router, cons
   int dev, sms;
   int rc = device_info(&dev, &sms);
   if (rc != MOE_OK) return rc;
+
+  // small batches: CUDA-core logits over many CTAs (MOE_ROUTER_SMALL=0 or =1 forces the choice)
+  int tb = small_tb(T, d);
+  {
+    const char* env = getenv("MOE_ROUTER_SMALL");
+    if (env && env[0] == '0' && env[1] == '\0') tb = 0;
+    if (env && env[0] == '1' && env[1] == '\0' && tb == 0) {
+      tb = 1;
+      while (tb > 0 && (size_t)tb * d * 2 > SMALL_X_BUDGET) tb = 0;
+    }
+  }
+  if (tb > 0 && n_routed + n_shared <= RED_COLS) {
+    Params p{};
+    p.bias = bias;
+    p.offset = logit_offset;
+    p.T = T;
+    p.d = d;
+    p.n_routed = n_routed;
+    p.n_shared = n_shared;
+    p.ksplit = 1;
+    p.topk_idx = topk_idx;
+    p.gates = gates;
+    p.gate_scale = route_scale;
+    p.counts = counts;
+    p.scores = scores_out;
+    p.timeout_ns = wait_timeout_ns();
+    p.status = status_ptr();
+    if (!p.status) return MOE_ERR_CUDA;
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* wb = reinterpret_cast<const __nv_bfloat16*>(w_router);
+    switch (top_k) {
+      case 1: return launch_small_k<1>(xb, wb, p, tb, s);
+      case 2: return launch_small_k<2>(xb, wb, p, tb, s);
+      case 3: return launch_small_k<3>(xb, wb, p, tb, s);
+      case 4: return launch_small_k<4>(xb, wb, p, tb, s);
+      case 5: return launch_small_k<5>(xb, wb, p, tb, s);
+      case 6: return launch_small_k<6>(xb, wb, p, tb, s);
+      case 7: return launch_small_k<7>(xb, wb, p, tb, s);
+      default: return launch_small_k<8>(xb, wb, p, tb, s);
+    }
+  }
 
   const int E = n_routed + n_shared;
   CUtensorMap tA, tB0, tB1;

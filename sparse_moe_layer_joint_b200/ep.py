@@ -173,3 +173,142 @@ class ExpertParallelLayer:
         from sparse_moe_layer_joint_b200 import dp
 
         dp.bias_step(self.local, bias, gamma, group=self.group)
+
+
+class PeerExpertParallelLayer:
+    """The expert-parallel step with the exchange fused into the library's kernels: rows go
+    straight from the source rank's x into the owner's receive buffer (moe_ep_dispatch, stores
+    through peer pointers), the owner runs one grouped GEMM over all rows it received, and each
+    source gathers its tokens' outputs back from the owners' buffers (moe_ep_combine, peer loads).
+    The only collectives are an all-gather of the per-expert counts (W x n_routed int32), two
+    barriers between the phases, and the bias step's all-reduce of the counts.
+
+    Every rank allocates ``recv_rows`` rows for its receive and output buffers (sized by the
+    caller: the rows its experts can receive in a step; more raise MOE_STATUS_RECV_OVERFLOW).
+    The buffers of the other ranks are mapped with CUDA IPC handles exchanged over the process
+    group; at one rank nothing is mapped.  With NCCL the barriers are stream-ordered collectives
+    (no host wait); with gloo the host synchronises the device and meets the other ranks, which
+    also lets several ranks share one GPU (no kernel of one rank ever waits on another's).
+    Weights: ``w1_local`` / ``w2_local`` hold this rank's routed experts followed by the shared
+    experts, as for ``ExpertParallelLayer``.
+    """
+
+    def __init__(self, shape, rank: int, world: int, recv_rows: int, device="cuda", group=None,
+                 activation: str = "gelu_tanh", route_scale: float = 1.0):
+        import torch
+        import torch.distributed as dist
+
+        from sparse_moe_layer_joint_b200 import MoELayer
+
+        import sparse_moe_layer_joint_b200 as moe
+
+        self.rank, self.world, self.group = rank, world, group
+        self.lo, self.hi = expert_range(shape.n_routed, world, rank)
+        self.local = MoELayer(shape, device=device, activation=activation, route_scale=route_scale)
+        self.dev = torch.device(device)
+        s = shape
+        self.recv_rows = int(recv_rows)
+        bf = torch.bfloat16
+        self.recv_x = torch.empty((max(self.recv_rows, 1), s.d), dtype=bf, device=self.dev)
+        self.recv_y = torch.empty((max(self.recv_rows, 1), s.d), dtype=bf, device=self.dev)
+        self.recv_h = torch.empty((max(self.recv_rows, 1), s.d_ff), dtype=bf, device=self.dev)
+        self.counts_all = torch.empty((world, s.n_routed), dtype=torch.int32, device=self.dev)
+        self.send_base = torch.empty((s.n_routed,), dtype=torch.int32, device=self.dev)
+        self.recv_offsets = torch.empty((self.hi - self.lo + 1,), dtype=torch.int32, device=self.dev)
+        self.nccl = world > 1 and dist.get_backend(group) == "nccl"
+        self.opened = []
+        ptr_x, ptr_y = [0] * world, [0] * world
+        ptr_x[rank], ptr_y[rank] = self.recv_x.data_ptr(), self.recv_y.data_ptr()
+        if world > 1:
+            mine = (moe.moe_ipc_get_handle(self.recv_x), moe.moe_ipc_get_handle(self.recv_y))
+            every = [None] * world
+            dist.all_gather_object(every, mine, group=group)
+            for q in range(world):
+                if q != rank:
+                    ptr_x[q] = moe.moe_ipc_open(*every[q][0])
+                    ptr_y[q] = moe.moe_ipc_open(*every[q][1])
+                    self.opened += [ptr_x[q], ptr_y[q]]
+        self.ptr_x = torch.tensor(ptr_x, dtype=torch.int64, device=self.dev)
+        self.ptr_y = torch.tensor(ptr_y, dtype=torch.int64, device=self.dev)
+        self.ev_routed = torch.cuda.Event()
+        self.ev_shared = torch.cuda.Event()
+        self.token = torch.zeros(1, dtype=torch.int32, device=self.dev)
+
+    def _gather_counts(self):
+        import torch.distributed as dist
+
+        L = self.local
+        if self.world == 1:
+            self.counts_all[0].copy_(L.counts)
+        elif self.nccl:
+            dist.all_gather_into_tensor(self.counts_all.view(-1), L.counts, group=self.group)
+        else:  # gloo: host tensors
+            import torch
+
+            parts = [torch.empty((L.counts.numel(),), dtype=torch.int32) for _ in range(self.world)]
+            dist.all_gather(parts, L.counts.cpu(), group=self.group)
+            self.counts_all.copy_(torch.stack(parts))
+
+    def _barrier(self):
+        """Every rank's work so far is complete before any rank goes on."""
+        import torch
+        import torch.distributed as dist
+
+        if self.world == 1:
+            return
+        if self.nccl:
+            dist.all_reduce(self.token, group=self.group)   # stream-ordered: no host wait
+        else:
+            torch.cuda.synchronize(self.dev)
+            dist.barrier(group=self.group)
+
+    def forward(self, x, w_router, w1_local, w2_local, bias, logit_offset=None):
+        import torch
+
+        import sparse_moe_layer_joint_b200 as moe
+
+        L, s = self.local, self.local.shape
+        T, d, f, k = s.T, s.d, s.d_ff, s.top_k
+        E_loc = self.hi - self.lo
+        main = torch.cuda.current_stream(self.dev)
+        moe.moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, L.route_scale,
+                            L.topk_idx, L.gates, L.counts, None, stream=main)
+        if s.n_shared > 0:
+            self.ev_routed.record(main)
+            L.side.wait_event(self.ev_routed)
+            moe.moe_grouped_ffn(x, None, s.n_shared, T, E_loc, w1_local, w2_local, d, f, L.activation,
+                                L.h_shared, L.y_shared, stream=L.side)
+            self.ev_shared.record(L.side)
+        moe.moe_permute(x, L.topk_idx, L.counts, T, d, s.n_routed, k, L.offsets, None, L.row_token, L.token_row,
+                        L.scratch, L.scratch_bytes, stream=main)
+        self._gather_counts()
+        moe.moe_ep_plan(self.counts_all, self.rank, self.world, s.n_routed, self.send_base, self.recv_offsets,
+                        stream=main)
+        moe.moe_ep_dispatch(x, L.topk_idx, L.token_row, L.offsets, self.send_base, T, d, s.n_routed, k, self.world,
+                            self.ptr_x, self.recv_rows, stream=main)
+        self._barrier()        # every rank's rows are in its owners' buffers
+        if E_loc > 0 and self.recv_rows > 0:
+            moe.moe_grouped_ffn(self.recv_x, self.recv_offsets, E_loc, self.recv_rows, 0, w1_local, w2_local, d, f,
+                                L.activation, self.recv_h, self.recv_y, stream=main)
+        self._barrier()        # every owner's outputs are written
+        if s.n_shared > 0:
+            main.wait_event(self.ev_shared)
+        moe.moe_ep_combine(self.ptr_y, L.topk_idx, L.token_row, L.offsets, self.send_base, L.gates,
+                           L.y_shared if s.n_shared > 0 else None, T, d, s.n_routed, k, s.n_shared, self.world,
+                           self.recv_rows, L.out, stream=main)
+        return L.out
+
+    def bias_update(self, bias, gamma: float):
+        """§02e after the step: the loads summed over all ranks, then the update with the whole
+        batch's token count (as ``ExpertParallelLayer.bias_update``)."""
+        from sparse_moe_layer_joint_b200 import dp
+
+        dp.bias_step(self.local, bias, gamma, group=self.group)
+
+    def close(self):
+        """Unmap the peers' buffers (call on every rank before the process group goes away)."""
+        import sparse_moe_layer_joint_b200 as moe
+
+        for p in self.opened:
+            moe.moe_ipc_close(p)
+        self.opened = []

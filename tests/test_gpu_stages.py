@@ -34,6 +34,17 @@ def _random_topk(T, k, E, seed):
 # ---------------------------------------------------------------------------
 # router
 # ---------------------------------------------------------------------------
+@pytest.fixture(params=["default", "tensor", "small"])
+def router_path(request, monkeypatch):
+    """Both router kernels on the same cases: the path the library picks, the tcgen05 router
+    (forced), and the small-batch CUDA-core router (forced, at any T)."""
+    if request.param == "default":
+        monkeypatch.delenv("MOE_ROUTER_SMALL", raising=False)
+    else:
+        monkeypatch.setenv("MOE_ROUTER_SMALL", "1" if request.param == "small" else "0")
+    return request.param
+
+
 def _run_router(x_u16, wr_u16, bias, k, n_routed, n_shared, offset=None, scores=False):
     T, d = x_u16.shape
     x = dev_bf16(x_u16)
@@ -51,7 +62,7 @@ def _run_router(x_u16, wr_u16, bias, k, n_routed, n_shared, offset=None, scores=
 
 
 @pytest.mark.parametrize("case", ["no_bias", "with_bias"])
-def test_router_worked_example(case):
+def test_router_worked_example(case, router_path):
     """The §02c hand example through the GPU: 4 routed experts, top-2, logits
     z fed as x = e_0 and W_r[:, 0] = z (z rounded to bf16, which keeps the order)."""
     with open(os.path.join(os.path.dirname(__file__), "golden", "worked_example_routing.json")) as fh:
@@ -74,7 +85,7 @@ def test_router_worked_example(case):
     # widths that are not a multiple of 64 (the last K block is read as zeros past d)
     (2048, 32, 64, 0, 6), (300, 96, 256, 2, 6), (129, 8, 16, 2, 4), (1000, 200, 256, 2, 6),
 ])
-def test_router_parity(T, d, n_routed, n_shared, k):
+def test_router_parity(T, d, n_routed, n_shared, k, router_path):
     E = n_routed + n_shared
     x = mi.normal_bf16(T * d, 1, mi.STREAM_X).reshape(T, d)
     wr = mi.normal_bf16(E * d, 1, mi.STREAM_WR, std=1 / np.sqrt(d)).reshape(E, d)
@@ -85,7 +96,7 @@ def test_router_parity(T, d, n_routed, n_shared, k):
     np.testing.assert_allclose(scores, ref["s"], atol=2e-6)
 
 
-def test_router_logit_offset_and_ties():
+def test_router_logit_offset_and_ties(router_path):
     """A logit offset enters the affinity (and so the gates); exact ties keep the lower index."""
     T, d, n_routed, k = 64, 64, 32, 4
     x = np.zeros((T, d), np.float32)
@@ -100,7 +111,7 @@ def test_router_logit_offset_and_ties():
     np.testing.assert_allclose(gates, ref["gates"], atol=1e-6)
 
 
-def test_router_bias_never_touches_gates():
+def test_router_bias_never_touches_gates(router_path):
     """Same token, two biases: where the kept set is the same, the gates are bit-identical."""
     T, d = 512, 256
     x = mi.normal_bf16(T * d, 2, mi.STREAM_X).reshape(T, d)
@@ -115,7 +126,7 @@ def test_router_bias_never_touches_gates():
         assert m0 == m1
 
 
-def test_router_zero_tokens_zeroes_counts():
+def test_router_zero_tokens_zeroes_counts(router_path):
     c = torch.full((256,), 99, dtype=torch.int32, device="cuda")
     x = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
     w = torch.zeros((258, 64), dtype=torch.bfloat16, device="cuda")
@@ -406,7 +417,7 @@ def test_experts_ffn_swiglu_parity(T, n_routed, n_shared, k, d, f, gemm_variant)
 
 
 @pytest.mark.parametrize("scale", [8.0, 2.83])
-def test_router_route_scale(scale):
+def test_router_route_scale(scale, router_path):
     """Joint weights times route_scale x global_scale: sums equal the scale, values the
     oracle's scaled weights, selection unchanged."""
     T, d = 700, 256
