@@ -155,7 +155,8 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
                            stream.cuda_stream)
     layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), device=dev,
                          gather_rows=args.gather_rows, capacity_factor=args.capacity_factor,
-                         activation=w.activation, route_scale=w.gate_scale, precision=args.precision)
+                         activation=w.activation, route_scale=w.gate_scale, precision=args.precision,
+                         fused_experts=not args.shared_stream)
     if args.precision == "nvfp4":
         layer.set_nvfp4_weights(t["w1"], t["w2"])
         torch.cuda.synchronize()
@@ -299,16 +300,20 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
         if want_cpu:
             line["cpu_baseline"] = cpu_baseline_nvfp4(w)
         return line
-    rows = routed_rows + w.T * w.n_shared
+    # the timed launch pair: all experts (routed and shared tiles in the same launches), or with
+    # --shared-stream the routed experts' pair alone (the shared experts' pair runs on the other stream)
+    n_sh = 0 if args.shared_stream else w.n_shared
+    rows = routed_rows + w.T * n_sh
     mats = 3 if w.activation == "swiglu" else 2   # weight matrices per expert
     ffn_flops = 2 * mats * rows * w.d * w.f
-    ffn_bytes = ((touched + w.n_shared) * mats * w.d * w.f * 2
+    ffn_bytes = ((touched + n_sh) * mats * w.d * w.f * 2
                  + rows * w.d * 2 + rows * w.f * 2 * 2 + rows * w.d * 2)
     tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
     gbs = ffn_bytes / (ffn_ms * 1e-3) / 1e9
-    kernel = f"grouped_gemm_kernel x2 (all experts: GEMM1+{'SwiGLU' if w.activation == 'swiglu' else 'GELU'}, GEMM2)"
+    kernel = (f"grouped_gemm_kernel x2 ({'routed experts' if args.shared_stream else 'all experts'}: "
+              f"GEMM1+{'SwiGLU' if w.activation == 'swiglu' else 'GELU'}, GEMM2)")
     traffic = None
-    if args.capacity_factor is None and not args.gather_rows:
+    if args.capacity_factor is None and not args.gather_rows and not args.shared_stream:
         if w.name in TRAFFIC_PER_LAUNCH_PAIR:
             traffic = TRAFFIC_PER_LAUNCH_PAIR[w.name]
         elif w.name in TRAFFIC_RATIO:
@@ -338,6 +343,8 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox, random-init weights)",
         "config": dict(config_of(w, world), dispatch="rows gathered by GEMM1 (TMA gather4)" if args.gather_rows
                        else "rows copied by moe_permute",
+                       shared_experts="own launches on a second stream" if args.shared_stream
+                       else "tiles of the routed experts' launches",
                        **({"cuda_graph": True, "ms_per_step_without_graph": round(eager_ms, 4)}
                           if eager_ms is not None else {}),
                        **({"capacity_factor": args.capacity_factor, "capacity": layer.capacity,
@@ -807,6 +814,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="prefill workload: skip the decode-scale record measured in the same run")
+    ap.add_argument("--shared-stream", action="store_true",
+                    help="shared experts as their own GEMM launches on a second stream (beside the router and "
+                         "dispatch) instead of tiles of the routed experts' launches")
     ap.add_argument("--decode-first", action="store_true",
                     help="prefill workload: measure the decode-scale record before the prefill steps")
     ap.add_argument("--gather-rows", action="store_true",

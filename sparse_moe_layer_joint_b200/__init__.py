@@ -472,12 +472,15 @@ class MoELayer:
         s = self.shape
         main = stream if stream is not None else torch.cuda.current_stream()
         T, d, f, k = s.T, s.d, s.d_ff, s.top_k
-        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, self.route_scale,
-                        self.topk_idx, self.gates, self.counts, scores_out, stream=main)
         side = s.n_shared > 0 and not self.fused_experts and not self.nvfp4
         if side:
+            # the shared experts need only x: their stream starts with the router, and the
+            # dispatch kernels (small, memory-bound) run beside their GEMM tiles
             self.ev_start.record(main)
             self.side.wait_event(self.ev_start)
+        moe_router_topk(x, w_router, bias, logit_offset, T, d, s.n_routed, s.n_shared, k, self.route_scale,
+                        self.topk_idx, self.gates, self.counts, scores_out, stream=main)
+        if side:
             moe_grouped_ffn(x, None, s.n_shared, T, s.n_routed, w1, w2, d, f, self.activation, self.h_shared,
                             self.y_shared, stream=self.side)
             self.ev_shared.record(self.side)
