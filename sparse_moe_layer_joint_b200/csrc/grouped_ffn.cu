@@ -112,6 +112,7 @@ struct Params {
   int b_up_row;  // EPI_SWIGLU: first weight row of the up projection (= d_ff)
   int n_tiles_n;
   int ldc;
+  int n_major_rows;  // groups of at most this many row tiles run column-tile-major (0: none)
   int hints;  // L2 policies: HINT_B_KEEP weight tiles evict_last, HINT_C_STREAM outputs evict_first,
               // HINT_A_STREAM A tiles evict_first
   uint64_t timeout_ns;
@@ -175,10 +176,14 @@ struct TileInfo {
   int g, m, nt;
 };
 
-__device__ __forceinline__ TileInfo tile_info(int tile, const int* prefix, int n_groups, int n_tiles_n) {
+// A group's tiles are the tile numbers [prefix[g] * n_tiles_n, prefix[g + 1] * n_tiles_n).  Within a
+// group they run row-tile-major (the column tiles of one row block together) or, for groups of at most
+// n_major_rows row tiles, column-tile-major (every row block of one weight tile together: each weight
+// tile is read from DRAM once while the group's few A blocks stay in L2).
+__device__ __forceinline__ TileInfo tile_info(int tile, const int* prefix, int n_groups, int n_tiles_n,
+                                              int n_major_rows) {
   TileInfo ti;
-  int mt = tile / n_tiles_n;
-  ti.nt = tile - mt * n_tiles_n;
+  const int mt = tile / n_tiles_n;
   int lo = 0, hi = n_groups;  // largest g with prefix[g] <= mt (never an empty group)
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
@@ -188,7 +193,15 @@ __device__ __forceinline__ TileInfo tile_info(int tile, const int* prefix, int n
       hi = mid;
   }
   ti.g = lo;
-  ti.m = mt - prefix[lo];
+  const int rows_g = prefix[lo + 1] - prefix[lo];  // row tiles of the group
+  if (rows_g <= n_major_rows) {
+    const int l = tile - prefix[lo] * n_tiles_n;
+    ti.nt = l / rows_g;
+    ti.m = l - ti.nt * rows_g;
+  } else {
+    ti.nt = tile - mt * n_tiles_n;
+    ti.m = mt - prefix[lo];
+  }
   return ti;
 }
 
@@ -298,7 +311,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
     const uint64_t pol_last = l2_policy_evict_last();
     const uint64_t pol_first = l2_policy_evict_first();
     for (int tile = unit; active && tile < total_tiles && ok; tile += n_units) {
-      const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
+      const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n, p.n_major_rows);
       const Group gr = group_info(p, st->gt, ti.g);
       const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
       const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
@@ -456,7 +469,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
       }
     };
     for (int tile = unit; tile < total_tiles; tile += n_units) {
-      const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n);
+      const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n, p.n_major_rows);
       const Group gr = group_info(p, st->gt, ti.g);
       const int r = ti.m * C::TILE_M + row_in_tile;
       const int c_row = gr.c_base + r;
@@ -609,6 +622,15 @@ int stages_for(bool pair, int which, double flop) {
   return st;
 }
 
+// Groups of at most this many row tiles run column-tile-major; MOE_GEMM_NMAJOR=<rows> overrides (0: all
+// row-tile-major).
+int n_major_rows_for() {
+  int r = 0;
+  const char* env = getenv("MOE_GEMM_NMAJOR");
+  if (env && env[0]) r = atoi(env);
+  return r < 0 ? 0 : r;
+}
+
 // L2 policies of a launch (HINT_* bits).  MOE_GEMM_HINTS=<0..7> overrides.
 int hints_for() {
   int h = 0;
@@ -705,6 +727,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
   p.hints = hints_for();
+  p.n_major_rows = n_major_rows_for();
 
   GemmSpec g1{};
   g1.a0 = rows;
@@ -791,6 +814,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
   p.hints = hints_for();
+  p.n_major_rows = n_major_rows_for();
 
   // GEMM1: routed rows from x_perm, or gathered from x through row_token (map 0), shared rows from x
   // (map 1); H = [routed rows | shared s rows]

@@ -699,6 +699,84 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1)
   }
 }
 
+// Narrow rows (d <= SINGLE_D_MAX): no cluster at all.  Each CTA takes TB <= 4 tokens and computes
+// the logits of every expert itself (W_r is at most 258 x 512 bf16 = 264 KB, read from L2 by every
+// CTA), keeps them in its own shared memory and routes its tokens: no cluster barrier, no DSMEM.
+constexpr int SINGLE_D_MAX = 512;
+
+template <int K, int TB>
+__global__ void __launch_bounds__(SMALL_THREADS, 1)
+    router_single_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
+  const int d = p.d;
+  uint4* xs = reinterpret_cast<uint4*>(smem);                           // [TB][d/8]
+  float* logits = reinterpret_cast<float*>(smem + (size_t)TB * d * 2);  // [TB][RED_LD]
+  SmallTail* st = reinterpret_cast<SmallTail*>(smem + (size_t)TB * d * 2 + (size_t)TB * RED_LD * 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t0 = (int)blockIdx.x * TB;
+  const int E = p.n_routed + p.n_shared;
+  const int nv = d / 8;
+  for (int i = tid; i < TB * nv; i += SMALL_THREADS) {
+    const int r = i / nv, v = i - r * nv;
+    xs[i] = t0 + r < p.T ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d) + v) : make_uint4(0, 0, 0, 0);
+  }
+  for (int i = tid; i < MOE_MAX_ROUTED; i += SMALL_THREADS) {
+    st->bias[i] = i < p.n_routed ? p.bias[i] : 0.0f;
+    st->off[i] = (p.offset != nullptr && i < p.n_routed) ? p.offset[i] : 0.0f;
+    st->hist[i] = 0;
+  }
+  for (int i = tid; i < TB * RED_LD; i += SMALL_THREADS) logits[i] = 0.0f;
+  __syncthreads();
+  constexpr int SHIFT = 5 - (TB == 1 ? 0 : TB == 2 ? 1 : 2);
+  for (int e0 = warp * SMALL_U; e0 < E; e0 += (SMALL_THREADS / 32) * SMALL_U) {
+    float acc[SMALL_U][TB];
+#pragma unroll
+    for (int u = 0; u < SMALL_U; ++u)
+#pragma unroll
+      for (int t = 0; t < TB; ++t) acc[u][t] = 0.0f;
+    for (int v = lane; v < nv; v += 32) {
+      float wf[SMALL_U][8];
+#pragma unroll
+      for (int u = 0; u < SMALL_U; ++u) {
+        const int e = min(e0 + u, E - 1);
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(w + (size_t)e * d) + v), wf[u]);
+      }
+#pragma unroll
+      for (int t = 0; t < TB; ++t) {
+        float xf[8];
+        bf16x8_to_f32(xs[t * nv + v], xf);
+#pragma unroll
+        for (int u = 0; u < SMALL_U; ++u)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[u][t] = fmaf(xf[j], wf[u][j], acc[u][t]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < SMALL_U; ++u) {
+      const float v = warp_sum_scatter<TB>(acc[u], lane);
+      if (e0 + u < E && (lane & ((1 << SHIFT) - 1)) == 0) logits[(lane >> SHIFT) * RED_LD + e0 + u] = v;
+    }
+  }
+  __syncthreads();
+  if (warp < TB && t0 + warp < p.T) route_tokens_warp<K, 1>(p, st, logits + (size_t)warp * RED_LD, RED_LD, t0 + warp, 1, lane);
+  __syncthreads();
+  for (int e = tid; e < p.n_routed; e += SMALL_THREADS) {
+    const int c = st->hist[e];
+    if (c) atomicAdd(&p.counts[e], c);
+  }
+}
+
+template <int K, int TB>
+int launch_single(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p, cudaStream_t s) {
+  auto kfn = router_single_kernel<K, TB>;
+  const size_t bytes = small_smem_bytes<TB>(p.d);
+  int rc = ensure_smem_attr((const void*)kfn, bytes);
+  if (rc != MOE_OK) return rc;
+  kfn<<<(p.T + TB - 1) / TB, SMALL_THREADS, bytes, s>>>(x, w, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 template <int K, int TB>
 int launch_small(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p, cudaStream_t s) {
   auto kfn = router_small_kernel<K, TB>;
@@ -721,6 +799,12 @@ int launch_small(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// MOE_ROUTER_SINGLE=0 keeps narrow rows on the cluster kernel (to test both small-batch kernels).
+bool single_allowed() {
+  const char* env = getenv("MOE_ROUTER_SINGLE");
+  return !(env && env[0] == '0' && env[1] == '\0');
+}
+
 // Tokens per cluster: about 128 CTAs in flight for the batch, at most 16 tokens, and the
 // staged rows within the shared-memory budget.  0: the small path does not apply.
 int small_tb(int T, int d) {
@@ -734,6 +818,12 @@ int small_tb(int T, int d) {
 
 template <int K>
 int launch_small_k(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p, int tb, cudaStream_t s) {
+  if (p.d <= SINGLE_D_MAX && single_allowed()) {  // tokens per CTA: about 128 CTAs, at most 4
+    const int tpc = p.T >= 512 ? 4 : (p.T >= 256 ? 2 : 1);
+    if (tpc == 4) return launch_single<K, 4>(x, w, p, s);
+    if (tpc == 2) return launch_single<K, 2>(x, w, p, s);
+    return launch_single<K, 1>(x, w, p, s);
+  }
   switch (tb) {
     case 1: return launch_small<K, 1>(x, w, p, s);
     case 2: return launch_small<K, 2>(x, w, p, s);

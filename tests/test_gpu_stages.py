@@ -34,14 +34,18 @@ def _random_topk(T, k, E, seed):
 # ---------------------------------------------------------------------------
 # router
 # ---------------------------------------------------------------------------
-@pytest.fixture(params=["default", "tensor", "small"])
+@pytest.fixture(params=["default", "tensor", "small", "cluster"])
 def router_path(request, monkeypatch):
-    """Both router kernels on the same cases: the path the library picks, the tcgen05 router
-    (forced), and the small-batch CUDA-core router (forced, at any T)."""
+    """Every router kernel on the same cases: the path the library picks, the tcgen05 router
+    (forced), and the small-batch CUDA-core routers forced at any T: the one-CTA kernel (narrow
+    rows) and the cluster kernel."""
+    monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
     if request.param == "default":
         monkeypatch.delenv("MOE_ROUTER_SMALL", raising=False)
     else:
-        monkeypatch.setenv("MOE_ROUTER_SMALL", "1" if request.param == "small" else "0")
+        monkeypatch.setenv("MOE_ROUTER_SMALL", "0" if request.param == "tensor" else "1")
+    if request.param == "cluster":
+        monkeypatch.setenv("MOE_ROUTER_SINGLE", "0")
     return request.param
 
 
@@ -217,11 +221,12 @@ def _ffn_weights(E, d, f, seed):
     return w1, w2
 
 
-@pytest.fixture(params=["pair", "pair4", "wide", "single"])
+@pytest.fixture(params=["pair", "pair4", "wide", "nmajor", "single"])
 def gemm_variant(request, monkeypatch):
     """Every grouped-GEMM kernel: CTA pairs with six pipeline stages (short launches), with four
     (long launches), pairs on 256 x 512 tiles (GELU and plain epilogues; SwiGLU launches keep
-    256-wide tiles), and single CTAs."""
+    256-wide tiles), pairs walking small groups column-tile-major, and single CTAs."""
+    monkeypatch.setenv("MOE_GEMM_NMAJOR", "4" if request.param == "nmajor" else "0")
     monkeypatch.setenv("MOE_GEMM_CTA", "1" if request.param == "single" else "2")
     if request.param == "pair4":
         monkeypatch.setenv("MOE_GEMM_STAGES", "4,4")
