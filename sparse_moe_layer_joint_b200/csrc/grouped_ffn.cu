@@ -113,11 +113,18 @@ struct Params {
   int n_tiles_n;
   int ldc;
   int n_major_rows;  // groups of at most this many row tiles run column-tile-major (0: none)
+  int tail_mode;     // TAIL_ALL: every row of every group; TAIL_WHOLE: only each group's whole blocks of
+                     // tail_unit rows; TAIL_ONLY: only the rows past them (two launches cover a group)
+  int tail_unit;
   int hints;  // L2 policies: HINT_B_KEEP weight tiles evict_last, HINT_C_STREAM outputs evict_first,
               // HINT_A_STREAM A tiles evict_first
   uint64_t timeout_ns;
   unsigned int* status;
 };
+
+constexpr int TAIL_ALL = 0;
+constexpr int TAIL_WHOLE = 1;
+constexpr int TAIL_ONLY = 2;
 
 constexpr int HINT_B_KEEP = 1;
 constexpr int HINT_C_STREAM = 2;
@@ -169,7 +176,23 @@ __device__ __forceinline__ Group group_info(const Params& p, const GroupTables& 
     G.c_sel = 1;
     G.c_base = p.c1_base + s * p.c1_stride;
   }
+  if (p.tail_mode == TAIL_ONLY) {  // the rows past the group's last whole tail_unit-row block
+    const int start = (G.rows / p.tail_unit) * p.tail_unit;
+    G.rows -= start;
+    G.a_base += start;
+    G.c_base += start;
+  }
   return G;
+}
+
+// Row tiles a group contributes to a launch (see Params::tail_mode).
+template <int TILE_M>
+__device__ __forceinline__ int group_row_tiles(const Params& p, int rows) {
+  if (rows <= 0) return 0;
+  if (p.tail_mode == TAIL_ALL) return (rows + TILE_M - 1) / TILE_M;
+  if (p.tail_mode == TAIL_WHOLE) return (rows / p.tail_unit) * (p.tail_unit / TILE_M);
+  rows -= (rows / p.tail_unit) * p.tail_unit;  // TAIL_ONLY
+  return (rows + TILE_M - 1) / TILE_M;
 }
 
 struct TileInfo {
@@ -221,7 +244,7 @@ __device__ __forceinline__ void build_tables(const Params& p, GroupTables& gt, i
       int cnt = 0;
       if (g < G) {
         int rows = g < p.G_r ? gt.off[g + 1] - gt.off[g] : p.shared_rows;
-        cnt = rows > 0 ? (rows + TILE_M - 1) / TILE_M : 0;
+        cnt = group_row_tiles<TILE_M>(p, rows);
       }
       int v = cnt;
 #pragma unroll
@@ -681,6 +704,32 @@ int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_
   return launch_one<EPI, false, 4>(a0, a1, b, p, (int)(units < sms ? units : sms), s);
 }
 
+// Pair launches with each group's last rows split off: the CTA pairs take every group's whole
+// 256-row blocks and single CTAs (128-row tiles) the rows past them, so a group's last block is
+// padded to 128 rows instead of 256.  MOE_GEMM_TAILS=1 or =0 forces it on or off.
+bool tails_for(bool pair) {
+  bool on = false;
+  const char* env = getenv("MOE_GEMM_TAILS");
+  if (env && env[0] == '1' && env[1] == '\0') on = true;
+  if (env && env[0] == '0' && env[1] == '\0') on = false;
+  return on && pair;
+}
+
+template <int EPI>
+int run_split(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_upper, cudaStream_t s) {
+  if (!tails_for(pair)) return run_gemm<EPI>(g, pair, stages, sms, tiles_upper, s);
+  GemmSpec whole = g;
+  whole.p.tail_mode = TAIL_WHOLE;
+  whole.p.tail_unit = Cfg<true, 4>::TILE_M;
+  int rc = run_gemm<EPI>(whole, true, stages, sms, tiles_upper, s);
+  if (rc != MOE_OK) return rc;
+  GemmSpec tail = g;
+  tail.p.tail_mode = TAIL_ONLY;
+  tail.p.tail_unit = Cfg<true, 4>::TILE_M;
+  const long long groups = (long long)g.p.G_r + g.p.G_s;
+  return run_gemm<EPI>(tail, false, 4, sms, groups * (Cfg<true, 4>::TILE_M / Cfg<false, 4>::TILE_M), s);
+}
+
 }  // namespace gffn
 }  // namespace moe
 
@@ -747,8 +796,8 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
   const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
-  rc = swiglu ? run_gemm<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
-              : run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
+  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
+              : run_split<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
   if (rc != MOE_OK) return rc;
 
   GemmSpec g2{};
@@ -766,7 +815,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g2.p.K = d_ff;
   g2.p.n_tiles_n = (d + BN - 1) / BN;
   g2.p.ldc = d;
-  return run_gemm<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
+  return run_split<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
 }
 
 extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* row_token,
@@ -844,8 +893,8 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
   const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
-  rc = swiglu ? run_gemm<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
-              : run_gemm<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
+  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
+              : run_split<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
   if (rc != MOE_OK) return rc;
 
   // GEMM2: all A rows from H (map 0); routed outputs to y_perm, shared outputs to y_shared
@@ -867,5 +916,5 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g2.p.K = d_ff;
   g2.p.n_tiles_n = (d + BN - 1) / BN;
   g2.p.ldc = d;
-  return run_gemm<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
+  return run_split<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
 }
