@@ -20,9 +20,11 @@
  * token dropping and per-batch balance statistics (§02d, §02g:
  * moe_permute_capped, moe_load_stats); the released configuration's SwiGLU
  * experts and routing-weight scale ("Under the hood", "MoE: the expert
- * configuration", "The routing strategy": MOE_ACT_SWIGLU, route_scale); and
+ * configuration", "The routing strategy": MOE_ACT_SWIGLU, route_scale);
  * NVFP4 W4A4 routed experts on the block-scaled tensor cores ("Under the hood",
- * "Quantization: BF16 vs NVFP4": moe_nvfp4_*).
+ * "Quantization: BF16 vs NVFP4": moe_nvfp4_*); and expert parallelism with the
+ * exchange done by the dispatch and combine kernels through peer pointers
+ * (§02d's all-to-all schedule: moe_ep_*, with CUDA IPC mappings moe_ipc_*).
  *
  * Conventions for every call
  * --------------------------
@@ -40,6 +42,9 @@
  *    that moe_get_status() reads and clears.
  *  - T = 0 (no tokens) is valid: the call does nothing except what it states
  *    (moe_router_topk still zeroes counts).
+ *  - Host-only calls (no stream, nothing launched): moe_permute_scratch_bytes,
+ *    moe_nvfp4_rows_capacity, moe_capacity_for, moe_status_string,
+ *    moe_set_wait_timeout_ns and the moe_ipc_* mappings.
  */
 #ifndef MOE_H
 #define MOE_H
