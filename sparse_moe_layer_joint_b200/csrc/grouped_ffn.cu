@@ -112,6 +112,7 @@ struct Params {
   int b_up_row;  // EPI_SWIGLU: first weight row of the up projection (= d_ff)
   int n_tiles_n;
   int ldc;
+  int prefetch_kb;   // > 0: also prefetch the tiles this many K blocks ahead into L2 (TMA prefetch)
   int n_major_rows;  // groups of at most this many row tiles run column-tile-major (0: none)
   int tail_mode;     // TAIL_ALL: every row of every group; TAIL_WHOLE: only each group's whole blocks of
                      // tail_unit rows; TAIL_ONLY: only the rows past them (two launches cover a group)
@@ -368,6 +369,16 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
             tma_gather4_pair(dst, &tmA0, &st->full[stage], kb * BK, src[0], src[1], src[2], src[3]);
           else
             tma_gather4(dst, &tmA0, &st->full[stage], kb * BK, src[0], src[1], src[2], src[3]);
+        }
+        if (lane == 0 && p.prefetch_kb > 0 && kb + p.prefetch_kb < num_kb) {
+          // the K block prefetch_kb ahead goes to L2 now, so its DRAM latency overlaps this stage
+          const int kp = (kb + p.prefetch_kb) * BK;
+          if (!gather) tma_prefetch_l2_2d(am, kp, a_row);
+#pragma unroll
+          for (int h = 0; h < C::NH; ++h) {
+            if (EPI == EPI_SWIGLU && !PAIR && h == 0) tma_prefetch_l2_3d(&tmB, kp, p.b_up_row + ti.nt * SWIGLU_OUT, ti.g);
+            tma_prefetch_l2_3d(&tmB, kp, b_row + h * BN, ti.g);
+          }
         }
         if (lane == 0) {
           if (PAIR) {
@@ -654,6 +665,14 @@ int n_major_rows_for() {
   return r < 0 ? 0 : r;
 }
 
+// L2 prefetch distance in K blocks (0: off).  MOE_GEMM_PREFETCH=<blocks> overrides.
+int prefetch_for() {
+  int r = 0;
+  const char* env = getenv("MOE_GEMM_PREFETCH");
+  if (env && env[0]) r = atoi(env);
+  return r < 0 ? 0 : (r > 64 ? 64 : r);
+}
+
 // L2 policies of a launch (HINT_* bits).  MOE_GEMM_HINTS=<0..7> overrides.
 int hints_for() {
   int h = 0;
@@ -777,6 +796,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   p.status = status;
   p.hints = hints_for();
   p.n_major_rows = n_major_rows_for();
+  p.prefetch_kb = prefetch_for();
 
   GemmSpec g1{};
   g1.a0 = rows;
@@ -864,6 +884,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   p.status = status;
   p.hints = hints_for();
   p.n_major_rows = n_major_rows_for();
+  p.prefetch_kb = prefetch_for();
 
   // GEMM1: routed rows from x_perm, or gathered from x through row_token (map 0), shared rows from x
   // (map 1); H = [routed rows | shared s rows]
