@@ -887,6 +887,7 @@ def main():
             dargs = copy.copy(args)
             dargs.steps = args.steps * DECODE_STEPS_PER_STEP
             dargs.log_balance = None
+            dargs.graph = world == 1  # a 2 ms step of 9 launches: replayed as one CUDA graph
             dec = run_ours(dargs, mi.WORKLOADS["decode"], rank, world, local_rank)
             return {k: dec[k] for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                                         "config", "clocks", "e2e", "gpu_launches", "roofline")}
