@@ -706,6 +706,8 @@ def run_kernel_case(args):
     import sparse_moe_layer_joint_b200 as moe
 
     G, per, d, f = 32, 1536, 7168, 2048
+    if args.kernel_case == "nvfp4_decode":
+        G, per = 64, 2  # decode-shaped: a couple of rows per expert, the weights streamed once
     n = G * per
     dev = torch.device("cuda", 0)
     s = torch.cuda.current_stream(dev).cuda_stream
@@ -732,7 +734,7 @@ def run_kernel_case(args):
     elif args.kernel_case == "grouped_ffn":
         def call():
             moe.moe_grouped_ffn(rows, offsets, G, n, 0, w1, w2, d, f, moe.MOE_ACT_GELU_TANH, h, y)
-    elif args.kernel_case == "nvfp4_ffn":
+    elif args.kernel_case in ("nvfp4_ffn", "nvfp4_decode"):
         # the same slice with NVFP4 operands: rows quantized once by the FP4 dispatch (one expert
         # per row, groups of 1536 = 12 x 128 rows, so no padding), then GEMM1 + GELU + FP4 and GEMM2
         u8 = torch.uint8
@@ -755,9 +757,11 @@ def run_kernel_case(args):
         offp = torch.empty(G + 1, dtype=torch.int32, device=dev)
         moe.moe_nvfp4_dispatch(rows, topk, trow, offsets, n, d, G, 1, xq, xsf, trp, offp)
 
+        real = offsets if args.kernel_case == "nvfp4_decode" else None  # load only the real A rows
+
         def call():
             moe.moe_nvfp4_grouped_gemm(xq, xsf, offp, G, rows_cap, w1q, w1sf, g1, f, d, moe.MOE_NVFP4_EPI_GELU_FP4,
-                                       hq, hsf, None, None, 0)
+                                       hq, hsf, None, real, n if real is not None else 0)
             moe.moe_nvfp4_grouped_gemm(hq, hsf, offp, G, rows_cap, w2q, w2sf, g2, d, f, moe.MOE_NVFP4_EPI_BF16,
                                        None, None, y, offsets, n)
     else:
@@ -790,8 +794,10 @@ def run_kernel_case(args):
                           "clocks": clk, "status": moe.moe_get_status()}), flush=True)
         return
     flops = 2 * 2.0 * n * d * f
+    wbytes = G * 2 * d * f * (0.5 + 1 / 16 if args.kernel_case.startswith("nvfp4") else 2)
     print(json.dumps({"kernel_case": args.kernel_case, "experts": G, "rows_per_expert": per, "d": d, "d_ff": f,
                       "ms_per_call": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                      "weight_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1),
                       "clocks": clk, "status": moe.moe_get_status()}), flush=True)
 
 
@@ -822,7 +828,8 @@ def main():
     ap.add_argument("--gather-rows", action="store_true",
                     help="GEMM1 gathers the routed rows from x (TMA tile::gather4) instead of reading rows copied "
                          "by dispatch")
-    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "nvfp4_ffn", "router"],
+    ap.add_argument("--kernel-case", choices=["grouped_ffn", "grouped_ffn_cublas", "nvfp4_ffn", "nvfp4_decode",
+                                              "router"],
                     default=None,
                     help="time one kernel alone on a small profiling case instead of the layer")
     args = ap.parse_args()
