@@ -219,3 +219,39 @@ def test_binding_arity_matches_the_header():
         fn = getattr(L, name)
         assert fn.argtypes is not None, name
         assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def test_expert_parallel_entry_points_reject():
+    E, U = moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_UNSUPPORTED
+    plan = L.moe_ep_plan
+    assert plan(A16, 0, 3, 256, A16, A16, NULL) == E          # 3 ranks do not split 256 experts
+    assert plan(A16, 0, 0, 256, A16, A16, NULL) == E          # no ranks
+    assert plan(A16, 2, 2, 256, A16, A16, NULL) == E          # rank outside [0, world)
+    assert plan(A16, 0, 128, 256, A16, A16, NULL) == E        # more ranks than MOE_EP_MAX_WORLD
+    assert plan(NULL, 0, 2, 256, A16, A16, NULL) == E
+    assert plan(A16, 0, 2, 256, 0x10002, A16, NULL) == E      # misaligned
+    disp = L.moe_ep_dispatch
+    assert disp(A16, A16, A16, A16, A16, 8, 64, 256, 9, 2, A16, 100, NULL) == E      # top_k > 8
+    assert disp(A16, A16, A16, A16, A16, 8, 60, 256, 6, 2, A16, 100, NULL) == U      # d % 8 != 0
+    assert disp(A16, A16, A16, A16, A16, 8, 64, 256, 6, 2, 0x10004, 100, NULL) == E  # pointer array misaligned
+    assert disp(A16, A16, A16, A16, NULL, 8, 64, 256, 6, 2, A16, 100, NULL) == E
+    assert disp(A16, A16, A16, A16, A16, 8, 64, 256, 6, 2, A16, -1, NULL) == E
+    assert disp(A16, A16, A16, A16, A16, 0, 64, 256, 6, 2, A16, 100, NULL) == moe.MOE_OK  # T = 0: nothing to do
+    comb = L.moe_ep_combine
+    assert comb(A16, A16, A16, A16, A16, A16, NULL, 8, 64, 256, 6, 2, 2, 100, A16, NULL) == E   # shared rows missing
+    assert comb(A16, A16, A16, A16, A16, A16, A16, 8, 64, 256, 6, 9, 2, 100, A16, NULL) == E    # n_shared > 8
+    assert comb(A16, A16, A16, A16, A16, A16, A16, 8, 64, 255, 6, 2, 2, 100, A16, NULL) == E    # 2 ranks, 255 experts
+    assert comb(A16, A16, A16, A16, A16, A16, A16, 8, 68, 256, 6, 2, 2, 100, A16, NULL) == U    # d % 8 != 0
+    assert comb(A16, A16, A16, A16, A16, A16, A16, 0, 64, 256, 6, 2, 2, 100, A16, NULL) == moe.MOE_OK
+
+
+def test_ipc_calls_reject_null():
+    assert L.moe_ipc_handle_bytes() == 64
+    off = ctypes.c_ulonglong(0)
+    buf = ctypes.create_string_buffer(64)
+    assert L.moe_ipc_get_handle(NULL, buf, ctypes.byref(off)) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ipc_get_handle(A16, NULL, ctypes.byref(off)) == moe.MOE_ERR_INVALID_ARG
+    ptr = ctypes.c_void_p()
+    assert L.moe_ipc_open(NULL, 0, ctypes.byref(ptr)) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ipc_open(buf, 0, NULL) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ipc_close(NULL) == moe.MOE_ERR_INVALID_ARG
