@@ -100,9 +100,10 @@ struct TmapKey {
   int elem_bytes;  // 2: bf16, 1: bytes (packed FP4 pairs)
   uint64_t dim0, dim1, dim2;
   uint32_t box0, box1;
+  bool swizzle;  // 128-byte swizzle (else none)
   bool operator==(const TmapKey& o) const {
     return base == o.base && rank == o.rank && elem_bytes == o.elem_bytes && dim0 == o.dim0 && dim1 == o.dim1 &&
-           dim2 == o.dim2 && box0 == o.box0 && box1 == o.box1;
+           dim2 == o.dim2 && box0 == o.box0 && box1 == o.box1 && swizzle == o.swizzle;
   }
 };
 
@@ -119,8 +120,8 @@ std::mutex g_tmap_mu;
 }  // namespace
 
 static int encode_tmap(CUtensorMap* map, const void* base, int elem_bytes, int rank, uint64_t dim0, uint64_t dim1,
-                       uint64_t dim2, uint32_t box0, uint32_t box1) {
-  const TmapKey key{base, rank, elem_bytes, dim0, dim1, rank == 3 ? dim2 : 1, box0, box1};
+                       uint64_t dim2, uint32_t box0, uint32_t box1, bool swizzle = true) {
+  const TmapKey key{base, rank, elem_bytes, dim0, dim1, rank == 3 ? dim2 : 1, box0, box1, swizzle};
   {
     std::lock_guard<std::mutex> lk(g_tmap_mu);
     for (int i = 0; i < kTmapCacheSize; ++i) {
@@ -138,7 +139,8 @@ static int encode_tmap(CUtensorMap* map, const void* base, int elem_bytes, int r
   cuuint32_t estr[3] = {1, 1, 1};
   memset(map, 0, sizeof(*map));
   CUresult r = fn(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_tmap_mu);
@@ -158,6 +160,11 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0
 int encode_tmap_u8(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                    uint32_t box0, uint32_t box1) {
   return encode_tmap(map, base, 1, rank, dim0, dim1, dim2, box0, box1);
+}
+
+int encode_tmap_u8_plain(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint32_t box0,
+                         uint32_t box1) {
+  return encode_tmap(map, base, 1, 2, dim0, dim1, 1, box0, box1, false);
 }
 
 namespace {

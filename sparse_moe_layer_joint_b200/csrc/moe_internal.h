@@ -28,6 +28,11 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, uint64_t dim0
 int encode_tmap_u8(CUtensorMap* map, const void* base, int rank, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                    uint32_t box0, uint32_t box1);
 
+// A rank-2 byte tensor without swizzle (boxes land in shared memory as they lie in global memory:
+// FP4 scale-factor atoms).
+int encode_tmap_u8_plain(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint32_t box0,
+                         uint32_t box1);
+
 // Limit on device-side waits for kernels launched from now on.
 uint64_t wait_timeout_ns();
 

@@ -254,25 +254,36 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(const uint4* __rest
 // grouped GEMM on NVFP4 operands
 // ---------------------------------------------------------------------------
 constexpr int NUM_THREADS = 192;
-constexpr int TM = 128;           // rows per tile
+constexpr int TM = 128;           // rows per CTA
 constexpr int ROW_BYTES = 128;    // code bytes per row per stage: 256 values
 constexpr int KV_STAGE = 256;     // values along K per stage
 constexpr int A_BYTES = TM * ROW_BYTES;
 constexpr int SF_BYTES = (KV_STAGE / ATOM_K) * ATOM_BYTES;  // 4 atoms = 2 KB per 128 rows per stage
+constexpr int SF_ROW = 256;       // scale atoms seen as rows of 256 bytes by the pair's TMA loads
 constexpr uint32_t TMEM_COLS = 512;
 
-// Tile width (MMA N).  128 (default): two accumulators (double-buffered epilogue), six 36 KB stages.
-// 256: twice the MMA work per stage, but two 256-column accumulators leave no TMEM for the scales, so one
-// accumulator (the next tile's MMAs wait for the epilogue) and four 54 KB stages -- measured slower.
-template <int TN_>
+// Tile shapes.
+//   TN = 128 (default): one CTA per 128 x 128 tile, two accumulators (double-buffered epilogue), six
+//     36 KB stages.
+//   TN = 256: twice the MMA work per stage, but two 256-column accumulators leave no TMEM for the scales,
+//     so one accumulator (the next tile's MMAs wait for the epilogue) and four 54 KB stages.
+//   PAIR (TN = 128): a cluster of two CTAs per 256 x 128 tile with tcgen05.mma.cta_group::2.  CTA rank r
+//     holds A rows r*128.. and weight rows r*64.. of the tile, its A rows' scales and the scales of all
+//     128 weight rows (the MMA reads SFB from both CTAs' TMEM); 28 KB per stage per CTA for the MMA work of
+//     a 36 KB single-CTA stage, seven stages, two accumulators.
+template <int TN_, bool PAIR_ = false>
 struct FCfg {
   static constexpr int TN = TN_;
+  static constexpr bool PAIR = PAIR_;
+  static_assert(!PAIR || TN == 128, "pair tiles are 256 x 128");
+  static constexpr int TILE_M = PAIR ? 2 * TM : TM;  // rows per tile (per pair, or per CTA)
+  static constexpr int B_ROWS = PAIR ? TN / 2 : TN;   // weight rows one CTA holds
   static constexpr int ACC_BUFS = TN == 256 ? 1 : 2;
-  static constexpr int STAGES = TN == 256 ? 4 : 6;
-  static constexpr int B_BYTES = TN * ROW_BYTES;
+  static constexpr int STAGES = PAIR ? 7 : (TN == 256 ? 4 : 6);
+  static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
   static constexpr int SFB_BYTES = (TN / ATOM_ROWS) * SF_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
-  static constexpr uint32_t STAGE_TX = (uint32_t)STAGE_BYTES;
+  static constexpr uint32_t STAGE_TX = (uint32_t)STAGE_BYTES * (PAIR ? 2u : 1u);  // on the (leader's) barrier
   static constexpr uint32_t SFA_COL = 256;  // 16 columns: 4 K-chunks x 4
   static constexpr uint32_t SFB_COL = 320;  // 4 K-chunks x TN/32 columns
   static_assert(ACC_BUFS * TN <= (int)SFA_COL && SFB_COL + 4 * (TN / 32) <= TMEM_COLS, "TMEM columns");
@@ -321,19 +332,23 @@ struct SmemTail {
   Tables t;
 };
 
-template <int TN>
+template <int TN, bool PAIR = false>
 constexpr size_t smem_bytes() {
-  using C = FCfg<TN>;
+  using C = FCfg<TN, PAIR>;
   return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + sizeof(SmemTail<C::STAGES>);
 }
-static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448, "shared memory per CTA");
+static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448 && smem_bytes<128, true>() <= 232448,
+              "shared memory per CTA");
 
-template <int EPI, int TN>
+// tmA / tmA32: A codes in 128-row / 32-row boxes; tmB: weight codes, boxes of FCfg::B_ROWS rows (128 for
+// SwiGLU); tmSA / tmSB (pair tiles only): the A / weight scale atoms as rows of 256 bytes, 8-row boxes.
+template <int EPI, int TN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
-                    const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using C = FCfg<TN>;
-  static_assert(EPI != EPI_SWIGLU_FP4 || TN == 256, "SwiGLU tiles hold gate and up columns side by side");
+                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSA,
+                    const __grid_constant__ CUtensorMap tmSB, const Params p) {
+  using C = FCfg<TN, PAIR>;
+  static_assert(EPI != EPI_SWIGLU_FP4 || (TN == 256 && !PAIR), "SwiGLU tiles hold gate and up columns side by side");
   constexpr int OUT_W = EPI == EPI_SWIGLU_FP4 ? TN / 2 : TN;  // output columns per tile
   constexpr int STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
@@ -347,6 +362,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sSFB = sSFA + STAGES * SF_BYTES;
   SmemTail<STAGES>* st = reinterpret_cast<SmemTail<STAGES>*>(sSFB + STAGES * SFB_BYTES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // pair or CTA index
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -355,7 +374,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&st->tfull[a], 1);
-      mbar_init(&st->tempty[a], 4);
+      mbar_init(&st->tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(&st->drain, 1);
     st->abort_flag = 0;
@@ -377,17 +396,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int g = 0; g < p.G; ++g) {
       st->t.prefix[g] = run;
       const int rows = st->t.off[g + 1] - st->t.off[g];
-      run += rows > 0 ? (rows + TM - 1) / TM : 0;
+      run += rows > 0 ? (rows + C::TILE_M - 1) / C::TILE_M : 0;
     }
     st->t.prefix[p.G] = run;
   }
   __syncthreads();
   const int total_tiles = st->t.prefix[p.G] * p.n_tiles_n;
-  if ((int)blockIdx.x >= total_tiles) return;
+  if (unit >= total_tiles) return;  // uniform across the CTA (and the pair), before TMEM is taken
 
-  if (warp == 1) tmem_alloc(&st->tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    if (PAIR)
+      tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
+    else
+      tmem_alloc(&st->tmem_base, TMEM_COLS);
+  }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync_all();  // both CTAs' barriers initialised and TMEM taken before any cross-CTA traffic
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = st->tmem_base;
   const int num_kb = p.K / KV_STAGE;
@@ -412,50 +439,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmA32);
       tma_prefetch_desc(&tmB);
+      if (PAIR) {
+        tma_prefetch_desc(&tmSA);
+        tma_prefetch_desc(&tmSB);
+      } else {
+        tma_prefetch_desc(&tmA32);
+      }
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
         int g, m, nt;
         tile_of(tile, g, m, nt);
-        const int a_row = st->t.off[g] + m * TM;
+        const int a_row = st->t.off[g] + m * C::TILE_M + (int)rank * TM;
         const int n0 = nt * OUT_W;  // first output column; for SwiGLU also the first gate row
         // A rows to load: the group's real rows in this tile, in 32-row boxes (few-row groups at small
         // T would otherwise fill three quarters of every A stage with padding)
         int a_boxes = 4;
-        if (p.offsets_out != nullptr) {
+        if (!PAIR && p.offsets_out != nullptr) {
           const int real = st->t.off_out[g + 1] - st->t.off_out[g] - m * TM;
           a_boxes = real >= TM ? 4 : (real <= 0 ? 1 : (real + 31) / 32);
         }
         const uint32_t tx = C::STAGE_TX - (uint32_t)(4 - a_boxes) * (A_BYTES / 4);
         const uint8_t* sfa = p.a_sf + ((size_t)(a_row / ATOM_ROWS) * atoms_k) * ATOM_BYTES;
         const uint8_t* sfb_g = p.b_sf + (size_t)g * p.b_sf_stride;
+        // pair tiles: the scale atoms' rows of 256 bytes (every offset below is a multiple of 2 KB)
+        const int sfa_row = (int)(((long long)(a_row / ATOM_ROWS) * atoms_k * ATOM_BYTES) / SF_ROW);
+        const int sfb_row =
+            (int)(((long long)g * p.b_sf_stride + (long long)(n0 / ATOM_ROWS) * atoms_k * ATOM_BYTES) / SF_ROW);
         for (int kb = 0; kb < num_kb; ++kb) {
           ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
           if (!ok) break;
           uint64_t* bar = &st->full[stage];
-          mbar_arrive_expect_tx(bar, tx);
-          if (a_boxes == 4) {
-            tma_load_2d(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
+          if (PAIR) {
+            // both CTAs' copies complete on the leader's barrier, which expects the pair's bytes
+            if (leader) mbar_arrive_expect_tx(bar, C::STAGE_TX);
+            tma_load_2d_pair(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
+            tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0 + (int)rank * C::B_ROWS, g);
+            tma_load_2d_pair(sSFA + stage * SF_BYTES, &tmSA, bar, 0, sfa_row + kb * (SF_BYTES / SF_ROW));
+            tma_load_2d_pair(sSFB + stage * SFB_BYTES, &tmSB, bar, 0, sfb_row + kb * (SF_BYTES / SF_ROW));
           } else {
-            for (int i = 0; i < a_boxes; ++i)
-              tma_load_2d(sA + stage * A_BYTES + i * (A_BYTES / 4), &tmA32, bar, kb * ROW_BYTES, a_row + 32 * i);
-          }
-          if (EPI == EPI_SWIGLU_FP4) {  // gate rows, then the matching up rows (128-row boxes)
-            tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
-            tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &tmB, bar, kb * ROW_BYTES, p.b_up_row + n0, g);
-          } else {
-            tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
-          }
-          bulk_load(sSFA + stage * SF_BYTES, sfa + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+            mbar_arrive_expect_tx(bar, tx);
+            if (a_boxes == 4) {
+              tma_load_2d(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
+            } else {
+              for (int i = 0; i < a_boxes; ++i)
+                tma_load_2d(sA + stage * A_BYTES + i * (A_BYTES / 4), &tmA32, bar, kb * ROW_BYTES, a_row + 32 * i);
+            }
+            if (EPI == EPI_SWIGLU_FP4) {  // gate rows, then the matching up rows (128-row boxes)
+              tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
+              tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &tmB, bar, kb * ROW_BYTES, p.b_up_row + n0, g);
+            } else {
+              tma_load_3d(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0, g);
+            }
+            bulk_load(sSFA + stage * SF_BYTES, sfa + (size_t)kb * SF_BYTES, SF_BYTES, bar);
 #pragma unroll
-          for (int rb = 0; rb < TN / ATOM_ROWS; ++rb) {  // the weight rows' 128-row blocks
-            const int blk = (EPI == EPI_SWIGLU_FP4 && rb == 1) ? (p.b_up_row + n0) / ATOM_ROWS : n0 / ATOM_ROWS + rb;
-            bulk_load(sSFB + stage * SFB_BYTES + rb * SF_BYTES,
-                      sfb_g + ((size_t)blk * atoms_k) * ATOM_BYTES + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+            for (int rb = 0; rb < TN / ATOM_ROWS; ++rb) {  // the weight rows' 128-row blocks
+              const int blk =
+                  (EPI == EPI_SWIGLU_FP4 && rb == 1) ? (p.b_up_row + n0) / ATOM_ROWS : n0 / ATOM_ROWS + rb;
+              bulk_load(sSFB + stage * SFB_BYTES + rb * SF_BYTES,
+                        sfb_g + ((size_t)blk * atoms_k) * ATOM_BYTES + (size_t)kb * SF_BYTES, SF_BYTES, bar);
+            }
           }
           ++issued;
           if (++stage == STAGES) {
@@ -464,7 +510,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
+      if (!ok && !PAIR) {
         // wind down: let the copies already issued land before the CTA exits
         int zero = 0;
         for (long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
@@ -472,14 +518,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_nvf4(TM, TN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc_nvf4(C::TILE_M, TN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
         if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TN);
@@ -497,44 +543,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // 128-row block (the layout the MMA reads: row r at lane r % 32, column r / 32)
 #pragma unroll
           for (int j = 0; j < KV_STAGE / ATOM_K; ++j) {
-            tmem_cp_sf(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
+            if (PAIR) {
+              tmem_cp_sf_pair(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
+              tmem_cp_sf_pair(tmem_base + SFB_COL + 4 * j, make_desc_sf(sfb_addr + j * ATOM_BYTES));
+            } else {
+              tmem_cp_sf(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
 #pragma unroll
-            for (int rb = 0; rb < TN / ATOM_ROWS; ++rb)
-              tmem_cp_sf(tmem_base + SFB_COL + (TN / 32) * j + 4 * rb,
-                         make_desc_sf(sfb_addr + rb * SF_BYTES + j * ATOM_BYTES));
+              for (int rb = 0; rb < TN / ATOM_ROWS; ++rb)
+                tmem_cp_sf(tmem_base + SFB_COL + (TN / 32) * j + 4 * rb,
+                           make_desc_sf(sfb_addr + rb * SF_BYTES + j * ATOM_BYTES));
+            }
           }
 #pragma unroll
-          for (int j = 0; j < KV_STAGE / ATOM_K; ++j)
-            mma_nvf4_ss(d_tmem, make_desc_sw128(a_addr + j * 32), make_desc_sw128(b_addr + j * 32), idesc,
-                        tmem_base + SFA_COL + 4 * j, tmem_base + SFB_COL + (TN / 32) * j, (kb | j) != 0 ? 1u : 0u);
-          mma_commit(&st->empty[stage]);
+          for (int j = 0; j < KV_STAGE / ATOM_K; ++j) {
+            const uint64_t ad = make_desc_sw128(a_addr + j * 32), bd = make_desc_sw128(b_addr + j * 32);
+            const uint32_t sfa_t = tmem_base + SFA_COL + 4 * j, sfb_t = tmem_base + SFB_COL + (TN / 32) * j;
+            if (PAIR)
+              mma_nvf4_ss_pair(d_tmem, ad, bd, idesc, sfa_t, sfb_t, (kb | j) != 0 ? 1u : 0u);
+            else
+              mma_nvf4_ss(d_tmem, ad, bd, idesc, sfa_t, sfb_t, (kb | j) != 0 ? 1u : 0u);
+          }
+          if (PAIR)
+            mma_commit_pair(&st->empty[stage], 0x3);
+          else
+            mma_commit(&st->empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&st->tfull[acc]);
+        if (PAIR)
+          mma_commit_pair(&st->tfull[acc], 0x3);
+        else
+          mma_commit(&st->tfull[acc]);
         if (++acc == C::ACC_BUFS) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
+      // no MMA may still be running when TMEM is released
       int zero = 0;
-      mma_commit(&st->drain);
+      if (PAIR)
+        mma_commit_pair(&st->drain, 0x1);
+      else
+        mma_commit(&st->drain);
       mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
     }
   } else {
     // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, one tile row per thread
     const int quarter = warp & 3;
+    const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(&st->tempty[0]), 0) : 0u;
+    const uint32_t tempty1 = PAIR ? mapa_shared(smem_u32(&st->tempty[1]), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int tile = unit; tile < total_tiles; tile += n_units) {
       int g, m, nt;
       tile_of(tile, g, m, nt);
-      const int in_group = m * TM + quarter * 32 + lane;  // row within the group
+      const int in_group = m * C::TILE_M + (int)rank * TM + quarter * 32 + lane;  // row within the group
       const long long r = (long long)st->t.off[g] + in_group;
-      bool valid = r < p.rows_cap;
+      // a pair tile's second half may run past the group's padded rows (into the next group's)
+      bool valid = r < p.rows_cap && in_group < st->t.off[g + 1] - st->t.off[g];
       long long r_out = r;  // output row
       if (EPI == EPI_BF16 && p.offsets_out != nullptr) {
         r_out = (long long)st->t.off_out[g] + in_group;
@@ -592,7 +661,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&st->tempty[acc]);
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(acc == 0 ? tempty0 : tempty1);
+        else
+          mbar_arrive(&st->tempty[acc]);
+      }
       if (++acc == C::ACC_BUFS) {
         acc = 0;
         acc_phase ^= 1u;
@@ -601,23 +675,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync_all();  // every MMA of the pair has landed; both CTAs are done with each other's memory
+  else
+    __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-template <int EPI, int TN>
-int launch_fp4(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const Params& p, int grid,
-               cudaStream_t s) {
-  auto kfn = fp4_gemm_kernel<EPI, TN>;
-  constexpr size_t bytes = smem_bytes<TN>();
+template <int EPI, int TN, bool PAIR = false>
+int launch_fp4(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const CUtensorMap& tsa,
+               const CUtensorMap& tsb, const Params& p, int grid, cudaStream_t s) {
+  auto kfn = fp4_gemm_kernel<EPI, TN, PAIR>;
+  constexpr size_t bytes = smem_bytes<TN, PAIR>();
   const int rc = ensure_smem_attr((const void*)kfn, bytes);
   if (rc != MOE_OK) return rc;
-  kfn<<<grid, NUM_THREADS, bytes, s>>>(ta, ta32, tb, p);
+  if (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kfn, ta, ta32, tb, tsa, tsb, p) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    kfn<<<grid, NUM_THREADS, bytes, s>>>(ta, ta32, tb, tsa, tsb, p);
+  }
   return MOE_OK;
+}
+
+// Pair tiles (256 x 128), an option (MOE_FP4_PAIR=1; GELU and bf16 epilogues) for groups long enough to
+// fill them (on average at least 256 padded rows a group).  Off by default: on a prefill-shaped slice they
+// ran at 2.05 against 1.99 ms per GEMM pair, as the epilogue, not operand delivery, sets the pace.
+bool fp4_pair_for(long long rows_cap, int n_groups) {
+  bool on = false;
+  (void)rows_cap;
+  (void)n_groups;
+  if (const char* env = getenv("MOE_FP4_PAIR")) {
+    if (env[0] == '1' && env[1] == '\0') on = true;
+    if (env[0] == '0' && env[1] == '\0') on = false;
+  }
+  return on;
 }
 
 }  // namespace fp4
@@ -716,12 +826,22 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (rc != MOE_OK) return rc;
   unsigned int* status = status_ptr();
   if (!status) return MOE_ERR_CUDA;
-  CUtensorMap ta, ta32, tb;
+  const bool pair = !swiglu && tn == 128 && fp4_pair_for(rows_cap, n_groups);
+  CUtensorMap ta, ta32, tb, tsa, tsb;
   if ((rc = encode_tmap_u8(&ta, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, TM)) != MOE_OK) return rc;
   if ((rc = encode_tmap_u8(&ta32, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, 32)) != MOE_OK) return rc;
-  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, b_rows, (uint64_t)n_groups, ROW_BYTES, swiglu ? 128 : tn)) !=
-      MOE_OK)
+  const uint32_t b_box = swiglu ? 128u : (pair ? (uint32_t)FCfg<128, true>::B_ROWS : (uint32_t)tn);
+  if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, b_rows, (uint64_t)n_groups, ROW_BYTES, b_box)) != MOE_OK)
     return rc;
+  if (pair) {  // the scale atoms as rows of 256 bytes: 8 rows (2 KB) per operand and stage
+    const uint64_t a_sf_bytes = (uint64_t)rows_cap * (K / 16), b_sf_bytes = (uint64_t)n_groups * b_rows * (K / 16);
+    if ((rc = encode_tmap_u8_plain(&tsa, asf, SF_ROW, a_sf_bytes / SF_ROW, SF_ROW, SF_BYTES / SF_ROW)) != MOE_OK)
+      return rc;
+    if ((rc = encode_tmap_u8_plain(&tsb, wsf, SF_ROW, b_sf_bytes / SF_ROW, SF_ROW, SF_BYTES / SF_ROW)) != MOE_OK)
+      return rc;
+  } else {
+    tsa = tsb = ta;  // not read
+  }
   Params p{};
   p.offsets_pad = offsets_pad;
   p.G = n_groups;
@@ -741,16 +861,26 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   p.out_rows = out_rows;
   p.timeout_ns = wait_timeout_ns();
   p.status = status;
+  if (pair) {
+    // every group may end in a partial 256-row tile
+    const long long tiles_upper = (rows_cap / FCfg<128, true>::TILE_M + n_groups) * p.n_tiles_n;
+    const long long pairs = tiles_upper < sms / 2 ? tiles_upper : sms / 2;
+    rc = epilogue == MOE_NVFP4_EPI_GELU_FP4
+             ? launch_fp4<EPI_GELU_FP4, 128, true>(ta, ta32, tb, tsa, tsb, p, (int)(2 * pairs), s)
+             : launch_fp4<EPI_BF16, 128, true>(ta, ta32, tb, tsa, tsb, p, (int)(2 * pairs), s);
+    if (rc != MOE_OK) return rc;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   const long long tiles_upper = (rows_cap / TM) * p.n_tiles_n;
   const int grid = (int)(tiles_upper < sms ? tiles_upper : sms);
   if (swiglu)
-    rc = launch_fp4<EPI_SWIGLU_FP4, 256>(ta, ta32, tb, p, grid, s);
+    rc = launch_fp4<EPI_SWIGLU_FP4, 256>(ta, ta32, tb, tsa, tsb, p, grid, s);
   else if (epilogue == MOE_NVFP4_EPI_GELU_FP4)
-    rc = tn == 256 ? launch_fp4<EPI_GELU_FP4, 256>(ta, ta32, tb, p, grid, s)
-                   : launch_fp4<EPI_GELU_FP4, 128>(ta, ta32, tb, p, grid, s);
+    rc = tn == 256 ? launch_fp4<EPI_GELU_FP4, 256>(ta, ta32, tb, tsa, tsb, p, grid, s)
+                   : launch_fp4<EPI_GELU_FP4, 128>(ta, ta32, tb, tsa, tsb, p, grid, s);
   else
-    rc = tn == 256 ? launch_fp4<EPI_BF16, 256>(ta, ta32, tb, p, grid, s)
-                   : launch_fp4<EPI_BF16, 128>(ta, ta32, tb, p, grid, s);
+    rc = tn == 256 ? launch_fp4<EPI_BF16, 256>(ta, ta32, tb, tsa, tsb, p, grid, s)
+                   : launch_fp4<EPI_BF16, 128>(ta, ta32, tb, tsa, tsb, p, grid, s);
   if (rc != MOE_OK) return rc;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -462,6 +462,26 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
       : "memory");
 }
 
+// tcgen05.cp for the pair, issued once by the leader: each CTA's 32 x 128-bit block at the same
+// shared-memory offset goes into its own TMEM columns [taddr, taddr + 4), broadcast to all four
+// lane quarters.
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Block-scaled FP4 MMA of the pair (M = 256): D[tmem of both CTAs] (+)= (A * SFA) x (B * SFB)^T over
+// K = 64, A rows and SFA from each CTA's own shared memory / TMEM, B split by rows between the CTAs,
+// SFB for all N columns in each CTA's TMEM.  Issued by the leader.
+__device__ __forceinline__ void mma_nvf4_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+
 }  // namespace moe
 
 namespace moe {

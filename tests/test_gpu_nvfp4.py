@@ -162,10 +162,16 @@ def test_quantize_at_exact_ties_divides():
         np.testing.assert_array_equal(sfs[rows[:, j]], s_ref)
 
 
-@pytest.fixture(params=["tn128", "tn256"])
+@pytest.fixture(params=["tn128", "tn256", "pair"])
 def fp4_tile(request, monkeypatch):
-    """Both FP4 GEMM tile widths (128, the default, and 256 where N is a multiple of 256)."""
-    monkeypatch.setenv("MOE_FP4_TN", request.param[2:])
+    """Every FP4 GEMM tile: 128 x 128 (the default at small sizes), 128 x 256 (where N is a multiple
+    of 256) and the CTA pair's 256 x 128 (the default for long groups), each forced."""
+    if request.param == "pair":
+        monkeypatch.setenv("MOE_FP4_TN", "128")
+        monkeypatch.setenv("MOE_FP4_PAIR", "1")
+    else:
+        monkeypatch.setenv("MOE_FP4_TN", request.param[2:])
+        monkeypatch.setenv("MOE_FP4_PAIR", "0")
     return request.param
 
 
