@@ -340,10 +340,11 @@ int moe_nvfp4_dispatch(const moe_bf16* x, const int32_t* topk_idx, const int32_t
  *              y_perm layout moe_combine reads with moe_permute's token_row
  *   offsets_out [n_groups + 1] int32 or NULL; values clamped to [0, out_rows].
  *              With either epilogue it also gives each group's real row count:
- *              rows past it are padding and are not loaded (their outputs are
- *              not meaningful), which saves most of the A traffic when groups
- *              have few rows (decode)
- * Padding rows are computed like any row (their FP4 outputs are not meaningful).
+ *              rows past it are padding; they are not loaded and, with the FP4
+ *              epilogues, not written, which saves most of the A traffic and the
+ *              epilogue work when groups have few rows (decode)
+ * Without offsets_out padding rows are computed and written like any row (their
+ * FP4 outputs are not meaningful).
  * Limits: N % 128 == 0, K % 256 == 0, rows_cap % 128 == 0, n_groups <= 256.
  */
 int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, const int32_t* offsets_pad, int n_groups,

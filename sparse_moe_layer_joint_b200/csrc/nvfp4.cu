@@ -25,11 +25,12 @@
 //   weight_amax / weight_quant / weight_scale   weights, once
 //   dispatch_quant   x rows quantized once per token and written to the padded
 //                    rows of its k experts (the FP4 dispatch)
-//   fp4_gemm_kernel<EPI>   persistent grouped GEMM, one CTA per 128 x 128 tile:
+//   fp4_gemm_kernel<EPI, TN, PAIR>   persistent grouped GEMM, one CTA per 128 x 128
+//                    tile (or 128 x 256; or a CTA pair per 256 x 128 tile):
 //                    warp 0 loads code tiles (TMA, 128-byte swizzle) and scale
 //                    atoms (bulk copies), warp 1 copies the scales to TMEM
 //                    (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4 with
-//                    block16 scales, warps 2-5 drain the accumulator: x the
+//                    block16 scales, warps 2-9 drain the accumulator: x the
 //                    weight matrix's g, then GELU and FP4 re-quantization
 //                    (GEMM1) or bf16 (GEMM2)
 #include <cuda_bf16.h>
@@ -94,13 +95,39 @@ __device__ __forceinline__ uint2 pack16(const float* v, float denom) {
   return make_uint2(w[0], w[1]);
 }
 
+// The same code, E2M1(fl32(v / s)), for a scale s > 0 that is an E4M3 value, decided without the
+// division.  Rounding is monotone, so fl32(q) against an E2M1 midpoint t is a test on q itself: every
+// midpoint has an even last mantissa bit, so a quotient halfway between t and a neighbour rounds to t,
+//   fl32(q) <= t  <=>  q <= t + h      fl32(q) < t  <=>  q < t - h      (h: half the fp32 spacing at t),
+// and with q = |v| / s these read |v| - t s <= h s and |v| - t s < -h s.  h s is exact (a power of two
+// times s), and the fma rounds |v| - t s once; wherever that difference is within a few of its own
+// spacings of h s, |v| and t s are within a factor of two of each other, so it is exact (Sterbenz) and
+// the comparison decides as over the reals.  (Checked against the rounded quotient for every positive
+// E4M3 scale at and around each midpoint.)  A NaN gives code 7, as the division form does.
+__device__ __forceinline__ uint32_t e2m1_code_of_quotient(float v, float s) {
+  const float a = fabsf(v);
+  const int n = (int)(fmaf(-0.25f, s, a) <= 0x1p-26f * s) + (int)(fmaf(-0.75f, s, a) < -0x1p-25f * s) +
+                (int)(fmaf(-1.25f, s, a) <= 0x1p-24f * s) + (int)(fmaf(-1.75f, s, a) < -0x1p-24f * s) +
+                (int)(fmaf(-2.5f, s, a) <= 0x1p-23f * s) + (int)(fmaf(-3.5f, s, a) < -0x1p-23f * s) +
+                (int)(fmaf(-5.0f, s, a) <= 0x1p-22f * s);
+  uint32_t c = 7u - (uint32_t)n;  // the midpoints fl32(q) has passed
+  if (c != 0u && v < 0.0f) c |= 8u;
+  return c;
+}
+
 // Activation block: dynamic scale, no tensor scale.
 __device__ __forceinline__ uint2 quant16_act(const float* v, uint32_t& sf) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
   sf = e4m3_code(__fdiv_rn(amax, E2M1_MAX));
-  return pack16(v, e4m3_value(sf));
+  const float s = e4m3_value(sf);
+  uint32_t w[2] = {0u, 0u};
+  if (s > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code_of_quotient(v[i], s) << (4 * (i & 7));
+  }
+  return make_uint2(w[0], w[1]);
 }
 
 __device__ __forceinline__ void bf16x8_to_float(const uint4& u, float* f) {
@@ -114,14 +141,16 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4& u, float* f) {
 }
 
 // GELU, tanh form, written through the identity (1 + tanh z) / 2 = 1 / (1 + e^-2z):
-// u / (1 + e^(-2 k0 (u + k1 u^3))).  No cancellation near 0 and one exp, so the
-// result is within a few fp32 ulps -- it decides FP4 codes, so it must stay close
-// to the exact value (the tanh.approx of the bf16 path would move ~0.1% of codes).
+// u / (1 + e^(-2 k0 (u + k1 u^3))).  No cancellation near 0, one exp and one
+// approximate division, so the result is within a few fp32 ulps -- it decides FP4
+// codes, so it must stay close to the exact value (the tanh.approx of the bf16 path
+// would move ~0.1% of codes).  For very negative u the denominator overflows and
+// the quotient is -0.
 __device__ __forceinline__ float gelu_tanh_accurate(float u) {
   const float k0x2 = 1.5957691216057308f;  // 2 sqrt(2/pi)
   const float k1 = 0.044715f;
   const float z = k0x2 * fmaf(k1 * u, u * u, u);
-  return u * __frcp_rn(1.0f + __expf(-z));
+  return __fdividef(u, 1.0f + __expf(-z));
 }
 
 // ---------------------------------------------------------------------------
@@ -253,7 +282,8 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(const uint4* __rest
 // ---------------------------------------------------------------------------
 // grouped GEMM on NVFP4 operands
 // ---------------------------------------------------------------------------
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;     // two per TMEM lane quarter, one per half of the tile's output columns
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;  // producer warp, MMA warp, epilogue warps
 constexpr int TM = 128;           // rows per CTA
 constexpr int ROW_BYTES = 128;    // code bytes per row per stage: 256 values
 constexpr int KV_STAGE = 256;     // values along K per stage
@@ -267,26 +297,31 @@ constexpr uint32_t TMEM_COLS = 512;
 //     36 KB stages.
 //   TN = 256: twice the MMA work per stage, but two 256-column accumulators leave no TMEM for the scales,
 //     so one accumulator (the next tile's MMAs wait for the epilogue) and four 54 KB stages.
-//   PAIR (TN = 128): a cluster of two CTAs per 256 x 128 tile with tcgen05.mma.cta_group::2.  CTA rank r
-//     holds A rows r*128.. and weight rows r*64.. of the tile, its A rows' scales and the scales of all
-//     128 weight rows (the MMA reads SFB from both CTAs' TMEM); 28 KB per stage per CTA for the MMA work of
-//     a 36 KB single-CTA stage, seven stages, two accumulators.
+//   PAIR: a cluster of two CTAs per 256 x TN tile with tcgen05.mma.cta_group::2.  CTA rank r holds A rows
+//     r*128.. and weight rows r*TN/2.. of the tile (SwiGLU: rank 0 the 128 gate rows, rank 1 the 128
+//     matching up rows), its A rows' scales and the scales of all TN weight rows (the MMA reads SFB from
+//     both CTAs' TMEM).  256 x 256: 38 KB per stage per CTA for the MMA work of a 54 KB single-CTA stage,
+//     five stages, one accumulator; 256 x 128: 28 KB for that of a 36 KB stage, seven stages, two.
 template <int TN_, bool PAIR_ = false>
 struct FCfg {
   static constexpr int TN = TN_;
   static constexpr bool PAIR = PAIR_;
-  static_assert(!PAIR || TN == 128, "pair tiles are 256 x 128");
+  static_assert(TN == 128 || TN == 256, "tile widths");
   static constexpr int TILE_M = PAIR ? 2 * TM : TM;  // rows per tile (per pair, or per CTA)
   static constexpr int B_ROWS = PAIR ? TN / 2 : TN;   // weight rows one CTA holds
   static constexpr int ACC_BUFS = TN == 256 ? 1 : 2;
-  static constexpr int STAGES = PAIR ? 7 : (TN == 256 ? 4 : 6);
+  static constexpr int STAGES = PAIR ? (TN == 256 ? 5 : 7) : (TN == 256 ? 4 : 6);
   static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
   static constexpr int SFB_BYTES = (TN / ATOM_ROWS) * SF_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
   static constexpr uint32_t STAGE_TX = (uint32_t)STAGE_BYTES * (PAIR ? 2u : 1u);  // on the (leader's) barrier
-  static constexpr uint32_t SFA_COL = 256;  // 16 columns: 4 K-chunks x 4
-  static constexpr uint32_t SFB_COL = 320;  // 4 K-chunks x TN/32 columns
-  static_assert(ACC_BUFS * TN <= (int)SFA_COL && SFB_COL + 4 * (TN / 32) <= TMEM_COLS, "TMEM columns");
+  // A stage's scales in the columns past the accumulators: 16 for A (4 K-chunks x 4), then TN/8 for the
+  // weights (4 K-chunks x TN/32).  Every stage reuses them: tcgen05 operations issued by one thread run in
+  // order, so a stage's copies land after the previous stage's MMAs have read them.  (Rotating buffers,
+  // one a stage, measured no faster.)
+  static constexpr uint32_t SFA_COL = (uint32_t)(ACC_BUFS * TN);
+  static constexpr uint32_t SFB_COL = SFA_COL + 16;
+  static_assert(SFB_COL + TN / 8 <= TMEM_COLS, "TMEM columns");
 };
 constexpr int EPI_GELU_FP4 = 0;   // GEMM1: x g1, GELU, FP4 out (the next GEMM's A)
 constexpr int EPI_BF16 = 1;       // GEMM2: x g2, bf16 out
@@ -308,7 +343,7 @@ struct Params {
   __nv_bfloat16* out;      // EPI_BF16: [rows_cap, N], or [out_rows, N] through offsets_out
   const int* offsets_out;  // nullable: the groups' real rows (offsets_out[e+1] - offsets_out[e] of them); with
                            // EPI_BF16 group e's row i goes to row offsets_out[e] + i.  Rows past a group's
-                           // real count are not loaded (their outputs are not meaningful)
+                           // real count are neither loaded nor (FP4 epilogues) written
   long long out_rows;
   uint64_t timeout_ns;
   unsigned int* status;
@@ -337,7 +372,8 @@ constexpr size_t smem_bytes() {
   using C = FCfg<TN, PAIR>;
   return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + sizeof(SmemTail<C::STAGES>);
 }
-static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448 && smem_bytes<128, true>() <= 232448,
+static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448 && smem_bytes<128, true>() <= 232448 &&
+                  smem_bytes<256, true>() <= 232448,
               "shared memory per CTA");
 
 // tmA / tmA32: A codes in 128-row / 32-row boxes; tmB: weight codes, boxes of FCfg::B_ROWS rows (128 for
@@ -348,12 +384,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSA,
                     const __grid_constant__ CUtensorMap tmSB, const Params p) {
   using C = FCfg<TN, PAIR>;
-  static_assert(EPI != EPI_SWIGLU_FP4 || (TN == 256 && !PAIR), "SwiGLU tiles hold gate and up columns side by side");
+  static_assert(EPI != EPI_SWIGLU_FP4 || TN == 256, "SwiGLU tiles hold gate and up columns side by side");
   constexpr int OUT_W = EPI == EPI_SWIGLU_FP4 ? TN / 2 : TN;  // output columns per tile
   constexpr int STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int SFB_BYTES = C::SFB_BYTES;
-  constexpr uint32_t SFA_COL = C::SFA_COL, SFB_COL = C::SFB_COL;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -374,7 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&st->tfull[a], 1);
-      mbar_init(&st->tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
+      mbar_init(&st->tempty[a], EPI_WARPS * (PAIR ? 2 : 1));  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(&st->drain, 1);
     st->abort_flag = 0;
@@ -469,6 +504,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int sfa_row = (int)(((long long)(a_row / ATOM_ROWS) * atoms_k * ATOM_BYTES) / SF_ROW);
         const int sfb_row =
             (int)(((long long)g * p.b_sf_stride + (long long)(n0 / ATOM_ROWS) * atoms_k * ATOM_BYTES) / SF_ROW);
+        const int sfb_up_row = (int)(((long long)g * p.b_sf_stride +
+                                      (long long)((p.b_up_row + n0) / ATOM_ROWS) * atoms_k * ATOM_BYTES) /
+                                     SF_ROW);
         for (int kb = 0; kb < num_kb; ++kb) {
           ok = mbar_wait(&st->empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, p.status);
           if (!ok) break;
@@ -476,10 +514,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (PAIR) {
             // both CTAs' copies complete on the leader's barrier, which expects the pair's bytes
             if (leader) mbar_arrive_expect_tx(bar, C::STAGE_TX);
+            const int b_row = EPI == EPI_SWIGLU_FP4 ? (rank == 0u ? n0 : p.b_up_row + n0) : n0 + (int)rank * C::B_ROWS;
             tma_load_2d_pair(sA + stage * A_BYTES, &tmA, bar, kb * ROW_BYTES, a_row);
-            tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, n0 + (int)rank * C::B_ROWS, g);
+            tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * ROW_BYTES, b_row, g);
             tma_load_2d_pair(sSFA + stage * SF_BYTES, &tmSA, bar, 0, sfa_row + kb * (SF_BYTES / SF_ROW));
-            tma_load_2d_pair(sSFB + stage * SFB_BYTES, &tmSB, bar, 0, sfb_row + kb * (SF_BYTES / SF_ROW));
+#pragma unroll
+            for (int rb = 0; rb < TN / ATOM_ROWS; ++rb) {  // the weight rows' 128-row blocks, in every CTA
+              const int blk_row = rb == 0 ? sfb_row : (EPI == EPI_SWIGLU_FP4 ? sfb_up_row : sfb_row + atoms_k * 2);
+              tma_load_2d_pair(sSFB + stage * SFB_BYTES + rb * SF_BYTES, &tmSB, bar, 0,
+                               blk_row + kb * (SF_BYTES / SF_ROW));
+            }
           } else {
             mbar_arrive_expect_tx(bar, tx);
             if (a_boxes == 4) {
@@ -539,25 +583,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
           const uint32_t sfa_addr = smem_u32(sSFA + stage * SF_BYTES);
           const uint32_t sfb_addr = smem_u32(sSFB + stage * SFB_BYTES);
+          const uint32_t sfa_col = tmem_base + C::SFA_COL, sfb_col = tmem_base + C::SFB_COL;
           // K-chunk j's scales: A's 128 rows in 4 columns; the weights' TN rows in TN/32 columns, 4 per
           // 128-row block (the layout the MMA reads: row r at lane r % 32, column r / 32)
 #pragma unroll
           for (int j = 0; j < KV_STAGE / ATOM_K; ++j) {
-            if (PAIR) {
-              tmem_cp_sf_pair(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
-              tmem_cp_sf_pair(tmem_base + SFB_COL + 4 * j, make_desc_sf(sfb_addr + j * ATOM_BYTES));
-            } else {
-              tmem_cp_sf(tmem_base + SFA_COL + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
+            if (PAIR)
+              tmem_cp_sf_pair(sfa_col + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
+            else
+              tmem_cp_sf(sfa_col + 4 * j, make_desc_sf(sfa_addr + j * ATOM_BYTES));
 #pragma unroll
-              for (int rb = 0; rb < TN / ATOM_ROWS; ++rb)
-                tmem_cp_sf(tmem_base + SFB_COL + (TN / 32) * j + 4 * rb,
-                           make_desc_sf(sfb_addr + rb * SF_BYTES + j * ATOM_BYTES));
+            for (int rb = 0; rb < TN / ATOM_ROWS; ++rb) {
+              const uint64_t d = make_desc_sf(sfb_addr + rb * SF_BYTES + j * ATOM_BYTES);
+              if (PAIR)
+                tmem_cp_sf_pair(sfb_col + (TN / 32) * j + 4 * rb, d);
+              else
+                tmem_cp_sf(sfb_col + (TN / 32) * j + 4 * rb, d);
             }
           }
 #pragma unroll
           for (int j = 0; j < KV_STAGE / ATOM_K; ++j) {
             const uint64_t ad = make_desc_sw128(a_addr + j * 32), bd = make_desc_sw128(b_addr + j * 32);
-            const uint32_t sfa_t = tmem_base + SFA_COL + 4 * j, sfb_t = tmem_base + SFB_COL + (TN / 32) * j;
+            const uint32_t sfa_t = sfa_col + 4 * j, sfb_t = sfb_col + (TN / 32) * j;
             if (PAIR)
               mma_nvf4_ss_pair(d_tmem, ad, bd, idesc, sfa_t, sfb_t, (kb | j) != 0 ? 1u : 0u);
             else
@@ -591,8 +638,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&st->drain, 0, p.timeout_ns, &zero, p.status);
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, one tile row per thread
+    // epilogue, EPI_WARPS warps: warp w reads TMEM lanes 32 * (w % 4) .. +31 (one tile row per thread)
+    // and drains the column half (w - 2) / 4 of the tile's outputs.  It reads its whole share of the
+    // accumulator, hands the accumulator back to the MMA, and only then computes and stores: the next
+    // tile's MMAs overlap the math and the stores, and the hand-back never waits for stores to land.
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int W = OUT_W / 2;                            // output columns per warp
+    constexpr int NV = EPI == EPI_SWIGLU_FP4 ? 2 * W : W;  // accumulator columns per thread (gate, up)
     const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(&st->tempty[0]), 0) : 0u;
     const uint32_t tempty1 = PAIR ? mapa_shared(smem_u32(&st->tempty[1]), 0) : 0u;
     int acc = 0;
@@ -605,59 +658,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // a pair tile's second half may run past the group's padded rows (into the next group's)
       bool valid = r < p.rows_cap && in_group < st->t.off[g + 1] - st->t.off[g];
       long long r_out = r;  // output row
-      if (EPI == EPI_BF16 && p.offsets_out != nullptr) {
-        r_out = (long long)st->t.off_out[g] + in_group;
-        valid = in_group < st->t.off_out[g + 1] - st->t.off_out[g] && r_out < p.out_rows;
+      if (p.offsets_out != nullptr) {
+        // only the groups' real rows are meaningful (and, with EPI_BF16, written to the unpadded rows)
+        const int real = st->t.off_out[g + 1] - st->t.off_out[g];
+        if (EPI == EPI_BF16) {
+          r_out = (long long)st->t.off_out[g] + in_group;
+          valid = in_group < real && r_out < p.out_rows;
+        } else {
+          valid = valid && in_group < real;
+        }
       }
       const float gs = __ldg(p.gscale + g);
       if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TN);
-#pragma unroll 1
-      for (int ch = 0; ch < OUT_W / 32; ++ch) {
-        const int col0 = nt * OUT_W + ch * 32;
-        if (col0 >= p.N) break;  // same for the whole warp
-        float v[32];
-        tmem_ld32(taddr + ch * 32, v);
-        if (EPI == EPI_SWIGLU_FP4) {
-          float u[32];
-          tmem_ld32(taddr + OUT_W + ch * 32, u);
-          if (!valid) continue;
+      float v[NV];
+      if (EPI == EPI_SWIGLU_FP4) {
+        tmem_ld64(taddr + half * W, v);              // gate columns
+        tmem_ld64(taddr + OUT_W + half * W, v + W);  // the matching up columns
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gate = __fmul_rn(v[i], gs);
-            v[i] = __fmul_rn(__fmul_rn(gate, __frcp_rn(1.0f + __expf(-gate))), __fmul_rn(u[i], gs));
-          }
-          uint32_t s0, s1;
-          const uint2 q0 = quant16_act(v, s0);
-          const uint2 q1 = quant16_act(v + 16, s1);
-          *reinterpret_cast<uint4*>(p.out_q + r * (p.N / 2) + col0 / 2) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-          const size_t so = sf_offset(r, col0 / 16, p.N);
-          p.out_sf[so] = (uint8_t)s0;
-          p.out_sf[so + 1] = (uint8_t)s1;
-          continue;
-        }
-        if (!valid) continue;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], gs);
-        if (EPI == EPI_GELU_FP4) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_accurate(v[i]);
-          uint32_t s0, s1;
-          const uint2 q0 = quant16_act(v, s0);
-          const uint2 q1 = quant16_act(v + 16, s1);
-          *reinterpret_cast<uint4*>(p.out_q + r * (p.N / 2) + col0 / 2) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-          const size_t so = sf_offset(r, col0 / 16, p.N);  // the two blocks share an atom line (b even)
-          p.out_sf[so] = (uint8_t)s0;
-          p.out_sf[so + 1] = (uint8_t)s1;
-        } else {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + r_out * p.N + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        for (int c = 0; c < W; c += 64) tmem_ld64(taddr + half * W + c, v + c);
       }
       tc_fence_before();
       __syncwarp();
@@ -671,9 +692,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+      if (!valid) continue;
+#pragma unroll
+      for (int ch = 0; ch < W / 32; ++ch) {
+        const int col0 = nt * OUT_W + half * W + ch * 32;
+        if (col0 >= p.N) break;  // same for the whole warp
+        float* x = v + ch * 32;
+        if (EPI == EPI_SWIGLU_FP4) {
+          const float* u = v + W + ch * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gate = __fmul_rn(x[i], gs);
+            x[i] = __fmul_rn(__fdividef(gate, 1.0f + __expf(-gate)), __fmul_rn(u[i], gs));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = __fmul_rn(x[i], gs);
+          if (EPI == EPI_GELU_FP4) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = gelu_tanh_accurate(x[i]);
+          }
+        }
+        if (EPI != EPI_BF16) {
+          uint32_t s0, s1;
+          const uint2 q0 = quant16_act(x, s0);
+          const uint2 q1 = quant16_act(x + 16, s1);
+          *reinterpret_cast<uint4*>(p.out_q + r * (p.N / 2) + col0 / 2) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+          const size_t so = sf_offset(r, col0 / 16, p.N);  // the two blocks share an atom line (b even)
+          p.out_sf[so] = (uint8_t)s0;
+          p.out_sf[so + 1] = (uint8_t)s1;
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + r_out * p.N + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
     }
   }
-
   tc_fence_before();
   if (PAIR)
     cluster_sync_all();  // every MMA of the pair has landed; both CTAs are done with each other's memory
@@ -716,9 +774,10 @@ int launch_fp4(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap
   return MOE_OK;
 }
 
-// Pair tiles (256 x 128), an option (MOE_FP4_PAIR=1; GELU and bf16 epilogues) for groups long enough to
-// fill them (on average at least 256 padded rows a group).  Off by default: on a prefill-shaped slice they
-// ran at 2.05 against 1.99 ms per GEMM pair, as the epilogue, not operand delivery, sets the pace.
+// Pair tiles (256 x TN), an option for groups long enough to fill them (MOE_FP4_PAIR=1; =0 or unset: off).
+// They move 30% fewer bytes per MMA into each SM than single-CTA tiles of the same width but were measured
+// slower on a prefill-shaped slice (256 x 256 pairs 1.12 ms against 1.03 ms per GEMM pair for 128 x 256
+// single-CTA tiles; 256 x 128 pairs 1.54 against 1.49 for 128 x 128).
 bool fp4_pair_for(long long rows_cap, int n_groups) {
   bool on = false;
   (void)rows_cap;
@@ -809,9 +868,10 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
       !aligned4(offsets_pad))
     return MOE_ERR_INVALID_ARG;
   if (N % 128 != 0 || K % KV_STAGE != 0 || rows_cap % ATOM_ROWS != 0) return MOE_ERR_UNSUPPORTED;
-  // tile width: 128 (measured faster at every size here: 1.87 against 2.19 ms on a prefill-shaped slice,
-  // 3.50 against 3.13 TB/s at decode); MOE_FP4_TN=256 selects the single-accumulator 256-wide tiles
-  int tn = 128;
+  // tile width: 256 where N allows (twice the MMA work per stage and 25% fewer bytes per MMA than 128; with
+  // the epilogue handing the accumulator back before its math, measured faster at every size: 1.03 against
+  // 1.49 ms on a prefill-shaped slice, 4.86 against 4.23 TB/s at decode); MOE_FP4_TN=128 or =256 forces one
+  int tn = N % 256 == 0 ? 256 : 128;
   if (const char* env = getenv("MOE_FP4_TN")) {
     if (env[0] == '1' && env[1] == '2' && env[2] == '8' && env[3] == '\0') tn = 128;
     if (env[0] == '2' && env[1] == '5' && env[2] == '6' && env[3] == '\0' && N % 256 == 0) tn = 256;
@@ -826,11 +886,11 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (rc != MOE_OK) return rc;
   unsigned int* status = status_ptr();
   if (!status) return MOE_ERR_CUDA;
-  const bool pair = !swiglu && tn == 128 && fp4_pair_for(rows_cap, n_groups);
+  const bool pair = fp4_pair_for(rows_cap, n_groups);
   CUtensorMap ta, ta32, tb, tsa, tsb;
   if ((rc = encode_tmap_u8(&ta, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, TM)) != MOE_OK) return rc;
   if ((rc = encode_tmap_u8(&ta32, aq, 2, (uint64_t)K / 2, (uint64_t)rows_cap, 1, ROW_BYTES, 32)) != MOE_OK) return rc;
-  const uint32_t b_box = swiglu ? 128u : (pair ? (uint32_t)FCfg<128, true>::B_ROWS : (uint32_t)tn);
+  const uint32_t b_box = swiglu ? 128u : (uint32_t)(pair ? tn / 2 : tn);  // weight rows a CTA loads per box
   if ((rc = encode_tmap_u8(&tb, wq, 3, (uint64_t)K / 2, b_rows, (uint64_t)n_groups, ROW_BYTES, b_box)) != MOE_OK)
     return rc;
   if (pair) {  // the scale atoms as rows of 256 bytes: 8 rows (2 KB) per operand and stage
@@ -864,10 +924,15 @@ extern "C" int moe_nvfp4_grouped_gemm(const uint8_t* aq, const uint8_t* asf, con
   if (pair) {
     // every group may end in a partial 256-row tile
     const long long tiles_upper = (rows_cap / FCfg<128, true>::TILE_M + n_groups) * p.n_tiles_n;
-    const long long pairs = tiles_upper < sms / 2 ? tiles_upper : sms / 2;
-    rc = epilogue == MOE_NVFP4_EPI_GELU_FP4
-             ? launch_fp4<EPI_GELU_FP4, 128, true>(ta, ta32, tb, tsa, tsb, p, (int)(2 * pairs), s)
-             : launch_fp4<EPI_BF16, 128, true>(ta, ta32, tb, tsa, tsb, p, (int)(2 * pairs), s);
+    const int grid = (int)(2 * (tiles_upper < sms / 2 ? tiles_upper : sms / 2));
+    if (swiglu)
+      rc = launch_fp4<EPI_SWIGLU_FP4, 256, true>(ta, ta32, tb, tsa, tsb, p, grid, s);
+    else if (epilogue == MOE_NVFP4_EPI_GELU_FP4)
+      rc = tn == 256 ? launch_fp4<EPI_GELU_FP4, 256, true>(ta, ta32, tb, tsa, tsb, p, grid, s)
+                     : launch_fp4<EPI_GELU_FP4, 128, true>(ta, ta32, tb, tsa, tsb, p, grid, s);
+    else
+      rc = tn == 256 ? launch_fp4<EPI_BF16, 256, true>(ta, ta32, tb, tsa, tsb, p, grid, s)
+                     : launch_fp4<EPI_BF16, 128, true>(ta, ta32, tb, tsa, tsb, p, grid, s);
     if (rc != MOE_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }

@@ -162,16 +162,13 @@ def test_quantize_at_exact_ties_divides():
         np.testing.assert_array_equal(sfs[rows[:, j]], s_ref)
 
 
-@pytest.fixture(params=["tn128", "tn256", "pair"])
+@pytest.fixture(params=["tn128", "tn256", "pair128", "pair256"])
 def fp4_tile(request, monkeypatch):
-    """Every FP4 GEMM tile: 128 x 128 (the default at small sizes), 128 x 256 (where N is a multiple
-    of 256) and the CTA pair's 256 x 128 (the default for long groups), each forced."""
-    if request.param == "pair":
-        monkeypatch.setenv("MOE_FP4_TN", "128")
-        monkeypatch.setenv("MOE_FP4_PAIR", "1")
-    else:
-        monkeypatch.setenv("MOE_FP4_TN", request.param[2:])
-        monkeypatch.setenv("MOE_FP4_PAIR", "0")
+    """Every FP4 GEMM tile, each forced: one CTA per 128 x 128 or 128 x 256 tile (256 where N is a
+    multiple of 256, the default for short groups), a CTA pair per 256 x 128 or 256 x 256 tile (the
+    default for long groups)."""
+    monkeypatch.setenv("MOE_FP4_TN", request.param[-3:])
+    monkeypatch.setenv("MOE_FP4_PAIR", "1" if request.param.startswith("pair") else "0")
     return request.param
 
 
@@ -248,9 +245,12 @@ def test_gemm_gelu_fp4_out_matches_oracle(sizes, real_rows, fp4_tile):
     assert n_code <= 1e-3 * total and n_sf <= 1e-3 * total / 16, (n_code, n_sf)
 
 
-def test_gemm_swiglu_fp4_out_matches_oracle():
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_gemm_swiglu_fp4_out_matches_oracle(pair, monkeypatch):
     """The SwiGLU first GEMM: gate and up rows of one quantized W1 [2N, K] side by side in a
-    256-wide tile, silu(g * gate) * (g * up), FP4 out; the same acceptance as the GELU epilogue."""
+    256-wide tile (on a CTA pair: the gate rows in one CTA, the up rows in the other),
+    silu(g * gate) * (g * up), FP4 out; the same acceptance as the GELU epilogue."""
+    monkeypatch.setenv("MOE_FP4_PAIR", pair)
     sizes, N, K = [1, 77, 128, 300], 256, 512
     G = len(sizes)
     off_pad = np.concatenate([[0], np.cumsum([(n + 127) // 128 * 128 for n in sizes])]).astype(np.int32)
