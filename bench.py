@@ -52,9 +52,9 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 DECODE_STEPS_PER_STEP = 10
 
 # DRAM bytes (read + write) of one GEMM1 + GEMM2 launch pair, from one single-pass ncu capture of the
-# full-size layer (profiles/grouped_gemm_prefill_dram.md: the mean of the two timed launch pairs);
-# workloads without a capture of the current kernels report null
-TRAFFIC_PER_LAUNCH_PAIR = {"prefill": ((20.85e9 + 2.14e9 + 12.57e9 + 7.48e9) + (21.05e9 + 2.14e9 + 12.99e9 + 7.48e9)) / 2}
+# full-size layer with the current kernels (profiles/grouped_gemm_prefill_dram.md: 256 x 512 pair tiles,
+# three stages); workloads without a capture of the current kernels report null
+TRAFFIC_PER_LAUNCH_PAIR = {"prefill": 18684339968 + 2137493760 + 14046192128 + 7475533056}
 # Weight-streaming launches read what their tokens touch, which drifts as the bias moves the loads, so the
 # capture gives DRAM bytes over algorithmic bytes at the captured launches (profiles/launches_decode.md),
 # applied to the timed launches' algorithmic bytes

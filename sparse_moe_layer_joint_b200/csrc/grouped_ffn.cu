@@ -35,10 +35,11 @@
 //                 CTAs' barriers, both epilogues release the accumulator on
 //                 the leader.  Per CTA this halves the B operand's shared-
 //                 memory traffic (6-stage ring of 32 KB).
-//   WIDE          pair tiles of 256 x 512 (see Cfg): 25% fewer L2 bytes per FLOP,
-//                 but one accumulator (the epilogue is not overlapped); measured
-//                 no faster than 256 x 256 on B200 at the prefill size, so off by
-//                 default (MOE_GEMM_WIDE=1).
+//   WIDE          pair tiles of 256 x 512 (see Cfg): 25% fewer L2 bytes per FLOP
+//                 and one accumulator, which the epilogue hands back as soon as
+//                 it holds its share as packed bf16 registers (the stores then
+//                 overlap the next tile's MMAs); the default for pair launches
+//                 with the GELU and plain epilogues (MOE_GEMM_WIDE=0: 256 x 256).
 // Ragged groups: a tile's A rows may run past its group (into the next
 // group's rows, or past the tensor where TMA fills zeros); the epilogue writes
 // only the group's own rows.
@@ -69,8 +70,9 @@ constexpr int SWIGLU_OUT = BN / 2;
 // WIDE (pairs only): a tile is 256 x 512, two 256-column halves that share the A stage; each CTA
 // holds 128 A rows and 2 x 128 weight rows per stage, so a K step moves 48 KB per CTA for twice
 // the MMA work of a 256 x 256 tile (32 KB): 25% fewer L2 -> shared-memory bytes per FLOP.  Its
-// 512-column accumulator fills TMEM, so there is one accumulator, drained by eight epilogue warps
-// (two per TMEM lane quarter, one per column half) before the next tile's MMAs start.
+// 512-column accumulator fills TMEM, so there is one accumulator, read by eight epilogue warps (two
+// per TMEM lane quarter, one per column half) into packed bf16 registers; the next tile's MMAs start
+// once every warp holds its share, while the warps store it.
 template <bool PAIR, int ST, bool WIDE = false>
 struct Cfg {
   static_assert(!WIDE || PAIR, "wide tiles are pair tiles");
@@ -515,6 +517,43 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
       const uint32_t taddr =
           tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::TILE_N + half * BN);
       __nv_bfloat16* crow = cbase + (size_t)c_row * p.ldc;
+      if (C::ACC_BUFS == 1 && EPI != EPI_SWIGLU) {
+        // one accumulator (wide tiles): convert this warp's whole share into packed bf16 registers, hand
+        // the accumulator back to the MMA, and only then store, so the next tile's MMAs overlap the stores
+        constexpr int NCH = BN / 32;
+        uint32_t pk[NCH * 16];
+#pragma unroll
+        for (int c16 = 0; c16 < 2 * NCH; ++c16) {  // 16 columns at a time (register pressure)
+          float v[16];
+          tmem_ld16(taddr + c16 * 16, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float a = v[2 * i], b = v[2 * i + 1];
+            if (EPI == EPI_GELU) {
+              a = gelu_tanh_f32(a);
+              b = gelu_tanh_f32(b);
+            }
+            pk[c16 * 8 + i] = pack_bf16x2(a, b);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR)
+            mbar_arrive_cluster(tempty0);
+          else
+            mbar_arrive(&st->tempty[0]);
+        }
+        acc_phase ^= 1u;
+        if (valid) {
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch) {
+            const int col0 = ti.nt * C::TILE_N + half * BN + ch * 32;
+            if (col0 < p.N) store16(reinterpret_cast<uint4*>(crow + col0), pk + ch * 16);
+          }
+        }
+        continue;
+      }
       if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
         for (int ch = 0; ch < SWIGLU_OUT / 32; ++ch) {
@@ -635,20 +674,24 @@ bool choose_pair(long long rows, int groups) {
   return pair;
 }
 
-// Pipeline depth of the pair kernel (stages of 64-deep K slices in flight per CTA).  Six stages hide
-// more load latency and win on short launches.  Launches of several TFLOP run for milliseconds under
-// the board's power cap; there four stages win: with less prefetch the pairs that share A rows or
-// weight tiles stay closer together in K, so more of their loads hit L2 (at 65536 tokens, d 7168,
-// d_ff 2048 the first GEMM reads about 21 GB from DRAM with four stages against about 50 GB with six).
-// MOE_GEMM_STAGES="s1,s2" (each 4 or 6) forces the depth of GEMM1, GEMM2.
+// Pipeline depth of the pair kernel (stages of 64-deep K slices in flight per CTA).  Deeper pipelines
+// hide more load latency and win on short launches.  Launches of several TFLOP run for milliseconds under
+// the board's power cap; there shallower ones win: with less prefetch the pairs that share A rows or
+// weight tiles stay closer together in K, so more of their loads hit L2.  At 65536 tokens, d 7168,
+// d_ff 2048 the first GEMM reads about 21 GB from DRAM with four stages of 256 x 256 tiles against about
+// 50 GB with six, and with 256 x 512 tiles (whose stages hold twice the MMA work) 19 GB with three
+// against 43 GB with four.  256 x 256 tiles: 6 short, 4 long; 256 x 512 tiles: 4 short, 3 long.
+// MOE_GEMM_STAGES="s1,s2" (each 3 .. 6; 3 for wide tiles only) forces the depth of GEMM1, GEMM2.
 constexpr double LONG_LAUNCH_FLOP = 4e12;
 
-int stages_for(bool pair, int which, double flop) {
+int stages_for(bool pair, bool wide, int which, double flop) {
   if (!pair) return 4;
-  int st = flop >= LONG_LAUNCH_FLOP ? 4 : 6;
+  const bool long_launch = flop >= LONG_LAUNCH_FLOP;
+  int st = wide ? (long_launch ? 3 : 4) : (long_launch ? 4 : 6);
   const char* env = getenv("MOE_GEMM_STAGES");
   if (env && env[0] && env[1] == ',' && env[2] && env[3] == '\0') {
     const char c = which == 1 ? env[0] : env[2];
+    if (c == '3') st = 3;  // wide tiles only (others take 4)
     if (c == '4') st = 4;
     if (c == '5') st = 5;
     if (c == '6') st = 6;
@@ -681,9 +724,10 @@ int hints_for() {
   return h;
 }
 
-// Wide 256 x 512 pair tiles (GELU and plain epilogues).  MOE_GEMM_WIDE=0 or =1 forces them off or on.
+// Wide 256 x 512 pair tiles (GELU and plain epilogues; measured 7-10% faster than 256 x 256 at the
+// prefill, skewed and slice sizes).  MOE_GEMM_WIDE=0 or =1 forces them off or on.
 bool wide_for(bool pair, int epi) {
-  bool wide = false;
+  bool wide = true;
   const char* env = getenv("MOE_GEMM_WIDE");
   if (env && env[0] == '1' && env[1] == '\0') wide = true;
   if (env && env[0] == '0' && env[1] == '\0') wide = false;
@@ -714,7 +758,10 @@ int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_
   if (pair) {
     long long pairs = units < sms / 2 ? units : sms / 2;
     if (wide) {
-      if constexpr (EPI != EPI_SWIGLU) return launch_one<EPI, true, 4, true>(a0, a1, b, p, (int)(2 * pairs), s);
+      if constexpr (EPI != EPI_SWIGLU) {
+        if (stages == 3) return launch_one<EPI, true, 3, true>(a0, a1, b, p, (int)(2 * pairs), s);
+        return launch_one<EPI, true, 4, true>(a0, a1, b, p, (int)(2 * pairs), s);
+      }
     }
     if (stages == 6) return launch_one<EPI, true, 6>(a0, a1, b, p, (int)(2 * pairs), s);
     if (stages == 5) return launch_one<EPI, true, 5>(a0, a1, b, p, (int)(2 * pairs), s);
@@ -816,8 +863,8 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
   const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
-  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
-              : run_split<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
+  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, false, 1, 2.0 * flop), sms, tiles_upper, s)
+              : run_split<EPI_GELU>(g1, pair, stages_for(pair, wide_for(pair, EPI_GELU), 1, flop), sms, tiles_upper, s);
   if (rc != MOE_OK) return rc;
 
   GemmSpec g2{};
@@ -835,7 +882,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g2.p.K = d_ff;
   g2.p.n_tiles_n = (d + BN - 1) / BN;
   g2.p.ldc = d;
-  return run_split<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
+  return run_split<EPI_NONE>(g2, pair, stages_for(pair, wide_for(pair, EPI_NONE), 2, flop), sms, tiles_upper, s);
 }
 
 extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const int32_t* row_token,
@@ -914,8 +961,8 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
   const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
-  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, 1, 2.0 * flop), sms, tiles_upper, s)
-              : run_split<EPI_GELU>(g1, pair, stages_for(pair, 1, flop), sms, tiles_upper, s);
+  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, false, 1, 2.0 * flop), sms, tiles_upper, s)
+              : run_split<EPI_GELU>(g1, pair, stages_for(pair, wide_for(pair, EPI_GELU), 1, flop), sms, tiles_upper, s);
   if (rc != MOE_OK) return rc;
 
   // GEMM2: all A rows from H (map 0); routed outputs to y_perm, shared outputs to y_shared
@@ -937,5 +984,5 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g2.p.K = d_ff;
   g2.p.n_tiles_n = (d + BN - 1) / BN;
   g2.p.ldc = d;
-  return run_split<EPI_NONE>(g2, pair, stages_for(pair, 2, flop), sms, tiles_upper, s);
+  return run_split<EPI_NONE>(g2, pair, stages_for(pair, wide_for(pair, EPI_NONE), 2, flop), sms, tiles_upper, s);
 }

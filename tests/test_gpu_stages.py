@@ -221,20 +221,22 @@ def _ffn_weights(E, d, f, seed):
     return w1, w2
 
 
-@pytest.fixture(params=["pair", "pair4", "wide", "nmajor", "tails", "single"])
+@pytest.fixture(params=["pair", "pair4", "wide", "wide3", "nmajor", "tails", "single"])
 def gemm_variant(request, monkeypatch):
-    """Every grouped-GEMM kernel: CTA pairs with six pipeline stages (short launches), with four
-    (long launches), pairs on 256 x 512 tiles (GELU and plain epilogues; SwiGLU launches keep
-    256-wide tiles), pairs walking small groups column-tile-major, pairs on each group's whole 256-row
-    blocks followed by single CTAs on the rows past them, and single CTAs."""
+    """Every grouped-GEMM kernel: CTA pairs on 256 x 256 tiles with six pipeline stages (short
+    launches) and with four (long launches), pairs on 256 x 512 tiles with four stages (the default for
+    pair launches with the GELU and plain epilogues; SwiGLU launches keep 256-wide tiles) and with
+    three, pairs walking small groups
+    column-tile-major, pairs on each group's whole 256-row blocks followed by single CTAs on the rows
+    past them, and single CTAs."""
     monkeypatch.setenv("MOE_GEMM_NMAJOR", "4" if request.param == "nmajor" else "0")
     monkeypatch.setenv("MOE_GEMM_TAILS", "1" if request.param == "tails" else "0")
     monkeypatch.setenv("MOE_GEMM_CTA", "1" if request.param == "single" else "2")
-    if request.param == "pair4":
-        monkeypatch.setenv("MOE_GEMM_STAGES", "4,4")
+    if request.param in ("pair4", "wide3"):
+        monkeypatch.setenv("MOE_GEMM_STAGES", "4,4" if request.param == "pair4" else "3,3")
     else:
         monkeypatch.delenv("MOE_GEMM_STAGES", raising=False)
-    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if request.param == "wide" else "0")
+    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if request.param.startswith("wide") else "0")
     return request.param
 
 
