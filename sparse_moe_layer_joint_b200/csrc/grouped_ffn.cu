@@ -40,6 +40,11 @@
 //                 it holds its share as packed bf16 registers (the stores then
 //                 overlap the next tile's MMAs); the default for pair launches
 //                 with the GELU and plain epilogues (MOE_GEMM_WIDE=0: 256 x 256).
+//   half tiles    (pairs, GELU and plain epilogues, groups of at most 1024 rows
+//                 on average) a group's last row tile with at most 128 rows runs
+//                 as an M = 128 pair MMA: 64 rows a CTA, whose 64 x 256 result
+//                 TMEM holds folded (lanes 0-63 the first 128 columns, lanes
+//                 64-127 the other 128), at half the MMA work.
 // Ragged groups: a tile's A rows may run past its group (into the next
 // group's rows, or past the tensor where TMA fills zeros); the epilogue writes
 // only the group's own rows.
@@ -48,6 +53,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
+
+#include <type_traits>
 
 #include "moe.h"
 #include "moe_internal.h"
@@ -121,6 +128,8 @@ struct Params {
   int tail_unit;
   int hints;  // L2 policies: HINT_B_KEEP weight tiles evict_last, HINT_C_STREAM outputs evict_first,
               // HINT_A_STREAM A tiles evict_first
+  int half_tiles;  // pair kernels, GELU / plain epilogues, tiled A loads: a group's last row tile with at
+                   // most 128 rows runs as an M = 128 pair MMA (64 rows a CTA) at half the MMA work
   uint64_t timeout_ns;
   unsigned int* status;
 };
@@ -201,6 +210,11 @@ __device__ __forceinline__ int group_row_tiles(const Params& p, int rows) {
 struct TileInfo {
   int g, m, nt;
 };
+
+// Whether a tile runs as a half (M = 128) pair tile: its group's rows end within its first 128.
+__device__ __forceinline__ bool half_tile(const Params& p, const Group& gr, const TileInfo& ti) {
+  return p.half_tiles != 0 && gr.rows - ti.m * 256 <= 128;
+}
 
 // A group's tiles are the tile numbers [prefix[g] * n_tiles_n, prefix[g + 1] * n_tiles_n).  Within a
 // group they run row-tile-major (the column tiles of one row block together) or, for groups of at most
@@ -340,7 +354,9 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
       const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n, p.n_major_rows);
       const Group gr = group_info(p, st->gt, ti.g);
       const CUtensorMap* am = gr.a_map ? &tmA1 : &tmA0;
-      const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * C::A_ROWS;
+      const bool half = half_tile(p, gr, ti);
+      // a half tile's CTA loads its usual 128-row box from its 64-row offset and uses the first 64 rows
+      const int a_row = gr.a_base + ti.m * C::TILE_M + (int)rank * (half ? C::A_ROWS / 2 : C::A_ROWS);
       // weight rows of this CTA's share of the tile's 256 columns; for SwiGLU the first 128
       // columns are gate rows and the other 128 the matching up rows
       // (a wide tile's second half: b_row + 256)
@@ -426,13 +442,20 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
   } else if (warp == 1) {
     // ================= MMA issuer (the pair's leader) =================
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc_bf16(C::TILE_M, BN);  // one MMA per 256-column half
+      constexpr uint32_t idesc_full = make_idesc_bf16(C::TILE_M, BN);  // one MMA per 256-column half
+      constexpr uint32_t idesc_half = make_idesc_bf16(C::TILE_M / 2, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
+        const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n, p.n_major_rows);
+        const bool half = half_tile(p, group_info(p, st->gt, ti.g), ti);
+        // an M = 128 pair MMA folds each CTA's 64 x 256 result into 128 TMEM columns: lanes 0-63 hold
+        // columns 0-127, lanes 64-127 columns 128-255
+        const uint32_t idesc = half ? idesc_half : idesc_full;
+        const uint32_t h_cols = half ? BN / 2 : BN;
         if (!mbar_wait(&st->tempty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::TILE_N);
@@ -451,9 +474,9 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
             for (int h = 0; h < C::NH; ++h) {
               const uint64_t bd = make_desc_sw128(b_addr + h * C::B_HALF_BYTES + k * 32);
               if (PAIR)
-                mma_bf16_ss_pair(d_tmem + h * BN, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                mma_bf16_ss_pair(d_tmem + h * h_cols, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
               else
-                mma_bf16_ss(d_tmem + h * BN, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                mma_bf16_ss(d_tmem + h * BN, ad, bd, idesc_full, (kb | k) != 0 ? 1u : 0u);
             }
           }
           if (PAIR)
@@ -507,7 +530,12 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
     for (int tile = unit; tile < total_tiles; tile += n_units) {
       const TileInfo ti = tile_info(tile, st->gt.prefix, G, p.n_tiles_n, p.n_major_rows);
       const Group gr = group_info(p, st->gt, ti.g);
-      const int r = ti.m * C::TILE_M + row_in_tile;
+      // a half tile (M = 128 pair MMA): this CTA's 64 rows, lanes 0-63 holding the first 128 of an MMA's
+      // 256 columns and lanes 64-127 the other 128, in 128 TMEM columns per MMA
+      const bool htile = PAIR && half_tile(p, gr, ti);
+      const int r = ti.m * C::TILE_M + (htile ? (int)rank * 64 + (quarter & 1) * 32 + lane : row_in_tile);
+      const int col_base = ti.nt * C::TILE_N + half * BN + (htile ? (quarter >> 1) * (BN / 2) : 0);
+      const int n_ch = htile ? BN / 64 : BN / 32;  // 32-column chunks this warp drains
       const int c_row = gr.c_base + r;
       __nv_bfloat16* cbase = gr.c_sel ? p.C1 : p.C0;
       const int climit = gr.c_sel ? p.c1_limit : p.c0_limit;
@@ -515,43 +543,50 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
       if (!mbar_wait(&st->tfull[acc], acc_phase, p.timeout_ns, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr =
-          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::TILE_N + half * BN);
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::TILE_N + half * (htile ? BN / 2 : BN));
       __nv_bfloat16* crow = cbase + (size_t)c_row * p.ldc;
       if (C::ACC_BUFS == 1 && EPI != EPI_SWIGLU) {
         // one accumulator (wide tiles): convert this warp's whole share into packed bf16 registers, hand
         // the accumulator back to the MMA, and only then store, so the next tile's MMAs overlap the stores
-        constexpr int NCH = BN / 32;
-        uint32_t pk[NCH * 16];
+        // (a half tile's share is half as wide; each width has its own fully unrolled copy)
+        auto drain = [&](auto n_chunks) {
+          constexpr int NCH = decltype(n_chunks)::value;
+          uint32_t pk[NCH * 16];
 #pragma unroll
-        for (int c16 = 0; c16 < 2 * NCH; ++c16) {  // 16 columns at a time (register pressure)
-          float v[16];
-          tmem_ld16(taddr + c16 * 16, v);
+          for (int c16 = 0; c16 < 2 * NCH; ++c16) {  // 16 columns at a time (register pressure)
+            float v[16];
+            tmem_ld16(taddr + c16 * 16, v);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float a = v[2 * i], b = v[2 * i + 1];
-            if (EPI == EPI_GELU) {
-              a = gelu_tanh_f32(a);
-              b = gelu_tanh_f32(b);
+            for (int i = 0; i < 8; ++i) {
+              float a = v[2 * i], b = v[2 * i + 1];
+              if (EPI == EPI_GELU) {
+                a = gelu_tanh_f32(a);
+                b = gelu_tanh_f32(b);
+              }
+              pk[c16 * 8 + i] = pack_bf16x2(a, b);
             }
-            pk[c16 * 8 + i] = pack_bf16x2(a, b);
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (PAIR)
-            mbar_arrive_cluster(tempty0);
-          else
-            mbar_arrive(&st->tempty[0]);
-        }
-        acc_phase ^= 1u;
-        if (valid) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (PAIR)
+              mbar_arrive_cluster(tempty0);
+            else
+              mbar_arrive(&st->tempty[0]);
+          }
+          if (valid) {
 #pragma unroll
-          for (int ch = 0; ch < NCH; ++ch) {
-            const int col0 = ti.nt * C::TILE_N + half * BN + ch * 32;
-            if (col0 < p.N) store16(reinterpret_cast<uint4*>(crow + col0), pk + ch * 16);
+            for (int ch = 0; ch < NCH; ++ch) {
+              const int col0 = col_base + ch * 32;
+              if (col0 < p.N) store16(reinterpret_cast<uint4*>(crow + col0), pk + ch * 16);
+            }
           }
-        }
+        };
+        if (htile)
+          drain(std::integral_constant<int, BN / 64>{});
+        else
+          drain(std::integral_constant<int, BN / 32>{});
+        acc_phase ^= 1u;
         continue;
       }
       if (EPI == EPI_SWIGLU) {
@@ -572,8 +607,8 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
         }
       }
 #pragma unroll 1
-      for (int ch = 0; ch < (EPI == EPI_SWIGLU ? 0 : BN / 32); ++ch) {
-        const int col0 = ti.nt * C::TILE_N + half * BN + ch * 32;
+      for (int ch = 0; ch < (EPI == EPI_SWIGLU ? 0 : n_ch); ++ch) {
+        const int col0 = col_base + ch * 32;
         if (col0 >= p.N) break;  // same for the whole warp
         float v[32];
         tmem_ld32(taddr + ch * 32, v);
@@ -734,6 +769,23 @@ bool wide_for(bool pair, int epi) {
   return wide && pair && epi != EPI_SWIGLU;
 }
 
+// Half (M = 128) pair tiles for groups' last row tiles of at most 128 rows: pair launches with the GELU
+// or plain epilogue and tiled A loads, where groups average at most 1024 rows.  A group's last 256-row
+// tile is on average half padding, so they save up to half of that: measured 3.5% on the expert pair at
+// the skewed workload (about 500 rows a group, 20% padding).  With long groups the saving is small and
+// the shorter tiles pull the CTA pairs that share A blocks and weight tiles apart in K: at the prefill
+// size (about 2000 rows a group) GEMM1 then read 34 GB from DRAM instead of 18 and the pair ran 4%
+// slower.  MOE_GEMM_HALF=1 / =0 forces them on / off.
+bool half_tiles_for(bool pair, int epi, const Params& p) {
+  const long long groups = (long long)p.G_r + p.G_s;
+  const long long rows = (long long)p.routed_rows * (p.G_r > 0 ? 1 : 0) + (long long)p.G_s * p.shared_rows;
+  bool on = groups > 0 && rows <= 1024LL * groups;
+  const char* env = getenv("MOE_GEMM_HALF");
+  if (env && env[0] == '0' && env[1] == '\0') on = false;
+  if (env && env[0] == '1' && env[1] == '\0') on = true;
+  return on && pair && epi != EPI_SWIGLU && p.gather_rows == nullptr && p.tail_mode == TAIL_ALL;
+}
+
 template <int EPI>
 int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_upper, cudaStream_t s) {
   // rows per weight box: a pair CTA loads 128 (per column half); a single CTA 256, or 2 x 128 (gate,
@@ -743,6 +795,7 @@ int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_
   const bool wide = wide_for(pair, EPI);
   Params p = g.p;
   if (wide) p.n_tiles_n = (p.N + Cfg<true, 4, true>::TILE_N - 1) / Cfg<true, 4, true>::TILE_N;
+  p.half_tiles = half_tiles_for(pair, EPI, p) ? 1 : 0;
   CUtensorMap a0, a1, b;
   int rc;
   const uint64_t K = (uint64_t)g.p.K, N = g.b_rows ? g.b_rows : (uint64_t)g.p.N;

@@ -221,12 +221,12 @@ def _ffn_weights(E, d, f, seed):
     return w1, w2
 
 
-@pytest.fixture(params=["pair", "pair4", "wide", "wide3", "nmajor", "tails", "single"])
+@pytest.fixture(params=["pair", "pair4", "wide", "wide3", "nohalf", "nmajor", "tails", "single"])
 def gemm_variant(request, monkeypatch):
     """Every grouped-GEMM kernel: CTA pairs on 256 x 256 tiles with six pipeline stages (short
     launches) and with four (long launches), pairs on 256 x 512 tiles with four stages (the default for
     pair launches with the GELU and plain epilogues; SwiGLU launches keep 256-wide tiles) and with
-    three, pairs walking small groups
+    three, the wide pairs without half (M = 128) tiles for the groups' last rows, pairs walking small groups
     column-tile-major, pairs on each group's whole 256-row blocks followed by single CTAs on the rows
     past them, and single CTAs."""
     monkeypatch.setenv("MOE_GEMM_NMAJOR", "4" if request.param == "nmajor" else "0")
@@ -236,7 +236,8 @@ def gemm_variant(request, monkeypatch):
         monkeypatch.setenv("MOE_GEMM_STAGES", "4,4" if request.param == "pair4" else "3,3")
     else:
         monkeypatch.delenv("MOE_GEMM_STAGES", raising=False)
-    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if request.param.startswith("wide") else "0")
+    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if request.param.startswith("wide") or request.param == "nohalf" else "0")
+    monkeypatch.setenv("MOE_GEMM_HALF", "0" if request.param == "nohalf" else "1")
     return request.param
 
 
