@@ -146,23 +146,32 @@ __global__ void __launch_bounds__(THREADS) rank_kernel(const int32_t* __restrict
   }
 }
 
-// x_perm[token_row[t][j]] = x[t] for every slot j: unit u = (token, slice of
-// 256 16-byte vectors); each thread reads one vector and writes it k times.
+// x_perm[token_row[t][j]] = x[t] for every slot j: a block copies one token at a time; each thread
+// loads up to COPY_VPT of the row's 16-byte vectors (v, v + THREADS, ...) before writing each of them k
+// times, so several loads are in flight per thread.
+constexpr int COPY_VPT = 4;
+
 __global__ void __launch_bounds__(THREADS) copy_rows_kernel(const uint4* __restrict__ x,
                                                             const int32_t* __restrict__ token_row, int T, int d_vec,
                                                             int k, int n_rows, uint4* __restrict__ x_perm) {
-  const int n_slices = (d_vec + THREADS - 1) / THREADS;
-  const long long units = (long long)T * n_slices;
-  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-    const int t = (int)(u / n_slices);
-    const int v = (int)(u - (long long)t * n_slices) * THREADS + threadIdx.x;
-    if (v >= d_vec) continue;
-    const uint4 val = __ldg(x + (size_t)t * d_vec + v);
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    int rows[MOE_MAX_TOP_K];
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
-      if (j < k) {
-        const int r = __ldg(token_row + (size_t)t * k + j);
-        if (r >= 0 && r < n_rows) x_perm[(size_t)r * d_vec + v] = val;
+    for (int j = 0; j < MOE_MAX_TOP_K; ++j) rows[j] = j < k ? __ldg(token_row + (size_t)t * k + j) : -1;
+    const uint4* src = x + (size_t)t * d_vec;
+    for (int v0 = threadIdx.x; v0 < d_vec; v0 += THREADS * COPY_VPT) {
+      uint4 val[COPY_VPT];
+#pragma unroll
+      for (int i = 0; i < COPY_VPT; ++i)
+        if (v0 + i * THREADS < d_vec) val[i] = __ldg(src + v0 + i * THREADS);
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+        const int r = rows[j];
+        if (r < 0 || r >= n_rows) continue;
+        uint4* dst = x_perm + (size_t)r * d_vec + v0;
+#pragma unroll
+        for (int i = 0; i < COPY_VPT; ++i)
+          if (v0 + i * THREADS < d_vec) dst[i * THREADS] = val[i];
       }
     }
   }
@@ -186,8 +195,7 @@ static int launch_permute(const moe_bf16* x, const int32_t* topk_idx, const int3
                                            token_row);
   if (x_perm == nullptr) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;  // indices only
   const int d_vec = d / 8;
-  const long long units = (long long)T * ((d_vec + THREADS - 1) / THREADS);
-  const int grid = (int)(units < (long long)sms * 8 ? units : (long long)sms * 8);
+  const int grid = (int)((long long)T < (long long)sms * 8 ? T : (long long)sms * 8);  // one token per block at a time
   copy_rows_kernel<<<grid, THREADS, 0, s>>>(reinterpret_cast<const uint4*>(x), token_row, T, d_vec, top_k,
                                             T * top_k, reinterpret_cast<uint4*>(x_perm));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
