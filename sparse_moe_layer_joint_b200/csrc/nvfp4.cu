@@ -683,8 +683,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
+        // the peer's hand-back orders no memory writes, so it need not wait for this warp's stores of
+        // the previous tile to land (a releasing arrive there cost 8% on a prefill-shaped slice)
         if (PAIR)
-          mbar_arrive_cluster(acc == 0 ? tempty0 : tempty1);
+          mbar_arrive_cluster_relaxed(acc == 0 ? tempty0 : tempty1);
         else
           mbar_arrive(&st->tempty[acc]);
       }
@@ -776,8 +778,8 @@ int launch_fp4(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap
 
 // Pair tiles (256 x TN), an option for groups long enough to fill them (MOE_FP4_PAIR=1; =0 or unset: off).
 // They move 30% fewer bytes per MMA into each SM than single-CTA tiles of the same width but were measured
-// slower on a prefill-shaped slice (256 x 256 pairs 1.12 ms against 1.03 ms per GEMM pair for 128 x 256
-// single-CTA tiles; 256 x 128 pairs 1.54 against 1.49 for 128 x 128).
+// no faster on a prefill-shaped slice (256 x 256 pairs 1.04 ms against 1.03 ms per GEMM pair for 128 x 256
+// single-CTA tiles; 256 x 128 pairs 1.53 against 1.49 for 128 x 128).
 bool fp4_pair_for(long long rows_cap, int n_groups) {
   bool on = false;
   (void)rows_cap;

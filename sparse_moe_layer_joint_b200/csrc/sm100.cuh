@@ -402,6 +402,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// The same without release semantics: for signals that order no memory writes, such as an epilogue warp
+// handing its TMEM accumulator back (its tcgen05.ld have completed at tcgen05.wait::ld), so the arrive does
+// not wait for the warp's earlier global stores to land.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // The pair's leader (rank 0) holds the barriers its MMA waits on; clearing the
 // rank bit of a CTA-local shared address gives the same offset in the leader.
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;
