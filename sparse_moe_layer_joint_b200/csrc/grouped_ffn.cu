@@ -35,11 +35,12 @@
 //                 CTAs' barriers, both epilogues release the accumulator on
 //                 the leader.  Per CTA this halves the B operand's shared-
 //                 memory traffic (6-stage ring of 32 KB).
-//   WIDE          pair tiles of 256 x 512 (see Cfg): 25% fewer L2 bytes per FLOP
-//                 and one accumulator, which the epilogue hands back as soon as
-//                 it holds its share as packed bf16 registers (the stores then
-//                 overlap the next tile's MMAs); the default for pair launches
-//                 with the GELU and plain epilogues (MOE_GEMM_WIDE=0: 256 x 256).
+//   WIDE          pair tiles of 256 x 512 accumulator columns (see Cfg): 25% fewer
+//                 L2 bytes per FLOP and one accumulator, which the epilogue hands
+//                 back as soon as it holds its share as packed bf16 registers
+//                 (the stores then overlap the next tile's MMAs); SwiGLU tiles
+//                 hold 256 gate and the 256 matching up columns; the default for
+//                 pair launches (MOE_GEMM_WIDE=0: 256 x 256).
 //   half tiles    (pairs, GELU and plain epilogues, groups of at most 1024 rows
 //                 on average) a group's last row tile with at most 128 rows runs
 //                 as an M = 128 pair MMA: 64 rows a CTA, whose 64 x 256 result
@@ -282,7 +283,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmB, const Params p) {
   using C = Cfg<PAIR, ST, WIDE>;
-  static_assert(!WIDE || EPI != EPI_SWIGLU, "SwiGLU tiles pair gate and up halves within 256 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smemA = smem;
@@ -360,8 +360,12 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
       // weight rows of this CTA's share of the tile's 256 columns; for SwiGLU the first 128
       // columns are gate rows and the other 128 the matching up rows
       // (a wide tile's second half: b_row + 256)
-      const int b_row = EPI == EPI_SWIGLU ? (rank == 0u ? ti.nt * SWIGLU_OUT : p.b_up_row + ti.nt * SWIGLU_OUT)
+      // (SwiGLU, wide: the first half's rows are gate rows, the second half's the matching up rows, so a
+      // tile computes 256 outputs; SwiGLU on 256-column pairs: one CTA loads gate rows, the other up rows)
+      const int b_row = EPI == EPI_SWIGLU ? (C::NH == 2 ? ti.nt * BN + (int)rank * C::B_HALF_ROWS
+                                                        : (rank == 0u ? ti.nt * SWIGLU_OUT : p.b_up_row + ti.nt * SWIGLU_OUT))
                                           : ti.nt * C::TILE_N + (int)rank * C::B_HALF_ROWS;
+      const int b_half_step = EPI == EPI_SWIGLU ? p.b_up_row : BN;  // weight rows between the two halves
       const bool gather = gathering && ti.g < p.G_r;
       int src[4] = {0, 0, 0, 0};  // this lane's four source rows (rows past the group: row 0, masked later)
       if (gather) {
@@ -395,7 +399,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
 #pragma unroll
           for (int h = 0; h < C::NH; ++h) {
             if (EPI == EPI_SWIGLU && !PAIR && h == 0) tma_prefetch_l2_3d(&tmB, kp, p.b_up_row + ti.nt * SWIGLU_OUT, ti.g);
-            tma_prefetch_l2_3d(&tmB, kp, b_row + h * BN, ti.g);
+            tma_prefetch_l2_3d(&tmB, kp, b_row + h * b_half_step, ti.g);
           }
         }
         if (lane == 0) {
@@ -410,9 +414,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
             for (int h = 0; h < C::NH; ++h) {
               uint8_t* b_dst = smemB + stage * C::B_BYTES + h * C::B_HALF_BYTES;
               if (p.hints & HINT_B_KEEP)
-                tma_load_3d_pair_hint(b_dst, &tmB, &st->full[stage], kb * BK, b_row + h * BN, ti.g, pol_last);
+                tma_load_3d_pair_hint(b_dst, &tmB, &st->full[stage], kb * BK, b_row + h * b_half_step, ti.g,
+                                      pol_last);
               else
-                tma_load_3d_pair(b_dst, &tmB, &st->full[stage], kb * BK, b_row + h * BN, ti.g);
+                tma_load_3d_pair(b_dst, &tmB, &st->full[stage], kb * BK, b_row + h * b_half_step, ti.g);
             }
           } else {
             if (!gather) tma_load_2d(a_dst, am, &st->full[stage], kb * BK, a_row);
@@ -545,6 +550,40 @@ __global__ void __launch_bounds__(Cfg<PAIR, ST, WIDE>::THREADS, 1)
       const uint32_t taddr =
           tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::TILE_N + half * (htile ? BN / 2 : BN));
       __nv_bfloat16* crow = cbase + (size_t)c_row * p.ldc;
+      if (C::ACC_BUFS == 1 && EPI == EPI_SWIGLU) {
+        // wide SwiGLU tile: accumulator columns 0-255 hold the gate and 256-511 the matching up columns of
+        // the tile's 256 outputs; this warp forms outputs half * 128 .. + 127 as packed bf16 registers, hands
+        // the accumulator back, then stores
+        constexpr int NCH = SWIGLU_OUT / 32;
+        uint32_t pk[NCH * 16];
+        const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * SWIGLU_OUT);
+#pragma unroll
+        for (int c16 = 0; c16 < 2 * NCH; ++c16) {  // 16 outputs at a time (register pressure)
+          float g[16], u[16];
+          tmem_ld16(tbase + c16 * 16, g);
+          tmem_ld16(tbase + BN + c16 * 16, u);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[c16 * 8 + i] = pack_bf16x2(silu_f32(g[2 * i]) * u[2 * i], silu_f32(g[2 * i + 1]) * u[2 * i + 1]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR)
+            mbar_arrive_cluster(tempty0);
+          else
+            mbar_arrive(&st->tempty[0]);
+        }
+        acc_phase ^= 1u;
+        if (valid) {
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch) {
+            const int col0 = ti.nt * BN + half * SWIGLU_OUT + ch * 32;
+            if (col0 < p.N) store16(reinterpret_cast<uint4*>(crow + col0), pk + ch * 16);
+          }
+        }
+        continue;
+      }
       if (C::ACC_BUFS == 1 && EPI != EPI_SWIGLU) {
         // one accumulator (wide tiles): convert this warp's whole share into packed bf16 registers, hand
         // the accumulator back to the MMA, and only then store, so the next tile's MMAs overlap the stores
@@ -759,14 +798,16 @@ int hints_for() {
   return h;
 }
 
-// Wide 256 x 512 pair tiles (GELU and plain epilogues; measured 7-10% faster than 256 x 256 at the
-// prefill, skewed and slice sizes).  MOE_GEMM_WIDE=0 or =1 forces them off or on.
+// Wide pair tiles: 256 x 512 (GELU and plain epilogues; measured 7-10% faster than 256 x 256 at the
+// prefill, skewed and slice sizes), or 256 x 256 outputs from 256 gate and 256 up accumulator columns
+// (SwiGLU).  MOE_GEMM_WIDE=0 or =1 forces them off or on.
 bool wide_for(bool pair, int epi) {
   bool wide = true;
   const char* env = getenv("MOE_GEMM_WIDE");
   if (env && env[0] == '1' && env[1] == '\0') wide = true;
   if (env && env[0] == '0' && env[1] == '\0') wide = false;
-  return wide && pair && epi != EPI_SWIGLU;
+  (void)epi;
+  return wide && pair;
 }
 
 // Half (M = 128) pair tiles for groups' last row tiles of at most 128 rows: pair launches with the GELU
@@ -794,7 +835,9 @@ int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_
                                                      : (uint32_t)Cfg<false, 4>::B_HALF_ROWS;
   const bool wide = wide_for(pair, EPI);
   Params p = g.p;
-  if (wide) p.n_tiles_n = (p.N + Cfg<true, 4, true>::TILE_N - 1) / Cfg<true, 4, true>::TILE_N;
+  if (wide)  // 512 output columns a tile; SwiGLU: 256 outputs (256 gate + 256 up accumulator columns)
+    p.n_tiles_n = EPI == EPI_SWIGLU ? (p.N + BN - 1) / BN
+                                    : (p.N + Cfg<true, 4, true>::TILE_N - 1) / Cfg<true, 4, true>::TILE_N;
   p.half_tiles = half_tiles_for(pair, EPI, p) ? 1 : 0;
   CUtensorMap a0, a1, b;
   int rc;
@@ -811,10 +854,8 @@ int run_gemm(const GemmSpec& g, bool pair, int stages, int sms, long long tiles_
   if (pair) {
     long long pairs = units < sms / 2 ? units : sms / 2;
     if (wide) {
-      if constexpr (EPI != EPI_SWIGLU) {
-        if (stages == 3) return launch_one<EPI, true, 3, true>(a0, a1, b, p, (int)(2 * pairs), s);
-        return launch_one<EPI, true, 4, true>(a0, a1, b, p, (int)(2 * pairs), s);
-      }
+      if (stages == 3) return launch_one<EPI, true, 3, true>(a0, a1, b, p, (int)(2 * pairs), s);
+      return launch_one<EPI, true, 4, true>(a0, a1, b, p, (int)(2 * pairs), s);
     }
     if (stages == 6) return launch_one<EPI, true, 6>(a0, a1, b, p, (int)(2 * pairs), s);
     if (stages == 5) return launch_one<EPI, true, 5>(a0, a1, b, p, (int)(2 * pairs), s);
@@ -916,7 +957,7 @@ extern "C" int moe_grouped_ffn(const moe_bf16* rows, const int32_t* offsets, int
   g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
   const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
-  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, false, 1, 2.0 * flop), sms, tiles_upper, s)
+  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, wide_for(pair, EPI_SWIGLU), 1, 2.0 * flop), sms, tiles_upper, s)
               : run_split<EPI_GELU>(g1, pair, stages_for(pair, wide_for(pair, EPI_GELU), 1, flop), sms, tiles_upper, s);
   if (rc != MOE_OK) return rc;
 
@@ -1014,7 +1055,7 @@ extern "C" int moe_experts_ffn(const moe_bf16* x, const moe_bf16* x_perm, const 
   g1.p.b_up_row = d_ff;
   g1.p.ldc = d_ff;
   const double flop = 2.0 * (double)h_rows * d * d_ff;  // GEMM2; GEMM1 has w1_rows / d_ff times as many
-  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, false, 1, 2.0 * flop), sms, tiles_upper, s)
+  rc = swiglu ? run_split<EPI_SWIGLU>(g1, pair, stages_for(pair, wide_for(pair, EPI_SWIGLU), 1, 2.0 * flop), sms, tiles_upper, s)
               : run_split<EPI_GELU>(g1, pair, stages_for(pair, wide_for(pair, EPI_GELU), 1, flop), sms, tiles_upper, s);
   if (rc != MOE_OK) return rc;
 
