@@ -54,7 +54,7 @@ DECODE_STEPS_PER_STEP = 10
 # DRAM bytes (read + write) of one GEMM1 + GEMM2 launch pair, from one single-pass ncu capture of the
 # full-size layer with the current kernels (profiles/grouped_gemm_prefill_dram.md: 256 x 512 pair tiles,
 # three stages); workloads without a capture of the current kernels report null
-TRAFFIC_PER_LAUNCH_PAIR = {"prefill": 18684339968 + 2137493760 + 14046192128 + 7475533056}
+TRAFFIC_PER_LAUNCH_PAIR = {"prefill": 18729761792 + 2210518528 + 13690001152 + 7472903168}
 # Weight-streaming launches read what their tokens touch, which drifts as the bias moves the loads, so the
 # capture gives DRAM bytes over algorithmic bytes at the captured launches (profiles/launches_decode.md),
 # applied to the timed launches' algorithmic bytes
