@@ -197,7 +197,7 @@ def run_ours(args, w, rank, world, local_rank, want_cpu=False):
     ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ffn_ev)
     eager_ms = None
     if args.graph and world == 1:
-        # the whole step (its 9 launches) captured once as a CUDA graph and replayed: for the
+        # the whole step (its 7-9 launches) captured once as a CUDA graph and replayed: for the
         # latency-bound sizes the host's launch cost, not the GPU, sets the eager step time
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
@@ -894,7 +894,7 @@ def main():
             dargs = copy.copy(args)
             dargs.steps = args.steps * DECODE_STEPS_PER_STEP
             dargs.log_balance = None
-            dargs.graph = world == 1  # a 2 ms step of 9 launches: replayed as one CUDA graph
+            dargs.graph = world == 1  # a 2 ms step of 7 launches: replayed as one CUDA graph
             dec = run_ours(dargs, mi.WORKLOADS["decode"], rank, world, local_rank)
             return {k: dec[k] for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                                         "config", "clocks", "e2e", "gpu_launches", "roofline")}

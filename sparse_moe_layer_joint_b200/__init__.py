@@ -513,10 +513,12 @@ class MoELayer:
     # kernels of libmoe launched by one forward + bias update
     def launches_per_step(self) -> int:
         """libmoe kernels one forward + bias update launches."""
-        if self.nvfp4:  # permute (indices) 3, FP4 dispatch 1, FP4 GEMMs 2, shared bf16 GEMMs 2
-            return 1 + 3 + 1 + 2 + 2 + 1 + 1
+        one_chunk = self.shape.T <= 256 and os.environ.get("MOE_PERMUTE_ONE_CHUNK") != "0"
+        indices = 1 if one_chunk else 3  # the dispatch's index launches (one CTA when one chunk holds every token)
+        if self.nvfp4:  # permute (indices), FP4 dispatch 1, FP4 GEMMs 2, shared bf16 GEMMs 2
+            return 1 + indices + 1 + 2 + 2 + 1 + 1
         experts = 2 if self.fused_experts else 4
-        permute = 3 if self.gather_rows else 4
+        permute = indices + (0 if self.gather_rows else 1)
         return 1 + permute + experts + 1 + 1
 
     def balance(self, stream=None) -> dict:

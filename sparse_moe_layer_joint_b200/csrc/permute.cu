@@ -2,7 +2,8 @@
 // one expert in increasing token order ("Inkling, Dissected" §02: each token
 // goes to exactly its k routed experts; §02d: tokens queue per expert).
 //
-// Four launches, all deterministic (no atomics decide a position):
+// Four launches (two when every token fits one chunk: one_chunk_kernel does 1-3),
+// all deterministic (no atomics decide a position):
 //   1. chunk_hist   one CTA per 256-token chunk: hist[c][e] = picks of e in chunk c
 //   2. chunk_scan   one CTA: offsets[e] = exclusive scan over experts of the
 //                   rows each expert serves, min(picks, capacity);
@@ -21,6 +22,7 @@
 //                   token's k rows.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "moe.h"
 #include "moe_internal.h"
@@ -146,6 +148,91 @@ __global__ void __launch_bounds__(THREADS) rank_kernel(const int32_t* __restrict
   }
 }
 
+// Launches 1-3 in one CTA when all tokens fit one chunk (T <= 256): the histogram is the popcount of the
+// rank masks, the scan runs over the experts, and the ranks follow with a base of zero, so every output
+// equals the three launches' bit for bit.
+__global__ void __launch_bounds__(THREADS) one_chunk_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
+                                                            int n_routed, int capacity,
+                                                            const int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ row_token,
+                                                            int32_t* __restrict__ token_row, unsigned int* status) {
+  __shared__ uint32_t mask[WARPS][MOE_MAX_ROUTED];
+  __shared__ int pre[WARPS][MOE_MAX_ROUTED];
+  __shared__ int off[MOE_MAX_ROUTED];
+  __shared__ int warp_sum[WARPS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < WARPS * MOE_MAX_ROUTED; i += THREADS) (&mask[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = threadIdx.x;  // one token per thread
+  const bool valid = t < T;
+  int ex[MOE_MAX_TOP_K];
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+    ex[j] = -1;
+    if (j < k && valid) {
+      const int e = topk_idx[(size_t)t * k + j];
+      if (e >= 0 && e < n_routed) {
+        ex[j] = e;
+        atomicOr(&mask[warp][e], 1u << lane);
+      } else {
+        bad = true;
+      }
+    }
+  }
+  if (bad) set_status(status, MOE_STATUS_BAD_EXPERT);
+  __syncthreads();
+  // thread e owns expert e: its picks per warp, in token order, and its served rows
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < n_routed) {
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      pre[w][e] = total;
+      total += __popc(mask[w][e]);
+    }
+    if (counts != nullptr && counts[e] != total) set_status(status, MOE_STATUS_COUNT_MISMATCH);
+  }
+  const int served = total < capacity ? total : capacity;
+  int v = served;  // exclusive scan of the served rows over experts
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_sum[warp] = v;
+  __syncthreads();
+  int before = 0;
+  for (int i = 0; i < warp; ++i) before += warp_sum[i];
+  const int excl = before + v - served;
+  if (e < n_routed) {
+    offsets[e] = excl;
+    off[e] = excl;
+  }
+  if (e == n_routed - 1) offsets[n_routed] = excl + served;
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+    if (ex[j] >= 0) {
+      const int rank = pre[warp][ex[j]] + __popc(mask[warp][ex[j]] & lt);  // place in the expert's queue
+      const int pos = rank < capacity ? off[ex[j]] + rank : -1;
+      token_row[(size_t)t * k + j] = pos;
+      if (pos >= 0) row_token[pos] = t;
+    } else if (j < k && valid) {
+      token_row[(size_t)t * k + j] = -1;
+    }
+  }
+}
+
+// Launches 1-3 in one CTA where a single chunk holds every token; MOE_PERMUTE_ONE_CHUNK=0 keeps three.
+static bool one_chunk_for(int n_chunks) {
+  const char* env = getenv("MOE_PERMUTE_ONE_CHUNK");
+  if (env && env[0] == '0' && env[1] == '\0') return false;
+  return n_chunks == 1;
+}
+
 // x_perm[token_row[t][j]] = x[t] for every slot j: a block copies one token at a time; each thread
 // loads up to COPY_VPT of the row's 16-byte vectors (v, v + THREADS, ...) before writing each of them k
 // times, so several loads are in flight per thread.
@@ -187,12 +274,17 @@ static int launch_permute(const moe_bf16* x, const int32_t* topk_idx, const int3
   int rc = device_info(&dev, &sms);
   if (rc != MOE_OK) return rc;
   const int n_chunks = (T + CHUNK - 1) / CHUNK;
-  int32_t* hist = reinterpret_cast<int32_t*>(scratch);
-  int32_t* base = hist + (size_t)n_chunks * n_routed;
-  chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
-  chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, capacity, counts, offsets, base, status);
-  rank_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, base, offsets, T, top_k, n_routed, capacity, row_token,
-                                           token_row);
+  if (one_chunk_for(n_chunks)) {
+    one_chunk_kernel<<<1, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, capacity, counts, offsets, row_token,
+                                            token_row, status);
+  } else {
+    int32_t* hist = reinterpret_cast<int32_t*>(scratch);
+    int32_t* base = hist + (size_t)n_chunks * n_routed;
+    chunk_hist_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, T, top_k, n_routed, hist, status);
+    chunk_scan_kernel<<<1, THREADS, 0, s>>>(hist, n_chunks, n_routed, capacity, counts, offsets, base, status);
+    rank_kernel<<<n_chunks, THREADS, 0, s>>>(topk_idx, base, offsets, T, top_k, n_routed, capacity, row_token,
+                                             token_row);
+  }
   if (x_perm == nullptr) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;  // indices only
   const int d_vec = d / 8;
   const int grid = (int)((long long)T < (long long)sms * 8 ? T : (long long)sms * 8);  // one token per block at a time

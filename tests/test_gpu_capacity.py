@@ -49,7 +49,9 @@ def _permute_capped(topk, x, cap, n_routed):
     (1000, 8, 256, 128, 30, 0.2), (2048, 6, 64, 32, 240, 0.1), (4097, 6, 256, 256, 120, 0.05),
     (3000, 1, 16, 8, 150, 1.0), (777, 3, 8, 16, 10 ** 6, 0.5),
 ])
-def test_permute_capped_parity(T, k, E, d, cap, skew):
+@pytest.mark.parametrize("one_chunk", ["1", "0"])
+def test_permute_capped_parity(T, k, E, d, cap, skew, one_chunk, monkeypatch):
+    monkeypatch.setenv("MOE_PERMUTE_ONE_CHUNK", one_chunk)  # batches of <= 256 tokens: both index paths
     topk = _topk(T, k, E, T + E, skew)
     x = mi.normal_bf16(T * d, 5, mi.STREAM_X).reshape(T, d)
     keep = oracle.capacity_keep(topk, cap, E)

@@ -89,6 +89,8 @@ def _run_and_check(name, tokens=None, check_all_routing=True, fused=True, gather
             nb = oracle.bias_update(ref_counts, b_host, w.T, w.k, w.gamma)
             np.testing.assert_array_equal(t["bias"].cpu().numpy().view(np.uint32), nb.view(np.uint32))
     _check_dispatch_properties(layer, x_bits, w.T, w.k, w.n_routed)
+    if callable(expert_groups):  # chosen from the routed counts
+        expert_groups = expert_groups(layer.counts.cpu().numpy())
     if expert_groups is not None:
         _check_expert_groups(w, layer, t, x_bits, expert_groups, shared_tokens)
     # layer output on the sampled tokens
@@ -162,7 +164,16 @@ def test_layer_skew_sampled_and_bias_trajectory():
     the oracle's own 20 rounds (routing with the exemption rule; b bit-exact
     while the counts agree)."""
     w = mi.WORKLOADS["skew"]
-    _run_and_check("skew", tokens=np.arange(0, w.T, 509))
+
+    def groups(counts):
+        # the busiest expert, the smallest non-empty one, and two whose last 256-row tile holds at most 128
+        # rows (run as half tiles at this size)
+        nz = np.flatnonzero(counts)
+        half = [int(e) for e in nz if 0 < counts[e] % 256 <= 128 and counts[e] > 256][:2]
+        return sorted({int(np.argmax(counts)), int(nz[np.argmin(counts[nz])]), *half})
+
+    _run_and_check("skew", tokens=np.arange(0, w.T, 509), expert_groups=groups,
+                   shared_tokens=np.arange(0, w.T, 997))
     t, layer = _layer(w, with_weights=False)
     off = mi.host_logit_offset(w)
     x_bits = host_bf16_bits(t["x"])

@@ -284,7 +284,25 @@ def test_gemm_swiglu_fp4_out_matches_oracle(pair, monkeypatch):
     assert n_code <= 1e-3 * total and n_sf <= 1e-3 * total / 16, (n_code, n_sf)
 
 
-def _nvfp4_layer(name, tokens, cap=None):
+def _nvfp4_expert_groups(w, layer, t, experts):
+    """Whole row groups of the NVFP4 expert GEMMs at full size: every y_perm row of each listed expert
+    (its ragged last tile included) against the NVFP4 oracle's expert on the token that row holds.  The
+    hidden layer's FP4 codes decide on fp32 sums in a different order, so a few codes may sit on the
+    other side of a rounding boundary; the rows meet the usual output bar."""
+    off = layer.offsets.cpu().numpy().astype(np.int64)
+    rt = layer.row_token.cpu().numpy()
+    x_bits = host_bf16_bits(t["x"])
+    fn = nvfp4.expert_swiglu if w.activation == "swiglu" else nvfp4.expert
+    for e in experts:
+        lo, hi = int(off[e]), int(off[e + 1])
+        assert hi > lo
+        w1 = nvfp4.quantize_weight(mi.bf16_to_f64(host_bf16_bits(t["w1"][e])).astype(np.float32))
+        w2 = nvfp4.quantize_weight(mi.bf16_to_f64(host_bf16_bits(t["w2"][e])).astype(np.float32))
+        ref = fn(mi.bf16_to_f64(x_bits[rt[lo:hi]]).astype(np.float32), w1, w2)["y"]
+        check_output(host_bf16_f64(layer.y_perm[lo:hi]), ref, f"{w.name} nvfp4 expert {e} rows {lo}..{hi}")
+
+
+def _nvfp4_layer(name, tokens, cap=None, expert_groups=None):
     w = mi.WORKLOADS[name]
     t = mi.torch_workload(w)
     layer = moe.MoELayer(moe.LayerShape(w.T, w.d, w.f, w.n_routed, w.n_shared, w.k), precision="nvfp4",
@@ -294,6 +312,8 @@ def _nvfp4_layer(name, tokens, cap=None):
     out = layer.forward(t["x"], t["w_r"], t["w1"], t["w2"], t["bias"], t["logit_offset"])
     torch.cuda.synchronize()
     assert moe.moe_get_status() == 0
+    if expert_groups is not None:
+        _nvfp4_expert_groups(w, layer, t, expert_groups)
     gpu_idx = layer.topk_idx.cpu().numpy()
     keep = None
     if cap is not None:
@@ -326,8 +346,9 @@ def test_layer_nvfp4_mid_with_capacity():
 
 @pytest.mark.slow
 def test_layer_nvfp4_prefill_sampled():
-    """Full prefill size (65536 tokens, 256 experts of d 7168 / d_ff 2048) with NVFP4 experts."""
-    _nvfp4_layer("prefill", np.array([0, 40000, 65535]))
+    """Full prefill size (65536 tokens, 256 experts of d 7168 / d_ff 2048) with NVFP4 experts: sampled
+    tokens through the whole layer, and every row of the first, a middle and the last expert."""
+    _nvfp4_layer("prefill", np.array([0, 40000, 65535]), expert_groups=[0, 128, 255])
 
 
 def test_nvfp4_zero_tokens_and_empty_experts():

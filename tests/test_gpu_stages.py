@@ -145,11 +145,18 @@ def test_router_zero_tokens_zeroes_counts(router_path):
 # ---------------------------------------------------------------------------
 # permute (dispatch): integer work, bit-exact
 # ---------------------------------------------------------------------------
+@pytest.fixture(params=["one_chunk", "chunked"])
+def permute_path(request, monkeypatch):
+    """Batches of at most 256 tokens: the single-CTA index kernel (default) and the three chunked launches."""
+    monkeypatch.setenv("MOE_PERMUTE_ONE_CHUNK", "1" if request.param == "one_chunk" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T,k,n_routed,d", [
     (1, 6, 256, 64), (7, 2, 8, 16), (255, 6, 256, 128), (256, 6, 256, 64), (257, 3, 64, 72),
     (1000, 8, 256, 256), (4096, 6, 256, 2048), (3000, 1, 16, 8),
 ])
-def test_permute_parity(T, k, n_routed, d):
+def test_permute_parity(T, k, n_routed, d, permute_path):
     topk = _random_topk(T, k, n_routed, T + k)
     x = mi.normal_bf16(T * d, 3, mi.STREAM_X).reshape(T, d)
     ref = oracle.dispatch(topk, n_routed)
@@ -186,8 +193,9 @@ def test_permute_indices_only():
     np.testing.assert_array_equal(tr.cpu().numpy(), ref["token_row"])
 
 
-def test_permute_reports_bad_inputs():
-    T, k, n = 300, 2, 16
+@pytest.mark.parametrize("T", [300, 200])
+def test_permute_reports_bad_inputs(T):
+    k, n = 2, 16
     topk = _random_topk(T, k, n, 5)
     wrong = oracle.load_counts(topk, n)
     wrong[3] += 1
