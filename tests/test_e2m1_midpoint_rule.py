@@ -3,8 +3,10 @@
 An FP4 code is the E2M1 rounding of the value over its block scale, the quotient rounded once to fp32
 ("Under the hood", "Quantization: BF16 vs NVFP4": FP4 elements with FP8 block scales; the oracle takes the
 code of fl32(v / s)).  For a scale s that is a positive E4M3 value the kernels instead compare |v| - t*s,
-rounded once as an fma rounds it, against +-h*s for each E2M1 midpoint t (h: half the fp32 spacing at t;
-"<=" where t's last mantissa bit is even so a tie rounds down onto t, "<" where the tie rounds up onto t).
+rounded once as an fma rounds it, against +-h*s for each E2M1 midpoint t (h: half the fp32 spacing at t
+on the side that matters; "<=" at the midpoints where a value exactly on t takes the lower code, "<" where it
+takes the upper one; a quotient exactly halfway between t and its fp32 neighbour rounds onto t, since every
+midpoint's last mantissa bit is even).
 This test checks that rule, in exact rational arithmetic, against the rounded quotient for every positive
 E4M3 scale at, around and between the midpoints.  It checks the mathematics the kernels rely on; the
 kernels themselves are compared bit for bit with the oracle's division in the GPU tests.
