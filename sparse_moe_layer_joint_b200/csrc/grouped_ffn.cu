@@ -19,12 +19,12 @@
 //               the routed A rows come from the token rows through the row
 //               indices, one tile::gather4 load (four rows) per lane and stage
 //   warp 1      TMEM owner + MMA issuer (one thread): tcgen05.mma kind::f16,
-//               bf16 in, fp32 accumulators in TMEM, two 256-column
+//               bf16 in, fp32 accumulators in TMEM: two 256-column
 //               accumulator buffers so the epilogue of tile i overlaps the
-//               main loop of tile i+1
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, activation, bf16,
-//               16-byte stores of each row's 64-byte chunk
-// Two variants:
+//               main loop of tile i+1 (one 512-column buffer for WIDE tiles)
+//   warps 2-5   epilogue (2-9 for WIDE tiles): tcgen05.ld, activation, bf16,
+//               16-byte stores of each row's 64-byte chunks
+// Variants:
 //   PAIR = false  one CTA per 128 x 256 tile (4-stage ring of 48 KB)
 //   PAIR = true   a cluster of two CTAs per 256 x 256 tile with
 //                 tcgen05.mma.cta_group::2 (M = 256): CTA rank r holds A rows
@@ -736,9 +736,9 @@ struct GemmSpec {
   Params p;
 };
 
-// Kernel variant.  CTA pairs (cta_group::2, 256 x 256 tiles) halve each CTA's shared-memory operand
-// traffic and win when groups are large (compute-bound); with few rows per group the work is weight
-// streaming and single CTAs (128 x 256 tiles, more weight bytes in flight per SM) win.
+// Kernel variant.  CTA pairs (cta_group::2; 256 x 512 tiles by default, see wide_for) halve each CTA's
+// shared-memory operand traffic and win when groups are large (compute-bound); with few rows per group the
+// work is weight streaming and single CTAs (128 x 256 tiles, more weight bytes in flight per SM) win.
 // MOE_GEMM_CTA=1 or =2 forces one of them.
 bool choose_pair(long long rows, int groups) {
   bool pair = groups > 0 && rows / groups >= 256;

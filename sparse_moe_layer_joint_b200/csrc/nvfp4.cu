@@ -25,8 +25,9 @@
 //   weight_amax / weight_quant / weight_scale   weights, once
 //   dispatch_quant   x rows quantized once per token and written to the padded
 //                    rows of its k experts (the FP4 dispatch)
-//   fp4_gemm_kernel<EPI, TN, PAIR>   persistent grouped GEMM, one CTA per 128 x 128
-//                    tile (or 128 x 256; or a CTA pair per 256 x 128 tile):
+//   fp4_gemm_kernel<EPI, TN, PAIR>   persistent grouped GEMM, one CTA per 128 x 256
+//                    tile (128 x 128 where N is not a multiple of 256; or, as an
+//                    option, a CTA pair per 256 x TN tile):
 //                    warp 0 loads code tiles (TMA, 128-byte swizzle) and scale
 //                    atoms (bulk copies), warp 1 copies the scales to TMEM
 //                    (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4 with
@@ -293,10 +294,10 @@ constexpr int SF_ROW = 256;       // scale atoms seen as rows of 256 bytes by th
 constexpr uint32_t TMEM_COLS = 512;
 
 // Tile shapes.
-//   TN = 128 (default): one CTA per 128 x 128 tile, two accumulators (double-buffered epilogue), six
-//     36 KB stages.
-//   TN = 256: twice the MMA work per stage, but two 256-column accumulators leave no TMEM for the scales,
-//     so one accumulator (the next tile's MMAs wait for the epilogue) and four 54 KB stages.
+//   TN = 256 (default where N allows): twice the MMA work per stage of TN = 128; two 256-column
+//     accumulators would leave no TMEM for the scales, so one accumulator, which the epilogue hands back
+//     as soon as it has read it, and four 54 KB stages.
+//   TN = 128: one CTA per 128 x 128 tile, two accumulators, six 36 KB stages.
 //   PAIR: a cluster of two CTAs per 256 x TN tile with tcgen05.mma.cta_group::2.  CTA rank r holds A rows
 //     r*128.. and weight rows r*TN/2.. of the tile (SwiGLU: rank 0 the 128 gate rows, rank 1 the 128
 //     matching up rows), its A rows' scales and the scales of all TN weight rows (the MMA reads SFB from
