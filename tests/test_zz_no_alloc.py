@@ -2,15 +2,17 @@
 allocate device memory (a plugin whose host application owns every device
 allocation, a process that reserved all of HBM up front, a loop that must not
 call cudaMalloc/cudaFree).  Its scratch is a fixed device array inside the
-library; this checks, through the C ABI, that it gives the same outputs as
-moe_permute with a caller scratch buffer, on two calls in a row, and that it
-refuses sizes beyond its limit.  Kept in its own file, collected last."""
+library; this checks, through the C ABI, that it gives the oracle's dispatch
+and the same outputs as moe_permute with a caller scratch buffer, on calls in a
+row, and that it refuses sizes beyond its limit.  Kept in its own file,
+collected last."""
 import ctypes
 
 import numpy as np
 import pytest
 
 import moe_inputs as mi
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -49,8 +51,9 @@ def _with_scratch(x, topk, T, d, n_routed, k, outs):
 
 
 def test_noalloc_permute_matches_permute_on_two_calls_in_a_row():
-    # two different problems back to back: the second must not see the first's scratch
-    for (T, k, n_routed, d, seed) in [(4096, 6, 256, 512, 1), (1000, 8, 64, 136, 2)]:
+    # different problems back to back: a later one must not see an earlier one's scratch (the third fits one
+    # 256-token chunk and takes the single-CTA index kernel)
+    for (T, k, n_routed, d, seed) in [(4096, 6, 256, 512, 1), (1000, 8, 64, 136, 2), (200, 6, 256, 64, 3)]:
         x, topk = _inputs(T, k, n_routed, d, seed)
         ref = _outputs(T, k, n_routed, d)
         got = _outputs(T, k, n_routed, d)
@@ -62,6 +65,14 @@ def test_noalloc_permute_matches_permute_on_two_calls_in_a_row():
             if a.dtype == torch.bfloat16:
                 a, b = a.view(torch.int16), b.view(torch.int16)
             assert torch.equal(a, b)
+        # and directly against the oracle's dispatch
+        want = oracle.dispatch(topk.cpu().numpy(), n_routed)
+        off, xp, rt, tr = got
+        np.testing.assert_array_equal(off.cpu().numpy(), want["offsets"])
+        np.testing.assert_array_equal(rt.cpu().numpy(), want["row_token"])
+        np.testing.assert_array_equal(tr.cpu().numpy(), want["token_row"])
+        x_bits = x.view(torch.int16).cpu().numpy()
+        np.testing.assert_array_equal(xp.view(torch.int16).cpu().numpy(), x_bits[want["row_token"]])
 
 
 def test_noalloc_permute_rejects_sizes_beyond_its_limit():
