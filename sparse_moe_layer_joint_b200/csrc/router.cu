@@ -704,7 +704,10 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1)
 // CTA), keeps them in its own shared memory and routes its tokens: no cluster barrier, no DSMEM.
 constexpr int SINGLE_D_MAX = 512;
 
-template <int K, int TB>
+// U: experts a warp works on at once.  Each round of a warp is a chain of L2 loads and a butterfly
+// reduction, so with narrow rows the latency of the rounds sets the time: more experts a round means fewer
+// rounds (the order of every expert's own sum, and so every logit, is the same for any U).
+template <int K, int TB, int U = SMALL_U>
 __global__ void __launch_bounds__(SMALL_THREADS, 1)
     router_single_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -729,16 +732,16 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1)
   for (int i = tid; i < TB * RED_LD; i += SMALL_THREADS) logits[i] = 0.0f;
   __syncthreads();
   constexpr int SHIFT = 5 - (TB == 1 ? 0 : TB == 2 ? 1 : 2);
-  for (int e0 = warp * SMALL_U; e0 < E; e0 += (SMALL_THREADS / 32) * SMALL_U) {
-    float acc[SMALL_U][TB];
+  for (int e0 = warp * U; e0 < E; e0 += (SMALL_THREADS / 32) * U) {
+    float acc[U][TB];
 #pragma unroll
-    for (int u = 0; u < SMALL_U; ++u)
+    for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int t = 0; t < TB; ++t) acc[u][t] = 0.0f;
     for (int v = lane; v < nv; v += 32) {
-      float wf[SMALL_U][8];
+      float wf[U][8];
 #pragma unroll
-      for (int u = 0; u < SMALL_U; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int e = min(e0 + u, E - 1);
         bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(w + (size_t)e * d) + v), wf[u]);
       }
@@ -747,13 +750,13 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1)
         float xf[8];
         bf16x8_to_f32(xs[t * nv + v], xf);
 #pragma unroll
-        for (int u = 0; u < SMALL_U; ++u)
+        for (int u = 0; u < U; ++u)
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[u][t] = fmaf(xf[j], wf[u][j], acc[u][t]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < SMALL_U; ++u) {
+    for (int u = 0; u < U; ++u) {
       const float v = warp_sum_scatter<TB>(acc[u], lane);
       if (e0 + u < E && (lane & ((1 << SHIFT) - 1)) == 0) logits[(lane >> SHIFT) * RED_LD + e0 + u] = v;
     }
@@ -769,7 +772,12 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1)
 
 template <int K, int TB>
 int launch_single(const __nv_bfloat16* x, const __nv_bfloat16* w, const Params& p, cudaStream_t s) {
-  auto kfn = router_single_kernel<K, TB>;
+  // 16 experts a round for rows of at most 256 values (one 16-byte load per lane and expert) and up to two
+  // tokens a CTA, else 8
+  auto kfn = router_single_kernel<K, TB, 8>;
+  if constexpr (TB <= 2) {
+    if (p.d <= 256) kfn = router_single_kernel<K, TB, 16>;
+  }
   const size_t bytes = small_smem_bytes<TB>(p.d);
   int rc = ensure_smem_attr((const void*)kfn, bytes);
   if (rc != MOE_OK) return rc;
